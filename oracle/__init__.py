@@ -1,0 +1,22 @@
+"""Plain CPU oracle for the Sherry 1.25-bit ternary format (test infrastructure).
+
+Only the test suite, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (the CUDA library and
+its binding) never touches it.  See ``sherry_oracle.c`` for the definitions
+and the readings of the paper it follows.
+"""
+from .oracle import (  # noqa: F401
+    build,
+    packed_bytes,
+    prune_block,
+    block_code,
+    code_weights,
+    pack,
+    unpack,
+    gemv_acc,
+    gemv,
+    gemm_acc,
+    gemm,
+    num_threads,
+    set_num_threads,
+)

@@ -1,0 +1,172 @@
+"""ctypes binding of the C oracle (test infrastructure only).
+
+Argument marshalling only: every computation happens in ``sherry_oracle.c``.
+"""
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "sherry_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle_sherry.so")
+_lib = None
+
+
+def build(force=False):
+    """Compile the oracle with gcc (plain C, OpenMP over output rows)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp%d" % os.getpid()
+        subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-fopenmp", "-o", tmp, _SRC])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load(path=None):
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    lib = ctypes.CDLL(path or build())
+    i64, p = ctypes.c_int64, ctypes.c_void_p
+    lib.oracle_packed_bytes.argtypes = [i64, i64]
+    lib.oracle_packed_bytes.restype = i64
+    lib.oracle_prune_block.argtypes = [p, p, p]
+    lib.oracle_prune_block.restype = None
+    lib.oracle_block_code.argtypes = [ctypes.c_int32, p]
+    lib.oracle_block_code.restype = ctypes.c_int32
+    lib.oracle_code_weights.argtypes = [ctypes.c_int32, p]
+    lib.oracle_code_weights.restype = None
+    lib.oracle_pack.argtypes = [p, i64, i64, p, p]
+    lib.oracle_unpack.argtypes = [p, i64, i64, p]
+    lib.oracle_gemv_acc.argtypes = [p, p, i64, i64, i64, p]
+    lib.oracle_gemv.argtypes = [p, p, p, i64, i64, i64, p]
+    lib.oracle_gemm_acc.argtypes = [p, p, i64, i64, i64, p]
+    lib.oracle_gemm.argtypes = [p, p, p, i64, i64, i64, p]
+    for f in ("oracle_pack", "oracle_unpack", "oracle_gemv_acc", "oracle_gemv",
+              "oracle_gemm_acc", "oracle_gemm"):
+        getattr(lib, f).restype = ctypes.c_int
+    lib.oracle_num_threads.argtypes = []
+    lib.oracle_num_threads.restype = ctypes.c_int
+    lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
+    lib.oracle_set_num_threads.restype = None
+    _lib = lib
+    return lib
+
+
+def use_library(path):
+    """Point the binding at another build of the oracle source (mutation tests);
+    `use_library(None)` returns to the committed source."""
+    global _lib
+    _lib = None
+    if path is not None:
+        _load(path)
+
+
+def _ptr(a):
+    return ctypes.c_void_p(a.ctypes.data)
+
+
+def _check(rc, name):
+    if rc != 0:
+        raise ValueError("%s failed with status %d" % (name, rc))
+
+
+def num_threads():
+    return _load().oracle_num_threads()
+
+
+def set_num_threads(n):
+    _load().oracle_set_num_threads(int(n))
+
+
+def packed_bytes(N, K):
+    return int(_load().oracle_packed_bytes(N, K))
+
+
+def prune_block(w4):
+    w = np.ascontiguousarray(w4, dtype=np.float32)
+    assert w.shape == (4,)
+    p = np.zeros(1, np.int32)
+    neg = np.zeros(3, np.int32)
+    _load().oracle_prune_block(_ptr(w), _ptr(p), _ptr(neg))
+    return int(p[0]), [int(v) for v in neg]
+
+
+def block_code(zero_pos, neg):
+    n = np.ascontiguousarray(neg, dtype=np.int32)
+    return int(_load().oracle_block_code(int(zero_pos), _ptr(n)))
+
+
+def code_weights(code):
+    w = np.zeros(4, np.int8)
+    _load().oracle_code_weights(int(code), _ptr(w))
+    return w
+
+
+def pack(w):
+    """w: float32 [N, K] -> (codes uint32 [5, N, K/128], scales float32 [N])."""
+    w = np.ascontiguousarray(w, dtype=np.float32)
+    N, K = w.shape
+    codes = np.zeros((5, N, K // 128), np.uint32)
+    scales = np.zeros(N, np.float32)
+    _check(_load().oracle_pack(_ptr(w), N, K, _ptr(codes), _ptr(scales)), "oracle_pack")
+    return codes, scales
+
+
+def unpack(codes, K):
+    codes = np.ascontiguousarray(codes, dtype=np.uint32)
+    N = codes.shape[1]
+    wt = np.zeros((N, K), np.int8)
+    _check(_load().oracle_unpack(_ptr(codes), N, K, _ptr(wt)), "oracle_unpack")
+    return wt
+
+
+def _x2(x, K):
+    x = np.ascontiguousarray(x, dtype=np.int8)
+    if x.ndim == 1:
+        x = x.reshape(1, -1)
+    assert x.shape[1] == K
+    return x
+
+
+def gemv_acc(codes, x, K):
+    codes = np.ascontiguousarray(codes, dtype=np.uint32)
+    N = codes.shape[1]
+    x = _x2(x, K)
+    acc = np.zeros((x.shape[0], N), np.int64)
+    _check(_load().oracle_gemv_acc(_ptr(codes), _ptr(x), N, K, x.shape[0], _ptr(acc)),
+           "oracle_gemv_acc")
+    return acc
+
+
+def gemv(codes, scales, x, K):
+    codes = np.ascontiguousarray(codes, dtype=np.uint32)
+    scales = np.ascontiguousarray(scales, dtype=np.float32)
+    N = codes.shape[1]
+    x = _x2(x, K)
+    y = np.zeros((x.shape[0], N), np.float64)
+    _check(_load().oracle_gemv(_ptr(codes), _ptr(scales), _ptr(x), N, K, x.shape[0], _ptr(y)),
+           "oracle_gemv")
+    return y
+
+
+def gemm_acc(codes, x, K):
+    codes = np.ascontiguousarray(codes, dtype=np.uint32)
+    N = codes.shape[1]
+    x = _x2(x, K)
+    acc = np.zeros((x.shape[0], N), np.int64)
+    _check(_load().oracle_gemm_acc(_ptr(codes), _ptr(x), x.shape[0], N, K, _ptr(acc)),
+           "oracle_gemm_acc")
+    return acc
+
+
+def gemm(codes, scales, x, K):
+    codes = np.ascontiguousarray(codes, dtype=np.uint32)
+    scales = np.ascontiguousarray(scales, dtype=np.float32)
+    N = codes.shape[1]
+    x = _x2(x, K)
+    y = np.zeros((x.shape[0], N), np.float64)
+    _check(_load().oracle_gemm(_ptr(codes), _ptr(scales), _ptr(x), x.shape[0], N, K, _ptr(y)),
+           "oracle_gemm")
+    return y

@@ -1,0 +1,244 @@
+/*
+ * sherry_oracle.c -- plain CPU oracle for the Sherry 1.25-bit ternary format.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may call, link or
+ * load this file: only the test suite, the smoke check and the benchmark's
+ * CPU-baseline leg use it.  It shares no code, header, table or constant with
+ * the CUDA library; it restates the format from its written definition.
+ *
+ * What it computes (source: "Sherry: Hardware-Efficient 1.25-Bit Ternary
+ * Quantization via Fine-grained Sparsification", arXiv 2601.07892, abstract
+ * and Figure 2 caption): weights are ternary {-1, 0, +1}; every block of four
+ * consecutive weights along K holds exactly one zero (3:4 sparsity) and is
+ * coded in five bits (4 zero positions x 2^3 sign patterns = 32 states).
+ * The product computed is y = s (.) (W_ternary . x_int8) with one fp32 scale
+ * per output row.
+ *
+ * Readings where the pages are silent (each is restated in the design notes):
+ *  - prune: in each block the weight of smallest |w| becomes the zero; ties go
+ *    to the lowest index (strict '<' while scanning i = 0..3);
+ *  - sign: a kept weight is -1 when w < 0, else +1 (so a kept -0.0 is +1);
+ *  - scale: the mean |w| over the kept weights of the row, summed in double
+ *    in ascending k, divided by the kept count 3K/4, rounded once to fp32;
+ *  - layout: a row is cut into tiles of 128 weights (32 blocks); a tile is
+ *    five 32-bit words Z0, Z1, S0, S1, S2 stored planar:
+ *        word(plane, n, t) = codes[(plane * N + n) * T + t],  T = K / 128,
+ *    plane 0 = Z0, 1 = Z1, 2 = S0, 3 = S1, 4 = S2;
+ *    block j (j = 0..31, weights k = 128 t + 4 j + i, i = 0..3) keeps its
+ *    2-bit zero position p in bits [2*(j/2), 2*(j/2)+1] of Z_(j mod 2);
+ *    the r-th kept weight of block j (r = 0, 1, 2 in ascending i) has its
+ *    sign in bit j of S_r, 1 meaning -1.
+ *  - logical 5-bit code of one block: c = p | s0 << 2 | s1 << 3 | s2 << 4.
+ *
+ * Arithmetic: unpack to int8 {-1, 0, +1}; dot products in int64; the output
+ * is y = (double) s_n * (double) acc, which is exact in double here.
+ */
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#include <math.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+enum { ORC_OK = 0, ORC_BAD_ARG = 1, ORC_NO_MEM = 2 };
+
+#define ORC_TILE 128   /* weights per tile            */
+#define ORC_NBLK 32    /* 4-weight blocks per tile    */
+#define ORC_NPLANE 5   /* 32-bit words per tile       */
+
+static int64_t orc_word(int64_t plane, int64_t n, int64_t t, int64_t N, int64_t T)
+{
+    return (plane * N + n) * T + t;
+}
+
+/* Number of bytes of packed codes for an N x K matrix (scales excluded). */
+int64_t oracle_packed_bytes(int64_t N, int64_t K)
+{
+    if (N < 0 || K < 0 || K % ORC_TILE) return -1;
+    return N * (K / ORC_TILE) * ORC_NPLANE * 4;
+}
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+void oracle_set_num_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
+/* 3:4 prune of one block: zero position (argmin |w|, lowest index on ties)
+ * and the three kept signs in ascending position (1 = negative). */
+void oracle_prune_block(const float *w, int32_t *zero_pos, int32_t *neg)
+{
+    int p = 0;
+    for (int i = 1; i < 4; i++)
+        if (fabsf(w[i]) < fabsf(w[p])) p = i;
+    int r = 0;
+    for (int i = 0; i < 4; i++) {
+        if (i == p) continue;
+        neg[r++] = (w[i] < 0.0f) ? 1 : 0;
+    }
+    *zero_pos = p;
+}
+
+/* Logical 5-bit code of a block from its zero position and kept signs. */
+int32_t oracle_block_code(int32_t zero_pos, const int32_t *neg)
+{
+    return (zero_pos & 3) | (neg[0] & 1) << 2 | (neg[1] & 1) << 3 | (neg[2] & 1) << 4;
+}
+
+/* Ternary values of the four weights of a block given its 5-bit code. */
+void oracle_code_weights(int32_t code, int8_t *w)
+{
+    int p = code & 3, r = 0;
+    for (int i = 0; i < 4; i++) {
+        if (i == p) { w[i] = 0; continue; }
+        w[i] = ((code >> (2 + r)) & 1) ? -1 : 1;
+        r++;
+    }
+}
+
+/* Pack fp32 latent weights W[N][K] (row-major) into codes + per-row scales. */
+int oracle_pack(const float *w, int64_t N, int64_t K, uint32_t *codes, float *scales)
+{
+    if (!w || !codes || !scales || N < 1 || K < ORC_TILE || K % ORC_TILE) return ORC_BAD_ARG;
+    const int64_t T = K / ORC_TILE;
+    #pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; n++) {
+        double sum_abs = 0.0;
+        for (int64_t t = 0; t < T; t++) {
+            uint32_t z[2] = {0, 0}, s[3] = {0, 0, 0};
+            for (int j = 0; j < ORC_NBLK; j++) {
+                const float *blk = w + n * K + t * ORC_TILE + 4 * j;
+                int32_t p, neg[3];
+                oracle_prune_block(blk, &p, neg);
+                z[j & 1] |= (uint32_t)p << (2 * (j >> 1));
+                for (int r = 0; r < 3; r++) s[r] |= (uint32_t)neg[r] << j;
+                for (int i = 0; i < 4; i++)
+                    if (i != p) sum_abs += fabs((double)blk[i]);
+            }
+            codes[orc_word(0, n, t, N, T)] = z[0];
+            codes[orc_word(1, n, t, N, T)] = z[1];
+            codes[orc_word(2, n, t, N, T)] = s[0];
+            codes[orc_word(3, n, t, N, T)] = s[1];
+            codes[orc_word(4, n, t, N, T)] = s[2];
+        }
+        scales[n] = (float)(sum_abs / (0.75 * (double)K));
+    }
+    return ORC_OK;
+}
+
+/* Ternary row n (K int8 values) from the packed codes. */
+static void orc_unpack_row(const uint32_t *codes, int64_t n, int64_t N, int64_t K, int8_t *row)
+{
+    const int64_t T = K / ORC_TILE;
+    for (int64_t t = 0; t < T; t++) {
+        uint32_t z[2] = {codes[orc_word(0, n, t, N, T)], codes[orc_word(1, n, t, N, T)]};
+        uint32_t s[3] = {codes[orc_word(2, n, t, N, T)], codes[orc_word(3, n, t, N, T)],
+                         codes[orc_word(4, n, t, N, T)]};
+        for (int j = 0; j < ORC_NBLK; j++) {
+            int p = (int)((z[j & 1] >> (2 * (j >> 1))) & 3u);
+            int r = 0;
+            for (int i = 0; i < 4; i++) {
+                int8_t v = 0;
+                if (i != p) {
+                    v = ((s[r] >> j) & 1u) ? -1 : 1;
+                    r++;
+                }
+                row[t * ORC_TILE + 4 * j + i] = v;
+            }
+        }
+    }
+}
+
+/* Unpack the whole matrix to int8 Wt[N][K] in {-1, 0, +1}. */
+int oracle_unpack(const uint32_t *codes, int64_t N, int64_t K, int8_t *wt)
+{
+    if (!codes || !wt || N < 1 || K < ORC_TILE || K % ORC_TILE) return ORC_BAD_ARG;
+    #pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; n++) orc_unpack_row(codes, n, N, K, wt + n * K);
+    return ORC_OK;
+}
+
+/* acc[m][n] = sum_k Wt[n][k] * x[m][k] in int64, for M activation rows x[M][K].
+ * The decode GEMV (M = batch) and the prefill GEMM (M = tokens) are the same
+ * definition; both entry points below call this loop. */
+static int orc_matmul_acc(const uint32_t *codes, const int8_t *x, int64_t M, int64_t N,
+                          int64_t K, int64_t *acc)
+{
+    if (!codes || !x || !acc || M < 1 || N < 1 || K < ORC_TILE || K % ORC_TILE) return ORC_BAD_ARG;
+    int err = 0;
+    #pragma omp parallel
+    {
+        int8_t *row = (int8_t *)malloc((size_t)K);
+        if (!row) {
+            #pragma omp atomic write
+            err = 1;
+        }
+        #pragma omp for schedule(static)
+        for (int64_t n = 0; n < N; n++) {
+            if (!row) continue;
+            orc_unpack_row(codes, n, N, K, row);
+            for (int64_t m = 0; m < M; m++) {
+                const int8_t *xm = x + m * K;
+                int64_t a = 0;
+                for (int64_t k = 0; k < K; k++) a += (int64_t)row[k] * (int64_t)xm[k];
+                acc[m * N + n] = a;
+            }
+        }
+        free(row);
+    }
+    return err ? ORC_NO_MEM : ORC_OK;
+}
+
+static int orc_matmul(const uint32_t *codes, const float *scales, const int8_t *x, int64_t M,
+                      int64_t N, int64_t K, double *y)
+{
+    if (!scales || !y) return ORC_BAD_ARG;
+    int64_t *acc = (int64_t *)malloc((size_t)(M * N) * sizeof(int64_t));
+    if (!acc) return ORC_NO_MEM;
+    int rc = orc_matmul_acc(codes, x, M, N, K, acc);
+    if (rc == ORC_OK)
+        for (int64_t m = 0; m < M; m++)
+            for (int64_t n = 0; n < N; n++)
+                y[m * N + n] = (double)scales[n] * (double)acc[m * N + n];
+    free(acc);
+    return rc;
+}
+
+/* Decode GEMV: x[B][K] int8, acc/y[B][N]. */
+int oracle_gemv_acc(const uint32_t *codes, const int8_t *x, int64_t N, int64_t K, int64_t B,
+                    int64_t *acc)
+{
+    return orc_matmul_acc(codes, x, B, N, K, acc);
+}
+
+int oracle_gemv(const uint32_t *codes, const float *scales, const int8_t *x, int64_t N,
+                int64_t K, int64_t B, double *y)
+{
+    return orc_matmul(codes, scales, x, B, N, K, y);
+}
+
+/* Prefill GEMM: x[M][K] int8 (tokens), acc/y[M][N]. */
+int oracle_gemm_acc(const uint32_t *codes, const int8_t *x, int64_t M, int64_t N, int64_t K,
+                    int64_t *acc)
+{
+    return orc_matmul_acc(codes, x, M, N, K, acc);
+}
+
+int oracle_gemm(const uint32_t *codes, const float *scales, const int8_t *x, int64_t M,
+                int64_t N, int64_t K, double *y)
+{
+    return orc_matmul(codes, scales, x, M, N, K, y);
+}

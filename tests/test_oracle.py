@@ -1,0 +1,196 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix.
+
+The pages (arXiv 2601.07892, abstract and Figure 2 caption) fix: ternary
+weights, exactly one zero per block of four (3:4), four weights in five bits
+(1.25 bits/weight), against 2-bit and 1.67-bit (3 weights in 5 bits) packing.
+They print no worked example, so the expected values here are hand-derived
+from the written layout (tests/golden), closed forms, invariants, and brute
+force against numpy's dense int64 matmul on matrices built with a known
+prune.  None of these recompute the oracle's own code path.
+"""
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from tests.helpers import (VALID_BLOCKS, load_tiles, random_ternary, ternary_latents,
+                           ulp_diff_f32)
+
+
+def test_code_space_is_exactly_32_blocks():
+    # 4 zero positions x 2^3 sign patterns = 32 = 2^5 (four weights in five bits).
+    assert len(VALID_BLOCKS) == 32 == 2 ** 5
+    seen = set()
+    for c in range(32):
+        w = tuple(int(v) for v in oracle.code_weights(c))
+        assert w.count(0) == 1 and all(v in (-1, 1) for v in w if v != 0)
+        seen.add(w)
+        p = w.index(0)
+        neg = [1 if v < 0 else 0 for i, v in enumerate(w) if i != p]
+        assert oracle.block_code(p, neg) == c
+    assert seen == set(VALID_BLOCKS)
+
+
+@pytest.mark.parametrize("code,expected", [
+    (0, (0, 1, 1, 1)), (1, (1, 0, 1, 1)), (2, (1, 1, 0, 1)), (3, (1, 1, 1, 0)),
+    (7, (-1, 1, 1, 0)), (30, (-1, -1, 0, -1)), (17, (1, 0, 1, -1)), (12, (0, -1, -1, 1)),
+])
+def test_code_examples(code, expected):
+    # c = p | s0<<2 | s1<<3 | s2<<4, signs of the kept weights in ascending position.
+    assert tuple(int(v) for v in oracle.code_weights(code)) == expected
+
+
+def test_prune_cases(golden_dir):
+    with open(os.path.join(golden_dir, "prune_cases.txt")) as f:
+        lines = [ln for ln in f if ln.strip() and not ln.startswith("#")]
+    assert len(lines) >= 10
+    for ln in lines:
+        lhs, rhs = ln.split("|")
+        w = np.array([float(v) for v in lhs.split()], np.float32)
+        exp = [int(v) for v in rhs.split()]
+        p, neg = oracle.prune_block(w)
+        assert [p] + neg == exp, ln
+
+
+def test_golden_tiles(golden_dir):
+    for t in load_tiles(golden_dir):
+        codes, scales = oracle.pack(t["latent"].reshape(1, 128))
+        got = [int(codes[p, 0, 0]) for p in range(5)]
+        assert got == t["words"], (t["name"], [hex(v) for v in got])
+        assert scales[0] == t["scale"], (t["name"], scales[0], t["scale"])
+        assert np.array_equal(oracle.unpack(codes, 128)[0], t["dense"]), t["name"]
+
+
+def test_golden_words_unpack_without_pack(golden_dir):
+    # Unpack and dot straight from the hand-derived words (no pack involved).
+    for t in load_tiles(golden_dir):
+        codes = np.array(t["words"], np.uint32).reshape(5, 1, 1)
+        assert np.array_equal(oracle.unpack(codes, 128)[0], t["dense"]), t["name"]
+        x = synth.int8_uniform((3, 128), seed=11)
+        acc = oracle.gemv_acc(codes, x, 128)
+        assert np.array_equal(acc[:, 0], x.astype(np.int64) @ t["dense"].astype(np.int64))
+
+
+def test_planar_layout_across_rows_and_tiles(golden_dir):
+    tiles = {t["name"][0]: t for t in load_tiles(golden_dir)}
+    # row 0 = [A | B], row 1 = [C | E], row 2 = [G | F]
+    rows = [("A", "B"), ("C", "E"), ("G", "F")]
+    lat = np.stack([np.concatenate([tiles[a]["latent"], tiles[b]["latent"]]) for a, b in rows])
+    codes, scales = oracle.pack(lat)
+    assert codes.shape == (5, 3, 2)
+    flat = codes.reshape(-1)
+    N, T = 3, 2
+    for n, pair in enumerate(rows):
+        for t, name in enumerate(pair):
+            for p in range(5):
+                assert flat[(p * N + n) * T + t] == tiles[name]["words"][p]
+    # mean over 192 kept weights: [A|B] = (96*1 + 96*2)/192 = 1.5
+    assert scales[0] == np.float32(1.5)
+    assert scales[1] == np.float32((96 * 2 + 96 * 3) / 192)
+    assert scales[2] == np.float32((64 + 56) / 192)
+
+
+def test_all_32_codes_in_one_tile():
+    rng = np.random.default_rng(5)
+    T = np.array(VALID_BLOCKS, np.int8).reshape(1, 128)   # block j = pattern j
+    lat = ternary_latents(T, rng)
+    codes, _ = oracle.pack(lat)
+    assert np.array_equal(oracle.unpack(codes, 128), T)
+
+
+def test_random_words_decode_to_valid_blocks():
+    # Every 5-bit pattern is a valid block: any words unpack to exactly one zero per block.
+    rng = np.random.default_rng(7)
+    codes = rng.integers(0, 2 ** 32, size=(5, 7, 3), dtype=np.uint64).astype(np.uint32)
+    wt = oracle.unpack(codes, 384).reshape(7, 96, 4)
+    assert np.all((wt == 0).sum(axis=2) == 1)
+    assert np.all(np.isin(wt, (-1, 0, 1)))
+
+
+def test_pack_unpack_roundtrip_and_scale():
+    rng = np.random.default_rng(3)
+    for N, K in [(1, 128), (9, 384), (4, 1024)]:
+        T = random_ternary(N, K, rng)
+        lat = ternary_latents(T, rng)
+        codes, scales = oracle.pack(lat)
+        assert np.array_equal(oracle.unpack(codes, K), T)
+        kept_mean = np.where(T != 0, np.abs(lat.astype(np.float64)), 0).sum(1) / (0.75 * K)
+        assert np.all(ulp_diff_f32(scales, kept_mean.astype(np.float32)) <= 1)
+
+
+def test_constant_magnitude_rows_have_exact_scale():
+    rng = np.random.default_rng(9)
+    for a in (0.02, 1.0 / 3.0, 7.5e-3, 1e-20):
+        a32 = np.float32(a)
+        lat = (rng.choice([-1, 1], size=(3, 512)) * a32).astype(np.float32)
+        _, s = oracle.pack(lat)
+        assert np.all(s == a32)
+
+
+def test_zero_rows_and_zero_activations():
+    lat = np.zeros((2, 256), np.float32)
+    codes, s = oracle.pack(lat)
+    assert np.all(s == 0.0)
+    x = synth.int8_uniform((2, 256), seed=4)
+    assert np.all(oracle.gemv(codes, s, x, 256) == 0.0)
+    lat = synth.latent_weights(5, 256, seed=2)
+    codes, s = oracle.pack(lat)
+    assert np.all(oracle.gemv(codes, s, np.zeros((1, 256), np.int8), 256) == 0.0)
+
+
+def test_all_ones_activation_gives_sum_of_signs():
+    N, K = 33, 640
+    lat = synth.latent_weights(N, K, seed=0)
+    codes, _ = oracle.pack(lat)
+    acc = oracle.gemv_acc(codes, np.ones((1, K), np.int8), K)[0]
+    neg = np.array([sum(bin(int(w)).count("1") for w in codes[2:, n, :].reshape(-1))
+                    for n in range(N)])
+    assert np.array_equal(acc, 3 * K // 4 - 2 * neg)
+
+
+@pytest.mark.parametrize("N", [1, 3, 17])
+@pytest.mark.parametrize("K", [128, 256, 640])
+@pytest.mark.parametrize("B", [1, 2, 5])
+def test_bruteforce_dense_matmul(N, K, B):
+    rng = np.random.default_rng(N * 1000 + K + B)
+    T = random_ternary(N, K, rng)
+    lat = ternary_latents(T, rng)
+    codes, scales = oracle.pack(lat)
+    x = rng.integers(-128, 128, size=(B, K)).astype(np.int8)
+    ref = x.astype(np.int64) @ T.astype(np.int64).T
+    assert np.array_equal(oracle.gemv_acc(codes, x, K), ref)
+    assert np.array_equal(oracle.gemm_acc(codes, x, K), ref)
+    y = oracle.gemv(codes, scales, x, K)
+    assert np.array_equal(y, scales.astype(np.float64)[None, :] * ref)
+    assert np.array_equal(oracle.gemm(codes, scales, x, K), y)
+
+
+def test_extreme_activations_bound():
+    # |acc| <= (3K/4) * 128: all kept weights aligned with x = -128 / +127.
+    K = 1024
+    T = np.tile(np.array([1, 1, 1, 0], np.int8), (2, K // 4))
+    T[1] *= -1
+    lat = ternary_latents(T, np.random.default_rng(0))
+    codes, _ = oracle.pack(lat)
+    x = np.full((2, K), -128, np.int8)
+    x[1] = 127
+    acc = oracle.gemv_acc(codes, x, K)
+    assert acc[0, 0] == -128 * 3 * K // 4 and acc[0, 1] == 128 * 3 * K // 4
+    assert acc[1, 0] == 127 * 3 * K // 4 and acc[1, 1] == -127 * 3 * K // 4
+
+
+def test_size_closed_forms():
+    for N, K in [(1, 128), (256, 1024), (2048, 8192), (8192, 2048)]:
+        nbytes = oracle.packed_bytes(N, K)
+        assert nbytes * 32 == N * K * 5          # 5 bits per 4 weights
+        assert 8 * nbytes / (N * K) == 1.25      # 1.25 bits per weight (scales excluded)
+    assert 1 - 1.25 / (5 / 3) == pytest.approx(0.25, abs=1e-15)   # vs 3-in-5-bit packing
+    assert 1 - 1.25 / 2 == 0.375                                  # vs 2-bit packing
+    assert oracle.packed_bytes(4, 100) == -1
+
+
+def test_bad_shapes_rejected():
+    with pytest.raises(Exception):
+        oracle.pack(np.zeros((2, 100), np.float32))
