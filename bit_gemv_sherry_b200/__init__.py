@@ -1,0 +1,9 @@
+"""B200-native Sherry 1.25-bit ternary GEMV/GEMM (sm_100a CUDA kernels behind a C ABI).
+
+The compute path lives in ``libsherry.so`` (``csrc/``, header ``include/sherry.h``);
+``sherry`` is its thin Python binding.
+"""
+from .sherry import (  # noqa: F401
+    SherryError, device_error, gemm, gemm_acc, gemv, gemv_acc, gemv_grouped,
+    gemv_workspace_bytes, lib, library_path, pack, packed_bytes, workspace,
+)

@@ -1,0 +1,218 @@
+"""Python binding of libsherry.so (argument marshalling only).
+
+Every step of the path runs in the library's CUDA kernels; this module only
+checks tensor properties, passes raw device pointers and the current CUDA
+stream, and turns status codes into exceptions.  PyTorch provides device
+memory and streams.  There is no CPU fallback: if the library cannot be
+loaded, importing the functions raises.
+"""
+import ctypes
+import os
+
+import torch
+
+from . import build as _build
+
+_lib = None
+
+STATUS = {
+    0: "SHERRY_OK", 1: "SHERRY_ERR_NULL", 2: "SHERRY_ERR_SHAPE", 3: "SHERRY_ERR_ALIGN",
+    4: "SHERRY_ERR_UNSUPPORTED", 5: "SHERRY_ERR_CUDA", 6: "SHERRY_ERR_TIMEOUT",
+    7: "SHERRY_ERR_WORKSPACE",
+}
+TILE_K = 128
+MAX_GEMV_BATCH = 16
+MAX_GROUP = 128
+
+
+class SherryError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        msg = "%s: %s (%s)" % (where, STATUS.get(status, status),
+                               lib().sherry_status_string(status).decode())
+        if status == 5:
+            msg += ": " + lib().sherry_last_error().decode()
+        super().__init__(msg)
+
+
+class GemvDesc(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("x", ctypes.c_void_p),
+                ("y", ctypes.c_void_p), ("N", ctypes.c_int64), ("K", ctypes.c_int64)]
+
+
+def library_path():
+    return _build.LIB
+
+
+def lib():
+    """Load libsherry.so (built in-tree).  Raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = _build.LIB
+    if not os.path.exists(path):
+        raise RuntimeError("libsherry.so not built: run `python -m bit_gemv_sherry_b200.build` "
+                           "(expected at %s)" % path)
+    L = ctypes.CDLL(path)
+    p, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+    sig = {
+        "sherry_packed_bytes": ([i64, i64], sz),
+        "sherry_pack": ([p, i64, i64, p, p, p], i32),
+        "sherry_gemv_workspace_bytes": ([i64, i32], sz),
+        "sherry_gemv": ([p, p, p, p, i64, i64, i32, p, sz, p], i32),
+        "sherry_gemv_acc": ([p, p, p, i64, i64, i32, p, sz, p], i32),
+        "sherry_gemv_grouped": ([p, i32, i32, p, sz, p], i32),
+        "sherry_gemm": ([p, p, p, p, i64, i64, i64, p], i32),
+        "sherry_gemm_acc": ([p, p, p, i64, i64, i64, p], i32),
+        "sherry_device_error": ([], i32),
+        "sherry_status_string": ([i32], ctypes.c_char_p),
+        "sherry_last_error": ([], ctypes.c_char_p),
+        "sherry_version": ([], i32),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(L, name)
+        f.argtypes = args
+        f.restype = res
+    _lib = L
+    return L
+
+
+def _check(status, where):
+    if status != 0:
+        raise SherryError(status, where)
+
+
+def _stream(t):
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _need(t, dtype, name):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError("%s must be a CUDA tensor" % name)
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+
+
+_workspaces = {}
+
+
+def workspace(nbytes, device):
+    """A cached device scratch buffer of at least `nbytes` for (device, current stream)."""
+    device = torch.device(device)
+    key = (device.index, torch.cuda.current_stream(device).cuda_stream)
+    buf = _workspaces.get(key)
+    if buf is None or buf.numel() < nbytes:
+        buf = torch.empty(max(nbytes, 1 << 16), dtype=torch.uint8, device=device)
+        _workspaces[key] = buf
+    return buf
+
+
+def packed_bytes(N, K):
+    return int(lib().sherry_packed_bytes(N, K))
+
+
+def gemv_workspace_bytes(K, B):
+    return int(lib().sherry_gemv_workspace_bytes(K, B))
+
+
+def pack(w, codes=None, scales=None):
+    """w: float32 [N, K] CUDA -> (codes int32 [5, N, K/128] (uint32 bit patterns), scales [N])."""
+    _need(w, torch.float32, "w")
+    N, K = w.shape
+    if codes is None:
+        codes = torch.empty((5, N, max(K // TILE_K, 1)), dtype=torch.int32, device=w.device)
+    if scales is None:
+        scales = torch.empty(N, dtype=torch.float32, device=w.device)
+    _check(lib().sherry_pack(_ptr(w), N, K, _ptr(codes), _ptr(scales), _stream(w)), "sherry_pack")
+    return codes, scales
+
+
+def _codes_shape(codes):
+    _need(codes, torch.int32, "codes")
+    if codes.dim() != 3 or codes.shape[0] != 5:
+        raise ValueError("codes must have shape [5, N, K/128]")
+    return codes.shape[1], codes.shape[2] * TILE_K
+
+
+def gemv(codes, scales, x, y=None, ws=None):
+    """y[B, N] = scales * (W . x^T); x int8 [B, K] (or [K])."""
+    N, K = _codes_shape(codes)
+    _need(scales, torch.float32, "scales")
+    _need(x, torch.int8, "x")
+    x2 = x.view(1, -1) if x.dim() == 1 else x
+    B = x2.shape[0]
+    if y is None:
+        y = torch.empty((B, N), dtype=torch.float32, device=x.device)
+    nb = gemv_workspace_bytes(K, B)
+    ws = workspace(nb, x.device) if ws is None else ws
+    _check(lib().sherry_gemv(_ptr(codes), _ptr(scales), _ptr(x2), _ptr(y), N, K, B, _ptr(ws),
+                             ws.numel(), _stream(x)), "sherry_gemv")
+    return y
+
+
+def gemv_acc(codes, x, acc=None, ws=None):
+    N, K = _codes_shape(codes)
+    _need(x, torch.int8, "x")
+    x2 = x.view(1, -1) if x.dim() == 1 else x
+    B = x2.shape[0]
+    if acc is None:
+        acc = torch.empty((B, N), dtype=torch.int32, device=x.device)
+    nb = gemv_workspace_bytes(K, B)
+    ws = workspace(nb, x.device) if ws is None else ws
+    _check(lib().sherry_gemv_acc(_ptr(codes), _ptr(x2), _ptr(acc), N, K, B, _ptr(ws), ws.numel(),
+                                 _stream(x)), "sherry_gemv_acc")
+    return acc
+
+
+def gemv_grouped(items, B, ws=None):
+    """items: list of (codes, scales, x [B, K], y [B, N]); runs every GEMV in one pass."""
+    n = len(items)
+    descs = (GemvDesc * n)()
+    total = 0
+    dev = None
+    for i, (codes, scales, x, y) in enumerate(items):
+        N, K = _codes_shape(codes)
+        _need(scales, torch.float32, "scales")
+        _need(x, torch.int8, "x")
+        _need(y, torch.float32, "y")
+        descs[i] = GemvDesc(codes.data_ptr(), scales.data_ptr(), x.data_ptr(), y.data_ptr(), N, K)
+        total += gemv_workspace_bytes(K, B)
+        dev = x.device
+    ws = workspace(total, dev) if ws is None else ws
+    _check(lib().sherry_gemv_grouped(ctypes.cast(descs, ctypes.c_void_p), n, B, _ptr(ws),
+                                     ws.numel(), _stream(items[0][2])), "sherry_gemv_grouped")
+
+
+def gemm(codes, scales, x, y=None):
+    """y[M, N] = scales * (x . W^T); x int8 [M, K]."""
+    N, K = _codes_shape(codes)
+    _need(scales, torch.float32, "scales")
+    _need(x, torch.int8, "x")
+    M = x.shape[0]
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.float32, device=x.device)
+    _check(lib().sherry_gemm(_ptr(codes), _ptr(scales), _ptr(x), _ptr(y), M, N, K, _stream(x)),
+           "sherry_gemm")
+    return y
+
+
+def gemm_acc(codes, x, acc=None):
+    N, K = _codes_shape(codes)
+    _need(x, torch.int8, "x")
+    M = x.shape[0]
+    if acc is None:
+        acc = torch.empty((M, N), dtype=torch.int32, device=x.device)
+    _check(lib().sherry_gemm_acc(_ptr(codes), _ptr(x), _ptr(acc), M, N, K, _stream(x)),
+           "sherry_gemm_acc")
+    return acc
+
+
+def device_error():
+    """Synchronise and return (and clear) the device-side error word (0 = none)."""
+    return int(lib().sherry_device_error())

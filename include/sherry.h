@@ -1,0 +1,201 @@
+/*
+ * sherry.h -- C ABI of libsherry.so: the Sherry 1.25-bit ternary weight format
+ * on NVIDIA B200 (sm_100a).
+ *
+ * The method ("Sherry: Hardware-Efficient 1.25-Bit Ternary Quantization via
+ * Fine-grained Sparsification", arXiv 2601.07892, abstract; Figure 2 caption)
+ * keeps weights in {-1, 0, +1} with 3:4 fine-grained sparsity -- every block of
+ * four consecutive weights along K holds exactly one zero -- and codes each
+ * block in five bits (4 zero positions x 2^3 signs = 32 states), a regular
+ * 1.25 bits per weight.  The product it serves is
+ *
+ *     y[b][n] = s[n] * sum_k W[n][k] * x[b][k],    W ternary, x int8, s fp32.
+ *
+ * ---------------------------------------------------------------------------
+ * Packed layout (the pages fix only "four weights in five bits"; this layout is
+ * the library's reading, chosen so that 32 blocks decode with 32-bit SWAR
+ * logic):
+ *   - a row of K weights (K a multiple of 128) is cut into T = K / 128 tiles of
+ *     128 weights = 32 blocks; weight k = 128 t + 4 j + i is position i of
+ *     block j of tile t;
+ *   - a tile is five uint32 words Z0, Z1, S0, S1, S2 (20 bytes per 128
+ *     weights, exactly 1.25 bits per weight), stored planar:
+ *         codes[(plane * N + n) * T + t],  plane 0..4 = Z0, Z1, S0, S1, S2,
+ *     so each plane of a row is contiguous and vector-loadable;
+ *   - block j's zero position p (0..3) is the 2-bit field at bits
+ *     [2*(j/2), 2*(j/2)+1] of Z_(j mod 2) (Z0 holds the even blocks, Z1 the
+ *     odd ones);
+ *   - the r-th kept weight of block j (r = 0, 1, 2, in ascending position)
+ *     has its sign at bit j of S_r, 1 meaning -1.
+ *   - scales[n] is one fp32 per output row.
+ * Pack rule (not on the pages; the library's reading): in each block the
+ * weight of smallest |w| is zeroed (ties go to the lowest index), a kept
+ * weight becomes -1 if w < 0 and +1 otherwise, and scales[n] is the mean |w|
+ * of the row's kept weights (3K/4 of them), accumulated in double and rounded
+ * once to fp32.
+ *
+ * ---------------------------------------------------------------------------
+ * Conventions shared by every call
+ *   - Every pointer argument is a DEVICE pointer unless stated otherwise; the
+ *     caller allocates and owns every buffer.  The library keeps no device
+ *     allocation between calls.
+ *   - Calls are asynchronous on `stream` (NULL = legacy default stream).  The
+ *     checks listed under each call run on the host before any launch and
+ *     return an error without touching the GPU.  A launch failure returns
+ *     SHERRY_ERR_CUDA; the CUDA error text is then available from
+ *     sherry_last_error().  Errors inside a running kernel surface as CUDA
+ *     errors at the caller's next synchronisation.
+ *   - No C++ exception crosses this interface.  Calls are thread-safe; two
+ *     calls that share an output or a workspace must not overlap on the GPU.
+ *   - Integer results are exact: the dot products are accumulated in int32,
+ *     which cannot overflow for K <= SHERRY_MAX_K, and converted to fp32
+ *     exactly (|acc| <= 3K/4 * 128 < 2^24), so y = fl32(s * acc) with one
+ *     rounding.
+ */
+#ifndef SHERRY_H
+#define SHERRY_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Opaque CUDA stream handle; identical to cudaStream_t / CUstream. */
+struct CUstream_st;
+typedef struct CUstream_st *sherry_stream_t;
+
+typedef enum {
+    SHERRY_OK = 0,
+    SHERRY_ERR_NULL = 1,        /* a required pointer is NULL                          */
+    SHERRY_ERR_SHAPE = 2,       /* N, M or B < 1, K < 128 or K % 128 != 0, K too large */
+    SHERRY_ERR_ALIGN = 3,       /* a pointer is not aligned as the call requires        */
+    SHERRY_ERR_UNSUPPORTED = 4, /* a size beyond what the kernels support (e.g. B > 16) */
+    SHERRY_ERR_CUDA = 5,        /* a CUDA call or launch failed                         */
+    SHERRY_ERR_TIMEOUT = 6,     /* a bounded device-side wait ran out (see below)       */
+    SHERRY_ERR_WORKSPACE = 7    /* workspace missing or smaller than required           */
+} sherry_status;
+
+#define SHERRY_TILE_K 128         /* weights per tile                     */
+#define SHERRY_WORDS_PER_TILE 5   /* uint32 words per tile                */
+#define SHERRY_MAX_K 131072       /* keeps |acc| < 2^24                   */
+#define SHERRY_MAX_GEMV_BATCH 16  /* activation rows per GEMV call        */
+#define SHERRY_MAX_GROUP 128      /* GEMVs per grouped call               */
+
+/* Bytes of packed codes for an N x K matrix: N * K * 5 / 32 (scales excluded).
+ * Returns 0 when K is not a positive multiple of 128 or N < 1. */
+size_t sherry_packed_bytes(int64_t N, int64_t K);
+
+/*
+ * sherry_pack -- 3:4 prune, ternarise, encode and scale (arXiv 2601.07892,
+ * abstract: "packing blocks of four weights into five bits").
+ *   w       [N][K] fp32, row-major, finite values (NaN/Inf give an unspecified
+ *           but deterministic code); 16-byte aligned.
+ *   codes   output, sherry_packed_bytes(N, K) bytes, layout above; 4-byte aligned.
+ *   scales  output, N fp32.
+ * Errors: NULL, SHAPE (N < 1, K not a positive multiple of 128, K > SHERRY_MAX_K),
+ * ALIGN, CUDA.
+ */
+sherry_status sherry_pack(const float *w, int64_t N, int64_t K, uint32_t *codes,
+                          float *scales, sherry_stream_t stream);
+
+/*
+ * Workspace of the GEMV calls: the activations are re-ordered once per call
+ * into the order in which the decoded weights meet the tensor-core fragments.
+ * sherry_gemv_workspace_bytes(K, B) is the size one GEMV needs (B * K bytes,
+ * rounded up to 256); the grouped call needs the sum over its GEMVs.  The
+ * workspace is a device buffer, 256-byte aligned, owned by the caller; its
+ * contents are scratch and are overwritten by every call.
+ */
+size_t sherry_gemv_workspace_bytes(int64_t K, int B);
+
+/*
+ * sherry_gemv -- decode GEMV, y = s (.) (W_ternary . x_int8) for B <= 16
+ * activation rows (arXiv 2601.07892, abstract: ternary weights served by
+ * hardware-aligned packing; the batch-1 case is the decode step).
+ *   codes   [5][N][K/128] uint32 from sherry_pack (or the same layout); 4-byte aligned.
+ *   scales  [N] fp32.
+ *   x       [B][K] int8, row-major, any value in [-128, 127]; 4-byte aligned.
+ *   y       [B][N] fp32 output, row-major.
+ *   workspace / workspace_bytes: see sherry_gemv_workspace_bytes.
+ * Errors: NULL, SHAPE, ALIGN, UNSUPPORTED (B > 16), WORKSPACE, CUDA.
+ */
+sherry_status sherry_gemv(const uint32_t *codes, const float *scales, const int8_t *x,
+                          float *y, int64_t N, int64_t K, int B, void *workspace,
+                          size_t workspace_bytes, sherry_stream_t stream);
+
+/* As sherry_gemv, but writes the exact integer accumulators acc[B][N] (int32,
+ * row-major) instead of scaled outputs; no scales are read.  For bit-exact
+ * checks of the decode and the dot products. */
+sherry_status sherry_gemv_acc(const uint32_t *codes, const int8_t *x, int32_t *acc,
+                              int64_t N, int64_t K, int B, void *workspace,
+                              size_t workspace_bytes, sherry_stream_t stream);
+
+/* One GEMV of a grouped call.  All pointers are device pointers with the
+ * alignment sherry_gemv requires. */
+typedef struct {
+    const uint32_t *codes;
+    const float *scales;
+    const int8_t *x;   /* [B][K] */
+    float *y;          /* [B][N] */
+    int64_t N;
+    int64_t K;
+} sherry_gemv_desc;
+
+/*
+ * sherry_gemv_grouped -- `count` independent GEMVs (count <= SHERRY_MAX_GROUP),
+ * all with the same batch B, in one pass: one activation re-ordering launch
+ * and one GEMV launch whose warps stream the codes of every GEMV.  This is the
+ * decode step of a whole stack of layers whose inputs are already known.
+ *   descs  HOST array of `count` descriptors (copied into the launch
+ *          parameters; may be reused as soon as the call returns).
+ *   workspace: at least the sum over the group of
+ *          sherry_gemv_workspace_bytes(K_i, B) bytes.
+ * Errors: as sherry_gemv, per descriptor; UNSUPPORTED if count > SHERRY_MAX_GROUP.
+ */
+sherry_status sherry_gemv_grouped(const sherry_gemv_desc *descs, int count, int B,
+                                  void *workspace, size_t workspace_bytes,
+                                  sherry_stream_t stream);
+
+/*
+ * sherry_gemm -- prefill GEMM, Y = X . W^T scaled per output column,
+ *   Y[m][n] = s[n] * sum_k X[m][k] * W[n][k]   (the same product for M tokens).
+ * The kernel decodes weight tiles to int8 in shared memory and runs them on
+ * the tcgen05 int8 tensor-core path with int32 accumulators in tensor memory.
+ *   codes   [5][N][K/128] uint32; 4-byte aligned.
+ *   scales  [N] fp32.
+ *   x       [M][K] int8 row-major; 16-byte aligned (tensor-memory-access copies).
+ *   y       [M][N] fp32 output, row-major.
+ * Errors: NULL, SHAPE, ALIGN, CUDA, TIMEOUT (only through sherry_device_error).
+ */
+sherry_status sherry_gemm(const uint32_t *codes, const float *scales, const int8_t *x,
+                          float *y, int64_t M, int64_t N, int64_t K, sherry_stream_t stream);
+
+/* As sherry_gemm, writing exact int32 accumulators acc[M][N]. */
+sherry_status sherry_gemm_acc(const uint32_t *codes, const int8_t *x, int32_t *acc,
+                              int64_t M, int64_t N, int64_t K, sherry_stream_t stream);
+
+/*
+ * Device-side error word.  Kernels that wait on barriers bound every wait;
+ * when one runs out the kernel records SHERRY_ERR_TIMEOUT here, releases what
+ * it holds and returns instead of hanging.  sherry_device_error() synchronises
+ * the current device, returns the recorded status (SHERRY_OK if none) and
+ * clears it.
+ */
+sherry_status sherry_device_error(void);
+
+/* Text of a status code (static string). */
+const char *sherry_status_string(sherry_status status);
+
+/* Text of the last CUDA error seen by this thread in a library call. */
+const char *sherry_last_error(void);
+
+/* Library version as MAJOR * 10000 + MINOR * 100 + PATCH. */
+int sherry_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SHERRY_H */

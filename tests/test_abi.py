@@ -1,0 +1,100 @@
+"""The C ABI library loads, exports every declared entry point, and rejects bad
+arguments on the host before touching a GPU (no CUDA device needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from bit_gemv_sherry_b200 import sherry as S
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sherry.h")
+FAKE = ctypes.c_void_p(0x100000)      # never dereferenced: checks fail first
+FAKE_WS = ctypes.c_void_p(0x200000)   # 256-aligned fake workspace
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(sherry_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_function():
+    L = S.lib()
+    names = declared_functions()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings_and_version():
+    L = S.lib()
+    for code in range(8):
+        assert L.sherry_status_string(code)
+    assert L.sherry_version() >= 100
+
+
+def test_packed_and_workspace_sizes():
+    assert S.packed_bytes(256, 1024) == 256 * 1024 * 5 // 32
+    assert S.packed_bytes(3, 100) == 0
+    assert S.packed_bytes(0, 128) == 0
+    assert S.gemv_workspace_bytes(2048, 1) == 2048
+    assert S.gemv_workspace_bytes(384, 3) == 1280       # 1152 rounded up to 256
+    assert S.gemv_workspace_bytes(128, 0) == 0
+
+
+def test_pack_argument_checks():
+    L = S.lib()
+    assert L.sherry_pack(None, 4, 128, FAKE, FAKE, None) == 1
+    assert L.sherry_pack(FAKE, 0, 128, FAKE, FAKE, None) == 2
+    assert L.sherry_pack(FAKE, 4, 100, FAKE, FAKE, None) == 2
+    assert L.sherry_pack(FAKE, 4, 131072 + 128, FAKE, FAKE, None) == 2
+    assert L.sherry_pack(ctypes.c_void_p(0x100004), 4, 128, FAKE, FAKE, None) == 3
+
+
+def test_gemv_argument_checks():
+    L = S.lib()
+    ws = 1 << 20
+    assert L.sherry_gemv(None, FAKE, FAKE, FAKE, 4, 128, 1, FAKE_WS, ws, None) == 1
+    assert L.sherry_gemv(FAKE, None, FAKE, FAKE, 4, 128, 1, FAKE_WS, ws, None) == 1
+    assert L.sherry_gemv(FAKE, FAKE, FAKE, FAKE, 0, 128, 1, FAKE_WS, ws, None) == 2
+    assert L.sherry_gemv(FAKE, FAKE, FAKE, FAKE, 4, 130, 1, FAKE_WS, ws, None) == 2
+    assert L.sherry_gemv(FAKE, FAKE, FAKE, FAKE, 4, 128, 0, FAKE_WS, ws, None) == 2
+    assert L.sherry_gemv(FAKE, FAKE, FAKE, FAKE, 4, 128, 17, FAKE_WS, ws, None) == 4
+    assert L.sherry_gemv(FAKE, FAKE, ctypes.c_void_p(0x100002), FAKE, 4, 128, 1, FAKE_WS, ws,
+                         None) == 3
+    assert L.sherry_gemv(FAKE, FAKE, FAKE, FAKE, 4, 128, 1, None, ws, None) == 7
+    assert L.sherry_gemv(FAKE, FAKE, FAKE, FAKE, 4, 128, 1, ctypes.c_void_p(0x200010), ws,
+                         None) == 3
+    assert L.sherry_gemv(FAKE, FAKE, FAKE, FAKE, 4, 1024, 2, FAKE_WS, 1024, None) == 7
+    assert L.sherry_gemv_acc(FAKE, FAKE, None, 4, 128, 1, FAKE_WS, ws, None) == 1
+
+
+def test_grouped_argument_checks():
+    L = S.lib()
+    d = (S.GemvDesc * 2)()
+    d[0] = S.GemvDesc(0x100000, 0x100000, 0x100000, 0x100000, 16, 128)
+    d[1] = S.GemvDesc(0x100000, 0, 0x100000, 0x100000, 16, 128)
+    p = ctypes.cast(d, ctypes.c_void_p)
+    assert L.sherry_gemv_grouped(None, 1, 1, FAKE_WS, 1 << 20, None) == 1
+    assert L.sherry_gemv_grouped(p, 0, 1, FAKE_WS, 1 << 20, None) == 2
+    assert L.sherry_gemv_grouped(p, 129, 1, FAKE_WS, 1 << 20, None) == 4
+    assert L.sherry_gemv_grouped(p, 2, 1, FAKE_WS, 1 << 20, None) == 1    # desc 1 has no scales
+    d[1] = S.GemvDesc(0x100000, 0x100000, 0x100000, 0x100000, 16, 200)
+    assert L.sherry_gemv_grouped(p, 2, 1, FAKE_WS, 1 << 20, None) == 2
+
+
+def test_gemm_argument_checks():
+    L = S.lib()
+    assert L.sherry_gemm(None, FAKE, FAKE, FAKE, 4, 4, 128, None) == 1
+    assert L.sherry_gemm(FAKE, FAKE, FAKE, FAKE, 0, 4, 128, None) == 2
+    assert L.sherry_gemm(FAKE, FAKE, FAKE, FAKE, 4, 4, 64, None) == 2
+    assert L.sherry_gemm(FAKE, FAKE, ctypes.c_void_p(0x100008), FAKE, 4, 4, 128, None) == 3
+    assert L.sherry_gemm_acc(FAKE, FAKE, None, 4, 4, 128, None) == 1
+
+
+def test_python_binding_rejects_cpu_tensors():
+    import torch
+    with pytest.raises(TypeError):
+        S.pack(torch.zeros(4, 128))

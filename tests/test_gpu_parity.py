@@ -1,0 +1,184 @@
+"""CUDA path vs the CPU oracle on the same seeded inputs (needs a B200).
+
+Bars: packed codes and integer accumulators bit-exact; scales within 1 ulp
+(double sums in a different order; the count of non-identical rows is
+checked too); fp32 outputs equal to the fp32 rounding of the exact
+s * acc, hence within 1e-6 relative.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from bit_gemv_sherry_b200 import sherry as S
+from tests.gpu_helpers import assert_y_matches, dev, dev_codes, host_codes, rows_subset
+from tests.helpers import load_tiles, ulp_diff_f32
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    S.lib()
+    yield
+    assert S.device_error() == 0
+
+
+# ----------------------------------------------------------------------------- pack
+@pytest.mark.parametrize("N,K", [(256, 1024), (1, 128), (7, 384), (33, 640), (5, 1152),
+                                 (300, 2048), (9, 8192)])
+def test_pack_matches_oracle(N, K):
+    w = synth.latent_weights(N, K, seed=0)
+    codes_ref, scales_ref = oracle.pack(w)
+    codes, scales = S.pack(dev(w))
+    torch.cuda.synchronize()
+    assert np.array_equal(host_codes(codes), codes_ref)
+    d = ulp_diff_f32(scales.cpu().numpy(), scales_ref)
+    assert d.max() <= 1
+    assert (d > 0).sum() <= max(1, N // 1000)
+
+
+def test_pack_golden_tiles(golden_dir):
+    tiles = load_tiles(golden_dir)
+    w = np.stack([t["latent"] for t in tiles])
+    codes_ref, scales_ref = oracle.pack(w)
+    codes, scales = S.pack(dev(w))
+    assert np.array_equal(host_codes(codes), codes_ref)
+    assert np.array_equal(scales.cpu().numpy(), scales_ref)
+    for n, t in enumerate(tiles):
+        assert [int(host_codes(codes)[p, n, 0]) for p in range(5)] == t["words"]
+
+
+@pytest.mark.parametrize("layer", range(7))
+def test_pack_full_size_1b_layers(layer):
+    name, N, K = synth.LLAMA_1B_LAYERS[layer]
+    w = synth.latent_weights(N, K, seed=synth.layer_seed(0, layer))
+    codes_ref, scales_ref = oracle.pack(w)
+    codes, scales = S.pack(dev(w))
+    assert np.array_equal(host_codes(codes), codes_ref), name
+    d = ulp_diff_f32(scales.cpu().numpy(), scales_ref)
+    assert d.max() <= 1 and (d > 0).sum() <= max(1, N // 1000), name
+
+
+# ----------------------------------------------------------------------------- gemv
+GEMV_CASES = [(256, 1024, 1), (1, 128, 1), (17, 384, 3), (33, 640, 5), (40, 1152, 8),
+              (19, 256, 9), (64, 512, 16), (2048, 2048, 1), (512, 2048, 4), (100, 3072, 2),
+              (31, 8192, 1), (48, 8192, 16)]
+
+
+@pytest.mark.parametrize("N,K,B", GEMV_CASES)
+def test_gemv_matches_oracle(N, K, B):
+    w = synth.latent_weights(N, K, seed=0)
+    codes, scales = oracle.pack(w)
+    x = synth.int8_uniform((B, K), seed=1)
+    tc, ts, tx = dev_codes(codes), dev(scales), dev(x)
+    acc = S.gemv_acc(tc, tx)
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), oracle.gemv_acc(codes, x, K))
+    y = S.gemv(tc, ts, tx)
+    assert_y_matches(y.cpu().numpy(), oracle.gemv(codes, scales, x, K))
+
+
+@pytest.mark.parametrize("N,K,B", [(37, 640, 1), (16, 1152, 7), (70, 384, 12)])
+def test_gemv_random_words_full_int8_range(N, K, B):
+    # every 32-bit pattern is a valid code; activations cover [-128, 127]
+    rng = np.random.default_rng(N + K + B)
+    codes = rng.integers(0, 2 ** 32, size=(5, N, K // 128), dtype=np.uint64).astype(np.uint32)
+    x = rng.integers(-128, 128, size=(B, K)).astype(np.int8)
+    acc = S.gemv_acc(dev_codes(codes), dev(x))
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), oracle.gemv_acc(codes, x, K))
+
+
+def test_gemv_extreme_and_zero_activations():
+    N, K = 64, 2048
+    codes, scales = oracle.pack(synth.latent_weights(N, K, seed=3))
+    x = np.stack([np.full(K, -128, np.int8), np.full(K, 127, np.int8), np.zeros(K, np.int8)])
+    y = S.gemv(dev_codes(codes), dev(scales), dev(x)).cpu().numpy()
+    assert_y_matches(y, oracle.gemv(codes, scales, x, K))
+    assert np.all(y[2] == 0)
+
+
+@pytest.mark.parametrize("B", [1, 4, 16])
+def test_gemv_full_size_3b_layers(B):
+    for li, (name, N, K) in enumerate(synth.LLAMA_3B_LAYERS):
+        if name in ("k", "v", "o"):
+            continue  # same kernels and shapes as q and the K=3072 layers
+        codes, scales = oracle.pack(synth.latent_weights(N, K, seed=synth.layer_seed(0, li)))
+        x = synth.int8_uniform((B, K), seed={1: 1, 4: 2, 16: 3}[B])
+        y = S.gemv(dev_codes(codes), dev(scales), dev(x)).cpu().numpy()
+        rows = np.random.default_rng(li).choice(N, size=min(N, 96), replace=False)
+        sub = rows_subset(codes, rows)
+        assert_y_matches(y[:, rows], oracle.gemv(sub, scales[rows], x, K))
+
+
+def test_gemv_grouped_1b_stack_layer():
+    items, refs = [], []
+    for li, (name, N, K) in enumerate(synth.LLAMA_1B_LAYERS):
+        codes, scales = oracle.pack(synth.latent_weights(N, K, seed=synth.layer_seed(0, li)))
+        x = synth.int8_uniform((1, K), seed=100 + li)
+        y = torch.empty((1, N), dtype=torch.float32, device="cuda")
+        items.append((dev_codes(codes), dev(scales), dev(x), y))
+        refs.append(oracle.gemv(codes, scales, x, K))
+    S.gemv_grouped(items, B=1)
+    for (_, _, _, y), ref in zip(items, refs):
+        assert_y_matches(y.cpu().numpy(), ref)
+
+
+def test_gemv_on_gpu_packed_codes():
+    # end to end on the device: pack on the GPU, then GEMV
+    N, K = 2048, 2048
+    w = synth.latent_weights(N, K, seed=0)
+    codes, scales = S.pack(dev(w))
+    x = synth.int8_uniform((1, K), seed=1)
+    y = S.gemv(codes, scales, dev(x)).cpu().numpy()
+    c_ref, s_ref = oracle.pack(w)
+    acc_ref = oracle.gemv_acc(c_ref, x, K)
+    y_ref = scales.cpu().numpy().astype(np.float64)[None, :] * acc_ref
+    assert_y_matches(y, y_ref)
+
+
+# ----------------------------------------------------------------------------- gemm
+GEMM_CASES = [(1, 128, 128), (100, 200, 384), (256, 128, 128), (300, 256, 640),
+              (513, 129, 1152), (64, 1000, 256), (1024, 384, 2048)]
+
+
+@pytest.mark.parametrize("M,N,K", GEMM_CASES)
+def test_gemm_matches_oracle(M, N, K):
+    codes, scales = oracle.pack(synth.latent_weights(N, K, seed=0))
+    x = synth.int8_clipped_normal((M, K), seed=1)
+    tc, ts, tx = dev_codes(codes), dev(scales), dev(x)
+    acc = S.gemm_acc(tc, tx)
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), oracle.gemm_acc(codes, x, K))
+    y = S.gemm(tc, ts, tx)
+    assert_y_matches(y.cpu().numpy(), oracle.gemm(codes, scales, x, K))
+
+
+def test_gemm_random_words_full_int8_range():
+    rng = np.random.default_rng(11)
+    M, N, K = 200, 160, 768
+    codes = rng.integers(0, 2 ** 32, size=(5, N, K // 128), dtype=np.uint64).astype(np.uint32)
+    x = rng.integers(-128, 128, size=(M, K)).astype(np.int8)
+    acc = S.gemm_acc(dev_codes(codes), dev(x))
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), oracle.gemm_acc(codes, x, K))
+
+
+@pytest.mark.parametrize("case", synth.PREFILL_GEMMS, ids=lambda c: c[0])
+def test_gemm_full_size_prefill(case):
+    _, M, N, K = case
+    codes, scales = oracle.pack(synth.latent_weights(N, K, seed=0))
+    x = synth.int8_clipped_normal((M, K), seed=1)
+    y = S.gemm(dev_codes(codes), dev(scales), dev(x)).cpu().numpy()
+    rows = np.random.default_rng(N).choice(N, size=48, replace=False)
+    rows[:2] = [0, N - 1]
+    sub = rows_subset(codes, rows)
+    assert_y_matches(y[:, rows], oracle.gemm(sub, scales[rows], x, K))
+
+
+def test_gemm_m1_equals_gemv():
+    N, K = 384, 1024
+    codes, scales = oracle.pack(synth.latent_weights(N, K, seed=5))
+    x = synth.int8_uniform((1, K), seed=6)
+    tc, ts, tx = dev_codes(codes), dev(scales), dev(x)
+    assert torch.equal(S.gemm(tc, ts, tx), S.gemv(tc, ts, tx))
