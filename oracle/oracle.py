@@ -104,19 +104,24 @@ def code_weights(code):
     return w
 
 
+GROUP = 32  # rows per group of the layout
+
+
 def pack(w):
-    """w: float32 [N, K] -> (codes uint32 [5, N, K/128], scales float32 [N])."""
+    """w: float32 [N, K] -> (codes uint32 [ceil(N/32), K/128, 5, 32], scales float32 [N]).
+
+    codes[g, t, p, r] is word p (Z0, Z1, S0, S1, S2) of tile t of row 32 g + r;
+    rows past N are padding (zeros)."""
     w = np.ascontiguousarray(w, dtype=np.float32)
     N, K = w.shape
-    codes = np.zeros((5, N, K // 128), np.uint32)
+    codes = np.zeros(((N + GROUP - 1) // GROUP, max(K // 128, 1), 5, GROUP), np.uint32)
     scales = np.zeros(N, np.float32)
     _check(_load().oracle_pack(_ptr(w), N, K, _ptr(codes), _ptr(scales)), "oracle_pack")
     return codes, scales
 
 
-def unpack(codes, K):
+def unpack(codes, N, K):
     codes = np.ascontiguousarray(codes, dtype=np.uint32)
-    N = codes.shape[1]
     wt = np.zeros((N, K), np.int8)
     _check(_load().oracle_unpack(_ptr(codes), N, K, _ptr(wt)), "oracle_unpack")
     return wt
@@ -130,9 +135,8 @@ def _x2(x, K):
     return x
 
 
-def gemv_acc(codes, x, K):
+def gemv_acc(codes, x, N, K):
     codes = np.ascontiguousarray(codes, dtype=np.uint32)
-    N = codes.shape[1]
     x = _x2(x, K)
     acc = np.zeros((x.shape[0], N), np.int64)
     _check(_load().oracle_gemv_acc(_ptr(codes), _ptr(x), N, K, x.shape[0], _ptr(acc)),
@@ -143,7 +147,7 @@ def gemv_acc(codes, x, K):
 def gemv(codes, scales, x, K):
     codes = np.ascontiguousarray(codes, dtype=np.uint32)
     scales = np.ascontiguousarray(scales, dtype=np.float32)
-    N = codes.shape[1]
+    N = scales.shape[0]
     x = _x2(x, K)
     y = np.zeros((x.shape[0], N), np.float64)
     _check(_load().oracle_gemv(_ptr(codes), _ptr(scales), _ptr(x), N, K, x.shape[0], _ptr(y)),
@@ -151,9 +155,8 @@ def gemv(codes, scales, x, K):
     return y
 
 
-def gemm_acc(codes, x, K):
+def gemm_acc(codes, x, N, K):
     codes = np.ascontiguousarray(codes, dtype=np.uint32)
-    N = codes.shape[1]
     x = _x2(x, K)
     acc = np.zeros((x.shape[0], N), np.int64)
     _check(_load().oracle_gemm_acc(_ptr(codes), _ptr(x), x.shape[0], N, K, _ptr(acc)),
@@ -164,7 +167,7 @@ def gemm_acc(codes, x, K):
 def gemm(codes, scales, x, K):
     codes = np.ascontiguousarray(codes, dtype=np.uint32)
     scales = np.ascontiguousarray(scales, dtype=np.float32)
-    N = codes.shape[1]
+    N = scales.shape[0]
     x = _x2(x, K)
     y = np.zeros((x.shape[0], N), np.float64)
     _check(_load().oracle_gemm(_ptr(codes), _ptr(scales), _ptr(x), x.shape[0], N, K, _ptr(y)),

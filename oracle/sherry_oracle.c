@@ -21,9 +21,12 @@
  *  - scale: the mean |w| over the kept weights of the row, summed in double
  *    in ascending k, divided by the kept count 3K/4, rounded once to fp32;
  *  - layout: a row is cut into tiles of 128 weights (32 blocks); a tile is
- *    five 32-bit words Z0, Z1, S0, S1, S2 stored planar:
- *        word(plane, n, t) = codes[(plane * N + n) * T + t],  T = K / 128,
- *    plane 0 = Z0, 1 = Z1, 2 = S0, 3 = S1, 4 = S2;
+ *    five 32-bit words Z0, Z1, S0, S1, S2 (plane 0 = Z0, 1 = Z1, 2 = S0,
+ *    3 = S1, 4 = S2).  Rows are taken in groups of 32; within a group the
+ *    tiles follow each other and, within a tile, each plane holds the 32 rows
+ *    of the group:
+ *        word(plane, n, t) = codes[((n / 32) * T + t) * 160 + plane * 32 + n % 32],
+ *    T = K / 128.  Rows past N in the last group are padding and hold zeros;
  *    block j (j = 0..31, weights k = 128 t + 4 j + i, i = 0..3) keeps its
  *    2-bit zero position p in bits [2*(j/2), 2*(j/2)+1] of Z_(j mod 2);
  *    the r-th kept weight of block j (r = 0, 1, 2 in ascending i) has its
@@ -47,16 +50,24 @@ enum { ORC_OK = 0, ORC_BAD_ARG = 1, ORC_NO_MEM = 2 };
 #define ORC_NBLK 32    /* 4-weight blocks per tile    */
 #define ORC_NPLANE 5   /* 32-bit words per tile       */
 
-static int64_t orc_word(int64_t plane, int64_t n, int64_t t, int64_t N, int64_t T)
+#define ORC_GROUP 32    /* rows per group in the layout */
+
+static int64_t orc_word(int64_t plane, int64_t n, int64_t t, int64_t T)
 {
-    return (plane * N + n) * T + t;
+    return ((n / ORC_GROUP) * T + t) * (ORC_NPLANE * ORC_GROUP) + plane * ORC_GROUP + n % ORC_GROUP;
 }
 
-/* Number of bytes of packed codes for an N x K matrix (scales excluded). */
+static int64_t orc_padded_rows(int64_t N)
+{
+    return (N + ORC_GROUP - 1) / ORC_GROUP * ORC_GROUP;
+}
+
+/* Number of bytes of packed codes for an N x K matrix (scales excluded),
+ * rows padded to a whole group. */
 int64_t oracle_packed_bytes(int64_t N, int64_t K)
 {
     if (N < 0 || K < 0 || K % ORC_TILE) return -1;
-    return N * (K / ORC_TILE) * ORC_NPLANE * 4;
+    return orc_padded_rows(N) * (K / ORC_TILE) * ORC_NPLANE * 4;
 }
 
 int oracle_num_threads(void)
@@ -128,25 +139,28 @@ int oracle_pack(const float *w, int64_t N, int64_t K, uint32_t *codes, float *sc
                 for (int i = 0; i < 4; i++)
                     if (i != p) sum_abs += fabs((double)blk[i]);
             }
-            codes[orc_word(0, n, t, N, T)] = z[0];
-            codes[orc_word(1, n, t, N, T)] = z[1];
-            codes[orc_word(2, n, t, N, T)] = s[0];
-            codes[orc_word(3, n, t, N, T)] = s[1];
-            codes[orc_word(4, n, t, N, T)] = s[2];
+            codes[orc_word(0, n, t, T)] = z[0];
+            codes[orc_word(1, n, t, T)] = z[1];
+            codes[orc_word(2, n, t, T)] = s[0];
+            codes[orc_word(3, n, t, T)] = s[1];
+            codes[orc_word(4, n, t, T)] = s[2];
         }
         scales[n] = (float)(sum_abs / (0.75 * (double)K));
     }
+    for (int64_t n = N; n < orc_padded_rows(N); n++)
+        for (int64_t t = 0; t < T; t++)
+            for (int p = 0; p < ORC_NPLANE; p++) codes[orc_word(p, n, t, T)] = 0u;
     return ORC_OK;
 }
 
 /* Ternary row n (K int8 values) from the packed codes. */
-static void orc_unpack_row(const uint32_t *codes, int64_t n, int64_t N, int64_t K, int8_t *row)
+static void orc_unpack_row(const uint32_t *codes, int64_t n, int64_t K, int8_t *row)
 {
     const int64_t T = K / ORC_TILE;
     for (int64_t t = 0; t < T; t++) {
-        uint32_t z[2] = {codes[orc_word(0, n, t, N, T)], codes[orc_word(1, n, t, N, T)]};
-        uint32_t s[3] = {codes[orc_word(2, n, t, N, T)], codes[orc_word(3, n, t, N, T)],
-                         codes[orc_word(4, n, t, N, T)]};
+        uint32_t z[2] = {codes[orc_word(0, n, t, T)], codes[orc_word(1, n, t, T)]};
+        uint32_t s[3] = {codes[orc_word(2, n, t, T)], codes[orc_word(3, n, t, T)],
+                         codes[orc_word(4, n, t, T)]};
         for (int j = 0; j < ORC_NBLK; j++) {
             int p = (int)((z[j & 1] >> (2 * (j >> 1))) & 3u);
             int r = 0;
@@ -167,7 +181,7 @@ int oracle_unpack(const uint32_t *codes, int64_t N, int64_t K, int8_t *wt)
 {
     if (!codes || !wt || N < 1 || K < ORC_TILE || K % ORC_TILE) return ORC_BAD_ARG;
     #pragma omp parallel for schedule(static)
-    for (int64_t n = 0; n < N; n++) orc_unpack_row(codes, n, N, K, wt + n * K);
+    for (int64_t n = 0; n < N; n++) orc_unpack_row(codes, n, K, wt + n * K);
     return ORC_OK;
 }
 
@@ -189,7 +203,7 @@ static int orc_matmul_acc(const uint32_t *codes, const int8_t *x, int64_t M, int
         #pragma omp for schedule(static)
         for (int64_t n = 0; n < N; n++) {
             if (!row) continue;
-            orc_unpack_row(codes, n, N, K, row);
+            orc_unpack_row(codes, n, K, row);
             for (int64_t m = 0; m < M; m++) {
                 const int8_t *xm = x + m * K;
                 int64_t a = 0;

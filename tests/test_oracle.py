@@ -57,35 +57,53 @@ def test_prune_cases(golden_dir):
 def test_golden_tiles(golden_dir):
     for t in load_tiles(golden_dir):
         codes, scales = oracle.pack(t["latent"].reshape(1, 128))
-        got = [int(codes[p, 0, 0]) for p in range(5)]
+        assert codes.shape == (1, 1, 5, 32)
+        got = [int(codes[0, 0, p, 0]) for p in range(5)]
         assert got == t["words"], (t["name"], [hex(v) for v in got])
+        assert not codes[0, 0, :, 1:].any()          # padding rows 1..31 are zero
         assert scales[0] == t["scale"], (t["name"], scales[0], t["scale"])
-        assert np.array_equal(oracle.unpack(codes, 128)[0], t["dense"]), t["name"]
+        assert np.array_equal(oracle.unpack(codes, 1, 128)[0], t["dense"]), t["name"]
 
 
 def test_golden_words_unpack_without_pack(golden_dir):
     # Unpack and dot straight from the hand-derived words (no pack involved).
     for t in load_tiles(golden_dir):
-        codes = np.array(t["words"], np.uint32).reshape(5, 1, 1)
-        assert np.array_equal(oracle.unpack(codes, 128)[0], t["dense"]), t["name"]
+        codes = np.zeros((1, 1, 5, 32), np.uint32)
+        codes[0, 0, :, 0] = t["words"]
+        assert np.array_equal(oracle.unpack(codes, 1, 128)[0], t["dense"]), t["name"]
         x = synth.int8_uniform((3, 128), seed=11)
-        acc = oracle.gemv_acc(codes, x, 128)
+        acc = oracle.gemv_acc(codes, x, 1, 128)
         assert np.array_equal(acc[:, 0], x.astype(np.int64) @ t["dense"].astype(np.int64))
 
 
-def test_planar_layout_across_rows_and_tiles(golden_dir):
+def test_blocked_layout_across_rows_and_tiles(golden_dir):
     tiles = {t["name"][0]: t for t in load_tiles(golden_dir)}
     # row 0 = [A | B], row 1 = [C | E], row 2 = [G | F]
     rows = [("A", "B"), ("C", "E"), ("G", "F")]
     lat = np.stack([np.concatenate([tiles[a]["latent"], tiles[b]["latent"]]) for a, b in rows])
     codes, scales = oracle.pack(lat)
-    assert codes.shape == (5, 3, 2)
+    assert codes.shape == (1, 2, 5, 32)
     flat = codes.reshape(-1)
-    N, T = 3, 2
+    # word (plane p, row n, tile t) sits at ((n // 32) * T + t) * 160 + 32 p + n % 32;
+    # hand-computed positions (T = 2):
+    assert flat[1 * 160 + 2 * 32 + 0] == tiles["B"]["words"][2]    # row 0, tile 1, S0 of B
+    assert flat[0 * 160 + 3 * 32 + 2] == tiles["G"]["words"][3]    # row 2, tile 0, S1 of G
+    assert flat[0 * 160 + 0 * 32 + 1] == tiles["C"]["words"][0]    # row 1, tile 0, Z0 of C
+    assert flat[1 * 160 + 1 * 32 + 1] == tiles["E"]["words"][1]    # row 1, tile 1, Z1 of E
+    assert flat[1 * 160 + 4 * 32 + 2] == tiles["F"]["words"][4]    # row 2, tile 1, S2 of F
     for n, pair in enumerate(rows):
         for t, name in enumerate(pair):
             for p in range(5):
-                assert flat[(p * N + n) * T + t] == tiles[name]["words"][p]
+                assert codes[0, t, p, n] == tiles[name]["words"][p]
+    assert not codes[0, :, :, 3:].any()                            # padding rows
+    # second group: row 35 of a 40-row matrix sits in group 1 at position 3
+    lat2 = np.zeros((40, 256), np.float32)
+    lat2[35] = np.concatenate([tiles["D"]["latent"], tiles["C"]["latent"]])
+    c2, _ = oracle.pack(lat2)
+    f2 = c2.reshape(-1)
+    assert c2.shape == (2, 2, 5, 32)
+    assert f2[(1 * 2 + 0) * 160 + 1 * 32 + 3] == tiles["D"]["words"][1]   # Z1 of D
+    assert f2[(1 * 2 + 1) * 160 + 2 * 32 + 3] == tiles["C"]["words"][2]   # S0 of C
     # mean over 192 kept weights: [A|B] = (96*1 + 96*2)/192 = 1.5
     assert scales[0] == np.float32(1.5)
     assert scales[1] == np.float32((96 * 2 + 96 * 3) / 192)
@@ -97,14 +115,14 @@ def test_all_32_codes_in_one_tile():
     T = np.array(VALID_BLOCKS, np.int8).reshape(1, 128)   # block j = pattern j
     lat = ternary_latents(T, rng)
     codes, _ = oracle.pack(lat)
-    assert np.array_equal(oracle.unpack(codes, 128), T)
+    assert np.array_equal(oracle.unpack(codes, 1, 128), T)
 
 
 def test_random_words_decode_to_valid_blocks():
     # Every 5-bit pattern is a valid block: any words unpack to exactly one zero per block.
     rng = np.random.default_rng(7)
-    codes = rng.integers(0, 2 ** 32, size=(5, 7, 3), dtype=np.uint64).astype(np.uint32)
-    wt = oracle.unpack(codes, 384).reshape(7, 96, 4)
+    codes = rng.integers(0, 2 ** 32, size=(1, 3, 5, 32), dtype=np.uint64).astype(np.uint32)
+    wt = oracle.unpack(codes, 7, 384).reshape(7, 96, 4)
     assert np.all((wt == 0).sum(axis=2) == 1)
     assert np.all(np.isin(wt, (-1, 0, 1)))
 
@@ -115,7 +133,7 @@ def test_pack_unpack_roundtrip_and_scale():
         T = random_ternary(N, K, rng)
         lat = ternary_latents(T, rng)
         codes, scales = oracle.pack(lat)
-        assert np.array_equal(oracle.unpack(codes, K), T)
+        assert np.array_equal(oracle.unpack(codes, N, K), T)
         kept_mean = np.where(T != 0, np.abs(lat.astype(np.float64)), 0).sum(1) / (0.75 * K)
         assert np.all(ulp_diff_f32(scales, kept_mean.astype(np.float32)) <= 1)
 
@@ -144,8 +162,8 @@ def test_all_ones_activation_gives_sum_of_signs():
     N, K = 33, 640
     lat = synth.latent_weights(N, K, seed=0)
     codes, _ = oracle.pack(lat)
-    acc = oracle.gemv_acc(codes, np.ones((1, K), np.int8), K)[0]
-    neg = np.array([sum(bin(int(w)).count("1") for w in codes[2:, n, :].reshape(-1))
+    acc = oracle.gemv_acc(codes, np.ones((1, K), np.int8), N, K)[0]
+    neg = np.array([sum(bin(int(w)).count("1") for w in codes[n // 32, :, 2:, n % 32].reshape(-1))
                     for n in range(N)])
     assert np.array_equal(acc, 3 * K // 4 - 2 * neg)
 
@@ -160,8 +178,8 @@ def test_bruteforce_dense_matmul(N, K, B):
     codes, scales = oracle.pack(lat)
     x = rng.integers(-128, 128, size=(B, K)).astype(np.int8)
     ref = x.astype(np.int64) @ T.astype(np.int64).T
-    assert np.array_equal(oracle.gemv_acc(codes, x, K), ref)
-    assert np.array_equal(oracle.gemm_acc(codes, x, K), ref)
+    assert np.array_equal(oracle.gemv_acc(codes, x, N, K), ref)
+    assert np.array_equal(oracle.gemm_acc(codes, x, N, K), ref)
     y = oracle.gemv(codes, scales, x, K)
     assert np.array_equal(y, scales.astype(np.float64)[None, :] * ref)
     assert np.array_equal(oracle.gemm(codes, scales, x, K), y)
@@ -176,16 +194,18 @@ def test_extreme_activations_bound():
     codes, _ = oracle.pack(lat)
     x = np.full((2, K), -128, np.int8)
     x[1] = 127
-    acc = oracle.gemv_acc(codes, x, K)
+    acc = oracle.gemv_acc(codes, x, 2, K)
     assert acc[0, 0] == -128 * 3 * K // 4 and acc[0, 1] == 128 * 3 * K // 4
     assert acc[1, 0] == 127 * 3 * K // 4 and acc[1, 1] == -127 * 3 * K // 4
 
 
 def test_size_closed_forms():
-    for N, K in [(1, 128), (256, 1024), (2048, 8192), (8192, 2048)]:
+    for N, K in [(32, 128), (256, 1024), (2048, 8192), (8192, 2048)]:
         nbytes = oracle.packed_bytes(N, K)
         assert nbytes * 32 == N * K * 5          # 5 bits per 4 weights
         assert 8 * nbytes / (N * K) == 1.25      # 1.25 bits per weight (scales excluded)
+    assert oracle.packed_bytes(1, 128) == 32 * 20    # one 32-row group of one tile
+    assert oracle.packed_bytes(33, 256) == 64 * 2 * 20
     assert 1 - 1.25 / (5 / 3) == pytest.approx(0.25, abs=1e-15)   # vs 3-in-5-bit packing
     assert 1 - 1.25 / 2 == 0.375                                  # vs 2-bit packing
     assert oracle.packed_bytes(4, 100) == -1

@@ -37,8 +37,12 @@ MUTANTS = {
                                   "const int8_t *xm = x + (M - 1 - m) * K;"),
     "y_without_scale": ("y[m * N + n] = (double)scales[n] * (double)acc[m * N + n];",
                         "y[m * N + n] = (double)acc[m * N + n];"),
-    "planes_swapped": ("codes[orc_word(2, n, t, N, T)] = s[0];\n            codes[orc_word(3, n, t, N, T)] = s[1];",
-                       "codes[orc_word(3, n, t, N, T)] = s[0];\n            codes[orc_word(2, n, t, N, T)] = s[1];"),
+    "planes_swapped": ("codes[orc_word(2, n, t, T)] = s[0];\n            codes[orc_word(3, n, t, T)] = s[1];",
+                       "codes[orc_word(3, n, t, T)] = s[0];\n            codes[orc_word(2, n, t, T)] = s[1];"),
+    "group_of_16_rows": ("return ((n / ORC_GROUP) * T + t) * (ORC_NPLANE * ORC_GROUP) + plane * ORC_GROUP + n % ORC_GROUP;",
+                         "return ((n / 16) * T + t) * (ORC_NPLANE * 16) + plane * 16 + n % 16;"),
+    "rows_before_tiles": ("return ((n / ORC_GROUP) * T + t) * (ORC_NPLANE * ORC_GROUP) + plane * ORC_GROUP + n % ORC_GROUP;",
+                          "return ((n / ORC_GROUP) * T + t) * (ORC_NPLANE * ORC_GROUP) + (n % ORC_GROUP) * ORC_NPLANE + plane;"),
 }
 
 
@@ -49,7 +53,7 @@ def _run_pins(golden_dir):
         lambda: pins.test_prune_cases(golden_dir),
         lambda: pins.test_golden_tiles(golden_dir),
         lambda: pins.test_golden_words_unpack_without_pack(golden_dir),
-        lambda: pins.test_planar_layout_across_rows_and_tiles(golden_dir),
+        lambda: pins.test_blocked_layout_across_rows_and_tiles(golden_dir),
         pins.test_pack_unpack_roundtrip_and_scale,
         pins.test_all_ones_activation_gives_sum_of_signs,
         lambda: pins.test_bruteforce_dense_matmul(3, 256, 2),
