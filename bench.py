@@ -1,0 +1,475 @@
+#!/usr/bin/env python
+"""Benchmark of the Sherry 1.25-bit ternary path on B200.
+
+Step = one batch-1 decode pass through a LLaMA-3.2-1B-shaped stack: 16 layers
+x (q, k, v, o 2048x2048 / 512x2048, gate/up 8192x2048, down 2048x8192) =
+112 GEMVs, 973,078,528 ternary weights, 152,043,520 bytes of codes (more than
+the 126 MB L2, so no flush is needed between steps).  The codes are made on the
+device by sherry_pack from seeded fp32 latents; the activations are one seeded
+int8 vector per K.  Metric: packed-weight bytes streamed per second.
+
+Also measured in the same run (rank 0): sherry_pack over all 973M fp32
+latents, the two prefill GEMMs (int8 TOPS, L2 flushed between launches), the
+per-projection GEMVs (L2 flushed), the end-to-end step with pinned host
+buffers, and the CPU oracle on a bounded sample.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl sherry|reference]
+For N > 1 run under torch.distributed.run: every rank runs its own replica of
+the step (the path has no exchange step), value = all ranks' bytes / max time.
+"""
+import argparse
+import ctypes
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "W1.25A8 GEMV weight GB/s at batch 1 (LLaMA-3.2-1B decode stack)"
+UNIT = "GB/s"
+L2_BYTES = 126 * 2 ** 20
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", choices=["sherry", "reference"], default="sherry")
+    ap.add_argument("--layers", type=int, default=16)
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the pack/GEMM/per-layer/CPU-baseline sub-measurements")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU time of the oracle baseline sample")
+    return ap.parse_args()
+
+
+def stack_spec(n_layers):
+    return synth.decode_stack(n_layers)
+
+
+def algorithmic_bytes(spec, B=1):
+    codes = sum(n * k * 5 // 32 for _, _, n, k, _ in spec)
+    scales = sum(4 * n for _, _, n, _, _ in spec)
+    xs = sum(B * k for _, _, _, k, _ in spec)
+    ys = sum(4 * B * n for _, _, n, _, _ in spec)
+    return codes, codes + scales + xs + ys
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of the GPU this process uses (timestamps on the host)."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.samples = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=uuid," + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9 or (self.uuid and parts[0] != self.uuid):
+                continue
+            self.samples.append((time.time(), parts[1:]))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        sel = [s for ts, s in self.samples if t0 <= ts <= t1]
+        if not sel:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return None
+        sm = [num(s[0]) for s in sel if num(s[0]) is not None]
+        smax = [num(s[1]) for s in sel if num(s[1]) is not None]
+        pw = [num(s[2]) for s in sel if num(s[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for s in sel for i in range(4) if s[4 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(pw) if pw else None,
+                "reasons": reasons, "samples": len(sel)}
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args, rank):
+    """Times the CPU oracle on a bounded sample of the same workload."""
+    import oracle
+    if rank != 0:
+        return None
+    spec = stack_spec(args.layers)
+    layer0 = [s for s in spec if s[0] == 0]
+    data = []
+    for _, name, n, k, seed in layer0:
+        codes, scales = oracle.pack(synth.latent_weights(n, k, seed=seed))
+        data.append((codes, scales, k))
+    xs = {2048: synth.int8_uniform((1, 2048), seed=1), 8192: synth.int8_uniform((1, 8192), seed=2)}
+    sample_bytes = sum(c.nbytes for c, _, _ in data)
+
+    def step():
+        for codes, scales, k in data:
+            oracle.gemv(codes, scales, xs[k], k)
+    for _ in range(max(0, min(args.warmup, 2))):
+        step()
+    steps = max(1, min(args.steps, 50))
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        step()
+    dt = (time.perf_counter() - t0) / steps
+    value = sample_bytes / dt / 1e9
+    cores = oracle.num_threads()
+    sample = "decoder layer 0 of the stack (7 GEMVs, %d weights, %d code bytes) per step" % (
+        sum(n * k for _, _, n, k, _ in layer0), sample_bytes)
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": args.gpus, "steps": steps, "warmup": min(args.warmup, 2),
+        "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "config": {"workload": "llama-3.2-1b decode stack sample (CPU oracle)", "batch": 1},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ----------------------------------------------------------------------------- sherry arm
+def build_stack(spec, dev, S, torch, keep_latents=False):
+    """Pack every layer on the device from seeded latents; return device tensors."""
+    layers, latents = [], []
+    for layer, name, n, k, seed in spec:
+        w = torch.from_numpy(synth.latent_weights(n, k, seed=seed)).to(dev)
+        codes, scales = S.pack(w)
+        layers.append((layer, name, n, k, codes, scales))
+        if keep_latents:
+            latents.append(w)
+        else:
+            del w
+    torch.cuda.synchronize(dev)
+    return layers, latents
+
+
+def time_pack(latents, layers, S, torch, reps=3):
+    """sherry_pack over every latent matrix of the stack (3.9 GB fp32 read)."""
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    outs = [(torch.empty_like(l[4]), torch.empty_like(l[5])) for l in layers]
+
+    def one():
+        for w, (c, s) in zip(latents, outs):
+            S.pack(w, c, s)
+    one()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(reps):
+        start.record()
+        one()
+        end.record()
+        end.synchronize()
+        times.append(start.elapsed_time(end) / 1e3)
+    t = min(times)
+    n_w = sum(l.numel() for l in latents)
+    read = 4 * n_w
+    written = sum(o[0].numel() * 4 + o[1].numel() * 4 for o in outs)
+    return {"weights": n_w, "ms": t * 1e3, "gweights_per_s": n_w / t / 1e9,
+            "gbs": (read + written) / t / 1e9, "launches": len(latents),
+            "bytes_read": read, "bytes_written": written}
+
+
+def l2_flusher(torch, dev):
+    buf = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def flush():
+        buf.add_(1.0)
+    return flush
+
+
+def time_gemm(S, torch, dev, flush, reps=5):
+    out = {}
+    for name, M, N, K in synth.PREFILL_GEMMS:
+        w = torch.from_numpy(synth.latent_weights(N, K, seed=0)).to(dev)
+        codes, scales = S.pack(w)
+        del w
+        x = torch.from_numpy(synth.int8_clipped_normal((M, K), seed=1)).to(dev)
+        y = torch.empty((M, N), dtype=torch.float32, device=dev)
+        for _ in range(3):
+            S.gemm(codes, scales, x, y)
+        torch.cuda.synchronize()
+        ts = []
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for _ in range(reps):
+            flush()
+            e0.record()
+            S.gemm(codes, scales, x, y)
+            e1.record()
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1) / 1e3)
+        t = statistics.median(ts)
+        ops = 2.0 * M * N * K
+        out[name] = {"M": M, "N": N, "K": K, "ms": t * 1e3, "tops": ops / t / 1e12,
+                     "bytes": M * K + N * K * 5 // 32 + 4 * N + 4 * M * N}
+    return out
+
+
+def time_layers(layers, xs, S, torch, dev, flush, reps=20):
+    """Single-projection GEMVs of layer 0 with the L2 flushed before each launch."""
+    res = {}
+    for layer, name, n, k, codes, scales in layers:
+        if layer != 0:
+            continue
+        x = xs[k]
+        y = torch.empty((1, n), dtype=torch.float32, device=dev)
+        ws = S.workspace(S.gemv_workspace_bytes(n, k, 1), dev)
+        for _ in range(3):
+            S.gemv(codes, scales, x, y, ws)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ts = []
+        for _ in range(reps):
+            flush()
+            e0.record()
+            S.gemv(codes, scales, x, y, ws)
+            e1.record()
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1) / 1e3)
+        t = statistics.median(ts)
+        cb = n * k * 5 // 32
+        res[name] = {"N": n, "K": k, "us": t * 1e6, "weight_gbs": cb / t / 1e9}
+    return res
+
+
+def cpu_baseline(layers, xs_host, seconds):
+    """The oracle, as it stands, on a bounded sample of the stack (host cores)."""
+    import oracle
+    t_start = time.perf_counter()
+    done_bytes, done_w, n_gemv = 0, 0, 0
+    t_compute = 0.0
+    for layer, name, n, k, codes, scales in layers:
+        c = codes.cpu().numpy().view(np.uint32)
+        s = scales.cpu().numpy()
+        t0 = time.perf_counter()
+        oracle.gemv(c, s, xs_host[k], k)
+        t_compute += time.perf_counter() - t0
+        done_bytes += c.nbytes
+        done_w += n * k
+        n_gemv += 1
+        if time.perf_counter() - t_start > seconds:
+            break
+    return {"value": done_bytes / t_compute / 1e9, "unit": UNIT, "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": "first %d GEMVs of the stack in order (%d weights, %d code bytes), each "
+                      "timed once" % (n_gemv, done_w, done_bytes)}
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if world > 1 and rank != 0:
+            return 0
+        line = run_reference(args, rank)
+        print(json.dumps(line))
+        return 0
+
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+    from bit_gemv_sherry_b200 import sherry as S
+
+    if args.warmup < 3:
+        args.warmup = 3
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    S.lib()
+
+    spec = stack_spec(args.layers)
+    codes_bytes, alg_bytes = algorithmic_bytes(spec)
+    extras = (rank == 0) and not args.no_extras
+    layers, latents = build_stack(spec, dev, S, torch, keep_latents=extras)
+    xs_host = {2048: synth.int8_uniform((1, 2048), seed=1), 8192: synth.int8_uniform((1, 8192), seed=2)}
+    xs = {k: torch.from_numpy(v).to(dev) for k, v in xs_host.items()}
+    ys = [torch.empty((1, n), dtype=torch.float32, device=dev) for _, _, n, _, _, _ in layers]
+    items = [(codes, scales, xs[k], y) for (_, _, n, k, codes, scales), y in zip(layers, ys)]
+    step = S.GroupedGemv(items, B=1)
+    stream = torch.cuda.current_stream(dev)
+    sptr = stream.cuda_stream
+
+    for _ in range(args.warmup):
+        step.prepare(sptr)
+        step.run(sptr)
+    torch.cuda.synchronize(dev)
+
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+    except Exception:
+        uuid = None
+    clocks = ClockSampler(uuid)
+    clocks.start()
+    time.sleep(0.3)
+
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    t_host0 = time.time()
+    for i in range(K):
+        a, b, c = ev[i]
+        a.record(stream)
+        step.prepare(sptr)
+        b.record(stream)
+        step.run(sptr)
+        c.record(stream)
+    torch.cuda.synchronize(dev)
+    t_host1 = time.time()
+    if world > 1:
+        dist.barrier()
+    total_s = ev[0][0].elapsed_time(ev[-1][2]) / 1e3
+    gemv_s = sum(b.elapsed_time(c) for _, b, c in ev) / 1e3 / K
+    prep_s = sum(a.elapsed_time(b) for a, b, _ in ev) / 1e3 / K
+    busy_s = sum(a.elapsed_time(c) for a, _, c in ev) / 1e3
+    time.sleep(0.2)
+    clocks.stop()
+    clk = clocks.summary(t_host0, t_host1)
+
+    t_max = total_s
+    if world > 1:
+        tt = torch.tensor([total_s], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_max = float(tt.item())
+    ms_per_step = t_max / K * 1e3
+    value = world * codes_bytes * K / t_max / 1e9
+
+    # ---------------- end to end through the public API with pinned host buffers
+    x_pinned = {k: torch.from_numpy(v).pin_memory() for k, v in xs_host.items()}
+    y_pinned = [torch.empty((1, n), dtype=torch.float32).pin_memory() for _, _, n, _, _, _ in layers]
+    h2d = sum(v.numel() for v in x_pinned.values())
+    d2h = sum(4 * y.numel() for y in y_pinned)
+    K_e2e = max(3, min(K, 2000))
+
+    def e2e_step():
+        for k, v in x_pinned.items():
+            xs[k].copy_(v, non_blocking=True)
+        step(sptr)
+        for yp, yd in zip(y_pinned, ys):
+            yp.copy_(yd, non_blocking=True)
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K_e2e):
+        e2e_step()
+    e1.record(stream)
+    e1.synchronize()
+    e2e_s = e0.elapsed_time(e1) / 1e3
+    if world > 1:
+        tt = torch.tensor([e2e_s], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_s = float(tt.item())
+        dist.barrier()
+    e2e_value = world * codes_bytes * K_e2e / e2e_s / 1e9
+
+    peaks = {}
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            peaks = json.load(f)
+    except (OSError, ValueError):
+        peaks = {}
+    hbm_peak = peaks.get("hbm_gbs")
+    peak_src = "measured"
+    if hbm_peak is None:
+        hbm_peak, peak_src = 6650.0, "fallback"
+    achieved = alg_bytes / gemv_s / 1e9
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "config": {
+            "workload": "llama-3.2-1b decode stack, batch 1: %d layers x (q,o 2048x2048; k,v "
+                        "512x2048; gate,up 8192x2048; down 2048x8192)" % args.layers,
+            "gemvs": len(spec), "weights": sum(n * k for _, _, n, k, _ in spec),
+            "code_bytes": codes_bytes, "batch": 1,
+            "l2": "inputs larger than L2: %.0f MB of codes per step > 126 MB L2, no flush" % (
+                codes_bytes / 1e6),
+            "launch": "sherry_gemv_prepare + sherry_gemv_run (one activation re-order launch and "
+                      "one GEMV launch per step)",
+            "parallelism": "replicas x%d" % world,
+        },
+        "gpu_launches": 2 * K,
+        "clocks": clk,
+        "roofline": {"bound": "hbm", "kernel": "gemv_kernel (sherry_gemv_run)",
+                     "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "peak_source": peak_src,
+                     "bytes_per_launch": alg_bytes, "kernel_us": gemv_s * 1e6,
+                     "prepare_us": prep_s * 1e6, "traffic": None},
+        "gpu_busy_frac": busy_s / total_s if total_s > 0 else None,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": K_e2e, "ms_per_step": e2e_s / K_e2e * 1e3},
+    }
+    if extras:
+        flush = l2_flusher(torch, dev)
+        line["pack"] = time_pack(latents, layers, S, torch)
+        del latents
+        torch.cuda.empty_cache()
+        line["gemm"] = time_gemm(S, torch, dev, flush)
+        line["gemv_layers_l2_flushed"] = time_layers(layers, xs, S, torch, dev, flush)
+        if world == 1:
+            line["cpu_baseline"] = cpu_baseline(layers, xs_host, args.cpu_seconds)
+    err = S.device_error()
+    if err != 0:
+        line["device_error"] = err
+    if rank == 0:
+        print(json.dumps(line))
+    del step
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

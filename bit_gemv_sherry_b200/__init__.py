@@ -4,6 +4,6 @@ The compute path lives in ``libsherry.so`` (``csrc/``, header ``include/sherry.h
 ``sherry`` is its thin Python binding.
 """
 from .sherry import (  # noqa: F401
-    SherryError, device_error, gemm, gemm_acc, gemv, gemv_acc, gemv_grouped,
+    GroupedGemv, SherryError, codes_shape, device_error, gemm, gemm_acc, gemv, gemv_acc, gemv_grouped,
     gemv_workspace_bytes, lib, library_path, pack, packed_bytes, workspace,
 )

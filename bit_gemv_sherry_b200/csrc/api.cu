@@ -43,7 +43,8 @@ int sm_count() {
 
 extern "C" size_t sherry_packed_bytes(int64_t N, int64_t K) {
     if (N < 1 || K < SHERRY_TILE_K || K % SHERRY_TILE_K) return 0;
-    return (size_t)N * (size_t)(K / SHERRY_TILE_K) * SHERRY_WORDS_PER_TILE * 4;
+    const size_t rows = (size_t)((N + SHERRY_ROW_GROUP - 1) / SHERRY_ROW_GROUP) * SHERRY_ROW_GROUP;
+    return rows * (size_t)(K / SHERRY_TILE_K) * SHERRY_WORDS_PER_TILE * 4;
 }
 
 extern "C" const char *sherry_status_string(sherry_status s) {

@@ -184,15 +184,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---------------- decoders: one weight row per thread ----------------
         const int r = threadIdx.x - 64;
         uint32_t it = 0;
-        const size_t plane = (size_t)N * T;
         for (int tile = blockIdx.x; tile < num_tiles && !*abort; tile += gridDim.x) {
             const int wb = tile % tiles_n;
             const int row = wb * kBM + r;
             const bool valid = row < N;
-            const uint32_t *crow = codes + (size_t)row * T;
+            // word (p, row, kt) = ((row / 32) * T + kt) * 160 + 32 p + row % 32: a warp
+            // (32 consecutive rows) reads 128 contiguous bytes per plane
+            const uint32_t *crow = codes + (size_t)(row / 32) * T * 160 + (row % 32);
             uint32_t w[5];
 #pragma unroll
-            for (int p = 0; p < 5; p++) w[p] = valid ? ld_code(crow + p * plane) : 0u;
+            for (int p = 0; p < 5; p++) w[p] = valid ? ld_code(crow + p * 32) : 0u;
             bool ok = true;
             for (int kt = 0; kt < T; kt++, it++) {
                 const int s = it % kStages;
@@ -201,7 +202,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 dec.load(w[0], w[1], w[2], w[3], w[4]);
                 if (kt + 1 < T) {
 #pragma unroll
-                    for (int p = 0; p < 5; p++) w[p] = valid ? ld_code(crow + p * plane + kt + 1) : 0u;
+                    for (int p = 0; p < 5; p++)
+                        w[p] = valid ? ld_code(crow + (size_t)(kt + 1) * 160 + p * 32) : 0u;
                 }
                 if (!mbar_wait(&bar->empty[s], ph ^ 1, abort, err)) {
                     ok = false;

@@ -2,26 +2,27 @@
 //
 // The product is the one the pages state for ternary weights with 3:4 blocks
 // coded in five bits (arXiv 2601.07892, abstract; Figure 2 caption: "SIMD-
-// friendly 4-way patterns").  On B200 the batch-1 GEMV is bound by HBM reads of
+// friendly 4-way patterns").  On B200 a batch-1 GEMV is bound by HBM reads of
 // the codes (0.15625 bytes per weight) only if the decode costs a few
 // instructions per 4-weight block, so:
 //
-//   * each warp owns 16 output rows (the M of an int8 m16n8k32 tensor-core
-//     MMA) and walks K four tiles at a time, one tile per thread of a quad;
-//   * a thread decodes its tile for two rows with 32-bit SWAR logic: per
-//     (position i, block group beta) one selector word whose nibbles are
-//     (zero position | sign << 2) of eight blocks, and one byte permute
-//     (PRMT) per four weights against an 8-byte table -- ~2.8 instructions
-//     per 4-weight block, no shared memory, no lookup loads;
-//   * the int8 words go straight from registers into mma.sync as the A
-//     fragment; the activations, re-ordered once per call into the same
-//     order (xprep_kernel), are the B fragment, one batch row per column, so
-//     batches up to 8 cost the same MMA count as batch 1;
-//   * accumulation is exact int32; the epilogue applies the row scale once.
+//   * the int8 MMA m16n8k32 does the multiply-accumulate: the decoded weights
+//     are its A fragment straight from registers (16 rows x 32 K per MMA), the
+//     activations its B fragment (one batch row per column, so batches up to 8
+//     cost the same MMA count as batch 1), int32 accumulation is exact;
+//   * a thread decodes whole 128-weight tiles with 32-bit SWAR logic: for a
+//     (position i, block group beta) pair one selector word holds, per nibble,
+//     (zero position | sign << 2) of one block, and one byte permute (PRMT)
+//     against an 8-byte table per position turns four nibbles into four
+//     ternary bytes; shifts that move left run as IMAD on the FMA pipe, so the
+//     ALU pipe carries only the permutes, the selector merges and a few shifts;
+//   * the activations are re-ordered once per call (xprep_kernel) into the
+//     order in which the decoded bytes meet the MMA fragments.
 //
-// The MMA replaces the per-block dp4a of a plain SIMT kernel (one tensor-core
-// instruction per 128 blocks instead of 128 dp4a), leaving the issue slots to
-// the decode.
+// Two kernels share this scheme.  The pipelined kernel (K a multiple of 512,
+// codes 16-byte aligned) streams codes through per-warp shared-memory rings
+// filled by cp.async and splits long rows into K-parts that are summed exactly
+// with integer atomics; the register kernel is the general fallback.
 #include <algorithm>
 #include <cstring>
 
@@ -30,33 +31,48 @@
 namespace sherry {
 namespace {
 
-constexpr int kGemvThreads = 256;
-constexpr int kGemvWarps = kGemvThreads / 32;
-
+// ---------------------------------------------------------------------------
+// Launch parameters
+// ---------------------------------------------------------------------------
 struct GemvDesc {
     const uint32_t *codes;
     const float *scales;
-    const uint4 *xw;   // re-ordered activations [B][T][32 words]
-    void *out;         // float y[B][N] or int32 acc[B][N]
+    const uint4 *xw;      // re-ordered activations [B][Tp][32 words]
+    void *out;            // float y[B][N] or int32 acc[B][N]
+    int32_t *part_acc;    // K-part partial sums [B][N] (pipelined kernel, kparts > 1)
+    uint32_t *part_cnt;   // K-parts finished per unit (pipelined kernel, kparts > 1)
     int N;
-    int T;
-    int unit_begin;    // first 16-row unit of this GEMV in the group
-    int pad;
+    int T;                // tiles per row (K / 128)
+    int Tp;               // tile stride of xw (T rounded up to a whole chunk)
+    int unit_begin16;     // register kernel: first 16-row unit in the group
+    int units;            // pipelined kernel: 32-row units
+    int nchunk;           // pipelined kernel: 4-tile chunks per row
+    int kparts;           // pipelined kernel: K-parts per unit
+    int cpp;              // pipelined kernel: chunks per K-part
+    int item_begin;       // pipelined kernel: first (unit, K-part) item in the group
+    int chunk_begin;      // pipelined kernel: balancing position of the first item
 };
 
 struct GemvParams {
     int count;
     int B;
-    int total_units;
+    int total_units16;    // register kernel
+    int total_items;      // pipelined kernel
+    int total_chunks;     // pipelined kernel: balancing space
+    uint32_t mul4, mul2;  // 4 and 2, passed at run time (see imul)
     int pad;
     GemvDesc d[SHERRY_MAX_GROUP];
 };
 
 struct XprepDesc {
     const int8_t *x;
-    uint32_t *xw;
+    uint32_t *xw;         // first word of this GEMV's workspace region
     int K;
-    int word_begin;  // first output word of this GEMV
+    int Tp;
+    int word_begin;       // first thread index of this GEMV
+    int xw_words;         // B * Tp * 32 re-ordered words, then zero_words zeros
+    int zero_words;       // partial sums and counters to clear
+    int pad;
 };
 
 struct XprepParams {
@@ -67,8 +83,45 @@ struct XprepParams {
     XprepDesc d[SHERRY_MAX_GROUP];
 };
 
-// xw[b][t][q]: word q = 2 (4 i + beta) + h holds the activations met by
-// char4(i, beta, h) of tile t: bytes x[b][128 t + 16 k' + 64 h + 4 beta + i], k' = 0..3.
+constexpr int kGemvThreads = 256;
+constexpr int kGemvWarps = kGemvThreads / 32;
+
+constexpr int kUnitRows = 32;      // pipelined kernel: rows per unit (two m16 blocks)
+constexpr int kChunkTiles = 4;     // tiles per K-chunk = per ring stage
+constexpr int kMaxPartChunks = 4;  // longest K-part: 4 chunks = 2048 weights per row
+constexpr int kRing = 3;           // stages per warp
+// A stage holds one chunk: 4 tile blocks of 5 planes x 32 rows (160 words, a
+// contiguous 2560 bytes in global memory), each block padded to 168 words in
+// shared memory so that a read of (tile t, plane p, rows g + 8 rb) by lanes
+// (g, t) hits 32 distinct banks.
+constexpr int kTileWords = 5 * kUnitRows;            // 160
+constexpr int kTileWordsPadded = kTileWords + 8;     // 168
+constexpr int kStageWords = kChunkTiles * kTileWordsPadded;
+constexpr int kPipeThreads = 256;
+constexpr int kPipeWarps = kPipeThreads / 32;
+constexpr size_t kPipeSmem = (size_t)kPipeWarps * kRing * kStageWords * 4;
+
+int64_t padded_tiles(int64_t K) {
+    const int64_t T = K / SHERRY_TILE_K;
+    return (T + kChunkTiles - 1) / kChunkTiles * kChunkTiles;
+}
+int64_t round_words(int64_t w) { return (w + 63) / 64 * 64; }  // 256-byte regions
+
+// Workspace words of one GEMV: re-ordered activations, then (for the pipelined
+// kernel) the K-part partial sums and the per-unit counters.
+int64_t ws_words(int64_t N, int64_t K, int B) {
+    const int64_t units = (N + kUnitRows - 1) / kUnitRows;
+    return round_words((int64_t)B * padded_tiles(K) * 32) + round_words((int64_t)B * N + units);
+}
+
+// ---------------------------------------------------------------------------
+// Activation re-order
+// ---------------------------------------------------------------------------
+// xw[b][t][q] (t < Tp): word q = 2 (4 i + beta) + h holds the activations met
+// by char4(i, beta, h) of tile t: bytes x[b][128 t + 16 k' + 64 h + 4 beta + i],
+// k' = 0..3; tiles t >= K/128 are zero so that padded chunks contribute
+// nothing.  The words after the re-ordered block (partial sums, counters) are
+// cleared.
 __global__ void __launch_bounds__(256) xprep_kernel(const __grid_constant__ XprepParams P) {
     const int w = blockIdx.x * blockDim.x + threadIdx.x;
     if (w >= P.total_words) return;
@@ -79,18 +132,28 @@ __global__ void __launch_bounds__(256) xprep_kernel(const __grid_constant__ Xpre
     }
     const XprepDesc &D = P.d[lo];
     const int local = w - D.word_begin;
+    if (local >= D.xw_words) {
+        D.xw[local] = 0u;
+        return;
+    }
     const int T = D.K / SHERRY_TILE_K;
     const int q = local & 31;
-    const int t = (local >> 5) % T;
-    const int b = (local >> 5) / T;
+    const int t = (local >> 5) % D.Tp;
+    const int b = (local >> 5) / D.Tp;
+    if (t >= T || b >= P.B) {
+        D.xw[local] = 0u;
+        return;
+    }
     const int m = q >> 1, h = q & 1, i = m >> 2, beta = m & 3;
     const uint8_t *src = reinterpret_cast<const uint8_t *>(D.x) + (size_t)b * D.K +
                          (size_t)t * SHERRY_TILE_K + 64 * h + 4 * beta + i;
-    const uint32_t v = (uint32_t)src[0] | ((uint32_t)src[16] << 8) | ((uint32_t)src[32] << 16) |
-                       ((uint32_t)src[48] << 24);
-    D.xw[local] = v;
+    D.xw[local] = (uint32_t)src[0] | ((uint32_t)src[16] << 8) | ((uint32_t)src[32] << 16) |
+                  ((uint32_t)src[48] << 24);
 }
 
+// ---------------------------------------------------------------------------
+// Device helpers
+// ---------------------------------------------------------------------------
 __device__ __forceinline__ void mma_s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                        uint32_t a3, uint32_t b0, uint32_t b1) {
     asm volatile(
@@ -118,25 +181,89 @@ __device__ __forceinline__ uint32_t pick(const uint4 &v, int j) {
     return j == 0 ? v.x : j == 1 ? v.y : j == 2 ? v.z : v.w;
 }
 
+__device__ __forceinline__ uint32_t lop_mux(uint32_t m, uint32_t a, uint32_t b) {  // m ? a : b
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xCA;" : "=r"(d) : "r"(m), "r"(a), "r"(b));
+    return d;
+}
+__device__ __forceinline__ uint32_t lop_merge(uint32_t a, uint32_t b, uint32_t m) {  // (a&m)|(b&~m)
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xE4;" : "=r"(d) : "r"(a), "r"(b), "r"(m));
+    return d;
+}
+__device__ __forceinline__ uint32_t lop_or_masked(uint32_t x, uint32_t m, uint32_t z) {  // (x&m)|z
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(x), "r"(m), "r"(z));
+    return d;
+}
+// Multiplication by a power of two passed at run time, so that the compiler
+// keeps it on the FMA pipe instead of turning it into an ALU shift.
+__device__ __forceinline__ uint32_t imul(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("mul.lo.u32 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+struct Consts {
+    uint32_t mul4, mul2;
+};
+
+// Per-row tile state of the pipelined kernel: zero-position nibbles per block
+// group and the four per-position sign planes.  Selector of (i, beta):
+//   zm[beta] | (sign plane i moved so block 4k+beta's bit lands at 4k+2) & 0x44444444.
+struct TileDecoder6 {
+    uint32_t zm[4];
+    uint32_t sg[4];
+
+    __device__ __forceinline__ void load(const Consts &C, uint32_t z0, uint32_t z1, uint32_t s0,
+                                         uint32_t s1, uint32_t s2) {
+        zm[0] = z0 & 0x33333333u;
+        zm[1] = z1 & 0x33333333u;
+        zm[2] = (z0 >> 2) & 0x33333333u;
+        zm[3] = (z1 >> 2) & 0x33333333u;
+        // bit-sliced zero positions: lo bit (L) and hi bit (H) of p_j at bit j
+        const uint32_t L = lop_merge(z0, imul(z1, C.mul2), 0x55555555u);
+        const uint32_t H = lop_merge(z0 >> 1, z1, 0x55555555u);
+        // sign of position i when kept: rank 0; rank 0 if p == 0 else 1;
+        // rank 1 if p <= 1 else 2; rank 2
+        sg[0] = s0;
+        sg[1] = lop_mux(L | H, s1, s0);
+        sg[2] = lop_mux(H, s2, s1);
+        sg[3] = s2;
+    }
+    __device__ __forceinline__ uint32_t sel(const Consts &C, int i, int beta) const {
+        const uint32_t v = beta == 0 ? imul(sg[i], C.mul4)
+                         : beta == 1 ? imul(sg[i], C.mul2)
+                         : beta == 2 ? sg[i] : (sg[i] >> 1);
+        return lop_or_masked(v, 0x44444444u, zm[beta]);
+    }
+};
+
+// ---------------------------------------------------------------------------
+// Register kernel (general fallback): each warp owns 16 rows x all of K; a
+// thread decodes rows g and g+8 of tile 4s + t and keeps the next slice's code
+// words in registers.
+// ---------------------------------------------------------------------------
 // NB = number of 8-row batch groups (1: B <= 8, 2: B <= 16).
 template <int NB, bool ACC_OUT>
 __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const __grid_constant__ GemvParams P) {
     const int lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
     const int nwarps = gridDim.x * kGemvWarps;
-    for (int u = blockIdx.x * kGemvWarps + (threadIdx.x >> 5); u < P.total_units; u += nwarps) {
+    for (int u = blockIdx.x * kGemvWarps + (threadIdx.x >> 5); u < P.total_units16; u += nwarps) {
         int lo = 0, hi = P.count - 1;
         while (lo < hi) {
             const int mid = (lo + hi + 1) >> 1;
-            if (P.d[mid].unit_begin <= u) lo = mid; else hi = mid - 1;
+            if (P.d[mid].unit_begin16 <= u) lo = mid; else hi = mid - 1;
         }
         const GemvDesc &D = P.d[lo];
         const int N = D.N, T = D.T;
-        const int r0 = (u - D.unit_begin) * 16 + g, r1 = r0 + 8;
+        const int r0 = (u - D.unit_begin16) * 16 + g, r1 = r0 + 8;
         const bool v0 = r0 < N, v1 = r1 < N;
-        const size_t plane = (size_t)N * T;
-        const uint32_t *c0 = D.codes + (size_t)r0 * T;
-        const uint32_t *c1 = D.codes + (size_t)r1 * T;
+        // word (p, row, tile) = ((row / 32) * T + tile) * 160 + 32 p + row % 32;
+        // rows past N inside the last group are zero padding, so loads need no row test
+        const uint32_t *c0 = D.codes + (size_t)(r0 / 32) * T * 160 + (r0 % 32);
+        const uint32_t *c1 = D.codes + (size_t)(r1 / 32) * T * 160 + (r1 % 32);
 
         int acc[NB][4];
 #pragma unroll
@@ -149,8 +276,8 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const __grid_constan
             const bool tv = tile < T;
 #pragma unroll
             for (int p = 0; p < 5; p++) {
-                w0[p] = (tv && v0) ? ld_code(c0 + p * plane + tile) : 0u;
-                w1[p] = (tv && v1) ? ld_code(c1 + p * plane + tile) : 0u;
+                w0[p] = tv ? ld_code(c0 + (size_t)tile * 160 + p * 32) : 0u;
+                w1[p] = tv ? ld_code(c1 + (size_t)tile * 160 + p * 32) : 0u;
             }
         }
         for (int s = 0; s < nslices; s++) {
@@ -159,24 +286,22 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const __grid_constan
             TileDecoder d0, d1;
             d0.load(w0[0], w0[1], w0[2], w0[3], w0[4]);
             d1.load(w1[0], w1[1], w1[2], w1[3], w1[4]);
-            // activations of this tile for batch rows g (+8)
             uint4 xv[NB][8];
 #pragma unroll
             for (int nb = 0; nb < NB; nb++) {
                 const int b = nb * 8 + g;
                 const bool xvld = tv && b < P.B;
-                const uint4 *xp = D.xw + ((size_t)b * T + tile) * 8;
+                const uint4 *xp = D.xw + ((size_t)b * D.Tp + tile) * 8;
 #pragma unroll
                 for (int k = 0; k < 8; k++) xv[nb][k] = xvld ? ld_x(xp + k) : make_uint4(0, 0, 0, 0);
             }
-            // prefetch the next slice's code words
-            if (s + 1 < nslices) {
+            if (s + 1 < nslices) {  // prefetch the next slice's code words
                 const int nt = tile + 4;
                 const bool ntv = nt < T;
 #pragma unroll
                 for (int p = 0; p < 5; p++) {
-                    w0[p] = (ntv && v0) ? ld_code(c0 + p * plane + nt) : 0u;
-                    w1[p] = (ntv && v1) ? ld_code(c1 + p * plane + nt) : 0u;
+                    w0[p] = ntv ? ld_code(c0 + (size_t)nt * 160 + p * 32) : 0u;
+                    w1[p] = ntv ? ld_code(c1 + (size_t)nt * 160 + p * 32) : 0u;
                 }
             }
 #pragma unroll
@@ -193,8 +318,8 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const __grid_constan
 #pragma unroll
                     for (int nb = 0; nb < NB; nb++) {
                         const uint4 &xq = xv[nb][m >> 1];
-                        const uint32_t b0 = pick(xq, (m & 1) * 2), b1 = pick(xq, (m & 1) * 2 + 1);
-                        mma_s8(acc[nb], a0, a1, a2, a3, b0, b1);
+                        mma_s8(acc[nb], a0, a1, a2, a3, pick(xq, (m & 1) * 2),
+                               pick(xq, (m & 1) * 2 + 1));
                     }
                 }
             }
@@ -208,36 +333,283 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const __grid_constan
                 const bool rv = (e < 2) ? v0 : v1;
                 const int b = nb * 8 + 2 * t + (e & 1);
                 if (rv && b < P.B) {
-                    if (ACC_OUT) {
+                    if (ACC_OUT)
                         static_cast<int32_t *>(D.out)[(size_t)b * N + row] = acc[nb][e];
-                    } else {
+                    else
                         static_cast<float *>(D.out)[(size_t)b * N + row] =
                             __ldg(D.scales + row) * (float)acc[nb][e];
-                    }
                 }
             }
         }
     }
 }
 
-size_t ws_bytes(int64_t K, int B) { return (size_t)((B * K + 255) / 256) * 256; }
+// ---------------------------------------------------------------------------
+// Pipelined kernel (K % 512 == 0, codes 16-byte aligned).
+//
+//   * work item = (32-row unit, K-part of at most 4 chunks = 2048 weights per
+//     row); thread (g, t) decodes rows g, g+8, g+16, g+24 of the unit for tile
+//     4c + t of chunk c, so the activation fragments it loads feed 32 MMAs;
+//   * a chunk of a unit (32 rows x 4 tiles) is one contiguous 2560-byte block
+//     of the code layout; each warp streams its items' chunks through a
+//     private ring of kRing shared-memory stages filled by cp.async with
+//     consecutive lanes on consecutive 16 bytes, so an SM keeps ~100 KB of
+//     fully coalesced HBM reads in flight;
+//   * items are split into contiguous ranges of equal chunk count, one range
+//     per warp, in GEMV order, so no warp carries much more than the average;
+//   * a unit with several K-parts adds its partial int32 sums into part_acc
+//     with atomics; the warp that completes the last part (per-unit counter)
+//     scales, writes y and clears its part_acc entries and the counter, so
+//     the workspace is ready for the next launch.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+                 "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
 
-template <int NB, bool ACC>
-int gemv_grid(int units) {
-    static int blocks_per_sm[64] = {0};
+__device__ __forceinline__ int find_desc_by_item(const GemvParams &P, int item) {
+    int lo = 0, hi = P.count - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (P.d[mid].item_begin <= item) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+// First item whose balancing position is >= c (total_items if none).
+__device__ __forceinline__ int first_item_at_or_after(const GemvParams &P, int c) {
+    if (c >= P.total_chunks) return P.total_items;
+    int lo = 0, hi = P.count - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (P.d[mid].chunk_begin <= c) lo = mid; else hi = mid - 1;
+    }
+    const GemvDesc &D = P.d[lo];
+    const int items = D.units * D.kparts;
+    const int k = (c - D.chunk_begin + D.cpp - 1) / D.cpp;
+    return k < items ? D.item_begin + k
+                     : (lo + 1 < P.count ? P.d[lo + 1].item_begin : P.total_items);
+}
+
+template <int NB, bool ACC_OUT>
+__global__ void __launch_bounds__(kPipeThreads, 3)
+    gemv_pipe_kernel(const __grid_constant__ GemvParams P) {
+    extern __shared__ __align__(16) uint32_t pipe_smem[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    const long long nw = (long long)gridDim.x * kPipeWarps;
+    const long long wg = (long long)blockIdx.x * kPipeWarps + warp;
+    const int it_begin = first_item_at_or_after(P, (int)(wg * P.total_chunks / nw));
+    const int it_end = first_item_at_or_after(P, (int)((wg + 1) * P.total_chunks / nw));
+    if (it_begin >= it_end) return;
+    uint32_t *ring = pipe_smem + (size_t)warp * kRing * kStageWords;
+    const Consts C{P.mul4, P.mul2};
+
+    // ---- producer side: the issue cursor runs kRing-1 stages ahead ----
+    // lane l copies 16-byte pieces l + 32 j (j = 0..4) of the 2560-byte chunk;
+    // piece words 4i..4i+3 belong to tile block 4i / 160
+    int iitem = it_begin, id = find_desc_by_item(P, it_begin);
+    int ic = 0, ic_end = 0;          // chunk cursor within the current item
+    const uint32_t *isrc = nullptr;  // first word of the current unit's group
+    auto set_issue_item = [&]() {
+        const GemvDesc &D = P.d[id];
+        const int local = iitem - D.item_begin;
+        const int unit = local / D.kparts, kp = local - unit * D.kparts;
+        isrc = D.codes + (size_t)unit * D.T * kTileWords + 4 * lane;
+        ic = kp * D.cpp;
+        ic_end = min(D.nchunk, ic + D.cpp);
+    };
+    set_issue_item();
+    uint32_t dst_piece[5];
+#pragma unroll
+    for (int j = 0; j < 5; j++) {
+        const int wd = 4 * (lane + 32 * j);
+        const int tb = wd / kTileWords;
+        dst_piece[j] = smem_u32(ring) + 4u * (uint32_t)(tb * kTileWordsPadded + (wd - tb * kTileWords));
+    }
+    auto issue = [&](int slot) {
+        if (iitem < it_end) {
+            const uint32_t *src = isrc + (size_t)ic * kChunkTiles * kTileWords;
+            const uint32_t sofs = (uint32_t)slot * kStageWords * 4;
+#pragma unroll
+            for (int j = 0; j < 5; j++) cp_async16(dst_piece[j] + sofs, src + 128 * j, 16u);
+            if (++ic == ic_end && ++iitem < it_end) {
+                if (iitem >= P.d[id].item_begin + P.d[id].units * P.d[id].kparts) id++;
+                set_issue_item();
+            }
+        }
+        cp_async_commit();
+    };
+#pragma unroll
+    for (int s = 0; s < kRing - 1; s++) issue(s);
+
+    // ---- consumer side ----
+    int slot = 0;
+    for (int item = it_begin; item < it_end; item++) {
+        const GemvDesc &D = P.d[find_desc_by_item(P, item)];
+        const int N = D.N;
+        const int local = item - D.item_begin;
+        const int unit = local / D.kparts, kp = local - unit * D.kparts;
+        const int rbase = unit * kUnitRows;
+        const int c_begin = kp * D.cpp, c_end = min(D.nchunk, c_begin + D.cpp);
+        const uint4 *xrow[NB];
+#pragma unroll
+        for (int nb = 0; nb < NB; nb++) {
+            const int b = min(nb * 8 + g, P.B - 1);  // lanes past the batch: never stored
+            xrow[nb] = D.xw + (size_t)b * D.Tp * 8 + (size_t)t * 8;
+        }
+        int acc[2][NB][4];  // [row block][batch group][fragment]
+#pragma unroll
+        for (int a = 0; a < 2; a++)
+#pragma unroll
+            for (int nb = 0; nb < NB; nb++) acc[a][nb][0] = acc[a][nb][1] = acc[a][nb][2] = acc[a][nb][3] = 0;
+        for (int c = c_begin; c < c_end; c++) {
+            cp_async_wait<kRing - 2>();
+            __syncwarp();
+            // tile t of the chunk, plane p, row g + 8 r: word t * 168 + 32 p + g + 8 r
+            const uint32_t *st = ring + slot * kStageWords + t * kTileWordsPadded + g;
+            TileDecoder6 dec[4];  // rows g, g+8, g+16, g+24
+#pragma unroll
+            for (int r = 0; r < 4; r++)
+                dec[r].load(C, st[0 * 32 + r * 8], st[1 * 32 + r * 8], st[2 * 32 + r * 8],
+                            st[3 * 32 + r * 8], st[4 * 32 + r * 8]);
+            __syncwarp();  // every lane has its words: the stage can be refilled
+            issue(slot == 0 ? kRing - 1 : slot - 1);
+            slot = (slot + 1 == kRing) ? 0 : slot + 1;
+            // padded tiles hold zero activations, so no load is predicated
+            const size_t xoff = (size_t)c * kChunkTiles * 8;
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                uint4 xq[NB][2];
+#pragma unroll
+                for (int nb = 0; nb < NB; nb++) {
+                    xq[nb][0] = ld_x(xrow[nb] + xoff + 2 * i);
+                    xq[nb][1] = ld_x(xrow[nb] + xoff + 2 * i + 1);
+                }
+                const uint32_t tlo = table_lo(i), thi = table_hi(i);
+#pragma unroll
+                for (int beta = 0; beta < 4; beta++) {
+                    const int m = 4 * i + beta;  // MMA index: activation words 2m, 2m+1
+#pragma unroll
+                    for (int rb = 0; rb < 2; rb++) {
+                        const uint32_t s0 = dec[2 * rb].sel(C, i, beta);
+                        const uint32_t s1 = dec[2 * rb + 1].sel(C, i, beta);
+                        const uint32_t a0 = prmt(tlo, thi, s0);
+                        const uint32_t a2 = prmt(tlo, thi, s0 >> 16);
+                        const uint32_t a1 = prmt(tlo, thi, s1);
+                        const uint32_t a3 = prmt(tlo, thi, s1 >> 16);
+#pragma unroll
+                        for (int nb = 0; nb < NB; nb++) {
+                            const uint4 &xx = xq[nb][(m >> 1) & 1];
+                            mma_s8(acc[rb][nb], a0, a1, a2, a3, pick(xx, (m & 1) * 2),
+                                   pick(xx, (m & 1) * 2 + 1));
+                        }
+                    }
+                }
+            }
+        }
+        // epilogue: per row block, c0/c1 = (row g, cols 2t, 2t+1), c2/c3 = row g+8
+        bool finish = true;
+        if (D.kparts > 1) {
+#pragma unroll
+            for (int rb = 0; rb < 2; rb++)
+#pragma unroll
+                for (int nb = 0; nb < NB; nb++)
+#pragma unroll
+                    for (int e = 0; e < 4; e++) {
+                        const int row = rbase + rb * 16 + g + ((e & 2) ? 8 : 0);
+                        const int b = nb * 8 + 2 * t + (e & 1);
+                        if (row < N && b < P.B)
+                            atomicAdd(D.part_acc + (size_t)b * N + row, acc[rb][nb][e]);
+                    }
+            __threadfence();
+            __syncwarp();
+            uint32_t done = 0;
+            if (lane == 0) done = atomicAdd(D.part_cnt + unit, 1u);
+            finish = __shfl_sync(0xFFFFFFFFu, done, 0) == (uint32_t)(D.kparts - 1);
+            if (finish) {
+                __threadfence();
+#pragma unroll
+                for (int rb = 0; rb < 2; rb++)
+#pragma unroll
+                    for (int nb = 0; nb < NB; nb++)
+#pragma unroll
+                        for (int e = 0; e < 4; e++) {
+                            const int row = rbase + rb * 16 + g + ((e & 2) ? 8 : 0);
+                            const int b = nb * 8 + 2 * t + (e & 1);
+                            if (row < N && b < P.B) {
+                                int32_t *pa = D.part_acc + (size_t)b * N + row;
+                                acc[rb][nb][e] = __ldcg(pa);
+                                *pa = 0;
+                            }
+                        }
+                if (lane == 0) D.part_cnt[unit] = 0u;
+            }
+        }
+        if (finish) {
+#pragma unroll
+            for (int rb = 0; rb < 2; rb++)
+#pragma unroll
+                for (int nb = 0; nb < NB; nb++)
+#pragma unroll
+                    for (int e = 0; e < 4; e++) {
+                        const int row = rbase + rb * 16 + g + ((e & 2) ? 8 : 0);
+                        const int b = nb * 8 + 2 * t + (e & 1);
+                        if (row < N && b < P.B) {
+                            if (ACC_OUT)
+                                static_cast<int32_t *>(D.out)[(size_t)b * N + row] = acc[rb][nb][e];
+                            else
+                                static_cast<float *>(D.out)[(size_t)b * N + row] =
+                                    __ldg(D.scales + row) * (float)acc[rb][nb][e];
+                        }
+                    }
+        }
+    }
+    cp_async_wait<0>();
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+template <typename KernelT>
+int grid_for(KernelT kernel, int threads, size_t smem, int want, int *cache) {
     int dev = 0;
     cudaGetDevice(&dev);
-    int &bps = blocks_per_sm[dev & 63];
+    int &bps = cache[dev & 63];
     if (bps == 0) {
+        if (smem > 48 * 1024)
+            cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         int n = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, gemv_kernel<NB, ACC>, kGemvThreads, 0) !=
-                cudaSuccess ||
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, smem) != cudaSuccess ||
             n < 1)
             n = 1;
         bps = n;
     }
-    const int want = (units + kGemvWarps - 1) / kGemvWarps;
     return std::max(1, std::min(want, bps * sm_count()));
+}
+
+template <int NB, bool ACC>
+void launch_pipe(const GemvParams &gp, cudaStream_t stream) {
+    static int cache[64] = {0};
+    const int want = (gp.total_chunks + kPipeWarps * 4 - 1) / (kPipeWarps * 4);
+    const int grid = grid_for(gemv_pipe_kernel<NB, ACC>, kPipeThreads, kPipeSmem, want, cache);
+    gemv_pipe_kernel<NB, ACC><<<grid, kPipeThreads, kPipeSmem, stream>>>(gp);
+}
+
+template <int NB, bool ACC>
+void launch_regs(const GemvParams &gp, cudaStream_t stream) {
+    static int cache[64] = {0};
+    const int want = (gp.total_units16 + kGemvWarps - 1) / kGemvWarps;
+    const int grid = grid_for(gemv_kernel<NB, ACC>, kGemvThreads, 0, want, cache);
+    gemv_kernel<NB, ACC><<<grid, kGemvThreads, 0, stream>>>(gp);
 }
 
 struct GemvCall {
@@ -248,30 +620,45 @@ struct GemvCall {
     int64_t N, K;
 };
 
+enum Phase { kPrepare = 1, kRun = 2, kBoth = 3 };
+
 sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out, void *workspace,
-                          size_t workspace_bytes, cudaStream_t stream) {
+                          size_t workspace_bytes, cudaStream_t stream, int phase) {
     if (count < 1) return SHERRY_ERR_SHAPE;
     if (count > SHERRY_MAX_GROUP) return SHERRY_ERR_UNSUPPORTED;
     if (B < 1) return SHERRY_ERR_SHAPE;
     if (B > SHERRY_MAX_GEMV_BATCH) return SHERRY_ERR_UNSUPPORTED;
     if (!workspace) return SHERRY_ERR_WORKSPACE;
     if (!aligned(workspace, 256)) return SHERRY_ERR_ALIGN;
-    size_t need = 0;
-    int64_t units = 0, words = 0;
+    int64_t words = 0, units16 = 0, items = 0, chunks = 0;
     for (int i = 0; i < count; i++) {
         const GemvCall &c = calls[i];
-        if (!c.codes || !c.x || !c.out || (!acc_out && !c.scales)) return SHERRY_ERR_NULL;
+        const bool need_x = (phase & kPrepare) != 0, need_out = (phase & kRun) != 0;
+        if ((need_x && !c.x) || (need_out && (!c.codes || !c.out || (!acc_out && !c.scales))))
+            return SHERRY_ERR_NULL;
         if (c.N < 1 || !valid_k(c.K)) return SHERRY_ERR_SHAPE;
-        if (!aligned(c.codes, 4) || !aligned(c.x, 4) || !aligned(c.out, 4) ||
-            (c.scales && !aligned(c.scales, 4)))
+        if ((need_x && !aligned(c.x, 4)) ||
+            (need_out && (!aligned(c.codes, 4) || !aligned(c.out, 4) ||
+                          (c.scales && !aligned(c.scales, 4)))))
             return SHERRY_ERR_ALIGN;
-        if (c.N > (int64_t)1 << 30) return SHERRY_ERR_UNSUPPORTED;
-        need += ws_bytes(c.K, B);
-        units += (c.N + 15) / 16;
-        words += (int64_t)B * c.K / 4;
+        if (c.N > (int64_t)1 << 28) return SHERRY_ERR_UNSUPPORTED;
+        words += ws_words(c.N, c.K, B);
+        units16 += (c.N + 15) / 16;
+        const int64_t nchunk = padded_tiles(c.K) / kChunkTiles;
+        const int64_t kparts = (nchunk + kMaxPartChunks - 1) / kMaxPartChunks;
+        items += (c.N + kUnitRows - 1) / kUnitRows * kparts;
+        chunks += (c.N + kUnitRows - 1) / kUnitRows * kparts * ((nchunk + kparts - 1) / kparts);
     }
-    if (workspace_bytes < need) return SHERRY_ERR_WORKSPACE;
-    if (units > 0x7FFFFFFF || words > 0x7FFFFFFF) return SHERRY_ERR_UNSUPPORTED;
+    if (workspace_bytes < (size_t)words * 4) return SHERRY_ERR_WORKSPACE;
+    if (words > 0x7FFFFFFF || units16 > 0x7FFFFFFF || items > 0x7FFFFFFF || chunks > 0x7FFFFFFF)
+        return SHERRY_ERR_UNSUPPORTED;
+
+    // the pipelined kernel needs whole 4-tile chunks and 16-byte aligned code rows
+    bool pipelined = true;
+    for (int i = 0; i < count; i++)
+        if ((calls[i].K / SHERRY_TILE_K) % kChunkTiles != 0 ||
+            ((phase & kRun) && !aligned(calls[i].codes, 16)))
+            pipelined = false;
 
     static thread_local XprepParams xp;
     static thread_local GemvParams gp;
@@ -279,60 +666,103 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
     std::memset(&gp, 0, sizeof(gp));
     xp.count = gp.count = count;
     xp.B = gp.B = B;
-    size_t off = 0;
-    int ub = 0, wb = 0;
+    gp.mul4 = 4u;
+    gp.mul2 = 2u;
+    int64_t off = 0;
+    int wb = 0, ub16 = 0, ib = 0, cb = 0;
     for (int i = 0; i < count; i++) {
         const GemvCall &c = calls[i];
-        uint32_t *xw = reinterpret_cast<uint32_t *>(static_cast<char *>(workspace) + off);
-        xp.d[i].x = c.x;
-        xp.d[i].xw = xw;
-        xp.d[i].K = (int)c.K;
-        xp.d[i].word_begin = wb;
-        gp.d[i].codes = c.codes;
-        gp.d[i].scales = c.scales;
-        gp.d[i].xw = reinterpret_cast<const uint4 *>(xw);
-        gp.d[i].out = c.out;
-        gp.d[i].N = (int)c.N;
-        gp.d[i].T = (int)(c.K / SHERRY_TILE_K);
-        gp.d[i].unit_begin = ub;
-        off += ws_bytes(c.K, B);
-        ub += (int)((c.N + 15) / 16);
-        wb += (int)((int64_t)B * c.K / 4);
+        uint32_t *region = static_cast<uint32_t *>(workspace) + off;
+        const int Tp = (int)padded_tiles(c.K);
+        const int xw_words = (int)round_words((int64_t)B * Tp * 32);
+        const int units = (int)((c.N + kUnitRows - 1) / kUnitRows);
+        const int nchunk = Tp / kChunkTiles;
+        const int kparts = (nchunk + kMaxPartChunks - 1) / kMaxPartChunks;
+        const int cpp = (nchunk + kparts - 1) / kparts;
+        XprepDesc &X = xp.d[i];
+        X.x = c.x;
+        X.xw = region;
+        X.K = (int)c.K;
+        X.Tp = Tp;
+        X.word_begin = wb;
+        X.xw_words = xw_words;
+        X.zero_words = (int)round_words((int64_t)B * c.N + units);
+        GemvDesc &D = gp.d[i];
+        D.codes = c.codes;
+        D.scales = c.scales;
+        D.xw = reinterpret_cast<const uint4 *>(region);
+        D.out = c.out;
+        D.part_acc = reinterpret_cast<int32_t *>(region + xw_words);
+        D.part_cnt = region + xw_words + (int64_t)B * c.N;
+        D.N = (int)c.N;
+        D.T = (int)(c.K / SHERRY_TILE_K);
+        D.Tp = Tp;
+        D.unit_begin16 = ub16;
+        D.units = units;
+        D.nchunk = nchunk;
+        D.kparts = kparts;
+        D.cpp = cpp;
+        D.item_begin = ib;
+        D.chunk_begin = cb;
+        off += ws_words(c.N, c.K, B);
+        wb += X.xw_words + X.zero_words;
+        ub16 += (int)((c.N + 15) / 16);
+        ib += units * kparts;
+        cb += units * kparts * cpp;
     }
     xp.total_words = wb;
-    gp.total_units = ub;
-    xprep_kernel<<<(wb + 255) / 256, 256, 0, stream>>>(xp);
-    sherry_status st = launch_status("sherry_gemv (activation re-order)");
-    if (st != SHERRY_OK) return st;
-    if (B <= 8) {
-        if (acc_out)
-            gemv_kernel<1, true><<<gemv_grid<1, true>(ub), kGemvThreads, 0, stream>>>(gp);
-        else
-            gemv_kernel<1, false><<<gemv_grid<1, false>(ub), kGemvThreads, 0, stream>>>(gp);
+    gp.total_units16 = ub16;
+    gp.total_items = ib;
+    gp.total_chunks = cb;
+    if (phase & kPrepare) {
+        xprep_kernel<<<(wb + 255) / 256, 256, 0, stream>>>(xp);
+        const sherry_status st = launch_status("sherry_gemv (activation re-order)");
+        if (st != SHERRY_OK) return st;
+    }
+    if (!(phase & kRun)) return SHERRY_OK;
+    if (pipelined) {
+        if (B <= 8) {
+            if (acc_out) launch_pipe<1, true>(gp, stream); else launch_pipe<1, false>(gp, stream);
+        } else {
+            if (acc_out) launch_pipe<2, true>(gp, stream); else launch_pipe<2, false>(gp, stream);
+        }
     } else {
-        if (acc_out)
-            gemv_kernel<2, true><<<gemv_grid<2, true>(ub), kGemvThreads, 0, stream>>>(gp);
-        else
-            gemv_kernel<2, false><<<gemv_grid<2, false>(ub), kGemvThreads, 0, stream>>>(gp);
+        if (B <= 8) {
+            if (acc_out) launch_regs<1, true>(gp, stream); else launch_regs<1, false>(gp, stream);
+        } else {
+            if (acc_out) launch_regs<2, true>(gp, stream); else launch_regs<2, false>(gp, stream);
+        }
     }
     return launch_status("sherry_gemv");
+}
+
+sherry_status grouped(const sherry_gemv_desc *descs, int count, int B, void *workspace,
+                      size_t workspace_bytes, cudaStream_t stream, int phase) {
+    if (!descs) return SHERRY_ERR_NULL;
+    if (count < 1) return SHERRY_ERR_SHAPE;
+    if (count > SHERRY_MAX_GROUP) return SHERRY_ERR_UNSUPPORTED;
+    GemvCall calls[SHERRY_MAX_GROUP];
+    for (int i = 0; i < count; i++)
+        calls[i] = GemvCall{descs[i].codes, descs[i].scales, descs[i].x, descs[i].y, descs[i].N,
+                            descs[i].K};
+    return gemv_launch(calls, count, B, false, workspace, workspace_bytes, stream, phase);
 }
 
 }  // namespace
 }  // namespace sherry
 
-extern "C" size_t sherry_gemv_workspace_bytes(int64_t K, int B) {
-    if (B < 1 || K < 1) return 0;
-    return sherry::ws_bytes(K, B);
+extern "C" size_t sherry_gemv_workspace_bytes(int64_t N, int64_t K, int B) {
+    if (B < 1 || N < 1 || K < 1) return 0;
+    return (size_t)sherry::ws_words(N, K, B) * 4;
 }
 
 extern "C" sherry_status sherry_gemv(const uint32_t *codes, const float *scales, const int8_t *x,
                                      float *y, int64_t N, int64_t K, int B, void *workspace,
                                      size_t workspace_bytes, sherry_stream_t stream) {
-    const sherry::GemvCall c{codes, scales, x, y, N, K};
     if (!scales) return SHERRY_ERR_NULL;
+    const sherry::GemvCall c{codes, scales, x, y, N, K};
     return sherry::gemv_launch(&c, 1, B, false, workspace, workspace_bytes,
-                               reinterpret_cast<cudaStream_t>(stream));
+                               reinterpret_cast<cudaStream_t>(stream), sherry::kBoth);
 }
 
 extern "C" sherry_status sherry_gemv_acc(const uint32_t *codes, const int8_t *x, int32_t *acc,
@@ -340,21 +770,26 @@ extern "C" sherry_status sherry_gemv_acc(const uint32_t *codes, const int8_t *x,
                                          size_t workspace_bytes, sherry_stream_t stream) {
     const sherry::GemvCall c{codes, nullptr, x, acc, N, K};
     return sherry::gemv_launch(&c, 1, B, true, workspace, workspace_bytes,
-                               reinterpret_cast<cudaStream_t>(stream));
+                               reinterpret_cast<cudaStream_t>(stream), sherry::kBoth);
 }
 
 extern "C" sherry_status sherry_gemv_grouped(const sherry_gemv_desc *descs, int count, int B,
                                              void *workspace, size_t workspace_bytes,
                                              sherry_stream_t stream) {
-    if (!descs) return SHERRY_ERR_NULL;
-    if (count < 1) return SHERRY_ERR_SHAPE;
-    if (count > SHERRY_MAX_GROUP) return SHERRY_ERR_UNSUPPORTED;
-    sherry::GemvCall calls[SHERRY_MAX_GROUP];
-    for (int i = 0; i < count; i++) {
-        calls[i] = sherry::GemvCall{descs[i].codes, descs[i].scales, descs[i].x, descs[i].y,
-                                    descs[i].N, descs[i].K};
-        if (!descs[i].scales) return SHERRY_ERR_NULL;
-    }
-    return sherry::gemv_launch(calls, count, B, false, workspace, workspace_bytes,
-                               reinterpret_cast<cudaStream_t>(stream));
+    return sherry::grouped(descs, count, B, workspace, workspace_bytes,
+                           reinterpret_cast<cudaStream_t>(stream), sherry::kBoth);
+}
+
+extern "C" sherry_status sherry_gemv_prepare(const sherry_gemv_desc *descs, int count, int B,
+                                             void *workspace, size_t workspace_bytes,
+                                             sherry_stream_t stream) {
+    return sherry::grouped(descs, count, B, workspace, workspace_bytes,
+                           reinterpret_cast<cudaStream_t>(stream), sherry::kPrepare);
+}
+
+extern "C" sherry_status sherry_gemv_run(const sherry_gemv_desc *descs, int count, int B,
+                                         const void *workspace, size_t workspace_bytes,
+                                         sherry_stream_t stream) {
+    return sherry::grouped(descs, count, B, const_cast<void *>(workspace), workspace_bytes,
+                           reinterpret_cast<cudaStream_t>(stream), sherry::kRun);
 }

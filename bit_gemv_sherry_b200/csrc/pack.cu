@@ -63,9 +63,10 @@ __device__ __forceinline__ TileBits pack_tile(float4 v) {
 }
 
 // CTA = 8 warps; `wpr` warps share one row (tiles strided by wpr), the CTA
-// covers 8 / wpr rows.
+// covers 8 / wpr rows.  Rows N..Npad-1 (padding of the last 32-row group) are
+// written as zero words.
 __global__ void __launch_bounds__(kPackThreads) pack_kernel(const float *__restrict__ w, int64_t N,
-                                                            int64_t K, int wpr,
+                                                            int64_t Npad, int64_t K, int wpr,
                                                             uint32_t *__restrict__ codes,
                                                             float *__restrict__ scales) {
     __shared__ double partial[kPackWarps];
@@ -75,10 +76,10 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(const float *__restr
     const int sub = warp % wpr;
     const int64_t T = K / SHERRY_TILE_K;
     double row_sum = 0.0;
+    // word (p, n, t) = ((n / 32) * T + t) * 160 + 32 p + n % 32
+    uint32_t *out = codes + (n / SHERRY_ROW_GROUP) * T * (5 * SHERRY_ROW_GROUP) + n % SHERRY_ROW_GROUP;
     if (n < N) {
         const float4 *row = reinterpret_cast<const float4 *>(w + n * K);
-        const int64_t plane = N * T;
-        uint32_t *out = codes + n * T;
         for (int64_t t0 = sub; t0 < T; t0 += (int64_t)wpr * kPackUnroll) {
             float4 v[kPackUnroll];
 #pragma unroll
@@ -95,10 +96,13 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(const float *__restr
                 if (lane < 5) {
                     const uint32_t word = lane == 0 ? tb.z0 : lane == 1 ? tb.z1 : lane == 2 ? tb.s0
                                           : lane == 3 ? tb.s1 : tb.s2;
-                    out[lane * plane + t] = word;
+                    out[t * (5 * SHERRY_ROW_GROUP) + lane * SHERRY_ROW_GROUP] = word;
                 }
             }
         }
+    } else if (n < Npad) {
+        for (int64_t t = sub; t < T; t += wpr)
+            if (lane < 5) out[t * (5 * SHERRY_ROW_GROUP) + lane * SHERRY_ROW_GROUP] = 0u;
     }
     if (lane == 0) partial[warp] = row_sum;
     __syncthreads();
@@ -120,14 +124,15 @@ extern "C" sherry_status sherry_pack(const float *w, int64_t N, int64_t K, uint3
     using namespace sherry;
     if (!w || !codes || !scales) return SHERRY_ERR_NULL;
     if (N < 1 || !valid_k(K)) return SHERRY_ERR_SHAPE;
-    if (!aligned(w, 16) || !aligned(codes, 4) || !aligned(scales, 4)) return SHERRY_ERR_ALIGN;
+    if (!aligned(w, 16) || !aligned(codes, 16) || !aligned(scales, 4)) return SHERRY_ERR_ALIGN;
     const int64_t T = K / SHERRY_TILE_K;
+    const int64_t Npad = (N + SHERRY_ROW_GROUP - 1) / SHERRY_ROW_GROUP * SHERRY_ROW_GROUP;
     int wpr = 1;
     while (wpr < kPackWarps && wpr * 2 <= T) wpr *= 2;
     const int rpc = kPackWarps / wpr;
-    const int64_t grid = (N + rpc - 1) / rpc;
+    const int64_t grid = (Npad + rpc - 1) / rpc;
     if (grid > 0x7FFFFFFF) return SHERRY_ERR_UNSUPPORTED;
     pack_kernel<<<(unsigned)grid, kPackThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-        w, N, K, wpr, codes, scales);
+        w, N, Npad, K, wpr, codes, scales);
     return launch_status("sherry_pack");
 }

@@ -58,10 +58,12 @@ def lib():
     sig = {
         "sherry_packed_bytes": ([i64, i64], sz),
         "sherry_pack": ([p, i64, i64, p, p, p], i32),
-        "sherry_gemv_workspace_bytes": ([i64, i32], sz),
+        "sherry_gemv_workspace_bytes": ([i64, i64, i32], sz),
         "sherry_gemv": ([p, p, p, p, i64, i64, i32, p, sz, p], i32),
         "sherry_gemv_acc": ([p, p, p, i64, i64, i32, p, sz, p], i32),
         "sherry_gemv_grouped": ([p, i32, i32, p, sz, p], i32),
+        "sherry_gemv_prepare": ([p, i32, i32, p, sz, p], i32),
+        "sherry_gemv_run": ([p, i32, i32, p, sz, p], i32),
         "sherry_gemm": ([p, p, p, p, i64, i64, i64, p], i32),
         "sherry_gemm_acc": ([p, p, p, i64, i64, i64, p], i32),
         "sherry_device_error": ([], i32),
@@ -117,53 +119,66 @@ def packed_bytes(N, K):
     return int(lib().sherry_packed_bytes(N, K))
 
 
-def gemv_workspace_bytes(K, B):
-    return int(lib().sherry_gemv_workspace_bytes(K, B))
+def gemv_workspace_bytes(N, K, B):
+    return int(lib().sherry_gemv_workspace_bytes(N, K, B))
+
+
+GROUP = 32  # rows per group of the code layout
+
+
+def codes_shape(N, K):
+    """Shape of the int32 tensor holding the codes of an N x K matrix."""
+    return ((N + GROUP - 1) // GROUP, K // TILE_K, 5, GROUP)
 
 
 def pack(w, codes=None, scales=None):
-    """w: float32 [N, K] CUDA -> (codes int32 [5, N, K/128] (uint32 bit patterns), scales [N])."""
+    """w: float32 [N, K] CUDA -> (codes int32 [ceil(N/32), K/128, 5, 32] holding the
+    uint32 words, scales float32 [N])."""
     _need(w, torch.float32, "w")
     N, K = w.shape
     if codes is None:
-        codes = torch.empty((5, N, max(K // TILE_K, 1)), dtype=torch.int32, device=w.device)
+        codes = torch.empty(codes_shape(N, max(K, TILE_K)), dtype=torch.int32, device=w.device)
     if scales is None:
         scales = torch.empty(N, dtype=torch.float32, device=w.device)
     _check(lib().sherry_pack(_ptr(w), N, K, _ptr(codes), _ptr(scales), _stream(w)), "sherry_pack")
     return codes, scales
 
 
-def _codes_shape(codes):
+def _codes_shape(codes, N):
     _need(codes, torch.int32, "codes")
-    if codes.dim() != 3 or codes.shape[0] != 5:
-        raise ValueError("codes must have shape [5, N, K/128]")
-    return codes.shape[1], codes.shape[2] * TILE_K
+    if codes.dim() != 4 or codes.shape[2] != 5 or codes.shape[3] != GROUP:
+        raise ValueError("codes must have shape [ceil(N/32), K/128, 5, 32]")
+    if codes.shape[0] != (N + GROUP - 1) // GROUP:
+        raise ValueError("codes hold %d row groups, N = %d needs %d"
+                         % (codes.shape[0], N, (N + GROUP - 1) // GROUP))
+    return N, codes.shape[1] * TILE_K
 
 
 def gemv(codes, scales, x, y=None, ws=None):
     """y[B, N] = scales * (W . x^T); x int8 [B, K] (or [K])."""
-    N, K = _codes_shape(codes)
     _need(scales, torch.float32, "scales")
+    N, K = _codes_shape(codes, scales.numel())
     _need(x, torch.int8, "x")
     x2 = x.view(1, -1) if x.dim() == 1 else x
     B = x2.shape[0]
     if y is None:
         y = torch.empty((B, N), dtype=torch.float32, device=x.device)
-    nb = gemv_workspace_bytes(K, B)
+    nb = gemv_workspace_bytes(N, K, B)
     ws = workspace(nb, x.device) if ws is None else ws
     _check(lib().sherry_gemv(_ptr(codes), _ptr(scales), _ptr(x2), _ptr(y), N, K, B, _ptr(ws),
                              ws.numel(), _stream(x)), "sherry_gemv")
     return y
 
 
-def gemv_acc(codes, x, acc=None, ws=None):
-    N, K = _codes_shape(codes)
+def gemv_acc(codes, x, N, acc=None, ws=None):
+    """Exact int32 accumulators acc[B, N] = W . x^T."""
+    N, K = _codes_shape(codes, N)
     _need(x, torch.int8, "x")
     x2 = x.view(1, -1) if x.dim() == 1 else x
     B = x2.shape[0]
     if acc is None:
         acc = torch.empty((B, N), dtype=torch.int32, device=x.device)
-    nb = gemv_workspace_bytes(K, B)
+    nb = gemv_workspace_bytes(N, K, B)
     ws = workspace(nb, x.device) if ws is None else ws
     _check(lib().sherry_gemv_acc(_ptr(codes), _ptr(x2), _ptr(acc), N, K, B, _ptr(ws), ws.numel(),
                                  _stream(x)), "sherry_gemv_acc")
@@ -177,22 +192,63 @@ def gemv_grouped(items, B, ws=None):
     total = 0
     dev = None
     for i, (codes, scales, x, y) in enumerate(items):
-        N, K = _codes_shape(codes)
         _need(scales, torch.float32, "scales")
+        N, K = _codes_shape(codes, scales.numel())
         _need(x, torch.int8, "x")
         _need(y, torch.float32, "y")
         descs[i] = GemvDesc(codes.data_ptr(), scales.data_ptr(), x.data_ptr(), y.data_ptr(), N, K)
-        total += gemv_workspace_bytes(K, B)
+        total += gemv_workspace_bytes(N, K, B)
         dev = x.device
     ws = workspace(total, dev) if ws is None else ws
     _check(lib().sherry_gemv_grouped(ctypes.cast(descs, ctypes.c_void_p), n, B, _ptr(ws),
                                      ws.numel(), _stream(items[0][2])), "sherry_gemv_grouped")
 
 
+class GroupedGemv:
+    """Pre-marshalled grouped GEMV: descriptors and workspace are built once, and
+    each call only passes them to the library (used where per-call Python cost
+    matters, e.g. timing a decode step)."""
+
+    def __init__(self, items, B, ws=None):
+        n = len(items)
+        self.descs = (GemvDesc * n)()
+        total = 0
+        for i, (codes, scales, x, y) in enumerate(items):
+            _need(scales, torch.float32, "scales")
+            N, K = _codes_shape(codes, scales.numel())
+            _need(x, torch.int8, "x")
+            _need(y, torch.float32, "y")
+            self.descs[i] = GemvDesc(codes.data_ptr(), scales.data_ptr(), x.data_ptr(),
+                                     y.data_ptr(), N, K)
+            total += gemv_workspace_bytes(N, K, B)
+        self.items = items  # keep the tensors alive
+        self.n, self.B = n, B
+        dev = items[0][2].device
+        self.ws = torch.empty(max(total, 256), dtype=torch.uint8, device=dev) if ws is None else ws
+        self.args = (ctypes.cast(self.descs, ctypes.c_void_p), n, B, _ptr(self.ws),
+                     self.ws.numel())
+        self.device = dev
+
+    def __call__(self, stream=None):
+        s = ctypes.c_void_p(stream if stream is not None
+                            else torch.cuda.current_stream(self.device).cuda_stream)
+        _check(lib().sherry_gemv_grouped(*self.args, s), "sherry_gemv_grouped")
+
+    def prepare(self, stream=None):
+        s = ctypes.c_void_p(stream if stream is not None
+                            else torch.cuda.current_stream(self.device).cuda_stream)
+        _check(lib().sherry_gemv_prepare(*self.args, s), "sherry_gemv_prepare")
+
+    def run(self, stream=None):
+        s = ctypes.c_void_p(stream if stream is not None
+                            else torch.cuda.current_stream(self.device).cuda_stream)
+        _check(lib().sherry_gemv_run(*self.args, s), "sherry_gemv_run")
+
+
 def gemm(codes, scales, x, y=None):
     """y[M, N] = scales * (x . W^T); x int8 [M, K]."""
-    N, K = _codes_shape(codes)
     _need(scales, torch.float32, "scales")
+    N, K = _codes_shape(codes, scales.numel())
     _need(x, torch.int8, "x")
     M = x.shape[0]
     if y is None:
@@ -202,8 +258,9 @@ def gemm(codes, scales, x, y=None):
     return y
 
 
-def gemm_acc(codes, x, acc=None):
-    N, K = _codes_shape(codes)
+def gemm_acc(codes, x, N, acc=None):
+    """Exact int32 accumulators acc[M, N] = x . W^T."""
+    N, K = _codes_shape(codes, N)
     _need(x, torch.int8, "x")
     M = x.shape[0]
     if acc is None:

@@ -14,14 +14,17 @@
  * ---------------------------------------------------------------------------
  * Packed layout (the pages fix only "four weights in five bits"; this layout is
  * the library's reading, chosen so that 32 blocks decode with 32-bit SWAR
- * logic):
+ * logic and a GEMV work chunk is one contiguous block of memory):
  *   - a row of K weights (K a multiple of 128) is cut into T = K / 128 tiles of
  *     128 weights = 32 blocks; weight k = 128 t + 4 j + i is position i of
  *     block j of tile t;
- *   - a tile is five uint32 words Z0, Z1, S0, S1, S2 (20 bytes per 128
- *     weights, exactly 1.25 bits per weight), stored planar:
- *         codes[(plane * N + n) * T + t],  plane 0..4 = Z0, Z1, S0, S1, S2,
- *     so each plane of a row is contiguous and vector-loadable;
+ *   - a tile is five uint32 words Z0, Z1, S0, S1, S2 (planes 0..4; 20 bytes per
+ *     128 weights, exactly 1.25 bits per weight);
+ *   - rows are taken in groups of 32; within a group the tiles follow each
+ *     other and within a tile each plane holds the 32 rows of the group:
+ *         codes[((n / 32) * T + t) * 160 + plane * 32 + n % 32],
+ *     i.e. a [ceil(N/32)][T][5][32] array of uint32; rows past N in the last
+ *     group are padding and hold zeros;
  *   - block j's zero position p (0..3) is the 2-bit field at bits
  *     [2*(j/2), 2*(j/2)+1] of Z_(j mod 2) (Z0 holds the even blocks, Z1 the
  *     odd ones);
@@ -79,11 +82,13 @@ typedef enum {
 
 #define SHERRY_TILE_K 128         /* weights per tile                     */
 #define SHERRY_WORDS_PER_TILE 5   /* uint32 words per tile                */
+#define SHERRY_ROW_GROUP 32       /* rows per group of the code layout    */
 #define SHERRY_MAX_K 131072       /* keeps |acc| < 2^24                   */
 #define SHERRY_MAX_GEMV_BATCH 16  /* activation rows per GEMV call        */
 #define SHERRY_MAX_GROUP 128      /* GEMVs per grouped call               */
 
-/* Bytes of packed codes for an N x K matrix: N * K * 5 / 32 (scales excluded).
+/* Bytes of packed codes for an N x K matrix: ceil(N/32)*32 * K * 5 / 32
+ * (N * K * 5 / 32 when N is a multiple of 32; scales excluded).
  * Returns 0 when K is not a positive multiple of 128 or N < 1. */
 size_t sherry_packed_bytes(int64_t N, int64_t K);
 
@@ -92,7 +97,8 @@ size_t sherry_packed_bytes(int64_t N, int64_t K);
  * abstract: "packing blocks of four weights into five bits").
  *   w       [N][K] fp32, row-major, finite values (NaN/Inf give an unspecified
  *           but deterministic code); 16-byte aligned.
- *   codes   output, sherry_packed_bytes(N, K) bytes, layout above; 4-byte aligned.
+ *   codes   output, sherry_packed_bytes(N, K) bytes, layout above (padding rows
+ *           are written as zeros); 16-byte aligned.
  *   scales  output, N fp32.
  * Errors: NULL, SHAPE (N < 1, K not a positive multiple of 128, K > SHERRY_MAX_K),
  * ALIGN, CUDA.
@@ -101,20 +107,25 @@ sherry_status sherry_pack(const float *w, int64_t N, int64_t K, uint32_t *codes,
                           float *scales, sherry_stream_t stream);
 
 /*
- * Workspace of the GEMV calls: the activations are re-ordered once per call
- * into the order in which the decoded weights meet the tensor-core fragments.
- * sherry_gemv_workspace_bytes(K, B) is the size one GEMV needs (B * K bytes,
- * rounded up to 256); the grouped call needs the sum over its GEMVs.  The
- * workspace is a device buffer, 256-byte aligned, owned by the caller; its
- * contents are scratch and are overwritten by every call.
+ * Workspace of the GEMV calls.  Each call re-orders its activations once into
+ * the order in which the decoded weights meet the tensor-core fragments, and
+ * long rows are processed as several K-parts whose int32 partial sums meet in
+ * the workspace.  sherry_gemv_workspace_bytes(N, K, B) is the size one GEMV
+ * needs; a grouped call needs the sum over its GEMVs, laid out in descriptor
+ * order.  The workspace is a device buffer, 256-byte aligned, owned by the
+ * caller; its contents are scratch: every call that prepares activations
+ * (sherry_gemv, sherry_gemv_acc, sherry_gemv_grouped, sherry_gemv_prepare)
+ * rewrites it, and a run leaves its partial-sum area cleared.  Calls that
+ * overlap on the GPU must not share a workspace.
  */
-size_t sherry_gemv_workspace_bytes(int64_t K, int B);
+size_t sherry_gemv_workspace_bytes(int64_t N, int64_t K, int B);
 
 /*
  * sherry_gemv -- decode GEMV, y = s (.) (W_ternary . x_int8) for B <= 16
  * activation rows (arXiv 2601.07892, abstract: ternary weights served by
  * hardware-aligned packing; the batch-1 case is the decode step).
- *   codes   [5][N][K/128] uint32 from sherry_pack (or the same layout); 4-byte aligned.
+ *   codes   [ceil(N/32)][K/128][5][32] uint32 from sherry_pack; 4-byte aligned
+ *           (16-byte aligned and K a multiple of 512 select the pipelined kernel).
  *   scales  [N] fp32.
  *   x       [B][K] int8, row-major, any value in [-128, 127]; 4-byte aligned.
  *   y       [B][N] fp32 output, row-major.
@@ -151,7 +162,7 @@ typedef struct {
  *   descs  HOST array of `count` descriptors (copied into the launch
  *          parameters; may be reused as soon as the call returns).
  *   workspace: at least the sum over the group of
- *          sherry_gemv_workspace_bytes(K_i, B) bytes.
+ *          sherry_gemv_workspace_bytes(N_i, K_i, B) bytes.
  * Errors: as sherry_gemv, per descriptor; UNSUPPORTED if count > SHERRY_MAX_GROUP.
  */
 sherry_status sherry_gemv_grouped(const sherry_gemv_desc *descs, int count, int B,
@@ -159,11 +170,30 @@ sherry_status sherry_gemv_grouped(const sherry_gemv_desc *descs, int count, int 
                                   sherry_stream_t stream);
 
 /*
+ * The two halves of sherry_gemv_grouped, for callers that reuse one input
+ * across several GEMVs or time the GEMV kernel alone:
+ *   sherry_gemv_prepare  re-orders each descriptor's x into the workspace
+ *                        (reads descs[i].x, N, K; codes, scales, y unused);
+ *   sherry_gemv_run      runs the GEMVs on a workspace prepared by a previous
+ *                        sherry_gemv_prepare with the same descriptors' K and
+ *                        order and the same B, on the same stream (descs[i].x
+ *                        is not read).
+ * sherry_gemv_grouped(d, n, B, ws) == prepare(d, n, B, ws) then run(d, n, B, ws).
+ * Errors: as sherry_gemv_grouped, each for the fields it reads.
+ */
+sherry_status sherry_gemv_prepare(const sherry_gemv_desc *descs, int count, int B,
+                                  void *workspace, size_t workspace_bytes,
+                                  sherry_stream_t stream);
+sherry_status sherry_gemv_run(const sherry_gemv_desc *descs, int count, int B,
+                              const void *workspace, size_t workspace_bytes,
+                              sherry_stream_t stream);
+
+/*
  * sherry_gemm -- prefill GEMM, Y = X . W^T scaled per output column,
  *   Y[m][n] = s[n] * sum_k X[m][k] * W[n][k]   (the same product for M tokens).
  * The kernel decodes weight tiles to int8 in shared memory and runs them on
  * the tcgen05 int8 tensor-core path with int32 accumulators in tensor memory.
- *   codes   [5][N][K/128] uint32; 4-byte aligned.
+ *   codes   [ceil(N/32)][K/128][5][32] uint32; 4-byte aligned.
  *   scales  [N] fp32.
  *   x       [M][K] int8 row-major; 16-byte aligned (tensor-memory-access copies).
  *   y       [M][N] fp32 output, row-major.

@@ -16,8 +16,12 @@ def dev(a):
 
 
 def rows_subset(codes_np, rows):
-    """Codes of a subset of output rows (planar layout [5][N][T])."""
-    return np.ascontiguousarray(codes_np[:, rows, :])
+    """Codes of a subset of output rows, re-grouped ([ceil(n/32)][T][5][32] layout)."""
+    rows = np.asarray(rows)
+    out = np.zeros(((len(rows) + 31) // 32, codes_np.shape[1], 5, 32), np.uint32)
+    for j, r in enumerate(rows):
+        out[j // 32, :, :, j % 32] = codes_np[r // 32, :, :, r % 32]
+    return out
 
 
 def assert_y_matches(y_gpu, y_ref):

@@ -37,11 +37,14 @@ def test_status_strings_and_version():
 
 def test_packed_and_workspace_sizes():
     assert S.packed_bytes(256, 1024) == 256 * 1024 * 5 // 32
+    assert S.packed_bytes(1, 1024) == 32 * 1024 * 5 // 32      # rows padded to a 32-row group
+    assert S.codes_shape(33, 2048) == (2, 16, 5, 32)
     assert S.packed_bytes(3, 100) == 0
     assert S.packed_bytes(0, 128) == 0
-    assert S.gemv_workspace_bytes(2048, 1) == 2048
-    assert S.gemv_workspace_bytes(384, 3) == 1280       # 1152 rounded up to 256
-    assert S.gemv_workspace_bytes(128, 0) == 0
+    # re-ordered activations (B rows of K padded to 512) + partial sums and counters
+    assert S.gemv_workspace_bytes(2048, 2048, 1) == 2048 + 4 * (2048 + 64)
+    assert S.gemv_workspace_bytes(100, 384, 3) == 3 * 512 + 256 * ((4 * (300 + 4) + 255) // 256)
+    assert S.gemv_workspace_bytes(16, 128, 0) == 0
 
 
 def test_pack_argument_checks():
@@ -68,6 +71,8 @@ def test_gemv_argument_checks():
     assert L.sherry_gemv(FAKE, FAKE, FAKE, FAKE, 4, 128, 1, ctypes.c_void_p(0x200010), ws,
                          None) == 3
     assert L.sherry_gemv(FAKE, FAKE, FAKE, FAKE, 4, 1024, 2, FAKE_WS, 1024, None) == 7
+    assert L.sherry_gemv(FAKE, FAKE, FAKE, FAKE, 4, 1024, 2, FAKE_WS,
+                         S.gemv_workspace_bytes(4, 1024, 2) - 4, None) == 7
     assert L.sherry_gemv_acc(FAKE, FAKE, None, 4, 128, 1, FAKE_WS, ws, None) == 1
 
 

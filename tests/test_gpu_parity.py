@@ -49,7 +49,7 @@ def test_pack_golden_tiles(golden_dir):
     assert np.array_equal(host_codes(codes), codes_ref)
     assert np.array_equal(scales.cpu().numpy(), scales_ref)
     for n, t in enumerate(tiles):
-        assert [int(host_codes(codes)[p, n, 0]) for p in range(5)] == t["words"]
+        assert [int(host_codes(codes)[0, 0, p, n]) for p in range(5)] == t["words"]
 
 
 @pytest.mark.parametrize("layer", range(7))
@@ -66,7 +66,8 @@ def test_pack_full_size_1b_layers(layer):
 # ----------------------------------------------------------------------------- gemv
 GEMV_CASES = [(256, 1024, 1), (1, 128, 1), (17, 384, 3), (33, 640, 5), (40, 1152, 8),
               (19, 256, 9), (64, 512, 16), (2048, 2048, 1), (512, 2048, 4), (100, 3072, 2),
-              (31, 8192, 1), (48, 8192, 16)]
+              (31, 8192, 1), (48, 8192, 16), (50, 1536, 2), (23, 512, 1), (70, 2560, 9),
+              (129, 4096, 8)]
 
 
 @pytest.mark.parametrize("N,K,B", GEMV_CASES)
@@ -75,8 +76,8 @@ def test_gemv_matches_oracle(N, K, B):
     codes, scales = oracle.pack(w)
     x = synth.int8_uniform((B, K), seed=1)
     tc, ts, tx = dev_codes(codes), dev(scales), dev(x)
-    acc = S.gemv_acc(tc, tx)
-    assert np.array_equal(acc.cpu().numpy().astype(np.int64), oracle.gemv_acc(codes, x, K))
+    acc = S.gemv_acc(tc, tx, N)
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), oracle.gemv_acc(codes, x, N, K))
     y = S.gemv(tc, ts, tx)
     assert_y_matches(y.cpu().numpy(), oracle.gemv(codes, scales, x, K))
 
@@ -85,10 +86,24 @@ def test_gemv_matches_oracle(N, K, B):
 def test_gemv_random_words_full_int8_range(N, K, B):
     # every 32-bit pattern is a valid code; activations cover [-128, 127]
     rng = np.random.default_rng(N + K + B)
-    codes = rng.integers(0, 2 ** 32, size=(5, N, K // 128), dtype=np.uint64).astype(np.uint32)
+    codes = rng.integers(0, 2 ** 32, size=((N + 31) // 32, K // 128, 5, 32),
+                         dtype=np.uint64).astype(np.uint32)
     x = rng.integers(-128, 128, size=(B, K)).astype(np.int8)
-    acc = S.gemv_acc(dev_codes(codes), dev(x))
-    assert np.array_equal(acc.cpu().numpy().astype(np.int64), oracle.gemv_acc(codes, x, K))
+    acc = S.gemv_acc(dev_codes(codes), dev(x), N)
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), oracle.gemv_acc(codes, x, N, K))
+
+
+def test_gemv_unaligned_codes_take_the_register_path():
+    # codes only 4-byte aligned: the cp.async path needs 16; results must not change
+    N, K, B = 40, 2048, 3
+    codes, scales = oracle.pack(synth.latent_weights(N, K, seed=8))
+    x = synth.int8_uniform((B, K), seed=9)
+    flat = torch.zeros(codes.size + 1, dtype=torch.int32, device="cuda")
+    flat[1:].copy_(dev_codes(codes).view(-1))
+    shifted = flat[1:].view(codes.shape)
+    assert shifted.data_ptr() % 16 == 4
+    acc = S.gemv_acc(shifted, dev(x), N)
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), oracle.gemv_acc(codes, x, N, K))
 
 
 def test_gemv_extreme_and_zero_activations():
@@ -134,7 +149,7 @@ def test_gemv_on_gpu_packed_codes():
     x = synth.int8_uniform((1, K), seed=1)
     y = S.gemv(codes, scales, dev(x)).cpu().numpy()
     c_ref, s_ref = oracle.pack(w)
-    acc_ref = oracle.gemv_acc(c_ref, x, K)
+    acc_ref = oracle.gemv_acc(c_ref, x, N, K)
     y_ref = scales.cpu().numpy().astype(np.float64)[None, :] * acc_ref
     assert_y_matches(y, y_ref)
 
@@ -149,8 +164,8 @@ def test_gemm_matches_oracle(M, N, K):
     codes, scales = oracle.pack(synth.latent_weights(N, K, seed=0))
     x = synth.int8_clipped_normal((M, K), seed=1)
     tc, ts, tx = dev_codes(codes), dev(scales), dev(x)
-    acc = S.gemm_acc(tc, tx)
-    assert np.array_equal(acc.cpu().numpy().astype(np.int64), oracle.gemm_acc(codes, x, K))
+    acc = S.gemm_acc(tc, tx, N)
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), oracle.gemm_acc(codes, x, N, K))
     y = S.gemm(tc, ts, tx)
     assert_y_matches(y.cpu().numpy(), oracle.gemm(codes, scales, x, K))
 
@@ -158,10 +173,11 @@ def test_gemm_matches_oracle(M, N, K):
 def test_gemm_random_words_full_int8_range():
     rng = np.random.default_rng(11)
     M, N, K = 200, 160, 768
-    codes = rng.integers(0, 2 ** 32, size=(5, N, K // 128), dtype=np.uint64).astype(np.uint32)
+    codes = rng.integers(0, 2 ** 32, size=((N + 31) // 32, K // 128, 5, 32),
+                         dtype=np.uint64).astype(np.uint32)
     x = rng.integers(-128, 128, size=(M, K)).astype(np.int8)
-    acc = S.gemm_acc(dev_codes(codes), dev(x))
-    assert np.array_equal(acc.cpu().numpy().astype(np.int64), oracle.gemm_acc(codes, x, K))
+    acc = S.gemm_acc(dev_codes(codes), dev(x), N)
+    assert np.array_equal(acc.cpu().numpy().astype(np.int64), oracle.gemm_acc(codes, x, N, K))
 
 
 @pytest.mark.parametrize("case", synth.PREFILL_GEMMS, ids=lambda c: c[0])
@@ -182,3 +198,42 @@ def test_gemm_m1_equals_gemv():
     x = synth.int8_uniform((1, K), seed=6)
     tc, ts, tx = dev_codes(codes), dev(scales), dev(x)
     assert torch.equal(S.gemm(tc, ts, tx), S.gemv(tc, ts, tx))
+
+
+def test_gemv_prepare_then_run_equals_grouped():
+    items, refs = [], []
+    for li, (N, K) in enumerate([(64, 2048), (48, 8192), (100, 384)]):
+        codes, scales = oracle.pack(synth.latent_weights(N, K, seed=40 + li))
+        x = synth.int8_uniform((3, K), seed=50 + li)
+        y = torch.zeros((3, N), dtype=torch.float32, device="cuda")
+        items.append((dev_codes(codes), dev(scales), dev(x), y))
+        refs.append(oracle.gemv(codes, scales, x, K))
+    g = S.GroupedGemv(items, B=3)
+    g.prepare()
+    g.run()
+    for (_, _, _, y), ref in zip(items, refs):
+        assert_y_matches(y.cpu().numpy(), ref)
+    for it in items:
+        it[3].zero_()
+    g()
+    for (_, _, _, y), ref in zip(items, refs):
+        assert_y_matches(y.cpu().numpy(), ref)
+
+
+def test_gemv_run_repeats_after_one_prepare():
+    # K-parts meet in the workspace; every run must leave it ready for the next
+    items, refs = [], []
+    for li, (N, K) in enumerate([(96, 8192), (70, 3072), (33, 2048)]):
+        codes, scales = oracle.pack(synth.latent_weights(N, K, seed=60 + li))
+        x = synth.int8_uniform((2, K), seed=70 + li)
+        y = torch.zeros((2, N), dtype=torch.float32, device="cuda")
+        items.append((dev_codes(codes), dev(scales), dev(x), y))
+        refs.append(oracle.gemv(codes, scales, x, K))
+    g = S.GroupedGemv(items, B=2)
+    g.prepare()
+    for _ in range(3):
+        for it in items:
+            it[3].zero_()
+        g.run()
+        for (_, _, _, y), ref in zip(items, refs):
+            assert_y_matches(y.cpu().numpy(), ref)
