@@ -59,8 +59,13 @@ struct GemvParams {
     int total_units16;    // register kernel
     int total_items;      // pipelined kernel
     int total_chunks;     // pipelined kernel: balancing space
-    uint32_t mul4, mul2;  // 4 and 2, passed at run time (see imul)
-    int pad;
+    // Constants passed at run time so that they live in registers instead of
+    // being re-created per use, and so that shifts by a power of two stay
+    // multiplications (IMAD / IMAD.HI on the FMA pipe) instead of ALU shifts.
+    uint32_t mul4, mul2;          // 4, 2
+    uint32_t hi1, hi2, hi16;      // 2^31, 2^30, 2^16: mul.hi gives >> 1, >> 2, >> 16
+    uint32_t m33, m55, m44;       // masks
+    uint32_t tlo[4], thi[4];      // PRMT byte tables of the four positions
     GemvDesc d[SHERRY_MAX_GROUP];
 };
 
@@ -204,26 +209,35 @@ __device__ __forceinline__ uint32_t imul(uint32_t a, uint32_t b) {
     return d;
 }
 
+__device__ __forceinline__ uint32_t imulhi(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("mul.hi.u32 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
 struct Consts {
-    uint32_t mul4, mul2;
+    uint32_t mul4, mul2, hi1, hi2, hi16, m33, m55, m44;
+    uint32_t tlo[4], thi[4];
 };
 
 // Per-row tile state of the pipelined kernel: zero-position nibbles per block
 // group and the four per-position sign planes.  Selector of (i, beta):
 //   zm[beta] | (sign plane i moved so block 4k+beta's bit lands at 4k+2) & 0x44444444.
+// Work split: masks, merges and permutes on the ALU pipe (2 cycles per warp
+// instruction); every shift on the FMA pipe as IMAD (left) or IMAD.HI (right).
 struct TileDecoder6 {
     uint32_t zm[4];
     uint32_t sg[4];
 
     __device__ __forceinline__ void load(const Consts &C, uint32_t z0, uint32_t z1, uint32_t s0,
                                          uint32_t s1, uint32_t s2) {
-        zm[0] = z0 & 0x33333333u;
-        zm[1] = z1 & 0x33333333u;
-        zm[2] = (z0 >> 2) & 0x33333333u;
-        zm[3] = (z1 >> 2) & 0x33333333u;
+        zm[0] = z0 & C.m33;
+        zm[1] = z1 & C.m33;
+        zm[2] = imulhi(z0, C.hi2) & C.m33;
+        zm[3] = imulhi(z1, C.hi2) & C.m33;
         // bit-sliced zero positions: lo bit (L) and hi bit (H) of p_j at bit j
-        const uint32_t L = lop_merge(z0, imul(z1, C.mul2), 0x55555555u);
-        const uint32_t H = lop_merge(z0 >> 1, z1, 0x55555555u);
+        const uint32_t L = lop_merge(z0, imul(z1, C.mul2), C.m55);
+        const uint32_t H = lop_merge(imulhi(z0, C.hi1), z1, C.m55);
         // sign of position i when kept: rank 0; rank 0 if p == 0 else 1;
         // rank 1 if p <= 1 else 2; rank 2
         sg[0] = s0;
@@ -234,8 +248,8 @@ struct TileDecoder6 {
     __device__ __forceinline__ uint32_t sel(const Consts &C, int i, int beta) const {
         const uint32_t v = beta == 0 ? imul(sg[i], C.mul4)
                          : beta == 1 ? imul(sg[i], C.mul2)
-                         : beta == 2 ? sg[i] : (sg[i] >> 1);
-        return lop_or_masked(v, 0x44444444u, zm[beta]);
+                         : beta == 2 ? sg[i] : imulhi(sg[i], C.hi1);
+        return lop_or_masked(v, C.m44, zm[beta]);
     }
 };
 
@@ -399,8 +413,11 @@ __device__ __forceinline__ int first_item_at_or_after(const GemvParams &P, int c
                      : (lo + 1 < P.count ? P.d[lo + 1].item_begin : P.total_items);
 }
 
+#ifndef SHERRY_PIPE_MIN_BLOCKS
+#define SHERRY_PIPE_MIN_BLOCKS 2
+#endif
 template <int NB, bool ACC_OUT>
-__global__ void __launch_bounds__(kPipeThreads, 3)
+__global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
     gemv_pipe_kernel(const __grid_constant__ GemvParams P) {
     extern __shared__ __align__(16) uint32_t pipe_smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -411,7 +428,20 @@ __global__ void __launch_bounds__(kPipeThreads, 3)
     const int it_end = first_item_at_or_after(P, (int)((wg + 1) * P.total_chunks / nw));
     if (it_begin >= it_end) return;
     uint32_t *ring = pipe_smem + (size_t)warp * kRing * kStageWords;
-    const Consts C{P.mul4, P.mul2};
+    Consts C;
+    C.mul4 = P.mul4;
+    C.mul2 = P.mul2;
+    C.hi1 = P.hi1;
+    C.hi2 = P.hi2;
+    C.hi16 = P.hi16;
+    C.m33 = P.m33;
+    C.m55 = P.m55;
+    C.m44 = P.m44;
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        C.tlo[i] = P.tlo[i];
+        C.thi[i] = P.thi[i];
+    }
 
     // ---- producer side: the issue cursor runs kRing-1 stages ahead ----
     // lane l copies 16-byte pieces l + 32 j (j = 0..4) of the 2560-byte chunk;
@@ -476,36 +506,38 @@ __global__ void __launch_bounds__(kPipeThreads, 3)
             __syncwarp();
             // tile t of the chunk, plane p, row g + 8 r: word t * 168 + 32 p + g + 8 r
             const uint32_t *st = ring + slot * kStageWords + t * kTileWordsPadded + g;
-            TileDecoder6 dec[4];  // rows g, g+8, g+16, g+24
-#pragma unroll
-            for (int r = 0; r < 4; r++)
-                dec[r].load(C, st[0 * 32 + r * 8], st[1 * 32 + r * 8], st[2 * 32 + r * 8],
-                            st[3 * 32 + r * 8], st[4 * 32 + r * 8]);
-            __syncwarp();  // every lane has its words: the stage can be refilled
-            issue(slot == 0 ? kRing - 1 : slot - 1);
-            slot = (slot + 1 == kRing) ? 0 : slot + 1;
             // padded tiles hold zero activations, so no load is predicated
             const size_t xoff = (size_t)c * kChunkTiles * 8;
 #pragma unroll
-            for (int i = 0; i < 4; i++) {
-                uint4 xq[NB][2];
-#pragma unroll
-                for (int nb = 0; nb < NB; nb++) {
-                    xq[nb][0] = ld_x(xrow[nb] + xoff + 2 * i);
-                    xq[nb][1] = ld_x(xrow[nb] + xoff + 2 * i + 1);
+            for (int rb = 0; rb < 2; rb++) {  // row block rb: rows g + 16 rb, g + 8 + 16 rb
+                TileDecoder6 d0, d1;
+                d0.load(C, st[0 * 32 + 16 * rb], st[1 * 32 + 16 * rb], st[2 * 32 + 16 * rb],
+                        st[3 * 32 + 16 * rb], st[4 * 32 + 16 * rb]);
+                d1.load(C, st[0 * 32 + 16 * rb + 8], st[1 * 32 + 16 * rb + 8],
+                        st[2 * 32 + 16 * rb + 8], st[3 * 32 + 16 * rb + 8], st[4 * 32 + 16 * rb + 8]);
+                if (rb == 1) {
+                    __syncwarp();  // every lane has its words: the stage can be refilled
+                    issue(slot == 0 ? kRing - 1 : slot - 1);
+                    slot = (slot + 1 == kRing) ? 0 : slot + 1;
                 }
-                const uint32_t tlo = table_lo(i), thi = table_hi(i);
 #pragma unroll
-                for (int beta = 0; beta < 4; beta++) {
-                    const int m = 4 * i + beta;  // MMA index: activation words 2m, 2m+1
+                for (int i = 0; i < 4; i++) {
+                    uint4 xq[NB][2];
 #pragma unroll
-                    for (int rb = 0; rb < 2; rb++) {
-                        const uint32_t s0 = dec[2 * rb].sel(C, i, beta);
-                        const uint32_t s1 = dec[2 * rb + 1].sel(C, i, beta);
+                    for (int nb = 0; nb < NB; nb++) {
+                        xq[nb][0] = ld_x(xrow[nb] + xoff + 2 * i);
+                        xq[nb][1] = ld_x(xrow[nb] + xoff + 2 * i + 1);
+                    }
+                    const uint32_t tlo = C.tlo[i], thi = C.thi[i];
+#pragma unroll
+                    for (int beta = 0; beta < 4; beta++) {
+                        const int m = 4 * i + beta;  // MMA index: activation words 2m, 2m+1
+                        const uint32_t s0 = d0.sel(C, i, beta);
+                        const uint32_t s1 = d1.sel(C, i, beta);
                         const uint32_t a0 = prmt(tlo, thi, s0);
-                        const uint32_t a2 = prmt(tlo, thi, s0 >> 16);
+                        const uint32_t a2 = prmt(tlo, thi, imulhi(s0, C.hi16));
                         const uint32_t a1 = prmt(tlo, thi, s1);
-                        const uint32_t a3 = prmt(tlo, thi, s1 >> 16);
+                        const uint32_t a3 = prmt(tlo, thi, imulhi(s1, C.hi16));
 #pragma unroll
                         for (int nb = 0; nb < NB; nb++) {
                             const uint4 &xx = xq[nb][(m >> 1) & 1];
@@ -668,6 +700,20 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
     xp.B = gp.B = B;
     gp.mul4 = 4u;
     gp.mul2 = 2u;
+    gp.hi1 = 0x80000000u;
+    gp.hi2 = 0x40000000u;
+    gp.hi16 = 0x10000u;
+    gp.m33 = 0x33333333u;
+    gp.m55 = 0x55555555u;
+    gp.m44 = 0x44444444u;
+    {
+        const uint32_t lo[4] = {0x01010100u, 0x01010001u, 0x01000101u, 0x00010101u};
+        const uint32_t hi[4] = {0xFFFFFF00u, 0xFFFF00FFu, 0xFF00FFFFu, 0x00FFFFFFu};
+        for (int i = 0; i < 4; i++) {
+            gp.tlo[i] = lo[i];
+            gp.thi[i] = hi[i];
+        }
+    }
     int64_t off = 0;
     int wb = 0, ub16 = 0, ib = 0, cb = 0;
     for (int i = 0; i < count; i++) {
