@@ -76,7 +76,7 @@ struct XprepDesc {
     int Tp;
     int word_begin;       // first thread index of this GEMV
     int xw_words;         // B * Tp * 32 re-ordered words, then zero_words zeros
-    int zero_words;       // partial sums and counters to clear
+    int zero_words;       // split-K partial sums and counters to clear (0 if unsplit)
     int pad;
 };
 
@@ -112,11 +112,22 @@ int64_t padded_tiles(int64_t K) {
 }
 int64_t round_words(int64_t w) { return (w + 63) / 64 * 64; }  // 256-byte regions
 
-// Workspace words of one GEMV: re-ordered activations, then (for the pipelined
-// kernel) the K-part partial sums and the per-unit counters.
+// K-parts per 32-row unit in the pipelined kernel.
+int64_t kparts_for(int64_t K) {
+    const int64_t nchunk = padded_tiles(K) / kChunkTiles;
+    return (nchunk + kMaxPartChunks - 1) / kMaxPartChunks;
+}
+
+// Split-K words of one GEMV: partial sums [B][N] and per-unit counters, only
+// when the rows are split into several K-parts.
+int64_t split_words(int64_t N, int64_t K, int B) {
+    if (kparts_for(K) <= 1) return 0;
+    return round_words((int64_t)B * N + (N + kUnitRows - 1) / kUnitRows);
+}
+
+// Workspace words of one GEMV: re-ordered activations, then the split-K words.
 int64_t ws_words(int64_t N, int64_t K, int B) {
-    const int64_t units = (N + kUnitRows - 1) / kUnitRows;
-    return round_words((int64_t)B * padded_tiles(K) * 32) + round_words((int64_t)B * N + units);
+    return round_words((int64_t)B * padded_tiles(K) * 32) + split_words(N, K, B);
 }
 
 // ---------------------------------------------------------------------------
@@ -677,7 +688,7 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
         words += ws_words(c.N, c.K, B);
         units16 += (c.N + 15) / 16;
         const int64_t nchunk = padded_tiles(c.K) / kChunkTiles;
-        const int64_t kparts = (nchunk + kMaxPartChunks - 1) / kMaxPartChunks;
+        const int64_t kparts = kparts_for(c.K);
         items += (c.N + kUnitRows - 1) / kUnitRows * kparts;
         chunks += (c.N + kUnitRows - 1) / kUnitRows * kparts * ((nchunk + kparts - 1) / kparts);
     }
@@ -723,7 +734,7 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
         const int xw_words = (int)round_words((int64_t)B * Tp * 32);
         const int units = (int)((c.N + kUnitRows - 1) / kUnitRows);
         const int nchunk = Tp / kChunkTiles;
-        const int kparts = (nchunk + kMaxPartChunks - 1) / kMaxPartChunks;
+        const int kparts = (int)kparts_for(c.K);
         const int cpp = (nchunk + kparts - 1) / kparts;
         XprepDesc &X = xp.d[i];
         X.x = c.x;
@@ -732,14 +743,14 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
         X.Tp = Tp;
         X.word_begin = wb;
         X.xw_words = xw_words;
-        X.zero_words = (int)round_words((int64_t)B * c.N + units);
+        X.zero_words = (int)split_words(c.N, c.K, B);
         GemvDesc &D = gp.d[i];
         D.codes = c.codes;
         D.scales = c.scales;
         D.xw = reinterpret_cast<const uint4 *>(region);
         D.out = c.out;
-        D.part_acc = reinterpret_cast<int32_t *>(region + xw_words);
-        D.part_cnt = region + xw_words + (int64_t)B * c.N;
+        D.part_acc = kparts > 1 ? reinterpret_cast<int32_t *>(region + xw_words) : nullptr;
+        D.part_cnt = kparts > 1 ? region + xw_words + (int64_t)B * c.N : nullptr;
         D.N = (int)c.N;
         D.T = (int)(c.K / SHERRY_TILE_K);
         D.Tp = Tp;

@@ -42,8 +42,12 @@ def test_packed_and_workspace_sizes():
     assert S.packed_bytes(3, 100) == 0
     assert S.packed_bytes(0, 128) == 0
     # re-ordered activations (B rows of K padded to 512) + partial sums and counters
-    assert S.gemv_workspace_bytes(2048, 2048, 1) == 2048 + 4 * (2048 + 64)
-    assert S.gemv_workspace_bytes(100, 384, 3) == 3 * 512 + 256 * ((4 * (300 + 4) + 255) // 256)
+    # re-ordered activations only: 4 chunks per row need no split-K region
+    assert S.gemv_workspace_bytes(2048, 2048, 1) == 2048
+    assert S.gemv_workspace_bytes(100, 384, 3) == 3 * 512
+    # 16 chunks per row -> 4 K-parts: partial sums [B][N] and 64 unit counters
+    assert S.gemv_workspace_bytes(2048, 8192, 1) == 4 * 64 * 32 + 4 * (2048 + 64)
+    assert S.gemv_workspace_bytes(100, 8192, 3) == 3 * 4 * 64 * 32 + 256 * ((4 * (300 + 4) + 255) // 256)
     assert S.gemv_workspace_bytes(16, 128, 0) == 0
 
 
