@@ -5,5 +5,6 @@ The compute path lives in ``libsherry.so`` (``csrc/``, header ``include/sherry.h
 """
 from .sherry import (  # noqa: F401
     GroupedGemv, SherryError, codes_shape, device_error, gemm, gemm_acc, gemv, gemv_acc, gemv_grouped,
+    gemv_static,
     gemv_workspace_bytes, lib, library_path, pack, packed_bytes, workspace,
 )

@@ -16,6 +16,10 @@ void set_last_error(const char *what, cudaError_t err) {
                   cudaGetErrorString(err));
 }
 
+void set_last_error_text(const char *text) {
+    std::snprintf(g_last_error, sizeof(g_last_error), "%s", text);
+}
+
 sherry_status launch_status(const char *what) {
     const cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) {

@@ -17,6 +17,7 @@ namespace sherry {
 // Host-side helpers
 // ---------------------------------------------------------------------------
 void set_last_error(const char *what, cudaError_t err);
+void set_last_error_text(const char *text);
 sherry_status launch_status(const char *what);
 
 inline bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }

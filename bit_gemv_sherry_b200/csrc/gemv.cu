@@ -24,7 +24,9 @@
 // filled by cp.async and splits long rows into K-parts that are summed exactly
 // with integer atomics; the register kernel is the general fallback.
 #include <algorithm>
+#include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include "common.cuh"
 
@@ -849,4 +851,69 @@ extern "C" sherry_status sherry_gemv_run(const sherry_gemv_desc *descs, int coun
                                          sherry_stream_t stream) {
     return sherry::grouped(descs, count, B, const_cast<void *>(workspace), workspace_bytes,
                            reinterpret_cast<cudaStream_t>(stream), sherry::kRun);
+}
+
+// ---------------------------------------------------------------------------
+// sherry_gemv_static: the GEMV above with its scratch in a fixed device array.
+// ---------------------------------------------------------------------------
+namespace sherry {
+namespace {
+
+static __device__ __align__(256) uint32_t g_gemv_static_scratch[SHERRY_STATIC_SCRATCH_BYTES / 4];
+
+constexpr int kStaticMaxDevices = 64;
+std::mutex g_static_mu;
+void *g_static_ptr[kStaticMaxDevices] = {};
+
+// Device address of the scratch array on the current device, looked up once
+// per device.
+sherry_status static_scratch(void **out) {
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) {
+        set_last_error("sherry_gemv_static (cudaGetDevice)", err);
+        return SHERRY_ERR_CUDA;
+    }
+    if (dev < 0 || dev >= kStaticMaxDevices) return SHERRY_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (g_static_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        err = cudaGetSymbolAddress(&p, g_gemv_static_scratch);
+        if (err != cudaSuccess || p == nullptr) {
+            set_last_error("sherry_gemv_static (cudaGetSymbolAddress)",
+                           err != cudaSuccess ? err : cudaErrorInvalidSymbol);
+            return SHERRY_ERR_CUDA;
+        }
+        g_static_ptr[dev] = p;
+    }
+    *out = g_static_ptr[dev];
+    return SHERRY_OK;
+}
+
+}  // namespace
+}  // namespace sherry
+
+extern "C" sherry_status sherry_gemv_static(const uint32_t *codes, const float *scales,
+                                            const int8_t *x, float *y, int64_t N, int64_t K, int B,
+                                            sherry_stream_t stream) {
+    using namespace sherry;
+    if (!codes || !scales || !x || !y) return SHERRY_ERR_NULL;
+    if (N < 1 || !valid_k(K) || B < 1) return SHERRY_ERR_SHAPE;
+    if (B > SHERRY_MAX_GEMV_BATCH || N > (int64_t)1 << 28) return SHERRY_ERR_UNSUPPORTED;
+    const size_t need = (size_t)ws_words(N, K, B) * 4;
+    if (need > (size_t)SHERRY_STATIC_SCRATCH_BYTES) {
+        char msg[200];
+        std::snprintf(msg, sizeof(msg),
+                      "sherry_gemv_static: N=%lld K=%lld B=%d needs %zu bytes of scratch; the "
+                      "static scratch holds %zu",
+                      (long long)N, (long long)K, B, need, (size_t)SHERRY_STATIC_SCRATCH_BYTES);
+        set_last_error_text(msg);
+        return SHERRY_ERR_WORKSPACE;
+    }
+    void *scratch = nullptr;
+    const sherry_status st = static_scratch(&scratch);
+    if (st != SHERRY_OK) return st;
+    const GemvCall c{codes, scales, x, y, N, K};
+    return gemv_launch(&c, 1, B, false, scratch, SHERRY_STATIC_SCRATCH_BYTES,
+                       reinterpret_cast<cudaStream_t>(stream), kBoth);
 }

@@ -61,6 +61,7 @@ def lib():
         "sherry_gemv_workspace_bytes": ([i64, i64, i32], sz),
         "sherry_gemv": ([p, p, p, p, i64, i64, i32, p, sz, p], i32),
         "sherry_gemv_acc": ([p, p, p, i64, i64, i32, p, sz, p], i32),
+        "sherry_gemv_static": ([p, p, p, p, i64, i64, i32, p], i32),
         "sherry_gemv_grouped": ([p, i32, i32, p, sz, p], i32),
         "sherry_gemv_prepare": ([p, i32, i32, p, sz, p], i32),
         "sherry_gemv_run": ([p, i32, i32, p, sz, p], i32),
@@ -167,6 +168,25 @@ def gemv(codes, scales, x, y=None, ws=None):
     ws = workspace(nb, x.device) if ws is None else ws
     _check(lib().sherry_gemv(_ptr(codes), _ptr(scales), _ptr(x2), _ptr(y), N, K, B, _ptr(ws),
                              ws.numel(), _stream(x)), "sherry_gemv")
+    return y
+
+
+STATIC_SCRATCH_BYTES = 4 << 20
+
+
+def gemv_static(codes, scales, x, y=None):
+    """As gemv, with the library's fixed scratch array instead of a workspace
+    (sherry_gemv_static: the C call allocates nothing; y is allocated here
+    only when not given)."""
+    _need(scales, torch.float32, "scales")
+    N, K = _codes_shape(codes, scales.numel())
+    _need(x, torch.int8, "x")
+    x2 = x.view(1, -1) if x.dim() == 1 else x
+    B = x2.shape[0]
+    if y is None:
+        y = torch.empty((B, N), dtype=torch.float32, device=x.device)
+    _check(lib().sherry_gemv_static(_ptr(codes), _ptr(scales), _ptr(x2), _ptr(y), N, K, B,
+                                    _stream(x)), "sherry_gemv_static")
     return y
 
 

@@ -86,6 +86,7 @@ typedef enum {
 #define SHERRY_MAX_K 131072       /* keeps |acc| < 2^24                   */
 #define SHERRY_MAX_GEMV_BATCH 16  /* activation rows per GEMV call        */
 #define SHERRY_MAX_GROUP 128      /* GEMVs per grouped call               */
+#define SHERRY_STATIC_SCRATCH_BYTES (4u << 20)  /* scratch of sherry_gemv_static */
 
 /* Bytes of packed codes for an N x K matrix: ceil(N/32)*32 * K * 5 / 32
  * (N * K * 5 / 32 when N is a multiple of 32; scales excluded).
@@ -142,6 +143,32 @@ sherry_status sherry_gemv(const uint32_t *codes, const float *scales, const int8
 sherry_status sherry_gemv_acc(const uint32_t *codes, const int8_t *x, int32_t *acc,
                               int64_t N, int64_t K, int B, void *workspace,
                               size_t workspace_bytes, sherry_stream_t stream);
+
+/*
+ * sherry_gemv_static -- sherry_gemv without a caller workspace: the call
+ * allocates nothing.  The paper has no counterpart; this entry point exists
+ * for callers that may not allocate device memory on their decode path.
+ * Its scratch (re-ordered activations, split-K partial sums and counters) is
+ * one device array of SHERRY_STATIC_SCRATCH_BYTES (4 MiB) per device, inside
+ * this library.
+ *   Arguments, layouts and the result are those of sherry_gemv.
+ *   Size limit: sherry_gemv_workspace_bytes(N, K, B) must not exceed
+ *   SHERRY_STATIC_SCRATCH_BYTES, otherwise the call returns
+ *   SHERRY_ERR_WORKSPACE with the two sizes in sherry_last_error().
+ *   Set-up: the first call on a device (with that device current) looks up
+ *   the array's device address (cudaGetSymbolAddress) once and caches it;
+ *   make that first call before any stream capture.
+ *   Sharing: every call on a device uses the same array.  Each call re-writes
+ *   the activations and zeroes the partial sums and counters it needs before
+ *   its GEMV kernel reads them, so consecutive calls are independent; calls
+ *   that overlap on the GPU (other streams, other host threads) race on the
+ *   array and give undefined results.
+ *   No cudaMalloc, cudaFree or other allocating routine is called.
+ * Errors: as sherry_gemv; WORKSPACE for sizes beyond the limit; CUDA if the
+ * set-up fails.
+ */
+sherry_status sherry_gemv_static(const uint32_t *codes, const float *scales, const int8_t *x,
+                                 float *y, int64_t N, int64_t K, int B, sherry_stream_t stream);
 
 /* One GEMV of a grouped call.  All pointers are device pointers with the
  * alignment sherry_gemv requires. */

@@ -80,6 +80,16 @@ def test_gemv_argument_checks():
     assert L.sherry_gemv_acc(FAKE, FAKE, None, 4, 128, 1, FAKE_WS, ws, None) == 1
 
 
+def test_gemv_static_argument_checks():
+    L = S.lib()
+    assert L.sherry_gemv_static(None, FAKE, FAKE, FAKE, 4, 128, 1, None) == 1
+    assert L.sherry_gemv_static(FAKE, FAKE, FAKE, FAKE, 4, 130, 1, None) == 2
+    assert L.sherry_gemv_static(FAKE, FAKE, FAKE, FAKE, 4, 128, 17, None) == 4
+    # beyond the 4 MiB static scratch: rejected on the host with both sizes in the message
+    assert L.sherry_gemv_static(FAKE, FAKE, FAKE, FAKE, 100000, 8192, 16, None) == 7
+    assert b"4194304" in L.sherry_last_error()
+
+
 def test_grouped_argument_checks():
     L = S.lib()
     d = (S.GemvDesc * 2)()
