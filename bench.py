@@ -37,6 +37,9 @@ import synth  # noqa: E402
 METRIC = "W1.25A8 GEMV weight GB/s at batch 1 (LLaMA-3.2-1B decode stack)"
 UNIT = "GB/s"
 L2_BYTES = 126 * 2 ** 20
+# ncu capture of gemv_pipe_kernel<1,false> on the 16-layer stack, B = 1:
+# dram read 154,059,008 + write 4,094,720 bytes per launch
+NCU_TRAFFIC_BYTES = 154059008 + 4094720
 
 
 def parse_args():
@@ -127,15 +130,31 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- reference arm
+def max_over_ranks(value, dist=None, device=None):
+    """MAX of a float over the ranks of the default process group (the value
+    itself on one process)."""
+    if dist is None or not dist.is_available() or not dist.is_initialized() or \
+            dist.get_world_size() == 1:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_value(world, bytes_per_step, steps, t_max):
+    """Whole-job GB/s: every rank streams its own replica of the step."""
+    return world * bytes_per_step * steps / t_max / 1e9
+
+
 def run_reference(args, rank):
     """Times the CPU oracle on a bounded sample of the same workload."""
     import oracle
     if rank != 0:
         return None
     spec = stack_spec(args.layers)
-    layer0 = [s for s in spec if s[0] == 0]
     data = []
-    for _, name, n, k, seed in layer0:
+    for _, name, n, k, seed in spec:
         codes, scales = oracle.pack(synth.latent_weights(n, k, seed=seed))
         data.append((codes, scales, k))
     xs = {2048: synth.int8_uniform((1, 2048), seed=1), 8192: synth.int8_uniform((1, 8192), seed=2)}
@@ -144,23 +163,29 @@ def run_reference(args, rank):
     def step():
         for codes, scales, k in data:
             oracle.gemv(codes, scales, xs[k], k)
-    for _ in range(max(0, min(args.warmup, 2))):
+    warmup = max(0, min(args.warmup, 1))
+    for _ in range(warmup):
         step()
-    steps = max(1, min(args.steps, 50))
+    # one step = the whole stack; the number of timed steps is bounded so that
+    # the run stays within about a minute of oracle time
     t0 = time.perf_counter()
-    for _ in range(steps):
+    step()
+    first = time.perf_counter() - t0
+    steps = max(1, min(args.steps, int(60.0 / max(first, 1e-3))))
+    t0 = time.perf_counter()
+    for _ in range(steps - 1):
         step()
-    dt = (time.perf_counter() - t0) / steps
+    dt = (time.perf_counter() - t0 + first) / steps
     value = sample_bytes / dt / 1e9
     cores = oracle.num_threads()
-    sample = "decoder layer 0 of the stack (7 GEMVs, %d weights, %d code bytes) per step" % (
-        sum(n * k for _, _, n, k, _ in layer0), sample_bytes)
+    sample = "the whole stack per step (%d GEMVs, %d weights, %d code bytes), %d steps" % (
+        len(spec), sum(n * k for _, _, n, k, _ in spec), sample_bytes, steps)
     return {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
-        "n_gpus": args.gpus, "steps": steps, "warmup": min(args.warmup, 2),
+        "n_gpus": args.gpus, "steps": steps, "warmup": warmup,
         "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-        "config": {"workload": "llama-3.2-1b decode stack sample (CPU oracle)", "batch": 1},
+        "config": {"workload": "llama-3.2-1b decode stack, batch 1 (CPU oracle)", "batch": 1},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -273,24 +298,26 @@ def time_layers(layers, xs, S, torch, dev, flush, reps=20):
 def cpu_baseline(layers, xs_host, seconds):
     """The oracle, as it stands, on a bounded sample of the stack (host cores)."""
     import oracle
-    t_start = time.perf_counter()
-    done_bytes, done_w, n_gemv = 0, 0, 0
+    host = [(n, k, codes.cpu().numpy().view(np.uint32), scales.cpu().numpy())
+            for _, _, n, k, codes, scales in layers]
+    done_bytes, done_w, n_gemv, passes = 0, 0, 0, 0
     t_compute = 0.0
-    for layer, name, n, k, codes, scales in layers:
-        c = codes.cpu().numpy().view(np.uint32)
-        s = scales.cpu().numpy()
-        t0 = time.perf_counter()
-        oracle.gemv(c, s, xs_host[k], k)
-        t_compute += time.perf_counter() - t0
-        done_bytes += c.nbytes
-        done_w += n * k
-        n_gemv += 1
-        if time.perf_counter() - t_start > seconds:
-            break
+    while t_compute < seconds:
+        for n, k, c, s in host:
+            t0 = time.perf_counter()
+            oracle.gemv(c, s, xs_host[k], k)
+            t_compute += time.perf_counter() - t0
+            done_bytes += c.nbytes
+            done_w += n * k
+            n_gemv += 1
+            if t_compute >= seconds:
+                break
+        passes += 1
     return {"value": done_bytes / t_compute / 1e9, "unit": UNIT, "cores": oracle.num_threads(),
-            "kind": "oracle",
-            "sample": "first %d GEMVs of the stack in order (%d weights, %d code bytes), each "
-                      "timed once" % (n_gemv, done_w, done_bytes)}
+            "kind": "oracle", "seconds": t_compute,
+            "sample": "%d GEMVs of the stack in stack order (%d passes started; %d weights, %d "
+                      "code bytes), %.1f s of oracle time" % (n_gemv, passes, done_w, done_bytes,
+                                                              t_compute)}
 
 
 def main():
@@ -324,8 +351,16 @@ def main():
     extras = (rank == 0) and not args.no_extras
     layers, latents = build_stack(spec, dev, S, torch, keep_latents=extras)
     xs_host = {2048: synth.int8_uniform((1, 2048), seed=1), 8192: synth.int8_uniform((1, 8192), seed=2)}
-    xs = {k: torch.from_numpy(v).to(dev) for k, v in xs_host.items()}
-    ys = [torch.empty((1, n), dtype=torch.float32, device=dev) for _, _, n, _, _, _ in layers]
+    # one device buffer for the activations and one for all outputs, so that the
+    # end-to-end step moves each with a single copy
+    x_all = torch.from_numpy(np.concatenate([xs_host[2048], xs_host[8192]], axis=1)).to(dev)
+    xs = {2048: x_all[:, :2048], 8192: x_all[:, 2048:]}
+    n_out = sum(n for _, _, n, _, _, _ in layers)
+    y_all = torch.empty((n_out,), dtype=torch.float32, device=dev)
+    ys, o = [], 0
+    for _, _, n, _, _, _ in layers:
+        ys.append(y_all[o:o + n].view(1, n))
+        o += n
     items = [(codes, scales, xs[k], y) for (_, _, n, k, codes, scales), y in zip(layers, ys)]
     step = S.GroupedGemv(items, B=1)
     stream = torch.cuda.current_stream(dev)
@@ -372,27 +407,21 @@ def main():
     clocks.stop()
     clk = clocks.summary(t_host0, t_host1)
 
-    t_max = total_s
-    if world > 1:
-        tt = torch.tensor([total_s], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_max = float(tt.item())
+    t_max = max_over_ranks(total_s, dist if world > 1 else None, dev)
     ms_per_step = t_max / K * 1e3
-    value = world * codes_bytes * K / t_max / 1e9
+    value = whole_job_value(world, codes_bytes, K, t_max)
 
     # ---------------- end to end through the public API with pinned host buffers
-    x_pinned = {k: torch.from_numpy(v).pin_memory() for k, v in xs_host.items()}
-    y_pinned = [torch.empty((1, n), dtype=torch.float32).pin_memory() for _, _, n, _, _, _ in layers]
-    h2d = sum(v.numel() for v in x_pinned.values())
-    d2h = sum(4 * y.numel() for y in y_pinned)
+    x_pinned = x_all.cpu().pin_memory()
+    y_pinned = torch.empty_like(y_all, device="cpu").pin_memory()
+    h2d = x_pinned.numel()
+    d2h = 4 * y_pinned.numel()
     K_e2e = max(3, min(K, 2000))
 
     def e2e_step():
-        for k, v in x_pinned.items():
-            xs[k].copy_(v, non_blocking=True)
+        x_all.copy_(x_pinned, non_blocking=True)
         step(sptr)
-        for yp, yd in zip(y_pinned, ys):
-            yp.copy_(yd, non_blocking=True)
+        y_pinned.copy_(y_all, non_blocking=True)
     for _ in range(3):
         e2e_step()
     torch.cuda.synchronize(dev)
@@ -404,13 +433,10 @@ def main():
         e2e_step()
     e1.record(stream)
     e1.synchronize()
-    e2e_s = e0.elapsed_time(e1) / 1e3
+    e2e_s = max_over_ranks(e0.elapsed_time(e1) / 1e3, dist if world > 1 else None, dev)
     if world > 1:
-        tt = torch.tensor([e2e_s], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_s = float(tt.item())
         dist.barrier()
-    e2e_value = world * codes_bytes * K_e2e / e2e_s / 1e9
+    e2e_value = whole_job_value(world, codes_bytes, K_e2e, e2e_s)
 
     peaks = {}
     try:
@@ -423,6 +449,9 @@ def main():
     if hbm_peak is None:
         hbm_peak, peak_src = 6650.0, "fallback"
     achieved = alg_bytes / gemv_s / 1e9
+    # dram__bytes_read.sum + dram__bytes_write.sum of one gemv_pipe_kernel launch
+    # on this workload (ncu --set full); valid only for that kernel version
+    ncu_traffic = NCU_TRAFFIC_BYTES if args.layers == 16 else None
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
@@ -445,7 +474,8 @@ def main():
                      "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "peak_source": peak_src,
                      "bytes_per_launch": alg_bytes, "kernel_us": gemv_s * 1e6,
-                     "prepare_us": prep_s * 1e6, "traffic": None},
+                     "prepare_us": prep_s * 1e6, "traffic": ncu_traffic,
+                     "traffic_unit": "bytes per launch"},
         "gpu_busy_frac": busy_s / total_s if total_s > 0 else None,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": K_e2e, "ms_per_step": e2e_s / K_e2e * 1e3},
