@@ -37,9 +37,9 @@ import synth  # noqa: E402
 METRIC = "W1.25A8 GEMV weight GB/s at batch 1 (LLaMA-3.2-1B decode stack)"
 UNIT = "GB/s"
 L2_BYTES = 126 * 2 ** 20
-# ncu capture of gemv_pipe_kernel<1,false> on the 16-layer stack, B = 1:
-# dram read 154,059,008 + write 4,094,720 bytes per launch
-NCU_TRAFFIC_BYTES = 154059008 + 4094720
+# ncu capture of gemv_dot_kernel<1,false> on the 16-layer stack, B = 1:
+# dram read 154,064,896 + write 4,563,712 bytes per launch
+NCU_TRAFFIC_BYTES = 154064896 + 4563712
 
 
 def parse_args():
@@ -449,7 +449,7 @@ def main():
     if hbm_peak is None:
         hbm_peak, peak_src = 6650.0, "fallback"
     achieved = alg_bytes / gemv_s / 1e9
-    # dram__bytes_read.sum + dram__bytes_write.sum of one gemv_pipe_kernel launch
+    # dram__bytes_read.sum + dram__bytes_write.sum of one gemv_dot_kernel launch
     # on this workload (ncu --set full); valid only for that kernel version
     ncu_traffic = NCU_TRAFFIC_BYTES if args.layers == 16 else None
 
@@ -470,7 +470,7 @@ def main():
         },
         "gpu_launches": 2 * K,
         "clocks": clk,
-        "roofline": {"bound": "hbm", "kernel": "gemv_kernel (sherry_gemv_run)",
+        "roofline": {"bound": "hbm", "kernel": "gemv_dot_kernel (sherry_gemv_run)",
                      "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "peak_source": peak_src,
                      "bytes_per_launch": alg_bytes, "kernel_us": gemv_s * 1e6,

@@ -233,11 +233,29 @@ struct Consts {
     uint32_t tlo[4], thi[4];
 };
 
+__device__ __forceinline__ void load_consts(const GemvParams &P, Consts &C) {
+    C.mul4 = P.mul4;
+    C.mul2 = P.mul2;
+    C.hi1 = P.hi1;
+    C.hi2 = P.hi2;
+    C.hi16 = P.hi16;
+    C.m33 = P.m33;
+    C.m55 = P.m55;
+    C.m44 = P.m44;
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        C.tlo[i] = P.tlo[i];
+        C.thi[i] = P.thi[i];
+    }
+}
+
 // Per-row tile state of the pipelined kernel: zero-position nibbles per block
 // group and the four per-position sign planes.  Selector of (i, beta):
 //   zm[beta] | (sign plane i moved so block 4k+beta's bit lands at 4k+2) & 0x44444444.
 // Work split: masks, merges and permutes on the ALU pipe (2 cycles per warp
-// instruction); every shift on the FMA pipe as IMAD (left) or IMAD.HI (right).
+// instruction); left shifts on the FMA pipe as IMAD (2 cycles); right shifts
+// are split between the ALU (SHF, 2 cycles) and the FMA pipe (IMAD.HI, which
+// takes 4 cycles there), so that neither pipe carries them all.
 struct TileDecoder6 {
     uint32_t zm[4];
     uint32_t sg[4];
@@ -246,11 +264,11 @@ struct TileDecoder6 {
                                          uint32_t s1, uint32_t s2) {
         zm[0] = z0 & C.m33;
         zm[1] = z1 & C.m33;
-        zm[2] = imulhi(z0, C.hi2) & C.m33;
-        zm[3] = imulhi(z1, C.hi2) & C.m33;
+        zm[2] = (z0 >> 2) & C.m33;
+        zm[3] = (z1 >> 2) & C.m33;
         // bit-sliced zero positions: lo bit (L) and hi bit (H) of p_j at bit j
         const uint32_t L = lop_merge(z0, imul(z1, C.mul2), C.m55);
-        const uint32_t H = lop_merge(imulhi(z0, C.hi1), z1, C.m55);
+        const uint32_t H = lop_merge(z0 >> 1, z1, C.m55);
         // sign of position i when kept: rank 0; rank 0 if p == 0 else 1;
         // rank 1 if p <= 1 else 2; rank 2
         sg[0] = s0;
@@ -426,6 +444,30 @@ __device__ __forceinline__ int first_item_at_or_after(const GemvParams &P, int c
                      : (lo + 1 < P.count ? P.d[lo + 1].item_begin : P.total_items);
 }
 
+// (GEMV, unit, K-part) of an item, advanced item by item without searches or
+// divisions.
+struct ItemCursor {
+    int id, unit, kp;
+};
+__device__ __forceinline__ ItemCursor cursor_at(const GemvParams &P, int item) {
+    ItemCursor c;
+    c.id = find_desc_by_item(P, item);
+    const GemvDesc &D = P.d[c.id];
+    const int local = item - D.item_begin;
+    c.unit = local / D.kparts;
+    c.kp = local - c.unit * D.kparts;
+    return c;
+}
+__device__ __forceinline__ void cursor_next(const GemvParams &P, ItemCursor &c) {
+    if (++c.kp == P.d[c.id].kparts) {
+        c.kp = 0;
+        if (++c.unit == P.d[c.id].units) {
+            c.unit = 0;
+            ++c.id;
+        }
+    }
+}
+
 #ifndef SHERRY_PIPE_MIN_BLOCKS
 #define SHERRY_PIPE_MIN_BLOCKS 2
 #endif
@@ -442,19 +484,7 @@ __global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
     if (it_begin >= it_end) return;
     uint32_t *ring = pipe_smem + (size_t)warp * kRing * kStageWords;
     Consts C;
-    C.mul4 = P.mul4;
-    C.mul2 = P.mul2;
-    C.hi1 = P.hi1;
-    C.hi2 = P.hi2;
-    C.hi16 = P.hi16;
-    C.m33 = P.m33;
-    C.m55 = P.m55;
-    C.m44 = P.m44;
-#pragma unroll
-    for (int i = 0; i < 4; i++) {
-        C.tlo[i] = P.tlo[i];
-        C.thi[i] = P.thi[i];
-    }
+    load_consts(P, C);
 
     // ---- producer side: the issue cursor runs kRing-1 stages ahead ----
     // lane l copies 16-byte pieces l + 32 j (j = 0..4) of the 2560-byte chunk;
@@ -622,6 +652,184 @@ __global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
 }
 
 // ---------------------------------------------------------------------------
+// Small-batch kernel (B <= 4): dot products on the ALU/FMA pipes, no MMA.
+//   * one warp owns a (32-row unit, K-part) item at a time and lane l owns row
+//     l of the unit, so a tile's five words are five conflict-free shared
+//     loads and each lane ends with its row's complete sum (no reduction);
+//   * the unit's chunks (2560 contiguous bytes) and the chunk's re-ordered
+//     activations (128 words per batch row) stream through a private
+//     3-stage cp.async ring; the activation words are the same for all lanes
+//     (broadcast reads);
+//   * each decoded word (four ternary bytes) meets its activation word in one
+//     dp4a, so a batch row costs 32 dp4a per tile: for B <= 4 this is cheaper
+//     than an m16n8k32 MMA whose 8 columns would mostly be empty.
+// Items, K-parts and the split-K completion are those of the pipelined kernel.
+// ---------------------------------------------------------------------------
+constexpr int kDotThreads = 256;
+constexpr int kDotWarps = kDotThreads / 32;
+constexpr int kDotRing = 3;
+constexpr int kDotCodeWords = kChunkTiles * kTileWords;  // 640
+template <int NBX>
+struct DotShape {
+    static constexpr int kStageWords = kDotCodeWords + NBX * kChunkTiles * 32;
+    static constexpr size_t kSmem = (size_t)kDotWarps * kDotRing * kStageWords * 4;
+    static constexpr int kMinBlocks = NBX == 1 ? 3 : 2;
+};
+
+template <int NBX, bool ACC_OUT>
+__global__ void __launch_bounds__(kDotThreads, DotShape<NBX>::kMinBlocks)
+    gemv_dot_kernel(const __grid_constant__ GemvParams P) {
+    constexpr int SW = DotShape<NBX>::kStageWords;
+    extern __shared__ __align__(16) uint32_t dot_smem[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const long long nw = (long long)gridDim.x * kDotWarps;
+    const long long wg = (long long)blockIdx.x * kDotWarps + warp;
+    const int it_begin = first_item_at_or_after(P, (int)(wg * P.total_chunks / nw));
+    const int it_end = first_item_at_or_after(P, (int)((wg + 1) * P.total_chunks / nw));
+    if (it_begin >= it_end) return;
+    uint32_t *ring = dot_smem + (size_t)warp * kDotRing * SW;
+    const uint32_t ring_addr = smem_u32(ring);
+    Consts C;
+    load_consts(P, C);
+    const int B = P.B;
+
+    // ---- producer side: the issue cursor runs kDotRing-1 stages ahead ----
+    // lane l copies 16-byte pieces l + 32 j (j = 0..4) of the chunk's codes and
+    // piece l of each batch row's 128 activation words
+    int iitem = it_begin;
+    ItemCursor icur = cursor_at(P, it_begin);
+    int ic = 0, ic_end = 0, iTp = 0;
+    const uint32_t *isrc = nullptr, *ixw = nullptr;
+    auto set_issue_item = [&]() {
+        const GemvDesc &D = P.d[icur.id];
+        isrc = D.codes + (size_t)icur.unit * D.T * kTileWords + 4 * lane;
+        ixw = reinterpret_cast<const uint32_t *>(D.xw) + 4 * lane;
+        iTp = D.Tp;
+        ic = icur.kp * D.cpp;
+        ic_end = min(D.nchunk, ic + D.cpp);
+    };
+    set_issue_item();
+    auto issue = [&](int slot) {
+        if (iitem < it_end) {
+            const uint32_t *src = isrc + (size_t)ic * kChunkTiles * kTileWords;
+            const uint32_t dst = ring_addr + (uint32_t)slot * SW * 4 + 16u * lane;
+#pragma unroll
+            for (int j = 0; j < 5; j++) cp_async16(dst + 512u * j, src + 128 * j, 16u);
+#pragma unroll
+            for (int b = 0; b < NBX; b++)
+                if (b < B)
+                    cp_async16(dst + 4u * kDotCodeWords + 512u * b,
+                               ixw + ((size_t)b * iTp + (size_t)kChunkTiles * ic) * 32, 16u);
+            if (++ic == ic_end && ++iitem < it_end) {
+                cursor_next(P, icur);
+                set_issue_item();
+            }
+        }
+        cp_async_commit();
+    };
+#pragma unroll
+    for (int s = 0; s < kDotRing - 1; s++) issue(s);
+
+    // ---- consumer side ----
+    int slot = 0;
+    ItemCursor cur = cursor_at(P, it_begin);
+    for (int item = it_begin; item < it_end; item++, cursor_next(P, cur)) {
+        const GemvDesc &D = P.d[cur.id];
+        const int N = D.N;
+        const int unit = cur.unit;
+        const int c_begin = cur.kp * D.cpp, c_end = min(D.nchunk, c_begin + D.cpp);
+        int acc[NBX][2];
+#pragma unroll
+        for (int b = 0; b < NBX; b++) acc[b][0] = acc[b][1] = 0;
+        for (int c = c_begin; c < c_end; c++) {
+            cp_async_wait<kDotRing - 2>();
+            __syncwarp();  // every lane is done with the previous stage: refill it
+            issue(slot == 0 ? kDotRing - 1 : slot - 1);
+            const uint32_t *st = ring + slot * SW;
+            slot = (slot + 1 == kDotRing) ? 0 : slot + 1;
+#pragma unroll 1
+            for (int tt = 0; tt < kChunkTiles; tt++) {
+                const uint32_t *cw = st + tt * kTileWords + lane;
+                TileDecoder6 d;
+                d.load(C, cw[0], cw[32], cw[64], cw[96], cw[128]);
+                // activation words of tile tt: batch row b at b * 128, word q at q
+                const uint4 *xs = reinterpret_cast<const uint4 *>(st + kDotCodeWords + tt * 32);
+#pragma unroll
+                for (int i = 0; i < 4; i++) {
+                    uint4 xa[NBX], xb[NBX];  // words 8i..8i+3 (beta 0, 1) and 8i+4..8i+7 (beta 2, 3)
+#pragma unroll
+                    for (int b = 0; b < NBX; b++) {
+                        xa[b] = xs[b * 32 + 2 * i];
+                        xb[b] = xs[b * 32 + 2 * i + 1];
+                    }
+#pragma unroll
+                    for (int beta = 0; beta < 4; beta++) {
+                        const uint32_t sl = d.sel(C, i, beta);
+                        const int lo = (int)prmt(C.tlo[i], C.thi[i], sl);
+                        // high half of the selector: beta 0, 2 on the ALU, beta 1, 3 on the FMA pipe
+                        const int hi = (int)prmt(C.tlo[i], C.thi[i],
+                                                 (beta & 1) ? imulhi(sl, C.hi16) : (sl >> 16));
+#pragma unroll
+                        for (int b = 0; b < NBX; b++) {
+                            const uint4 &xv = beta < 2 ? xa[b] : xb[b];
+                            int &a = acc[b][beta & 1];
+                            a = __dp4a(lo, (int)pick(xv, 2 * (beta & 1)), a);
+                            a = __dp4a(hi, (int)pick(xv, 2 * (beta & 1) + 1), a);
+                        }
+                    }
+                }
+            }
+        }
+        // epilogue: lane = row of the unit
+        const int row = unit * kUnitRows + lane;
+        const bool rv = row < N;
+        int v[NBX];
+#pragma unroll
+        for (int b = 0; b < NBX; b++) v[b] = acc[b][0] + acc[b][1];
+        bool finish = true;
+        if (D.kparts > 1) {
+            if (rv) {
+#pragma unroll
+                for (int b = 0; b < NBX; b++)
+                    if (b < B) atomicAdd(D.part_acc + (size_t)b * N + row, v[b]);
+            }
+            __threadfence();
+            __syncwarp();
+            uint32_t done = 0;
+            if (lane == 0) done = atomicAdd(D.part_cnt + unit, 1u);
+            finish = __shfl_sync(0xFFFFFFFFu, done, 0) == (uint32_t)(D.kparts - 1);
+            if (finish) {
+                __threadfence();
+                if (rv) {
+#pragma unroll
+                    for (int b = 0; b < NBX; b++) {
+                        if (b < B) {
+                            int32_t *pa = D.part_acc + (size_t)b * N + row;
+                            v[b] = __ldcg(pa);
+                            *pa = 0;
+                        }
+                    }
+                }
+                if (lane == 0) D.part_cnt[unit] = 0u;
+            }
+        }
+        if (finish && rv) {
+            if (ACC_OUT) {
+#pragma unroll
+                for (int b = 0; b < NBX; b++)
+                    if (b < B) static_cast<int32_t *>(D.out)[(size_t)b * N + row] = v[b];
+            } else {
+                const float sc = __ldg(D.scales + row);
+#pragma unroll
+                for (int b = 0; b < NBX; b++)
+                    if (b < B) static_cast<float *>(D.out)[(size_t)b * N + row] = sc * (float)v[b];
+            }
+        }
+    }
+    cp_async_wait<0>();
+}
+
+// ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
 template <typename KernelT>
@@ -647,6 +855,15 @@ void launch_pipe(const GemvParams &gp, cudaStream_t stream) {
     const int want = (gp.total_chunks + kPipeWarps * 4 - 1) / (kPipeWarps * 4);
     const int grid = grid_for(gemv_pipe_kernel<NB, ACC>, kPipeThreads, kPipeSmem, want, cache);
     gemv_pipe_kernel<NB, ACC><<<grid, kPipeThreads, kPipeSmem, stream>>>(gp);
+}
+
+template <int NBX, bool ACC>
+void launch_dot(const GemvParams &gp, cudaStream_t stream) {
+    static int cache[64] = {0};
+    const size_t smem = DotShape<NBX>::kSmem;
+    const int want = (gp.total_chunks + kDotWarps * 4 - 1) / (kDotWarps * 4);
+    const int grid = grid_for(gemv_dot_kernel<NBX, ACC>, kDotThreads, smem, want, cache);
+    gemv_dot_kernel<NBX, ACC><<<grid, kDotThreads, smem, stream>>>(gp);
 }
 
 template <int NB, bool ACC>
@@ -779,7 +996,15 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
         if (st != SHERRY_OK) return st;
     }
     if (!(phase & kRun)) return SHERRY_OK;
-    if (pipelined) {
+    if (pipelined && B <= 4) {
+        if (B == 1) {
+            if (acc_out) launch_dot<1, true>(gp, stream); else launch_dot<1, false>(gp, stream);
+        } else if (B == 2) {
+            if (acc_out) launch_dot<2, true>(gp, stream); else launch_dot<2, false>(gp, stream);
+        } else {
+            if (acc_out) launch_dot<4, true>(gp, stream); else launch_dot<4, false>(gp, stream);
+        }
+    } else if (pipelined) {
         if (B <= 8) {
             if (acc_out) launch_pipe<1, true>(gp, stream); else launch_pipe<1, false>(gp, stream);
         } else {

@@ -42,10 +42,11 @@ def test_packed_and_workspace_sizes():
     assert S.packed_bytes(3, 100) == 0
     assert S.packed_bytes(0, 128) == 0
     # re-ordered activations (B rows of K padded to 512) + partial sums and counters
-    # re-ordered activations only: 4 chunks per row need no split-K region
-    assert S.gemv_workspace_bytes(2048, 2048, 1) == 2048
+    # up to 4 chunks per row: re-ordered activations only, no split-K region
     assert S.gemv_workspace_bytes(100, 384, 3) == 3 * 512
-    # 16 chunks per row -> 4 K-parts: partial sums [B][N] and 64 unit counters
+    assert S.gemv_workspace_bytes(40, 1024, 2) == 2 * 8 * 128
+    assert S.gemv_workspace_bytes(2048, 2048, 1) == 2048
+    # 16 chunks per row -> 4 K-parts: activations, then partial sums [B][N] and 64 unit counters
     assert S.gemv_workspace_bytes(2048, 8192, 1) == 4 * 64 * 32 + 4 * (2048 + 64)
     assert S.gemv_workspace_bytes(100, 8192, 3) == 3 * 4 * 64 * 32 + 256 * ((4 * (300 + 4) + 255) // 256)
     assert S.gemv_workspace_bytes(16, 128, 0) == 0
