@@ -577,10 +577,12 @@ __global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
                         const int m = 4 * i + beta;  // MMA index: activation words 2m, 2m+1
                         const uint32_t s0 = d0.sel(C, i, beta);
                         const uint32_t s1 = d1.sel(C, i, beta);
+                        // high halves of the selectors by ALU shifts: the FMA pipe
+                        // already carries the decoder's IMAD work here
                         const uint32_t a0 = prmt(tlo, thi, s0);
-                        const uint32_t a2 = prmt(tlo, thi, imulhi(s0, C.hi16));
+                        const uint32_t a2 = prmt(tlo, thi, s0 >> 16);
                         const uint32_t a1 = prmt(tlo, thi, s1);
-                        const uint32_t a3 = prmt(tlo, thi, imulhi(s1, C.hi16));
+                        const uint32_t a3 = prmt(tlo, thi, s1 >> 16);
 #pragma unroll
                         for (int nb = 0; nb < NB; nb++) {
                             const uint4 &xx = xq[nb][(m >> 1) & 1];
@@ -652,7 +654,7 @@ __global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
 }
 
 // ---------------------------------------------------------------------------
-// Small-batch kernel (B <= 4): dot products on the ALU/FMA pipes, no MMA.
+// Small-batch kernel (B <= 2): dot products on the ALU/FMA pipes, no MMA.
 //   * one warp owns a (32-row unit, K-part) item at a time and lane l owns row
 //     l of the unit, so a tile's five words are five conflict-free shared
 //     loads and each lane ends with its row's complete sum (no reduction);
@@ -661,7 +663,7 @@ __global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
 //     3-stage cp.async ring; the activation words are the same for all lanes
 //     (broadcast reads);
 //   * each decoded word (four ternary bytes) meets its activation word in one
-//     dp4a, so a batch row costs 32 dp4a per tile: for B <= 4 this is cheaper
+//     dp4a, so a batch row costs 32 dp4a per tile: for B <= 2 this is cheaper
 //     than an m16n8k32 MMA whose 8 columns would mostly be empty.
 // Items, K-parts and the split-K completion are those of the pipelined kernel.
 // ---------------------------------------------------------------------------
@@ -996,13 +998,13 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
         if (st != SHERRY_OK) return st;
     }
     if (!(phase & kRun)) return SHERRY_OK;
-    if (pipelined && B <= 4) {
+    // B <= 2: dp4a kernel; B >= 3: the MMA kernel (its 8 batch columns cost the
+    // same as one, while dp4a work grows with B) -- measured on the decode stack
+    if (pipelined && B <= 2) {
         if (B == 1) {
             if (acc_out) launch_dot<1, true>(gp, stream); else launch_dot<1, false>(gp, stream);
-        } else if (B == 2) {
-            if (acc_out) launch_dot<2, true>(gp, stream); else launch_dot<2, false>(gp, stream);
         } else {
-            if (acc_out) launch_dot<4, true>(gp, stream); else launch_dot<4, false>(gp, stream);
+            if (acc_out) launch_dot<2, true>(gp, stream); else launch_dot<2, false>(gp, stream);
         }
     } else if (pipelined) {
         if (B <= 8) {

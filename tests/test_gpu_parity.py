@@ -67,7 +67,7 @@ def test_pack_full_size_1b_layers(layer):
 GEMV_CASES = [(256, 1024, 1), (1, 128, 1), (17, 384, 3), (33, 640, 5), (40, 1152, 8),
               (19, 256, 9), (64, 512, 16), (2048, 2048, 1), (512, 2048, 4), (100, 3072, 2),
               (31, 8192, 1), (48, 8192, 16), (50, 1536, 2), (23, 512, 1), (70, 2560, 9),
-              (129, 4096, 8)]
+              (129, 4096, 8), (37, 8192, 2), (130, 2048, 3)]
 
 
 @pytest.mark.parametrize("N,K,B", GEMV_CASES)
