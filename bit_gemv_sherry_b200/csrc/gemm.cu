@@ -11,14 +11,16 @@
 //               into a 4-stage ring (completion via mbarrier transaction count);
 //   warp 1      allocates 512 TMEM columns (two 128 x 256 int32 accumulators)
 //               and, from one thread, issues tcgen05.mma.kind::i8 (M=128,
-//               N=256, K=32) four times per stage, committing each stage back
-//               to its producers and each finished tile to the epilogue;
-//   warps 2-5   decoders: thread r decodes weight row r of the 128-row tile for
-//               one 128-weight K tile (the five words of the Sherry tile) with
-//               the same SWAR/PRMT decode as the GEMV, re-orders the bytes to
-//               natural K order with a 4x4 byte transpose, and writes the
-//               row's 128 bytes into the swizzled K-major operand layout;
-//   warps 6-9   epilogue: tcgen05.ld of their 32-lane quarter of the finished
+//               N=256, K=32) four times per stage, committing every second
+//               stage back to its producers (a commit frees a pair of stages)
+//               and each finished tile to the epilogue;
+//   warps 2-9   decoders, two groups of four taking alternate stages: thread r
+//               of a group loads weight row r's five code words (two of its
+//               stages ahead), decodes them (SWAR + PRMT, as in the GEMV),
+//               re-orders the bytes to natural K order with 4x4 byte
+//               transposes and writes the row's 128 bytes into the swizzled
+//               K-major operand layout;
+//   warps 10-13 epilogue: tcgen05.ld of their 32-lane quarter of the finished
 //               accumulator, y = s * (float) acc, coalesced fp32 stores;
 //               double-buffered TMEM lets tile i's epilogue overlap tile i+1's MMAs.
 //
@@ -45,17 +47,18 @@ constexpr int kStages = 4;
 constexpr int kABytes = kBM * kBK;  // 16 KB
 constexpr int kBBytes = kBN * kBK;  // 32 KB
 constexpr int kStageBytes = kABytes + kBBytes;
-constexpr int kThreads = 320;
+constexpr int kDecGroups = 2;                   // decoder groups, taking alternate stages
+constexpr int kThreads = 32 * (2 + 4 * kDecGroups + 4);
 constexpr int kTmemCols = 512;
 constexpr uint32_t kIdesc = (2u << 4)                  // D = s32
                             | (1u << 7) | (1u << 10)   // A, B = signed int8
                             | ((uint32_t)(kBN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
-constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + 1024 + 256;
+constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + 1024 + 512;
 
 struct __align__(8) Barriers {
-    uint64_t full_a[kStages];
-    uint64_t full_b[kStages];
-    uint64_t empty[kStages];
+    uint64_t full_a[kStages];         // A tile written: 128 decoder threads
+    uint64_t full_b[kStages];         // X tile landed: 1 arrival + bytes
+    uint64_t empty[kStages / 2];      // stage pair (2p, 2p+1) read by the MMAs: 1 commit
     uint64_t tmem_full[2];
     uint64_t tmem_empty[2];
     uint64_t drain;
@@ -97,7 +100,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int s = 0; s < kStages; s++) {
             mbar_init(&bar->full_a[s], 128);
             mbar_init(&bar->full_b[s], 1);
-            mbar_init(&bar->empty[s], 1);
+            if (s % 2 == 0) mbar_init(&bar->empty[s / 2], 1);
         }
         for (int a = 0; a < 2; a++) {
             mbar_init(&bar->tmem_full[a], 1);
@@ -117,7 +120,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem_base = bar->tmem_base;
 
     if (warp == 0) {
-        // ---------------- TMA producer ----------------
+        // ---------------- TMA producer: X tiles ----------------
         if (lane == 0) {
             uint32_t it = 0;
             for (int tile = blockIdx.x; tile < num_tiles && !*abort; tile += gridDim.x) {
@@ -125,7 +128,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int kt = 0; kt < T; kt++, it++) {
                     const int s = it % kStages;
                     const uint32_t ph = (it / kStages) & 1;
-                    if (!mbar_wait(&bar->empty[s], ph ^ 1, abort, err)) break;
+                    if (!mbar_wait(&bar->empty[s >> 1], ph ^ 1, abort, err)) break;
                     uint8_t *b_smem = smem + (size_t)s * kStageBytes + kABytes;
                     mbar_arrive_expect_tx(&bar->full_b[s], kBBytes);
                     tma_load_2d(b_smem, &tmap_x, &bar->full_b[s], kt * kBK, xb * kBN);
@@ -169,7 +172,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 smem_desc_sw128(b_addr + 32 * k), kIdesc, (kt | k) != 0);
                     }
                     issued = true;
-                    umma_commit(&bar->empty[s]);
+                    // one commit frees a pair of stages: half the commits of the issuing thread
+                    if (s & 1) umma_commit(&bar->empty[s >> 1]);
                 }
                 if (!ok) break;
                 umma_commit(&bar->tmem_full[a]);
@@ -180,60 +184,71 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_wait(&bar->drain, 0, &no_abort, err, 1000000000LL);
             }
         }
-    } else if (warp < 6) {
-        // ---------------- decoders: one weight row per thread ----------------
-        const int r = threadIdx.x - 64;
-        uint32_t it = 0;
-        for (int tile = blockIdx.x; tile < num_tiles && !*abort; tile += gridDim.x) {
-            const int wb = tile % tiles_n;
-            const int row = wb * kBM + r;
-            const bool valid = row < N;
-            // word (p, row, kt) = ((row / 32) * T + kt) * 160 + 32 p + row % 32: a warp
-            // (32 consecutive rows) reads 128 contiguous bytes per plane
-            const uint32_t *crow = codes + (size_t)(row / 32) * T * 160 + (row % 32);
+    } else if (warp < 2 + 4 * kDecGroups) {
+        // ------- decoders: group g takes stages j = g mod kDecGroups, one row per thread -------
+        // Stage j of this CTA is (tile blockIdx.x + (j / T) * gridDim.x, K tile j % T).  A
+        // thread loads its row's five code words itself (a warp reads 128 contiguous bytes
+        // per plane) two of its group's stages ahead, so the loads overlap the decode.
+        const int g = (warp - 2) >> 2;
+        const int r = threadIdx.x - 64 - 128 * g;
+        const int my_tiles = num_tiles > (int)blockIdx.x
+                                 ? (num_tiles - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+        const uint32_t total = (uint32_t)my_tiles * (uint32_t)T;
+        auto load_stage = [&](uint32_t j, uint32_t (&w)[5]) {
+            const int tile = (int)blockIdx.x + (int)(j / T) * (int)gridDim.x;
+            const int row = (tile % tiles_n) * kBM + r;
+            if (j < total && row < N) {
+                // word (p, row, kt) = ((row / 32) * T + kt) * 160 + 32 p + row % 32
+                const uint32_t *c = codes + ((size_t)(row / 32) * T + j % T) * 160 + (row % 32);
+#pragma unroll
+                for (int p = 0; p < 5; p++) w[p] = ld_code(c + 32 * p);
+            } else {
+#pragma unroll
+                for (int p = 0; p < 5; p++) w[p] = 0u;
+            }
+        };
+        uint32_t wa[5], wb[5];
+        load_stage(g, wa);
+        load_stage(g + kDecGroups, wb);
+        for (uint32_t j = g; j < total; j += kDecGroups) {
             uint32_t w[5];
 #pragma unroll
-            for (int p = 0; p < 5; p++) w[p] = valid ? ld_code(crow + p * 32) : 0u;
-            bool ok = true;
-            for (int kt = 0; kt < T; kt++, it++) {
-                const int s = it % kStages;
-                const uint32_t ph = (it / kStages) & 1;
-                TileDecoder dec;
-                dec.load(w[0], w[1], w[2], w[3], w[4]);
-                if (kt + 1 < T) {
-#pragma unroll
-                    for (int p = 0; p < 5; p++)
-                        w[p] = valid ? ld_code(crow + (size_t)(kt + 1) * 160 + p * 32) : 0u;
-                }
-                if (!mbar_wait(&bar->empty[s], ph ^ 1, abort, err)) {
-                    ok = false;
-                    break;
-                }
-                uint8_t *a_row = smem + (size_t)s * kStageBytes + (size_t)r * kBK;
-#pragma unroll
-                for (int h = 0; h < 2; h++) {
-                    uint32_t nat[4][4];  // [beta][k'] natural-order words of block 4(k'+4h)+beta
-#pragma unroll
-                    for (int beta = 0; beta < 4; beta++) {
-                        uint32_t byi[4];
-#pragma unroll
-                        for (int i = 0; i < 4; i++) {
-                            const uint32_t sel = dec.sel(i, beta);
-                            byi[i] = valid ? prmt(table_lo(i), table_hi(i), h ? (sel >> 16) : sel) : 0u;
-                        }
-                        transpose4(byi, nat[beta]);
-                    }
-#pragma unroll
-                    for (int kp = 0; kp < 4; kp++) {
-                        const int c = 4 * h + kp;  // 16-byte chunk = blocks 4c..4c+3
-                        const uint4 v = make_uint4(nat[0][kp], nat[1][kp], nat[2][kp], nat[3][kp]);
-                        *reinterpret_cast<uint4 *>(a_row + ((c ^ (r & 7)) << 4)) = v;
-                    }
-                }
-                fence_proxy_async_smem();
-                mbar_arrive(&bar->full_a[s]);
+            for (int p = 0; p < 5; p++) {
+                w[p] = wa[p];
+                wa[p] = wb[p];
             }
-            if (!ok) break;
+            load_stage(j + 2 * kDecGroups, wb);
+            const int s = j % kStages;
+            const uint32_t ph = (j / kStages) & 1;
+            // the A slot's previous tile has been consumed by the MMAs
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&bar->empty[s >> 1], ph ^ 1, abort, err))) break;
+            const int tile = (int)blockIdx.x + (int)(j / T) * (int)gridDim.x;
+            const bool valid = (tile % tiles_n) * kBM + r < N;
+            TileDecoder dec;
+            dec.load(w[0], w[1], w[2], w[3], w[4]);
+            uint8_t *a_row = smem + (size_t)s * kStageBytes + (size_t)r * kBK;
+#pragma unroll
+            for (int h = 0; h < 2; h++) {
+                uint32_t nat[4][4];  // [beta][k'] natural-order words of block 4(k'+4h)+beta
+#pragma unroll
+                for (int beta = 0; beta < 4; beta++) {
+                    uint32_t byi[4];
+#pragma unroll
+                    for (int i = 0; i < 4; i++) {
+                        const uint32_t sel = dec.sel(i, beta);
+                        byi[i] = valid ? prmt(table_lo(i), table_hi(i), h ? (sel >> 16) : sel) : 0u;
+                    }
+                    transpose4(byi, nat[beta]);
+                }
+#pragma unroll
+                for (int kp = 0; kp < 4; kp++) {
+                    const int c = 4 * h + kp;  // 16-byte chunk = blocks 4c..4c+3
+                    const uint4 v = make_uint4(nat[0][kp], nat[1][kp], nat[2][kp], nat[3][kp]);
+                    *reinterpret_cast<uint4 *>(a_row + ((c ^ (r & 7)) << 4)) = v;
+                }
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&bar->full_a[s]);
         }
     } else {
         // ---------------- epilogue ----------------
@@ -242,7 +257,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int tile = blockIdx.x; tile < num_tiles && !*abort; tile += gridDim.x, acc_it++) {
             const int wb = tile % tiles_n, xb = tile / tiles_n;
             const uint32_t a = acc_it & 1, aph = (acc_it >> 1) & 1;
-            if (!mbar_wait(&bar->tmem_full[a], aph, abort, err)) break;
+            // every lane waits; the warp leaves together if any lane's wait gave up
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&bar->tmem_full[a], aph, abort, err))) break;
             tc_fence_after();
             const int row = wb * kBM + q * 32 + lane;
             const bool rv = row < N;
