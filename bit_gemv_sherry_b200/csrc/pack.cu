@@ -2,13 +2,14 @@
 //
 // The step the pages call "packing blocks of four weights into five bits" under
 // "3:4 fine-grained sparsity" (arXiv 2601.07892, abstract).  One warp handles a
-// 128-weight tile: lane j loads block j as a float4 (one coalesced 512-byte
-// row segment per warp), picks its zero (smallest |w|, lowest index on ties),
-// and the warp assembles the five words with ballots -- bit j of a ballot is
-// block j, which is exactly the bit-sliced sign layout.  Kept |w| are summed
-// in double per lane, reduced over the warp, then over the warps of the row in
-// a fixed order, so the scale is deterministic.  HBM-bound: 4 bytes read and
-// 0.16 bytes written per weight.
+// 128-weight tile at a time: lane j loads block j as a float4 (one coalesced
+// 512-byte row segment per warp), picks its zero (smallest |w|, lowest index
+// on ties), and the warp assembles the five words with ballots -- bit j of a
+// ballot is block j, which is exactly the bit-sliced sign layout.  A warp
+// takes a run of tiles of one row and keeps eight tile loads in flight.  Kept
+// |w| are summed in double per lane, reduced over the warp once, then over the
+// warps of the row in a fixed order, so the scale is deterministic.
+// HBM-bound: 4 bytes read and 0.16 bytes written per weight.
 #include "common.cuh"
 
 namespace sherry {
@@ -16,11 +17,11 @@ namespace {
 
 constexpr int kPackThreads = 256;
 constexpr int kPackWarps = kPackThreads / 32;
-constexpr int kPackUnroll = 4;
+constexpr int kPackBatch = 8;      // tiles loaded per batch
+constexpr int64_t kPackMinTiles = 8;  // fewest tiles a warp of a multi-warp row takes
 
 struct TileBits {
     uint32_t z0, z1, s0, s1, s2;
-    double sum;
 };
 
 __device__ __forceinline__ float4 ld_stream(const float4 *p) {
@@ -31,13 +32,18 @@ __device__ __forceinline__ float4 ld_stream(const float4 *p) {
     return v;
 }
 
-__device__ __forceinline__ TileBits pack_tile(float4 v) {
+// Zero position, kept signs and the five words of one tile (lane j = block j);
+// `kept` receives this lane's sum of kept |w| (not reduced over the warp).
+__device__ __forceinline__ TileBits pack_tile(float4 v, double &kept) {
     const float a0 = fabsf(v.x), a1 = fabsf(v.y), a2 = fabsf(v.z), a3 = fabsf(v.w);
-    int p = 0;
-    float m = a0;
-    if (a1 < m) { p = 1; m = a1; }
-    if (a2 < m) { p = 2; m = a2; }
-    if (a3 < m) { p = 3; m = a3; }
+    // argmin with the lowest index on ties, as selects (no branches)
+    const bool b1 = a1 < a0;
+    const float m01 = b1 ? a1 : a0;
+    const int p01 = b1 ? 1 : 0;
+    const bool b2 = a2 < m01;
+    const float m02 = b2 ? a2 : m01;
+    const int p02 = b2 ? 2 : p01;
+    const int p = (a3 < m02) ? 3 : p02;
     const bool f0 = v.x < 0.0f, f1 = v.y < 0.0f, f2 = v.z < 0.0f, f3 = v.w < 0.0f;
     // kept weights in ascending position -> ranks 0, 1, 2
     const bool r0 = (p == 0) ? f1 : f0;
@@ -55,19 +61,28 @@ __device__ __forceinline__ TileBits pack_tile(float4 v) {
     // Z0: fields of the even blocks, Z1: fields of the odd blocks.
     tb.z0 = (L & 0x55555555u) | ((H & 0x55555555u) << 1);
     tb.z1 = ((L >> 1) & 0x55555555u) | (H & 0xAAAAAAAAu);
-    double s = (double)k0 + (double)k1 + (double)k2;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
-    tb.sum = s;
+    kept += (double)k0 + (double)k1 + (double)k2;
     return tb;
 }
 
-// CTA = 8 warps; `wpr` warps share one row (tiles strided by wpr), the CTA
-// covers 8 / wpr rows.  Rows N..Npad-1 (padding of the last 32-row group) are
+// Lanes 0..4 store words Z0, Z1, S0, S1, S2 of a tile at plane offsets 32 p.
+__device__ __forceinline__ void store_words(uint32_t *tile_out, const TileBits &tb, int lane) {
+    const uint32_t lo = (lane & 1) ? tb.z1 : tb.z0;
+    const uint32_t sg = (lane & 1) ? tb.s1 : tb.s0;
+    const uint32_t word = (lane & 4) ? tb.s2 : ((lane & 2) ? sg : lo);
+    if (lane < 5) tile_out[lane * SHERRY_ROW_GROUP] = word;
+}
+
+// CTA = 8 warps; `wpr` warps share one row, warp `sub` of a row takes the
+// `tpw` consecutive tiles sub * tpw .. and loads them kPackBatch at a time
+// (all loads of a batch in flight before the first tile is packed).  Each
+// lane sums its kept |w| in double over all its tiles; the lanes are reduced
+// once per warp and the warps of a row in a fixed order, so the scale is
+// deterministic.  Rows N..Npad-1 (padding of the last 32-row group) are
 // written as zero words.
 __global__ void __launch_bounds__(kPackThreads) pack_kernel(const float *__restrict__ w, int64_t N,
                                                             int64_t Npad, int64_t K, int wpr,
-                                                            uint32_t *__restrict__ codes,
+                                                            int64_t tpw, uint32_t *__restrict__ codes,
                                                             float *__restrict__ scales) {
     __shared__ double partial[kPackWarps];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -75,36 +90,37 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(const float *__restr
     const int64_t n = (int64_t)blockIdx.x * rpc + warp / wpr;
     const int sub = warp % wpr;
     const int64_t T = K / SHERRY_TILE_K;
-    double row_sum = 0.0;
+    const int64_t t_begin = sub * tpw;
+    const int64_t t_end = t_begin + tpw < T ? t_begin + tpw : T;
+    double kept = 0.0;
     // word (p, n, t) = ((n / 32) * T + t) * 160 + 32 p + n % 32
     uint32_t *out = codes + (n / SHERRY_ROW_GROUP) * T * (5 * SHERRY_ROW_GROUP) + n % SHERRY_ROW_GROUP;
     if (n < N) {
         const float4 *row = reinterpret_cast<const float4 *>(w + n * K);
-        for (int64_t t0 = sub; t0 < T; t0 += (int64_t)wpr * kPackUnroll) {
-            float4 v[kPackUnroll];
+        for (int64_t t0 = t_begin; t0 < t_end; t0 += kPackBatch) {
+            if (t0 + kPackBatch <= t_end) {  // full batch: no per-tile bounds tests
+                float4 v[kPackBatch];
 #pragma unroll
-            for (int u = 0; u < kPackUnroll; u++) {
-                const int64_t t = t0 + (int64_t)u * wpr;
-                v[u] = (t < T) ? ld_stream(row + t * 32 + lane) : make_float4(0.f, 0.f, 0.f, 0.f);
-            }
+                for (int u = 0; u < kPackBatch; u++) v[u] = ld_stream(row + (t0 + u) * 32 + lane);
 #pragma unroll
-            for (int u = 0; u < kPackUnroll; u++) {
-                const int64_t t = t0 + (int64_t)u * wpr;
-                if (t >= T) break;  // warp-uniform
-                const TileBits tb = pack_tile(v[u]);
-                row_sum += tb.sum;
-                if (lane < 5) {
-                    const uint32_t word = lane == 0 ? tb.z0 : lane == 1 ? tb.z1 : lane == 2 ? tb.s0
-                                          : lane == 3 ? tb.s1 : tb.s2;
-                    out[t * (5 * SHERRY_ROW_GROUP) + lane * SHERRY_ROW_GROUP] = word;
+                for (int u = 0; u < kPackBatch; u++) {
+                    const TileBits tb = pack_tile(v[u], kept);
+                    store_words(out + (t0 + u) * (5 * SHERRY_ROW_GROUP), tb, lane);
+                }
+            } else {
+                for (int64_t t = t0; t < t_end; t++) {
+                    const TileBits tb = pack_tile(ld_stream(row + t * 32 + lane), kept);
+                    store_words(out + t * (5 * SHERRY_ROW_GROUP), tb, lane);
                 }
             }
         }
     } else if (n < Npad) {
-        for (int64_t t = sub; t < T; t += wpr)
+        for (int64_t t = t_begin; t < t_end; t++)
             if (lane < 5) out[t * (5 * SHERRY_ROW_GROUP) + lane * SHERRY_ROW_GROUP] = 0u;
     }
-    if (lane == 0) partial[warp] = row_sum;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) kept += __shfl_xor_sync(0xFFFFFFFFu, kept, o);
+    if (lane == 0) partial[warp] = kept;
     __syncthreads();
     if (threadIdx.x < rpc) {
         const int64_t rn = (int64_t)blockIdx.x * rpc + threadIdx.x;
@@ -127,12 +143,14 @@ extern "C" sherry_status sherry_pack(const float *w, int64_t N, int64_t K, uint3
     if (!aligned(w, 16) || !aligned(codes, 16) || !aligned(scales, 4)) return SHERRY_ERR_ALIGN;
     const int64_t T = K / SHERRY_TILE_K;
     const int64_t Npad = (N + SHERRY_ROW_GROUP - 1) / SHERRY_ROW_GROUP * SHERRY_ROW_GROUP;
+    // warps per row: as many as keep at least kPackMinTiles tiles each (up to 8)
     int wpr = 1;
-    while (wpr < kPackWarps && wpr * 2 <= T) wpr *= 2;
+    while (wpr < kPackWarps && (int64_t)wpr * 2 * kPackMinTiles <= T) wpr *= 2;
+    const int64_t tpw = (T + wpr - 1) / wpr;
     const int rpc = kPackWarps / wpr;
     const int64_t grid = (Npad + rpc - 1) / rpc;
     if (grid > 0x7FFFFFFF) return SHERRY_ERR_UNSUPPORTED;
     pack_kernel<<<(unsigned)grid, kPackThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-        w, N, Npad, K, wpr, codes, scales);
+        w, N, Npad, K, wpr, tpw, codes, scales);
     return launch_status("sherry_pack");
 }
