@@ -74,18 +74,19 @@ struct GemvParams {
 struct XprepDesc {
     const int8_t *x;
     uint32_t *xw;         // first word of this GEMV's workspace region
+    uint32_t *zero;       // split-K partial sums and counters to clear
     int K;
     int Tp;
-    int word_begin;       // first thread index of this GEMV
-    int xw_words;         // B * Tp * 32 re-ordered words, then zero_words zeros
-    int zero_words;       // split-K partial sums and counters to clear (0 if unsplit)
+    int unit_begin;       // first work unit of this GEMV
+    int xunits;           // B * Tp (batch row, tile) units
+    int zero_words;       // words at `zero` (0 if the rows are not split)
     int pad;
 };
 
 struct XprepParams {
     int count;
     int B;
-    int total_words;
+    int total_units;
     int pad;
     XprepDesc d[SHERRY_MAX_GROUP];
 };
@@ -138,35 +139,56 @@ int64_t ws_words(int64_t N, int64_t K, int B) {
 // xw[b][t][q] (t < Tp): word q = 2 (4 i + beta) + h holds the activations met
 // by char4(i, beta, h) of tile t: bytes x[b][128 t + 16 k' + 64 h + 4 beta + i],
 // k' = 0..3; tiles t >= K/128 are zero so that padded chunks contribute
-// nothing.  The words after the re-ordered block (partial sums, counters) are
-// cleared.
+// nothing.  The split-K partial sums and counters are cleared.
+//
+// One warp per work unit: a (batch row, tile) unit -- lane l loads raw word l
+// of the tile (128 contiguous bytes per warp); the bytes of output word q are
+// byte i of raw words 4 k' + 16 h + beta, fetched with four shuffles and
+// merged with three byte permutes -- or a unit of 32 words to clear.
+__device__ __forceinline__ uint32_t reorder_word(uint32_t raw, int lane) {
+    const int i = lane >> 3, beta = (lane >> 1) & 3, h = lane & 1;
+    const uint32_t pick2 = (uint32_t)i | ((uint32_t)(4 + i) << 4);  // byte i of a, byte i of b
+    const uint32_t v0 = __shfl_sync(0xFFFFFFFFu, raw, 0 + 16 * h + beta);
+    const uint32_t v1 = __shfl_sync(0xFFFFFFFFu, raw, 4 + 16 * h + beta);
+    const uint32_t v2 = __shfl_sync(0xFFFFFFFFu, raw, 8 + 16 * h + beta);
+    const uint32_t v3 = __shfl_sync(0xFFFFFFFFu, raw, 12 + 16 * h + beta);
+    return prmt(prmt(v0, v1, pick2), prmt(v2, v3, pick2), 0x5410u);
+}
+
+// Programmatic dependent launch: the GEMV kernels are launched so that they may
+// start while the re-order kernel before them still runs; they wait for it
+// (griddepcontrol.wait: the prior grid completed and its writes are visible)
+// before reading anything it writes.  Without a prior grid the wait returns.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_allow_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __global__ void __launch_bounds__(256) xprep_kernel(const __grid_constant__ XprepParams P) {
-    const int w = blockIdx.x * blockDim.x + threadIdx.x;
-    if (w >= P.total_words) return;
-    int lo = 0, hi = P.count - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (P.d[mid].word_begin <= w) lo = mid; else hi = mid - 1;
+    pdl_allow_dependents();
+    const int lane = threadIdx.x & 31;
+    const int nw = gridDim.x * (blockDim.x >> 5);
+    for (int u = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); u < P.total_units; u += nw) {
+        int lo = 0, hi = P.count - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (P.d[mid].unit_begin <= u) lo = mid; else hi = mid - 1;
+        }
+        const XprepDesc &D = P.d[lo];
+        const int local = u - D.unit_begin;
+        if (local < D.xunits) {
+            const int b = local / D.Tp, t = local - b * D.Tp;
+            const int T = D.K / SHERRY_TILE_K;
+            // x rows are 4-byte aligned (x is, and K is a multiple of 128)
+            const uint32_t raw = t < T ? __ldg(reinterpret_cast<const uint32_t *>(
+                                             D.x + (size_t)b * D.K + (size_t)t * SHERRY_TILE_K) + lane)
+                                       : 0u;
+            D.xw[(size_t)local * 32 + lane] = reorder_word(raw, lane);
+        } else {
+            const int w = (local - D.xunits) * 32 + lane;
+            if (w < D.zero_words) D.zero[w] = 0u;
+        }
     }
-    const XprepDesc &D = P.d[lo];
-    const int local = w - D.word_begin;
-    if (local >= D.xw_words) {
-        D.xw[local] = 0u;
-        return;
-    }
-    const int T = D.K / SHERRY_TILE_K;
-    const int q = local & 31;
-    const int t = (local >> 5) % D.Tp;
-    const int b = (local >> 5) / D.Tp;
-    if (t >= T || b >= P.B) {
-        D.xw[local] = 0u;
-        return;
-    }
-    const int m = q >> 1, h = q & 1, i = m >> 2, beta = m & 3;
-    const uint8_t *src = reinterpret_cast<const uint8_t *>(D.x) + (size_t)b * D.K +
-                         (size_t)t * SHERRY_TILE_K + 64 * h + 4 * beta + i;
-    D.xw[local] = (uint32_t)src[0] | ((uint32_t)src[16] << 8) | ((uint32_t)src[32] << 16) |
-                  ((uint32_t)src[48] << 24);
 }
 
 // ---------------------------------------------------------------------------
@@ -292,6 +314,7 @@ struct TileDecoder6 {
 // NB = number of 8-row batch groups (1: B <= 8, 2: B <= 16).
 template <int NB, bool ACC_OUT>
 __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const __grid_constant__ GemvParams P) {
+    pdl_wait();
     const int lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
     const int nwarps = gridDim.x * kGemvWarps;
@@ -474,6 +497,7 @@ __device__ __forceinline__ void cursor_next(const GemvParams &P, ItemCursor &c) 
 template <int NB, bool ACC_OUT>
 __global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
     gemv_pipe_kernel(const __grid_constant__ GemvParams P) {
+    pdl_wait();
     extern __shared__ __align__(16) uint32_t pipe_smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
@@ -681,6 +705,7 @@ struct DotShape {
 template <int NBX, bool ACC_OUT>
 __global__ void __launch_bounds__(kDotThreads, DotShape<NBX>::kMinBlocks)
     gemv_dot_kernel(const __grid_constant__ GemvParams P) {
+    pdl_wait();
     constexpr int SW = DotShape<NBX>::kStageWords;
     extern __shared__ __align__(16) uint32_t dot_smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -834,6 +859,23 @@ __global__ void __launch_bounds__(kDotThreads, DotShape<NBX>::kMinBlocks)
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
+// Launch with the programmatic-stream-serialization attribute (see pdl_wait).
+template <typename KernelT>
+void launch_pdl(KernelT kernel, int grid, int threads, size_t smem, cudaStream_t stream,
+                const GemvParams &gp) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3((unsigned)threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, kernel, gp);
+}
+
 template <typename KernelT>
 int grid_for(KernelT kernel, int threads, size_t smem, int want, int *cache) {
     int dev = 0;
@@ -856,7 +898,7 @@ void launch_pipe(const GemvParams &gp, cudaStream_t stream) {
     static int cache[64] = {0};
     const int want = (gp.total_chunks + kPipeWarps * 4 - 1) / (kPipeWarps * 4);
     const int grid = grid_for(gemv_pipe_kernel<NB, ACC>, kPipeThreads, kPipeSmem, want, cache);
-    gemv_pipe_kernel<NB, ACC><<<grid, kPipeThreads, kPipeSmem, stream>>>(gp);
+    launch_pdl(gemv_pipe_kernel<NB, ACC>, grid, kPipeThreads, kPipeSmem, stream, gp);
 }
 
 template <int NBX, bool ACC>
@@ -865,7 +907,7 @@ void launch_dot(const GemvParams &gp, cudaStream_t stream) {
     const size_t smem = DotShape<NBX>::kSmem;
     const int want = (gp.total_chunks + kDotWarps * 4 - 1) / (kDotWarps * 4);
     const int grid = grid_for(gemv_dot_kernel<NBX, ACC>, kDotThreads, smem, want, cache);
-    gemv_dot_kernel<NBX, ACC><<<grid, kDotThreads, smem, stream>>>(gp);
+    launch_pdl(gemv_dot_kernel<NBX, ACC>, grid, kDotThreads, smem, stream, gp);
 }
 
 template <int NB, bool ACC>
@@ -873,7 +915,7 @@ void launch_regs(const GemvParams &gp, cudaStream_t stream) {
     static int cache[64] = {0};
     const int want = (gp.total_units16 + kGemvWarps - 1) / kGemvWarps;
     const int grid = grid_for(gemv_kernel<NB, ACC>, kGemvThreads, 0, want, cache);
-    gemv_kernel<NB, ACC><<<grid, kGemvThreads, 0, stream>>>(gp);
+    launch_pdl(gemv_kernel<NB, ACC>, grid, kGemvThreads, 0, stream, gp);
 }
 
 struct GemvCall {
@@ -960,10 +1002,11 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
         XprepDesc &X = xp.d[i];
         X.x = c.x;
         X.xw = region;
+        X.zero = region + xw_words;
         X.K = (int)c.K;
         X.Tp = Tp;
-        X.word_begin = wb;
-        X.xw_words = xw_words;
+        X.unit_begin = wb;
+        X.xunits = B * Tp;
         X.zero_words = (int)split_words(c.N, c.K, B);
         GemvDesc &D = gp.d[i];
         D.codes = c.codes;
@@ -983,17 +1026,18 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
         D.item_begin = ib;
         D.chunk_begin = cb;
         off += ws_words(c.N, c.K, B);
-        wb += X.xw_words + X.zero_words;
+        wb += X.xunits + (X.zero_words + 31) / 32;
         ub16 += (int)((c.N + 15) / 16);
         ib += units * kparts;
         cb += units * kparts * cpp;
     }
-    xp.total_words = wb;
+    xp.total_units = wb;
     gp.total_units16 = ub16;
     gp.total_items = ib;
     gp.total_chunks = cb;
     if (phase & kPrepare) {
-        xprep_kernel<<<(wb + 255) / 256, 256, 0, stream>>>(xp);
+        const int blocks = std::max(1, std::min((wb + 7) / 8, sm_count() * 8));
+        xprep_kernel<<<blocks, 256, 0, stream>>>(xp);
         const sherry_status st = launch_status("sherry_gemv (activation re-order)");
         if (st != SHERRY_OK) return st;
     }
