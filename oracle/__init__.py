@@ -13,6 +13,9 @@ from .oracle import (  # noqa: F401
     code_weights,
     pack,
     unpack,
+    quantize_act,
+    gemv_act,
+    bf16_bits,
     gemv_acc,
     gemv,
     gemm_acc,

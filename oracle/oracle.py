@@ -43,8 +43,10 @@ def _load(path=None):
     lib.oracle_gemv.argtypes = [p, p, p, i64, i64, i64, p]
     lib.oracle_gemm_acc.argtypes = [p, p, i64, i64, i64, p]
     lib.oracle_gemm.argtypes = [p, p, p, i64, i64, i64, p]
+    lib.oracle_quantize_act.argtypes = [p, i64, i64, p, p]
+    lib.oracle_gemv_act.argtypes = [p, p, p, p, i64, i64, i64, p]
     for f in ("oracle_pack", "oracle_unpack", "oracle_gemv_acc", "oracle_gemv",
-              "oracle_gemm_acc", "oracle_gemm"):
+              "oracle_gemm_acc", "oracle_gemm", "oracle_quantize_act", "oracle_gemv_act"):
         getattr(lib, f).restype = ctypes.c_int
     lib.oracle_num_threads.argtypes = []
     lib.oracle_num_threads.restype = ctypes.c_int
@@ -173,3 +175,38 @@ def gemm(codes, scales, x, K):
     _check(_load().oracle_gemm(_ptr(codes), _ptr(scales), _ptr(x), x.shape[0], N, K, _ptr(y)),
            "oracle_gemm")
     return y
+
+
+def quantize_act(x_bf16):
+    """Per-token absmax int8 quantization of bf16 activations (uint16 bit
+    patterns, [B][K]) -> (q int8 [B][K], s float32 [B])."""
+    x = np.ascontiguousarray(x_bf16, dtype=np.uint16)
+    if x.ndim == 1:
+        x = x.reshape(1, -1)
+    B, K = x.shape
+    q = np.zeros((B, K), np.int8)
+    s = np.zeros(B, np.float32)
+    _check(_load().oracle_quantize_act(_ptr(x), B, K, _ptr(q), _ptr(s)), "oracle_quantize_act")
+    return q, s
+
+
+def gemv_act(codes, scales, q, sx, K):
+    """y[b][n] = scales[n] * sx[b] * (W . q^T)[b][n] in double."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint32)
+    scales = np.ascontiguousarray(scales, dtype=np.float32)
+    sx = np.ascontiguousarray(sx, dtype=np.float32)
+    N = scales.shape[0]
+    q = _x2(q, K)
+    y = np.zeros((q.shape[0], N), np.float64)
+    _check(_load().oracle_gemv_act(_ptr(codes), _ptr(scales), _ptr(q), _ptr(sx), N, K,
+                                   q.shape[0], _ptr(y)), "oracle_gemv_act")
+    return y
+
+
+def bf16_bits(values):
+    """bf16 bit patterns of float values that bf16 represents exactly (test data)."""
+    v = np.ascontiguousarray(values, dtype=np.float32)
+    u = v.view(np.uint32)
+    if np.any(u & 0xFFFF):
+        raise ValueError("value not representable in bf16")
+    return (u >> 16).astype(np.uint16)

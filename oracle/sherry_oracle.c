@@ -256,3 +256,65 @@ int oracle_gemm(const uint32_t *codes, const float *scales, const int8_t *x, int
 {
     return orc_matmul(codes, scales, x, M, N, K, y);
 }
+
+/*
+ * Activation front-end.  The setting the method is served in is W1.25A8
+ * (int8 activations); the pages do not say how the int8 activations are made.
+ * Reading taken (restated in the design notes): per token b,
+ *     amax_b = max_k |x[b][k]|,   s_b = amax_b / 127,
+ *     q[b][k] = clamp(rint(x[b][k] * (127 / amax_b)), -127, 127),
+ * every operation in IEEE single precision, rounding to nearest even (the
+ * default mode); an all-zero row gives s_b = 0 and q = 0.  x holds bf16 bit
+ * patterns: the upper 16 bits of an fp32 value.
+ */
+static float orc_bf16(uint16_t h)
+{
+    const uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+int oracle_quantize_act(const uint16_t *x, int64_t B, int64_t K, int8_t *q, float *s)
+{
+    if (!x || !q || !s || B < 1 || K < 1) return ORC_BAD_ARG;
+    for (int64_t b = 0; b < B; b++) {
+        const uint16_t *xr = x + b * K;
+        float amax = 0.0f;
+        for (int64_t k = 0; k < K; k++) {
+            const float a = fabsf(orc_bf16(xr[k]));
+            if (a > amax) amax = a;
+        }
+        if (amax == 0.0f) {
+            s[b] = 0.0f;
+            memset(q + b * K, 0, (size_t)K);
+            continue;
+        }
+        const float inv = 127.0f / amax;
+        s[b] = amax / 127.0f;
+        for (int64_t k = 0; k < K; k++) {
+            const float v = orc_bf16(xr[k]) * inv;
+            float r = nearbyintf(v);
+            if (r > 127.0f) r = 127.0f;
+            if (r < -127.0f) r = -127.0f;
+            q[b * K + k] = (int8_t)r;
+        }
+    }
+    return ORC_OK;
+}
+
+/* GEMV on quantized activations: y[b][n] = s[n] * sx[b] * acc[b][n], in double. */
+int oracle_gemv_act(const uint32_t *codes, const float *scales, const int8_t *q, const float *sx,
+                    int64_t N, int64_t K, int64_t B, double *y)
+{
+    if (!sx) return ORC_BAD_ARG;
+    int64_t *acc = (int64_t *)malloc(sizeof(int64_t) * (size_t)(B * N > 0 ? B * N : 1));
+    if (!acc) return ORC_NO_MEM;
+    int rc = orc_matmul_acc(codes, q, B, N, K, acc);
+    if (rc == ORC_OK)
+        for (int64_t b = 0; b < B; b++)
+            for (int64_t n = 0; n < N; n++)
+                y[b * N + n] = (double)scales[n] * (double)sx[b] * (double)acc[b * N + n];
+    free(acc);
+    return rc;
+}

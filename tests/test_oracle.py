@@ -214,3 +214,55 @@ def test_size_closed_forms():
 def test_bad_shapes_rejected():
     with pytest.raises(Exception):
         oracle.pack(np.zeros((2, 100), np.float32))
+
+
+# ---------------------------------------------------------------------------
+# Activation front-end (int8 activations of the W1.25A8 setting; the rule is
+# the reading stated in the oracle: per-token absmax, s = amax / 127,
+# q = clamp(rint(x * (127 / amax)), -127, 127) in fp32, ties to even).
+# Expected values below are derived by hand.
+# ---------------------------------------------------------------------------
+def test_quantize_act_hand_cases():
+    # amax = 127: s = 1 and 127 / amax = 1, so q = rint(x) with ties to even
+    q, s = oracle.quantize_act(oracle.bf16_bits([127.0, 1.0, -0.5, 0.25, -127.0, 63.5, 0.0, 126.5]))
+    assert s.tolist() == [1.0]
+    assert q.tolist() == [[127, 1, 0, 0, -127, 64, 0, 126]]
+    # amax = 2: 127 / 2 = 63.5 exactly; 1.0 -> 63.5 -> 64 (even), 0.5 -> 31.75 -> 32,
+    # 2^-6 -> 0.9921875 -> 1; s = fl32(2 / 127)
+    q, s = oracle.quantize_act(oracle.bf16_bits([2.0, 1.0, -1.0, 0.5, 0.015625, -2.0, 0.0, -0.75]))
+    assert s[0] == np.float32(2.0) / np.float32(127.0)
+    assert q.tolist() == [[127, 64, -64, 32, 1, -127, 0, -48]]   # -0.75 * 63.5 = -47.625 -> -48
+    # an all-zero row
+    q, s = oracle.quantize_act(np.zeros((1, 16), np.uint16))
+    assert s.tolist() == [0.0] and not q.any()
+
+
+def test_quantize_act_bounds_on_random_rows():
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((6, 384)).astype(np.float32) * np.array([1, 1e-3, 10, 1e4, 0.5, 3],
+                                                                    np.float32)[:, None]
+    bits = (x.view(np.uint32) >> 16).astype(np.uint16)          # truncate to bf16
+    xb = (bits.astype(np.uint32) << 16).view(np.float32)
+    q, s = oracle.quantize_act(bits)
+    amax = np.abs(xb).max(axis=1)
+    assert np.array_equal(s, (amax / np.float32(127.0)).astype(np.float32))
+    assert np.abs(q.astype(np.int32)).max() <= 127
+    for b in range(6):
+        k = np.argmax(np.abs(xb[b]))
+        assert abs(int(q[b, k])) == 127 and np.sign(q[b, k]) == np.sign(xb[b, k])
+        # dequantisation error: at most half a step (plus fp32 rounding of x * inv)
+        err = np.abs(q[b].astype(np.float64) * float(s[b]) - xb[b].astype(np.float64))
+        assert err.max() <= 0.5 * float(s[b]) * (1 + 1e-5)
+
+
+def test_gemv_act_equals_scaled_bruteforce():
+    N, K, B = 21, 384, 3
+    codes, scales = oracle.pack(synth.latent_weights(N, K, seed=8))
+    wt = oracle.unpack(codes, N, K).astype(np.int64)
+    rng = np.random.default_rng(9)
+    x = rng.standard_normal((B, K)).astype(np.float32)
+    bits = (x.view(np.uint32) >> 16).astype(np.uint16)
+    q, sx = oracle.quantize_act(bits)
+    acc = q.astype(np.int64) @ wt.T
+    ref = scales.astype(np.float64)[None, :] * sx.astype(np.float64)[:, None] * acc
+    assert np.array_equal(oracle.gemv_act(codes, scales, q, sx, K), ref)

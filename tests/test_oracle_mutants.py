@@ -43,6 +43,12 @@ MUTANTS = {
                          "return ((n / 16) * T + t) * (ORC_NPLANE * 16) + plane * 16 + n % 16;"),
     "rows_before_tiles": ("return ((n / ORC_GROUP) * T + t) * (ORC_NPLANE * ORC_GROUP) + plane * ORC_GROUP + n % ORC_GROUP;",
                           "return ((n / ORC_GROUP) * T + t) * (ORC_NPLANE * ORC_GROUP) + (n % ORC_GROUP) * ORC_NPLANE + plane;"),
+    "quantize_truncates": ("float r = nearbyintf(v);", "float r = truncf(v);"),
+    "quantize_ties_away": ("float r = nearbyintf(v);", "float r = roundf(v);"),
+    "quantize_scale_over_128": ("s[b] = amax / 127.0f;", "s[b] = amax / 128.0f;"),
+    "quantize_inverse_scale_128": ("const float inv = 127.0f / amax;", "const float inv = 128.0f / amax;"),
+    "act_scale_dropped": ("y[b * N + n] = (double)scales[n] * (double)sx[b] * (double)acc[b * N + n];",
+                          "y[b * N + n] = (double)scales[n] * (double)acc[b * N + n];"),
 }
 
 
@@ -58,6 +64,9 @@ def _run_pins(golden_dir):
         pins.test_all_ones_activation_gives_sum_of_signs,
         lambda: pins.test_bruteforce_dense_matmul(3, 256, 2),
         lambda: pins.test_bruteforce_dense_matmul(17, 640, 5),
+        pins.test_quantize_act_hand_cases,
+        pins.test_quantize_act_bounds_on_random_rows,
+        pins.test_gemv_act_equals_scaled_bruteforce,
     ]
     for c in checks:
         try:
