@@ -39,6 +39,7 @@ namespace {
 struct GemvDesc {
     const uint32_t *codes;
     const float *scales;
+    const float *xscale;  // per batch row activation scales (bf16 front-end), else null
     const uint4 *xw;      // re-ordered activations [B][Tp][32 words]
     void *out;            // float y[B][N] or int32 acc[B][N]
     int32_t *part_acc;    // K-part partial sums [B][N] (pipelined kernel, kparts > 1)
@@ -73,14 +74,16 @@ struct GemvParams {
 
 struct XprepDesc {
     const int8_t *x;
+    const uint16_t *xbf;  // bf16 activations to quantize (kind 1), else null
+    float *xscale;        // kind 1: per batch row activation scales written here
     uint32_t *xw;         // first word of this GEMV's workspace region
     uint32_t *zero;       // split-K partial sums and counters to clear
     int K;
     int Tp;
     int unit_begin;       // first work unit of this GEMV
-    int xunits;           // B * Tp (batch row, tile) units
+    int xunits;           // int8: B * Tp (batch row, tile) units; bf16: B row units
     int zero_words;       // words at `zero` (0 if the rows are not split)
-    int pad;
+    int kind;             // 0: int8 activations, 1: bf16 activations quantized here
 };
 
 struct XprepParams {
@@ -164,6 +167,40 @@ __device__ __forceinline__ void pdl_allow_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// Activation front-end (int8 activations of the W1.25A8 setting; the pages
+// do not say how they are made): per token, amax = max |x|, s = amax / 127,
+// q = clamp(rint(x * (127 / amax)), -127, 127), all in fp32 with round-to-
+// nearest-even; amax = 0 gives s = 0, q = 0.  x is bf16 (the upper half of an
+// fp32).
+__device__ __forceinline__ float bf16_lo(uint32_t two) { return __uint_as_float(two << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t two) { return __uint_as_float(two & 0xFFFF0000u); }
+
+__device__ __forceinline__ uint32_t quant_byte(float x, float inv) {
+    int q = __float2int_rn(__fmul_rn(x, inv));
+    q = max(-127, min(127, q));
+    return (uint32_t)(q & 0xFF);
+}
+// four consecutive bf16 values (two words) -> four int8 in one word, k order
+__device__ __forceinline__ uint32_t quant_word(uint2 v, float inv) {
+    return quant_byte(bf16_lo(v.x), inv) | (quant_byte(bf16_hi(v.x), inv) << 8) |
+           (quant_byte(bf16_lo(v.y), inv) << 16) | (quant_byte(bf16_hi(v.y), inv) << 24);
+}
+// max |x| over one bf16 row, reduced over the warp (all lanes get it)
+__device__ __forceinline__ float row_absmax_bf16(const uint16_t *row, int K, int lane) {
+    float m = 0.0f;
+    const uint4 *r4 = reinterpret_cast<const uint4 *>(row);  // 8 values per uint4
+    for (int i = lane; i < K / 8; i += 32) {
+        const uint4 v = __ldg(r4 + i);
+        m = fmaxf(m, fmaxf(fmaxf(fabsf(bf16_lo(v.x)), fabsf(bf16_hi(v.x))),
+                           fmaxf(fabsf(bf16_lo(v.y)), fabsf(bf16_hi(v.y)))));
+        m = fmaxf(m, fmaxf(fmaxf(fabsf(bf16_lo(v.z)), fabsf(bf16_hi(v.z))),
+                           fmaxf(fabsf(bf16_lo(v.w)), fabsf(bf16_hi(v.w)))));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    return m;
+}
+
 __global__ void __launch_bounds__(256) xprep_kernel(const __grid_constant__ XprepParams P) {
     pdl_allow_dependents();
     const int lane = threadIdx.x & 31;
@@ -176,7 +213,22 @@ __global__ void __launch_bounds__(256) xprep_kernel(const __grid_constant__ Xpre
         }
         const XprepDesc &D = P.d[lo];
         const int local = u - D.unit_begin;
-        if (local < D.xunits) {
+        if (local < D.xunits && D.kind == 1) {
+            // bf16 row b: absmax, then quantize and re-order tile by tile
+            const int b = local;
+            const int T = D.K / SHERRY_TILE_K;
+            const uint16_t *row = D.xbf + (size_t)b * D.K;
+            const float amax = row_absmax_bf16(row, D.K, lane);
+            const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+            if (lane == 0) D.xscale[b] = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
+            for (int t = 0; t < D.Tp; t++) {
+                uint32_t raw = 0u;
+                if (t < T)
+                    raw = quant_word(__ldg(reinterpret_cast<const uint2 *>(row + (size_t)t * SHERRY_TILE_K) + lane),
+                                     inv);
+                D.xw[((size_t)b * D.Tp + t) * 32 + lane] = reorder_word(raw, lane);
+            }
+        } else if (local < D.xunits) {
             const int b = local / D.Tp, t = local - b * D.Tp;
             const int T = D.K / SHERRY_TILE_K;
             // x rows are 4-byte aligned (x is, and K is a multiple of 128)
@@ -248,6 +300,13 @@ __device__ __forceinline__ uint32_t imulhi(uint32_t a, uint32_t b) {
     uint32_t d;
     asm("mul.hi.u32 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
     return d;
+}
+
+// Scale of output (row, batch row b): s[row], times the activation scale of b
+// when the activations came through the bf16 front-end (one fp32 rounding).
+__device__ __forceinline__ float out_scale(const GemvDesc &D, int row, int b) {
+    const float s = __ldg(D.scales + row);
+    return D.xscale ? __fmul_rn(s, __ldg(D.xscale + b)) : s;
 }
 
 struct Consts {
@@ -405,7 +464,7 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const __grid_constan
                         static_cast<int32_t *>(D.out)[(size_t)b * N + row] = acc[nb][e];
                     else
                         static_cast<float *>(D.out)[(size_t)b * N + row] =
-                            __ldg(D.scales + row) * (float)acc[nb][e];
+                            out_scale(D, row, b) * (float)acc[nb][e];
                 }
             }
         }
@@ -669,7 +728,7 @@ __global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
                                 static_cast<int32_t *>(D.out)[(size_t)b * N + row] = acc[rb][nb][e];
                             else
                                 static_cast<float *>(D.out)[(size_t)b * N + row] =
-                                    __ldg(D.scales + row) * (float)acc[rb][nb][e];
+                                    out_scale(D, row, b) * (float)acc[rb][nb][e];
                         }
                     }
         }
@@ -846,10 +905,10 @@ __global__ void __launch_bounds__(kDotThreads, DotShape<NBX>::kMinBlocks)
                 for (int b = 0; b < NBX; b++)
                     if (b < B) static_cast<int32_t *>(D.out)[(size_t)b * N + row] = v[b];
             } else {
-                const float sc = __ldg(D.scales + row);
 #pragma unroll
                 for (int b = 0; b < NBX; b++)
-                    if (b < B) static_cast<float *>(D.out)[(size_t)b * N + row] = sc * (float)v[b];
+                    if (b < B)
+                        static_cast<float *>(D.out)[(size_t)b * N + row] = out_scale(D, row, b) * (float)v[b];
             }
         }
     }
@@ -921,10 +980,14 @@ void launch_regs(const GemvParams &gp, cudaStream_t stream) {
 struct GemvCall {
     const uint32_t *codes;
     const float *scales;
-    const int8_t *x;
+    const int8_t *x;        // int8 activations, or null when xbf is given
     void *out;
     int64_t N, K;
+    const uint16_t *xbf;    // bf16 activations (quantized per token), or null
 };
+
+// Words after a GEMV's region for the activation scales of the bf16 front-end.
+constexpr int64_t kActScaleWords = 64;  // >= SHERRY_MAX_GEMV_BATCH, 256-byte region
 
 enum Phase { kPrepare = 1, kRun = 2, kBoth = 3 };
 
@@ -940,15 +1003,16 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
     for (int i = 0; i < count; i++) {
         const GemvCall &c = calls[i];
         const bool need_x = (phase & kPrepare) != 0, need_out = (phase & kRun) != 0;
-        if ((need_x && !c.x) || (need_out && (!c.codes || !c.out || (!acc_out && !c.scales))))
+        if ((need_x && !c.x && !c.xbf) ||
+            (need_out && (!c.codes || !c.out || (!acc_out && !c.scales))))
             return SHERRY_ERR_NULL;
         if (c.N < 1 || !valid_k(c.K)) return SHERRY_ERR_SHAPE;
-        if ((need_x && !aligned(c.x, 4)) ||
+        if ((need_x && c.x && !aligned(c.x, 4)) || (need_x && c.xbf && !aligned(c.xbf, 16)) ||
             (need_out && (!aligned(c.codes, 4) || !aligned(c.out, 4) ||
                           (c.scales && !aligned(c.scales, 4)))))
             return SHERRY_ERR_ALIGN;
         if (c.N > (int64_t)1 << 28) return SHERRY_ERR_UNSUPPORTED;
-        words += ws_words(c.N, c.K, B);
+        words += ws_words(c.N, c.K, B) + (c.xbf ? kActScaleWords : 0);
         units16 += (c.N + 15) / 16;
         const int64_t nchunk = padded_tiles(c.K) / kChunkTiles;
         const int64_t kparts = kparts_for(c.K);
@@ -999,18 +1063,25 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
         const int nchunk = Tp / kChunkTiles;
         const int kparts = (int)kparts_for(c.K);
         const int cpp = (nchunk + kparts - 1) / kparts;
+        const bool bf = c.xbf != nullptr;
+        // activation scales of the bf16 front-end follow the GEMV's regular words
+        float *act_scale = bf ? reinterpret_cast<float *>(region + ws_words(c.N, c.K, B)) : nullptr;
         XprepDesc &X = xp.d[i];
         X.x = c.x;
+        X.xbf = c.xbf;
+        X.xscale = act_scale;
         X.xw = region;
         X.zero = region + xw_words;
         X.K = (int)c.K;
         X.Tp = Tp;
         X.unit_begin = wb;
-        X.xunits = B * Tp;
+        X.xunits = bf ? B : B * Tp;
         X.zero_words = (int)split_words(c.N, c.K, B);
+        X.kind = bf ? 1 : 0;
         GemvDesc &D = gp.d[i];
         D.codes = c.codes;
         D.scales = c.scales;
+        D.xscale = act_scale;
         D.xw = reinterpret_cast<const uint4 *>(region);
         D.out = c.out;
         D.part_acc = kparts > 1 ? reinterpret_cast<int32_t *>(region + xw_words) : nullptr;
@@ -1025,7 +1096,7 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
         D.cpp = cpp;
         D.item_begin = ib;
         D.chunk_begin = cb;
-        off += ws_words(c.N, c.K, B);
+        off += ws_words(c.N, c.K, B) + (bf ? kActScaleWords : 0);
         wb += X.xunits + (X.zero_words + 31) / 32;
         ub16 += (int)((c.N + 15) / 16);
         ib += units * kparts;
@@ -1074,8 +1145,37 @@ sherry_status grouped(const sherry_gemv_desc *descs, int count, int B, void *wor
     GemvCall calls[SHERRY_MAX_GROUP];
     for (int i = 0; i < count; i++)
         calls[i] = GemvCall{descs[i].codes, descs[i].scales, descs[i].x, descs[i].y, descs[i].N,
-                            descs[i].K};
+                            descs[i].K, nullptr};
     return gemv_launch(calls, count, B, false, workspace, workspace_bytes, stream, phase);
+}
+
+sherry_status grouped_bf16(const sherry_gemv_bf16_desc *descs, int count, int B, void *workspace,
+                           size_t workspace_bytes, cudaStream_t stream) {
+    if (!descs) return SHERRY_ERR_NULL;
+    if (count < 1) return SHERRY_ERR_SHAPE;
+    if (count > SHERRY_MAX_GROUP) return SHERRY_ERR_UNSUPPORTED;
+    GemvCall calls[SHERRY_MAX_GROUP];
+    for (int i = 0; i < count; i++) {
+        if (!descs[i].x) return SHERRY_ERR_NULL;
+        calls[i] = GemvCall{descs[i].codes, descs[i].scales, nullptr, descs[i].y, descs[i].N,
+                            descs[i].K, descs[i].x};
+    }
+    return gemv_launch(calls, count, B, false, workspace, workspace_bytes, stream, kBoth);
+}
+
+// Per-token quantization of bf16 activations, natural order (one warp per row).
+__global__ void __launch_bounds__(256) quantize_act_kernel(const uint16_t *__restrict__ x, int B, int K,
+                                                           int8_t *__restrict__ q, float *__restrict__ s) {
+    const int lane = threadIdx.x & 31;
+    const int b = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (b >= B) return;
+    const uint16_t *row = x + (size_t)b * K;
+    const float amax = row_absmax_bf16(row, K, lane);
+    const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+    if (lane == 0) s[b] = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
+    const uint2 *r2 = reinterpret_cast<const uint2 *>(row);
+    uint32_t *qw = reinterpret_cast<uint32_t *>(q + (size_t)b * K);
+    for (int i = lane; i < K / 4; i += 32) qw[i] = quant_word(__ldg(r2 + i), inv);
 }
 
 }  // namespace
@@ -1090,7 +1190,7 @@ extern "C" sherry_status sherry_gemv(const uint32_t *codes, const float *scales,
                                      float *y, int64_t N, int64_t K, int B, void *workspace,
                                      size_t workspace_bytes, sherry_stream_t stream) {
     if (!scales) return SHERRY_ERR_NULL;
-    const sherry::GemvCall c{codes, scales, x, y, N, K};
+    const sherry::GemvCall c{codes, scales, x, y, N, K, nullptr};
     return sherry::gemv_launch(&c, 1, B, false, workspace, workspace_bytes,
                                reinterpret_cast<cudaStream_t>(stream), sherry::kBoth);
 }
@@ -1098,7 +1198,7 @@ extern "C" sherry_status sherry_gemv(const uint32_t *codes, const float *scales,
 extern "C" sherry_status sherry_gemv_acc(const uint32_t *codes, const int8_t *x, int32_t *acc,
                                          int64_t N, int64_t K, int B, void *workspace,
                                          size_t workspace_bytes, sherry_stream_t stream) {
-    const sherry::GemvCall c{codes, nullptr, x, acc, N, K};
+    const sherry::GemvCall c{codes, nullptr, x, acc, N, K, nullptr};
     return sherry::gemv_launch(&c, 1, B, true, workspace, workspace_bytes,
                                reinterpret_cast<cudaStream_t>(stream), sherry::kBoth);
 }
@@ -1122,6 +1222,41 @@ extern "C" sherry_status sherry_gemv_run(const sherry_gemv_desc *descs, int coun
                                          sherry_stream_t stream) {
     return sherry::grouped(descs, count, B, const_cast<void *>(workspace), workspace_bytes,
                            reinterpret_cast<cudaStream_t>(stream), sherry::kRun);
+}
+
+extern "C" size_t sherry_gemv_bf16_workspace_bytes(int64_t N, int64_t K, int B) {
+    if (B < 1 || N < 1 || K < 1) return 0;
+    return (size_t)(sherry::ws_words(N, K, B) + sherry::kActScaleWords) * 4;
+}
+
+extern "C" sherry_status sherry_gemv_bf16(const uint32_t *codes, const float *scales,
+                                          const uint16_t *x, float *y, int64_t N, int64_t K, int B,
+                                          void *workspace, size_t workspace_bytes,
+                                          sherry_stream_t stream) {
+    if (!scales || !x) return SHERRY_ERR_NULL;
+    const sherry::GemvCall c{codes, scales, nullptr, y, N, K, x};
+    return sherry::gemv_launch(&c, 1, B, false, workspace, workspace_bytes,
+                               reinterpret_cast<cudaStream_t>(stream), sherry::kBoth);
+}
+
+extern "C" sherry_status sherry_gemv_bf16_grouped(const sherry_gemv_bf16_desc *descs, int count,
+                                                  int B, void *workspace, size_t workspace_bytes,
+                                                  sherry_stream_t stream) {
+    return sherry::grouped_bf16(descs, count, B, workspace, workspace_bytes,
+                                reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" sherry_status sherry_quantize_act(const uint16_t *x, int64_t B, int64_t K, int8_t *q,
+                                             float *s, sherry_stream_t stream) {
+    using namespace sherry;
+    if (!x || !q || !s) return SHERRY_ERR_NULL;
+    if (B < 1 || K < 8 || K % 8 != 0) return SHERRY_ERR_SHAPE;
+    if (B > 0x7FFFFFFF || K > 0x7FFFFFFF) return SHERRY_ERR_UNSUPPORTED;
+    if (!aligned(x, 16) || !aligned(q, 4) || !aligned(s, 4)) return SHERRY_ERR_ALIGN;
+    const int blocks = (int)((B + 7) / 8);
+    quantize_act_kernel<<<blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, (int)B, (int)K,
+                                                                                    q, s);
+    return launch_status("sherry_quantize_act");
 }
 
 // ---------------------------------------------------------------------------
@@ -1184,7 +1319,7 @@ extern "C" sherry_status sherry_gemv_static(const uint32_t *codes, const float *
     void *scratch = nullptr;
     const sherry_status st = static_scratch(&scratch);
     if (st != SHERRY_OK) return st;
-    const GemvCall c{codes, scales, x, y, N, K};
+    const GemvCall c{codes, scales, x, y, N, K, nullptr};
     return gemv_launch(&c, 1, B, false, scratch, SHERRY_STATIC_SCRATCH_BYTES,
                        reinterpret_cast<cudaStream_t>(stream), kBoth);
 }

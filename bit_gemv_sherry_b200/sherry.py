@@ -62,6 +62,10 @@ def lib():
         "sherry_gemv": ([p, p, p, p, i64, i64, i32, p, sz, p], i32),
         "sherry_gemv_acc": ([p, p, p, i64, i64, i32, p, sz, p], i32),
         "sherry_gemv_static": ([p, p, p, p, i64, i64, i32, p], i32),
+        "sherry_quantize_act": ([p, i64, i64, p, p, p], i32),
+        "sherry_gemv_bf16_workspace_bytes": ([i64, i64, i32], sz),
+        "sherry_gemv_bf16": ([p, p, p, p, i64, i64, i32, p, sz, p], i32),
+        "sherry_gemv_bf16_grouped": ([p, i32, i32, p, sz, p], i32),
         "sherry_gemv_grouped": ([p, i32, i32, p, sz, p], i32),
         "sherry_gemv_prepare": ([p, i32, i32, p, sz, p], i32),
         "sherry_gemv_run": ([p, i32, i32, p, sz, p], i32),
@@ -222,6 +226,61 @@ def gemv_grouped(items, B, ws=None):
     ws = workspace(total, dev) if ws is None else ws
     _check(lib().sherry_gemv_grouped(ctypes.cast(descs, ctypes.c_void_p), n, B, _ptr(ws),
                                      ws.numel(), _stream(items[0][2])), "sherry_gemv_grouped")
+
+
+def quantize_act(x, q=None, s=None):
+    """Per-token absmax int8 quantization of bf16 activations x [B, K]:
+    returns (q int8 [B, K], s fp32 [B]) with x ~ s[:, None] * q."""
+    _need(x, torch.bfloat16, "x")
+    x2 = x.view(1, -1) if x.dim() == 1 else x
+    B, K = x2.shape
+    if q is None:
+        q = torch.empty((B, K), dtype=torch.int8, device=x.device)
+    if s is None:
+        s = torch.empty((B,), dtype=torch.float32, device=x.device)
+    _check(lib().sherry_quantize_act(_ptr(x2), B, K, _ptr(q), _ptr(s), _stream(x)),
+           "sherry_quantize_act")
+    return q, s
+
+
+def gemv_bf16_workspace_bytes(N, K, B):
+    return int(lib().sherry_gemv_bf16_workspace_bytes(N, K, B))
+
+
+def gemv_bf16(codes, scales, x, y=None, ws=None):
+    """y[B, N] = scales * s_x * (W . q^T) for bf16 activations x [B, K] quantized per token."""
+    _need(scales, torch.float32, "scales")
+    N, K = _codes_shape(codes, scales.numel())
+    _need(x, torch.bfloat16, "x")
+    x2 = x.view(1, -1) if x.dim() == 1 else x
+    B = x2.shape[0]
+    if y is None:
+        y = torch.empty((B, N), dtype=torch.float32, device=x.device)
+    nb = gemv_bf16_workspace_bytes(N, K, B)
+    ws = workspace(nb, x.device) if ws is None else ws
+    _check(lib().sherry_gemv_bf16(_ptr(codes), _ptr(scales), _ptr(x2), _ptr(y), N, K, B, _ptr(ws),
+                                  ws.numel(), _stream(x)), "sherry_gemv_bf16")
+    return y
+
+
+def gemv_bf16_grouped(items, B, ws=None):
+    """items: list of (codes, scales, x bf16 [B, K], y [B, N]); one pass over all GEMVs."""
+    n = len(items)
+    descs = (GemvDesc * n)()  # same field layout as sherry_gemv_bf16_desc
+    total = 0
+    dev = None
+    for i, (codes, scales, x, y) in enumerate(items):
+        _need(scales, torch.float32, "scales")
+        N, K = _codes_shape(codes, scales.numel())
+        _need(x, torch.bfloat16, "x")
+        _need(y, torch.float32, "y")
+        descs[i] = GemvDesc(codes.data_ptr(), scales.data_ptr(), x.data_ptr(), y.data_ptr(), N, K)
+        total += gemv_bf16_workspace_bytes(N, K, B)
+        dev = x.device
+    ws = workspace(total, dev) if ws is None else ws
+    _check(lib().sherry_gemv_bf16_grouped(ctypes.cast(descs, ctypes.c_void_p), n, B, _ptr(ws),
+                                          ws.numel(), _stream(items[0][2])),
+           "sherry_gemv_bf16_grouped")
 
 
 class GroupedGemv:

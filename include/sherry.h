@@ -145,6 +145,54 @@ sherry_status sherry_gemv_acc(const uint32_t *codes, const int8_t *x, int32_t *a
                               size_t workspace_bytes, sherry_stream_t stream);
 
 /*
+ * Activation front-end.  The method is served as W1.25A8 (1.25-bit weights,
+ * int8 activations: arXiv 2601.07892, abstract); the pages do not say how the
+ * int8 activations are produced.  Reading taken here: per token (batch row) b
+ *     amax_b = max_k |x[b][k]|,   s_b = amax_b / 127,
+ *     q[b][k] = clamp(rint(x[b][k] * (127 / amax_b)), -127, 127),
+ * every operation in fp32 with round-to-nearest-even; amax_b = 0 gives s_b = 0
+ * and q = 0.  x is bf16 (uint16 bit patterns: the upper half of an fp32).
+ *
+ * sherry_quantize_act -- the front-end alone.
+ *   x  [B][K] bf16, row-major, device, 16-byte aligned, K a multiple of 8.
+ *   q  [B][K] int8 output, 4-byte aligned.   s  [B] fp32 output.
+ * Errors: NULL, SHAPE, ALIGN, UNSUPPORTED, CUDA.
+ */
+sherry_status sherry_quantize_act(const uint16_t *x, int64_t B, int64_t K, int8_t *q, float *s,
+                                  sherry_stream_t stream);
+
+/*
+ * sherry_gemv_bf16 -- the decode GEMV on bf16 activations: the re-order launch
+ * quantizes each token as sherry_quantize_act does (keeping s_b in the
+ * workspace) and the GEMV scales by both the weight and the activation scale:
+ *   y[b][n] = fl32(fl32(s[n] * s_b) * acc[b][n]),  acc = W . q^T exactly.
+ *   x  [B][K] bf16, 16-byte aligned; other arguments as sherry_gemv.
+ *   workspace: sherry_gemv_bf16_workspace_bytes(N, K, B) bytes (a grouped call:
+ *   the sum over its GEMVs, in descriptor order), 256-byte aligned.
+ * Errors: as sherry_gemv.
+ */
+size_t sherry_gemv_bf16_workspace_bytes(int64_t N, int64_t K, int B);
+sherry_status sherry_gemv_bf16(const uint32_t *codes, const float *scales, const uint16_t *x,
+                               float *y, int64_t N, int64_t K, int B, void *workspace,
+                               size_t workspace_bytes, sherry_stream_t stream);
+
+/* One GEMV of a grouped bf16 call (device pointers). */
+typedef struct {
+    const uint32_t *codes;
+    const float *scales;
+    const uint16_t *x;  /* [B][K] bf16 */
+    float *y;           /* [B][N] */
+    int64_t N;
+    int64_t K;
+} sherry_gemv_bf16_desc;
+
+/* sherry_gemv_bf16 over `count` GEMVs with the same B in one pass (one
+ * re-order launch and one GEMV launch), as sherry_gemv_grouped. */
+sherry_status sherry_gemv_bf16_grouped(const sherry_gemv_bf16_desc *descs, int count, int B,
+                                       void *workspace, size_t workspace_bytes,
+                                       sherry_stream_t stream);
+
+/*
  * sherry_gemv_static -- sherry_gemv without a caller workspace: the call
  * allocates nothing.  The paper has no counterpart; this entry point exists
  * for callers that may not allocate device memory on their decode path.

@@ -91,6 +91,23 @@ def test_gemv_static_argument_checks():
     assert b"4194304" in L.sherry_last_error()
 
 
+def test_activation_front_end_argument_checks():
+    L = S.lib()
+    assert L.sherry_quantize_act(None, 1, 128, FAKE, FAKE, None) == 1
+    assert L.sherry_quantize_act(FAKE, 1, 12, FAKE, FAKE, None) == 2        # K % 8
+    assert L.sherry_quantize_act(FAKE, 0, 128, FAKE, FAKE, None) == 2
+    assert L.sherry_quantize_act(ctypes.c_void_p(0x100008), 1, 128, FAKE, FAKE, None) == 3
+    ws = 1 << 20
+    assert L.sherry_gemv_bf16(FAKE, FAKE, None, FAKE, 4, 128, 1, FAKE_WS, ws, None) == 1
+    assert L.sherry_gemv_bf16(FAKE, FAKE, ctypes.c_void_p(0x100008), FAKE, 4, 128, 1, FAKE_WS, ws,
+                              None) == 3                                  # bf16 x: 16-byte aligned
+    assert L.sherry_gemv_bf16(FAKE, FAKE, FAKE, FAKE, 4, 128, 17, FAKE_WS, ws, None) == 4
+    # the activation scales take 64 more words than the int8 workspace
+    assert S.gemv_bf16_workspace_bytes(2048, 2048, 1) == S.gemv_workspace_bytes(2048, 2048, 1) + 256
+    assert L.sherry_gemv_bf16(FAKE, FAKE, FAKE, FAKE, 4, 1024, 2, FAKE_WS,
+                              S.gemv_workspace_bytes(4, 1024, 2), None) == 7
+
+
 def test_grouped_argument_checks():
     L = S.lib()
     d = (S.GemvDesc * 2)()

@@ -1,0 +1,74 @@
+"""GPU parity of the activation front-end (bf16 -> per-token int8) and of the
+GEMV on bf16 activations, through the C ABI, against the oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from bit_gemv_sherry_b200 import sherry as S
+from tests.gpu_helpers import dev, dev_codes
+
+pytestmark = pytest.mark.gpu
+
+
+def bf16_rows(B, K, seed):
+    """Seeded bf16 bit patterns: normal rows of very different magnitudes, an
+    all-zero row, and a row of hand values with exact rounding ties."""
+    rng = np.random.default_rng(seed)
+    mags = np.array([1.0, 1e-3, 37.0, 2e4, 0.25, 3.0], np.float32)
+    x = rng.standard_normal((B, K)).astype(np.float32) * mags[np.arange(B) % len(mags)][:, None]
+    bits = (x.view(np.uint32) >> 16).astype(np.uint16)
+    if B >= 2:
+        bits[1] = 0
+    if B >= 3 and K >= 8:
+        bits[2, :8] = oracle.bf16_bits([127.0, 1.0, -0.5, 0.25, -127.0, 63.5, 0.0, 126.5])
+        bits[2, 8:] = 0
+    return bits
+
+
+def to_bf16(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda().view(torch.bfloat16)
+
+
+@pytest.mark.parametrize("B,K", [(1, 128), (3, 2048), (16, 1024), (5, 8), (2, 8192)])
+def test_quantize_act_matches_oracle(B, K):
+    bits = bf16_rows(B, K, seed=30 + B)
+    q_ref, s_ref = oracle.quantize_act(bits)
+    q, s = S.quantize_act(to_bf16(bits))
+    assert np.array_equal(q.cpu().numpy(), q_ref)
+    assert np.array_equal(s.cpu().numpy(), s_ref)
+
+
+@pytest.mark.parametrize("N,K,B", [(256, 1024, 1), (100, 3072, 2), (70, 2048, 5), (37, 640, 3),
+                                   (48, 8192, 16), (31, 8192, 1)])
+def test_gemv_bf16_matches_oracle(N, K, B):
+    codes, scales = oracle.pack(synth.latent_weights(N, K, seed=40 + N))
+    bits = bf16_rows(B, K, seed=50 + B)
+    q_ref, s_ref = oracle.quantize_act(bits)
+    acc = oracle.gemv_acc(codes, q_ref, N, K)
+    # one fp32 rounding for s_w * s_b, one for the product with the exact acc
+    expect = (scales[None, :] * s_ref[:, None]).astype(np.float32) * acc.astype(np.float32)
+    y = S.gemv_bf16(dev_codes(codes), dev(scales), to_bf16(bits)).cpu().numpy()
+    assert np.array_equal(y, expect.astype(np.float32))
+    ref = oracle.gemv_act(codes, scales, q_ref, s_ref, K)
+    rel = np.abs(y.astype(np.float64) - ref) / np.maximum(np.abs(ref), 1e-300)
+    rel[(ref == 0) & (y == 0)] = 0.0
+    assert rel.max() <= 1e-6
+
+
+def test_gemv_bf16_grouped_equals_single_calls():
+    dev_ = torch.device("cuda")
+    items, singles = [], []
+    for i, (name, n, k) in enumerate(synth.LLAMA_1B_LAYERS):
+        w = torch.from_numpy(synth.latent_weights(n, k, seed=60 + i)).to(dev_)
+        c, s = S.pack(w)
+        x = to_bf16(bf16_rows(1, k, seed=70 + i))
+        y = torch.empty((1, n), dtype=torch.float32, device=dev_)
+        items.append((c, s, x, y))
+        singles.append(S.gemv_bf16(c, s, x))
+    S.gemv_bf16_grouped(items, 1)
+    torch.cuda.synchronize()
+    for (_, _, _, y), ref in zip(items, singles):
+        assert torch.equal(y, ref)
+    assert S.device_error() == 0
