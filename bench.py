@@ -38,8 +38,8 @@ METRIC = "W1.25A8 GEMV weight GB/s at batch 1 (LLaMA-3.2-1B decode stack)"
 UNIT = "GB/s"
 L2_BYTES = 126 * 2 ** 20
 # ncu capture of gemv_dot_kernel<1,false> on the 16-layer stack, B = 1:
-# dram read 154,064,896 + write 4,563,712 bytes per launch
-NCU_TRAFFIC_BYTES = 154064896 + 4563712
+# dram read 154,071,552 + write 3,885,824 bytes per launch
+NCU_TRAFFIC_BYTES = 154071552 + 3885824
 
 
 def parse_args():
@@ -295,6 +295,29 @@ def time_layers(layers, xs, S, torch, dev, flush, reps=20):
     return res
 
 
+def time_bf16_stack(layers, S, torch, dev, reps=200):
+    """The same stack with bf16 activations: each step quantizes every GEMV's
+    activations per token (fused into the re-order launch) and runs the GEMVs."""
+    gen = torch.Generator(device="cpu").manual_seed(3)
+    xb = {k: torch.randn((1, k), generator=gen).to(torch.bfloat16).to(dev) for k in (2048, 8192)}
+    ys = [torch.empty((1, n), dtype=torch.float32, device=dev) for _, _, n, _, _, _ in layers]
+    items = [(codes, scales, xb[k], y) for (_, _, n, k, codes, scales), y in zip(layers, ys)]
+    step = S.GroupedGemvBf16(items, B=1)
+    for _ in range(5):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        step()
+    e1.record()
+    e1.synchronize()
+    t = e0.elapsed_time(e1) / 1e3 / reps
+    code_bytes = sum(codes.numel() * 4 for _, _, _, _, codes, _ in layers)
+    return {"us_per_step": t * 1e6, "weight_gbs": code_bytes / t / 1e9, "steps": reps,
+            "note": "bf16 activations quantized per token inside the step (x seed 3)"}
+
+
 def cpu_baseline(layers, xs_host, seconds):
     """The oracle, as it stands, on a bounded sample of the stack (host cores)."""
     import oracle
@@ -499,6 +522,7 @@ def main():
         torch.cuda.empty_cache()
         line["gemm"] = time_gemm(S, torch, dev, flush)
         line["gemv_layers_l2_flushed"] = time_layers(layers, xs, S, torch, dev, flush)
+        line["gemv_bf16_stack"] = time_bf16_stack(layers, S, torch, dev)
         if world == 1:
             line["cpu_baseline"] = cpu_baseline(layers, xs_host, args.cpu_seconds)
     err = S.device_error()
