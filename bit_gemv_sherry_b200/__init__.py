@@ -4,7 +4,7 @@ The compute path lives in ``libsherry.so`` (``csrc/``, header ``include/sherry.h
 ``sherry`` is its thin Python binding.
 """
 from .sherry import (  # noqa: F401
-    GroupedGemv, SherryError, codes_shape, device_error, gemm, gemm_acc, gemv, gemv_acc, gemv_grouped,
+    GroupedGemv, GroupedGemvBf16, SherryError, codes_shape, device_error, gemm, gemm_acc, gemv, gemv_acc, gemv_grouped,
     gemv_static, quantize_act, gemv_bf16, gemv_bf16_grouped, gemv_bf16_workspace_bytes,
     gemv_workspace_bytes, lib, library_path, pack, packed_bytes, workspace,
 )

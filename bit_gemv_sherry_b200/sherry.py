@@ -324,6 +324,35 @@ class GroupedGemv:
         _check(lib().sherry_gemv_run(*self.args, s), "sherry_gemv_run")
 
 
+class GroupedGemvBf16:
+    """Pre-marshalled grouped GEMV on bf16 activations (sherry_gemv_bf16_grouped):
+    items are (codes, scales, x bf16 [B, K], y [B, N])."""
+
+    def __init__(self, items, B, ws=None):
+        n = len(items)
+        self.descs = (GemvDesc * n)()  # same field layout as sherry_gemv_bf16_desc
+        total = 0
+        for i, (codes, scales, x, y) in enumerate(items):
+            _need(scales, torch.float32, "scales")
+            N, K = _codes_shape(codes, scales.numel())
+            _need(x, torch.bfloat16, "x")
+            _need(y, torch.float32, "y")
+            self.descs[i] = GemvDesc(codes.data_ptr(), scales.data_ptr(), x.data_ptr(),
+                                     y.data_ptr(), N, K)
+            total += gemv_bf16_workspace_bytes(N, K, B)
+        self.items = items
+        dev = items[0][2].device
+        self.ws = torch.empty(max(total, 256), dtype=torch.uint8, device=dev) if ws is None else ws
+        self.args = (ctypes.cast(self.descs, ctypes.c_void_p), n, B, _ptr(self.ws),
+                     self.ws.numel())
+        self.device = dev
+
+    def __call__(self, stream=None):
+        s = ctypes.c_void_p(stream if stream is not None
+                            else torch.cuda.current_stream(self.device).cuda_stream)
+        _check(lib().sherry_gemv_bf16_grouped(*self.args, s), "sherry_gemv_bf16_grouped")
+
+
 def gemm(codes, scales, x, y=None):
     """y[M, N] = scales * (x . W^T); x int8 [M, K]."""
     _need(scales, torch.float32, "scales")
