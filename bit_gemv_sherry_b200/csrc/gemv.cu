@@ -833,7 +833,7 @@ __global__ void __launch_bounds__(kDotThreads, DotShape<NBX>::kMinBlocks)
             issue(slot == 0 ? kDotRing - 1 : slot - 1);
             const uint32_t *st = ring + slot * SW;
             slot = (slot + 1 == kDotRing) ? 0 : slot + 1;
-#pragma unroll 1
+#pragma unroll
             for (int tt = 0; tt < kChunkTiles; tt++) {
                 const uint32_t *cw = st + tt * kTileWords + lane;
                 TileDecoder6 d;
