@@ -743,7 +743,8 @@ __global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
 //     loads and each lane ends with its row's complete sum (no reduction);
 //   * the unit's chunks (2560 contiguous bytes) and the chunk's re-ordered
 //     activations (128 words per batch row) stream through a private
-//     3-stage cp.async ring; the activation words are the same for all lanes
+//     2-stage cp.async ring (one chunk in flight while one is consumed, 32
+//     warps per SM); the activation words are the same for all lanes
 //     (broadcast reads);
 //   * each decoded word (four ternary bytes) meets its activation word in one
 //     dp4a, so a batch row costs 32 dp4a per tile: for B <= 2 this is cheaper
@@ -752,13 +753,13 @@ __global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
 // ---------------------------------------------------------------------------
 constexpr int kDotThreads = 256;
 constexpr int kDotWarps = kDotThreads / 32;
-constexpr int kDotRing = 3;
+constexpr int kDotRing = 2;  // 2 stages x 8 warps: 49 KB per CTA, 4 CTAs (32 warps) per SM
 constexpr int kDotCodeWords = kChunkTiles * kTileWords;  // 640
 template <int NBX>
 struct DotShape {
     static constexpr int kStageWords = kDotCodeWords + NBX * kChunkTiles * 32;
     static constexpr size_t kSmem = (size_t)kDotWarps * kDotRing * kStageWords * 4;
-    static constexpr int kMinBlocks = NBX == 1 ? 3 : 2;
+    static constexpr int kMinBlocks = NBX == 1 ? 4 : 2;
 };
 
 template <int NBX, bool ACC_OUT>
