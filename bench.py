@@ -295,6 +295,41 @@ def time_layers(layers, xs, S, torch, dev, flush, reps=20):
     return res
 
 
+def time_3b_layer(S, torch, dev, flush, reps=10):
+    """One LLaMA-3.2-3B-shaped layer (7 projections, one grouped call) at
+    B = 1, 4, 16 with int8 activations (seeds 1, 2, 3), L2 flushed before each
+    call."""
+    items_w = []
+    for pi, (name, n, k) in enumerate(synth.LLAMA_3B_LAYERS):
+        w = torch.from_numpy(synth.latent_weights(n, k, seed=synth.layer_seed(0, pi))).to(dev)
+        codes, scales = S.pack(w)
+        del w
+        items_w.append((n, k, codes, scales))
+    code_bytes = sum(c.numel() * 4 for _, _, c, _ in items_w)
+    out = {}
+    for B, seed in ((1, 1), (4, 2), (16, 3)):
+        xs = {k: torch.from_numpy(synth.int8_uniform((B, k), seed=seed)).to(dev)
+              for k in {k for _, k, _, _ in items_w}}
+        ys = [torch.empty((B, n), dtype=torch.float32, device=dev) for n, _, _, _ in items_w]
+        step = S.GroupedGemv([(c, s, xs[k], y) for (n, k, c, s), y in zip(items_w, ys)], B=B)
+        for _ in range(3):
+            step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ts = []
+        for _ in range(reps):
+            flush()
+            e0.record()
+            step()
+            e1.record()
+            e1.synchronize()
+            ts.append(e0.elapsed_time(e1) / 1e3)
+        t = statistics.median(ts)
+        out["B%d" % B] = {"us": t * 1e6, "weight_gbs": code_bytes / t / 1e9}
+    out["code_bytes"] = code_bytes
+    return out
+
+
 def time_bf16_stack(layers, S, torch, dev, reps=200):
     """The same stack with bf16 activations: each step quantizes every GEMV's
     activations per token (fused into the re-order launch) and runs the GEMVs."""
@@ -523,6 +558,7 @@ def main():
         line["gemm"] = time_gemm(S, torch, dev, flush)
         line["gemv_layers_l2_flushed"] = time_layers(layers, xs, S, torch, dev, flush)
         line["gemv_bf16_stack"] = time_bf16_stack(layers, S, torch, dev)
+        line["gemv_3b_layer_l2_flushed"] = time_3b_layer(S, torch, dev, flush)
         if world == 1:
             line["cpu_baseline"] = cpu_baseline(layers, xs_host, args.cpu_seconds)
     err = S.device_error()

@@ -81,7 +81,7 @@ struct XprepDesc {
     int K;
     int Tp;
     int unit_begin;       // first work unit of this GEMV
-    int xunits;           // int8: B * Tp (batch row, tile) units; bf16: B row units
+    int xunits;           // int8: B * Tp (batch row, tile) units; bf16: (row, 4 tiles) units
     int zero_words;       // words at `zero` (0 if the rows are not split)
     int kind;             // 0: int8 activations, 1: bf16 activations quantized here
 };
@@ -201,6 +201,8 @@ __device__ __forceinline__ float row_absmax_bf16(const uint16_t *row, int K, int
     return m;
 }
 
+constexpr int kXqTiles = 4;  // tiles per bf16 quantize unit
+
 __global__ void __launch_bounds__(256) xprep_kernel(const __grid_constant__ XprepParams P) {
     pdl_allow_dependents();
     const int lane = threadIdx.x & 31;
@@ -214,14 +216,18 @@ __global__ void __launch_bounds__(256) xprep_kernel(const __grid_constant__ Xpre
         const XprepDesc &D = P.d[lo];
         const int local = u - D.unit_begin;
         if (local < D.xunits && D.kind == 1) {
-            // bf16 row b: absmax, then quantize and re-order tile by tile
-            const int b = local;
+            // bf16: unit = (row b, kXqTiles tiles); every unit of a row computes the
+            // row's absmax (the row is re-read from L2), then quantizes and re-orders
+            // its own tiles; the row's first unit stores the activation scale
+            const int per_row = (D.Tp + kXqTiles - 1) / kXqTiles;
+            const int b = local / per_row, g = local - b * per_row;
             const int T = D.K / SHERRY_TILE_K;
             const uint16_t *row = D.xbf + (size_t)b * D.K;
             const float amax = row_absmax_bf16(row, D.K, lane);
             const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
-            if (lane == 0) D.xscale[b] = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
-            for (int t = 0; t < D.Tp; t++) {
+            if (lane == 0 && g == 0) D.xscale[b] = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
+            const int t_end = min(D.Tp, (g + 1) * kXqTiles);
+            for (int t = g * kXqTiles; t < t_end; t++) {
                 uint32_t raw = 0u;
                 if (t < T)
                     raw = quant_word(__ldg(reinterpret_cast<const uint2 *>(row + (size_t)t * SHERRY_TILE_K) + lane),
@@ -1076,7 +1082,7 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
         X.K = (int)c.K;
         X.Tp = Tp;
         X.unit_begin = wb;
-        X.xunits = bf ? B : B * Tp;
+        X.xunits = bf ? B * ((Tp + kXqTiles - 1) / kXqTiles) : B * Tp;
         X.zero_words = (int)split_words(c.N, c.K, B);
         X.kind = bf ? 1 : 0;
         GemvDesc &D = gp.d[i];
