@@ -53,7 +53,8 @@ struct GemvDesc {
     int kparts;           // pipelined kernel: K-parts per unit
     int cpp;              // pipelined kernel: chunks per K-part
     int item_begin;       // pipelined kernel: first (unit, K-part) item in the group
-    int chunk_begin;      // pipelined kernel: balancing position of the first item
+    int chunk_begin;      // pipelined kernel: first 4-tile chunk of the group (all groups' rows
+                          // in order, each row's K-parts in order)
 };
 
 struct GemvParams {
@@ -61,14 +62,14 @@ struct GemvParams {
     int B;
     int total_units16;    // register kernel
     int total_items;      // pipelined kernel
-    int total_chunks;     // pipelined kernel: balancing space
+    int total_chunks;     // pipelined kernel: chunks of all groups (the balancing space)
     // Constants passed at run time so that they live in registers instead of
-    // being re-created per use, and so that shifts by a power of two stay
-    // multiplications (IMAD / IMAD.HI on the FMA pipe) instead of ALU shifts.
+    // being re-created per use, and so that left shifts by a power of two stay
+    // multiplications (IMAD on the FMA pipe) instead of ALU shifts.
     uint32_t mul4, mul2;          // 4, 2
-    uint32_t hi1, hi2, hi16;      // 2^31, 2^30, 2^16: mul.hi gives >> 1, >> 2, >> 16
     uint32_t m33, m55, m44;       // masks
     uint32_t tlo[4], thi[4];      // PRMT byte tables of the four positions
+    uint32_t f16one, f16negz;     // fp16x2 1.0 and -0.0 (high-half copy, see hi_half)
     GemvDesc d[SHERRY_MAX_GROUP];
 };
 
@@ -158,10 +159,14 @@ __device__ __forceinline__ uint32_t reorder_word(uint32_t raw, int lane) {
     return prmt(prmt(v0, v1, pick2), prmt(v2, v3, pick2), 0x5410u);
 }
 
-// Programmatic dependent launch: the GEMV kernels are launched so that they may
-// start while the re-order kernel before them still runs; they wait for it
-// (griddepcontrol.wait: the prior grid completed and its writes are visible)
-// before reading anything it writes.  Without a prior grid the wait returns.
+// Programmatic dependent launch: the re-order and GEMV kernels are launched so
+// that they may start while the kernel before them in the stream still runs.
+// Each waits for it (griddepcontrol.wait: the prior grid completed and its
+// writes are visible) before reading or writing anything that grid may touch;
+// without a prior grid the wait returns.  Each lets its own dependents be
+// scheduled from its start (griddepcontrol.launch_dependents), which only
+// moves their launch work under this grid's tail: they still wait for its
+// completion.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_allow_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -205,6 +210,7 @@ constexpr int kXqTiles = 4;  // tiles per bf16 quantize unit
 
 __global__ void __launch_bounds__(256) xprep_kernel(const __grid_constant__ XprepParams P) {
     pdl_allow_dependents();
+    pdl_wait();  // x may come from the kernel before; the last GEMV may still read xw
     const int lane = threadIdx.x & 31;
     const int nw = gridDim.x * (blockDim.x >> 5);
     for (int u = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); u < P.total_units; u += nw) {
@@ -302,11 +308,6 @@ __device__ __forceinline__ uint32_t imul(uint32_t a, uint32_t b) {
     return d;
 }
 
-__device__ __forceinline__ uint32_t imulhi(uint32_t a, uint32_t b) {
-    uint32_t d;
-    asm("mul.hi.u32 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
-}
 
 // Scale of output (row, batch row b): s[row], times the activation scale of b
 // when the activations came through the bf16 front-end (one fp32 rounding).
@@ -316,16 +317,14 @@ __device__ __forceinline__ float out_scale(const GemvDesc &D, int row, int b) {
 }
 
 struct Consts {
-    uint32_t mul4, mul2, hi1, hi2, hi16, m33, m55, m44;
+    uint32_t mul4, mul2, m33, m55, m44;
     uint32_t tlo[4], thi[4];
+    uint32_t f16one, f16negz;
 };
 
 __device__ __forceinline__ void load_consts(const GemvParams &P, Consts &C) {
     C.mul4 = P.mul4;
     C.mul2 = P.mul2;
-    C.hi1 = P.hi1;
-    C.hi2 = P.hi2;
-    C.hi16 = P.hi16;
     C.m33 = P.m33;
     C.m55 = P.m55;
     C.m44 = P.m44;
@@ -334,15 +333,34 @@ __device__ __forceinline__ void load_consts(const GemvParams &P, Consts &C) {
         C.tlo[i] = P.tlo[i];
         C.thi[i] = P.thi[i];
     }
+    C.f16one = P.f16one;
+    C.f16negz = P.f16negz;
+}
+
+// High half of a selector word, moved to the low half for the next PRMT (which
+// reads selector bits 0..15 only).  Done as one fp16x2 FMA whose first operand
+// takes the high half in both lanes: h * 1.0 + (-0.0) = h exactly for every
+// finite h, subnormals included (no .ftz).  A selector nibble never has bit 3
+// set, so bit 11 of the half is clear, its exponent field is never all ones,
+// and h is never NaN or Inf.  The FMA runs on the FMA-lite pipe, which the
+// rest of the decode leaves idle, instead of taking an ALU shift or a two-
+// instruction mul.hi on the heavy FMA pipe.
+__device__ __forceinline__ uint32_t hi_half(const Consts &C, uint32_t sel) {
+    uint32_t d;
+    asm("{\n\t.reg .b16 l, h;\n\t.reg .b32 t;\n\t"
+        "mov.b32 {l, h}, %1;\n\tmov.b32 t, {h, h};\n\t"
+        "fma.rn.f16x2 %0, t, %2, %3;\n\t}"
+        : "=r"(d)
+        : "r"(sel), "r"(C.f16one), "r"(C.f16negz));
+    return d;
 }
 
 // Per-row tile state of the pipelined kernel: zero-position nibbles per block
 // group and the four per-position sign planes.  Selector of (i, beta):
 //   zm[beta] | (sign plane i moved so block 4k+beta's bit lands at 4k+2) & 0x44444444.
-// Work split: masks, merges and permutes on the ALU pipe (2 cycles per warp
-// instruction); left shifts on the FMA pipe as IMAD (2 cycles); right shifts
-// are split between the ALU (SHF, 2 cycles) and the FMA pipe (IMAD.HI, which
-// takes 4 cycles there), so that neither pipe carries them all.
+// Work split: masks, merges, permutes and right shifts on the ALU pipe (2
+// cycles per warp instruction); left shifts on the heavy FMA pipe as IMAD (2
+// cycles); the selectors' high halves on the FMA-lite pipe (hi_half).
 struct TileDecoder6 {
     uint32_t zm[4];
     uint32_t sg[4];
@@ -366,7 +384,7 @@ struct TileDecoder6 {
     __device__ __forceinline__ uint32_t sel(const Consts &C, int i, int beta) const {
         const uint32_t v = beta == 0 ? imul(sg[i], C.mul4)
                          : beta == 1 ? imul(sg[i], C.mul2)
-                         : beta == 2 ? sg[i] : imulhi(sg[i], C.hi1);
+                         : beta == 2 ? sg[i] : (sg[i] >> 1);
         return lop_or_masked(v, C.m44, zm[beta]);
     }
 };
@@ -379,6 +397,7 @@ struct TileDecoder6 {
 // NB = number of 8-row batch groups (1: B <= 8, 2: B <= 16).
 template <int NB, bool ACC_OUT>
 __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const __grid_constant__ GemvParams P) {
+    pdl_allow_dependents();
     pdl_wait();
     const int lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
@@ -517,19 +536,29 @@ __device__ __forceinline__ int find_desc_by_item(const GemvParams &P, int item) 
     return lo;
 }
 
-// First item whose balancing position is >= c (total_items if none).
-__device__ __forceinline__ int first_item_at_or_after(const GemvParams &P, int c) {
-    if (c >= P.total_chunks) return P.total_items;
+// Chunk space: the 4-tile chunks of all groups, group by group, each group's
+// 32-row units in order and each unit's chunks in K order.  An item (unit,
+// K-part kp) holds chunks kp*cpp .. min(nchunk, kp*cpp + cpp) - 1 of its unit.
+__device__ __forceinline__ int desc_by_chunk(const GemvParams &P, int c) {
     int lo = 0, hi = P.count - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
         if (P.d[mid].chunk_begin <= c) lo = mid; else hi = mid - 1;
     }
-    const GemvDesc &D = P.d[lo];
-    const int items = D.units * D.kparts;
-    const int k = (c - D.chunk_begin + D.cpp - 1) / D.cpp;
-    return k < items ? D.item_begin + k
-                     : (lo + 1 < P.count ? P.d[lo + 1].item_begin : P.total_items);
+    return lo;
+}
+
+// First item that starts at chunk c or later (total_items if none).
+__device__ __forceinline__ int first_item_at_or_after(const GemvParams &P, int c) {
+    if (c >= P.total_chunks) return P.total_items;
+    const int id = desc_by_chunk(P, c);
+    const GemvDesc &D = P.d[id];
+    const int rc = c - D.chunk_begin;
+    const int unit = rc / D.nchunk;
+    const int kp = (rc - unit * D.nchunk + D.cpp - 1) / D.cpp;  // kparts: the next unit
+    const int k = unit * D.kparts + kp;
+    return k < D.units * D.kparts ? D.item_begin + k
+                                  : (id + 1 < P.count ? P.d[id + 1].item_begin : P.total_items);
 }
 
 // (GEMV, unit, K-part) of an item, advanced item by item without searches or
@@ -537,14 +566,23 @@ __device__ __forceinline__ int first_item_at_or_after(const GemvParams &P, int c
 struct ItemCursor {
     int id, unit, kp;
 };
-__device__ __forceinline__ ItemCursor cursor_at(const GemvParams &P, int item) {
-    ItemCursor c;
-    c.id = find_desc_by_item(P, item);
-    const GemvDesc &D = P.d[c.id];
-    const int local = item - D.item_begin;
-    c.unit = local / D.kparts;
-    c.kp = local - c.unit * D.kparts;
-    return c;
+// The item holding chunk c (c < total_chunks), and the chunk it starts at.
+__device__ __forceinline__ ItemCursor cursor_at_chunk(const GemvParams &P, int c, int &start) {
+    ItemCursor r;
+    r.id = desc_by_chunk(P, c);
+    const GemvDesc &D = P.d[r.id];
+    const int rc = c - D.chunk_begin;
+    r.unit = rc / D.nchunk;
+    r.kp = (rc - r.unit * D.nchunk) / D.cpp;
+    start = D.chunk_begin + r.unit * D.nchunk + r.kp * D.cpp;
+    return r;
+}
+// First chunk of the item holding chunk c; total_chunks for c >= total_chunks.
+__device__ __forceinline__ int item_start_at_or_before(const GemvParams &P, int c) {
+    if (c >= P.total_chunks) return P.total_chunks;
+    int start;
+    cursor_at_chunk(P, c, start);
+    return start;
 }
 __device__ __forceinline__ void cursor_next(const GemvParams &P, ItemCursor &c) {
     if (++c.kp == P.d[c.id].kparts) {
@@ -562,6 +600,7 @@ __device__ __forceinline__ void cursor_next(const GemvParams &P, ItemCursor &c) 
 template <int NB, bool ACC_OUT>
 __global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
     gemv_pipe_kernel(const __grid_constant__ GemvParams P) {
+    pdl_allow_dependents();
     pdl_wait();
     extern __shared__ __align__(16) uint32_t pipe_smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -666,12 +705,10 @@ __global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
                         const int m = 4 * i + beta;  // MMA index: activation words 2m, 2m+1
                         const uint32_t s0 = d0.sel(C, i, beta);
                         const uint32_t s1 = d1.sel(C, i, beta);
-                        // high halves of the selectors by ALU shifts: the FMA pipe
-                        // already carries the decoder's IMAD work here
                         const uint32_t a0 = prmt(tlo, thi, s0);
-                        const uint32_t a2 = prmt(tlo, thi, s0 >> 16);
+                        const uint32_t a2 = prmt(tlo, thi, hi_half(C, s0));
                         const uint32_t a1 = prmt(tlo, thi, s1);
-                        const uint32_t a3 = prmt(tlo, thi, s1 >> 16);
+                        const uint32_t a3 = prmt(tlo, thi, hi_half(C, s1));
 #pragma unroll
                         for (int nb = 0; nb < NB; nb++) {
                             const uint4 &xx = xq[nb][(m >> 1) & 1];
@@ -744,93 +781,183 @@ __global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
 
 // ---------------------------------------------------------------------------
 // Small-batch kernel (B <= 2): dot products on the ALU/FMA pipes, no MMA.
-//   * one warp owns a (32-row unit, K-part) item at a time and lane l owns row
-//     l of the unit, so a tile's five words are five conflict-free shared
-//     loads and each lane ends with its row's complete sum (no reduction);
+//   * lane l owns row l of a 32-row unit, so a tile's five words are five
+//     conflict-free shared loads and each lane ends with its row's sum (no
+//     reduction across lanes);
+//   * work is split by chunk count.  Each CTA takes a run of whole items
+//     (unit, K-part) holding about 1/gridDim of the chunks, and its 8 warps
+//     split the run into equal chunk ranges, so no warp ends the launch with a
+//     whole extra item to do.  An item cut by a warp boundary is summed by the
+//     warps holding its pieces: later pieces leave their row sums in shared
+//     memory, and after one CTA barrier the warp holding the item's first
+//     chunk adds them and finishes the item;
 //   * the unit's chunks (2560 contiguous bytes) and the chunk's re-ordered
-//     activations (128 words per batch row) stream through a private
-//     2-stage cp.async ring (one chunk in flight while one is consumed, 32
+//     activations (128 words per batch row) stream through a private 2-stage
+//     cp.async ring per warp (one chunk in flight while one is consumed, 32
 //     warps per SM); the activation words are the same for all lanes
 //     (broadcast reads);
 //   * each decoded word (four ternary bytes) meets its activation word in one
 //     dp4a, so a batch row costs 32 dp4a per tile: for B <= 2 this is cheaper
 //     than an m16n8k32 MMA whose 8 columns would mostly be empty.
-// Items, K-parts and the split-K completion are those of the pipelined kernel.
+// K-parts and the split-K completion are those of the pipelined kernel.
 // ---------------------------------------------------------------------------
 constexpr int kDotThreads = 256;
 constexpr int kDotWarps = kDotThreads / 32;
-constexpr int kDotRing = 2;  // 2 stages x 8 warps: 49 KB per CTA, 4 CTAs (32 warps) per SM
+constexpr int kDotRing = 2;  // 2 stages x 8 warps: 50 KB per CTA, 4 CTAs (32 warps) per SM
 constexpr int kDotCodeWords = kChunkTiles * kTileWords;  // 640
 template <int NBX>
 struct DotShape {
     static constexpr int kStageWords = kDotCodeWords + NBX * kChunkTiles * 32;
-    static constexpr size_t kSmem = (size_t)kDotWarps * kDotRing * kStageWords * 4;
+    static constexpr int kRingWords = kDotWarps * kDotRing * kStageWords;
+    // after the rings: per warp, the row sums of a later piece of a cut item
+    // [warp][NBX][32] and the first chunk of that item [warp]
+    static constexpr size_t kSmem = ((size_t)kRingWords + kDotWarps * (NBX * 32 + 1)) * 4;
     static constexpr int kMinBlocks = NBX == 1 ? 4 : 2;
 };
+
+// Finishes an item: lane = row of the unit, v = the item's row sums.  A K-part
+// of a split row adds into the K-part sums; the last K-part to finish scales,
+// stores and clears them.
+template <int NBX, bool ACC_OUT>
+__device__ __forceinline__ void dot_finish(const GemvDesc &D, int unit, int B, int lane,
+                                           int (&v)[NBX]) {
+    const int N = D.N;
+    const int row = unit * kUnitRows + lane;
+    const bool rv = row < N;
+    bool finish = true;
+    if (D.kparts > 1) {
+        if (rv) {
+#pragma unroll
+            for (int b = 0; b < NBX; b++)
+                if (b < B) atomicAdd(D.part_acc + (size_t)b * N + row, v[b]);
+        }
+        __threadfence();
+        __syncwarp();
+        uint32_t done = 0;
+        if (lane == 0) done = atomicAdd(D.part_cnt + unit, 1u);
+        finish = __shfl_sync(0xFFFFFFFFu, done, 0) == (uint32_t)(D.kparts - 1);
+        if (finish) {
+            __threadfence();
+            if (rv) {
+#pragma unroll
+                for (int b = 0; b < NBX; b++) {
+                    if (b < B) {
+                        int32_t *pa = D.part_acc + (size_t)b * N + row;
+                        v[b] = __ldcg(pa);
+                        *pa = 0;
+                    }
+                }
+            }
+            if (lane == 0) D.part_cnt[unit] = 0u;
+        }
+    }
+    if (finish && rv) {
+        if (ACC_OUT) {
+#pragma unroll
+            for (int b = 0; b < NBX; b++)
+                if (b < B) static_cast<int32_t *>(D.out)[(size_t)b * N + row] = v[b];
+        } else {
+#pragma unroll
+            for (int b = 0; b < NBX; b++)
+                if (b < B)
+                    static_cast<float *>(D.out)[(size_t)b * N + row] = out_scale(D, row, b) * (float)v[b];
+        }
+    }
+}
 
 template <int NBX, bool ACC_OUT>
 __global__ void __launch_bounds__(kDotThreads, DotShape<NBX>::kMinBlocks)
     gemv_dot_kernel(const __grid_constant__ GemvParams P) {
-    pdl_wait();
+    pdl_allow_dependents();
     constexpr int SW = DotShape<NBX>::kStageWords;
     extern __shared__ __align__(16) uint32_t dot_smem[];
+    int *cut_sum = reinterpret_cast<int *>(dot_smem + DotShape<NBX>::kRingWords);
+    int *cut_start = cut_sum + kDotWarps * NBX * 32;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const long long nw = (long long)gridDim.x * kDotWarps;
-    const long long wg = (long long)blockIdx.x * kDotWarps + warp;
-    const int it_begin = first_item_at_or_after(P, (int)(wg * P.total_chunks / nw));
-    const int it_end = first_item_at_or_after(P, (int)((wg + 1) * P.total_chunks / nw));
-    if (it_begin >= it_end) return;
+    // chunk range [b0, b1) of this warp
+    const long long tc = P.total_chunks, nb = gridDim.x;
+    const int cta_lo = item_start_at_or_before(P, (int)(blockIdx.x * tc / nb));
+    const int cta_hi = item_start_at_or_before(P, (int)((blockIdx.x + 1) * tc / nb));
+    const long long len = cta_hi - cta_lo;
+    const int b0 = cta_lo + (int)(warp * len / kDotWarps);
+    const int b1 = cta_lo + (int)((warp + 1) * len / kDotWarps);
+    // -1: no cut item starts before b0; -2: empty range (skipped when summing)
+    if (lane == 0) cut_start[warp] = b0 < b1 ? -1 : -2;
     uint32_t *ring = dot_smem + (size_t)warp * kDotRing * SW;
     const uint32_t ring_addr = smem_u32(ring);
     Consts C;
     load_consts(P, C);
     const int B = P.B;
 
+    // the warp's items: from the one holding chunk b0, while they start before b1
+    int start = b1;
+    ItemCursor cur = {0, 0, 0};
+    if (b0 < b1) cur = cursor_at_chunk(P, b0, start);
+
     // ---- producer side: the issue cursor runs kDotRing-1 stages ahead ----
     // lane l copies 16-byte pieces l + 32 j (j = 0..4) of the chunk's codes and
-    // piece l of each batch row's 128 activation words
-    int iitem = it_begin;
-    ItemCursor icur = cursor_at(P, it_begin);
-    int ic = 0, ic_end = 0, iTp = 0;
+    // piece l of each batch row's 128 activation words.  Until pdl_wait() only
+    // codes are read: the activation words and the K-part sums belong to the
+    // re-order kernel before this one.
+    ItemCursor icur = cur;
+    int istart = start, ic = 0, ic_end = 0, iTp = 0;
     const uint32_t *isrc = nullptr, *ixw = nullptr;
     auto set_issue_item = [&]() {
         const GemvDesc &D = P.d[icur.id];
         isrc = D.codes + (size_t)icur.unit * D.T * kTileWords + 4 * lane;
         ixw = reinterpret_cast<const uint32_t *>(D.xw) + 4 * lane;
         iTp = D.Tp;
-        ic = icur.kp * D.cpp;
-        ic_end = min(D.nchunk, ic + D.cpp);
+        const int first = icur.kp * D.cpp;
+        ic = first + max(b0 - istart, 0);
+        ic_end = first + min(b1 - istart, min(D.cpp, D.nchunk - first));
     };
-    set_issue_item();
-    auto issue = [&](int slot) {
-        if (iitem < it_end) {
-            const uint32_t *src = isrc + (size_t)ic * kChunkTiles * kTileWords;
-            const uint32_t dst = ring_addr + (uint32_t)slot * SW * 4 + 16u * lane;
+    if (istart < b1) set_issue_item();
+    auto copy_codes = [&](int slot) {
+        const uint32_t *src = isrc + (size_t)ic * kChunkTiles * kTileWords;
+        const uint32_t dst = ring_addr + (uint32_t)slot * SW * 4 + 16u * lane;
 #pragma unroll
-            for (int j = 0; j < 5; j++) cp_async16(dst + 512u * j, src + 128 * j, 16u);
+        for (int j = 0; j < 5; j++) cp_async16(dst + 512u * j, src + 128 * j, 16u);
+    };
+    auto copy_x_and_advance = [&](int slot) {
+        const uint32_t dst = ring_addr + (uint32_t)slot * SW * 4 + 16u * lane;
 #pragma unroll
-            for (int b = 0; b < NBX; b++)
-                if (b < B)
-                    cp_async16(dst + 4u * kDotCodeWords + 512u * b,
-                               ixw + ((size_t)b * iTp + (size_t)kChunkTiles * ic) * 32, 16u);
-            if (++ic == ic_end && ++iitem < it_end) {
+        for (int b = 0; b < NBX; b++)
+            if (b < B)
+                cp_async16(dst + 4u * kDotCodeWords + 512u * b,
+                           ixw + ((size_t)b * iTp + (size_t)kChunkTiles * ic) * 32, 16u);
+        if (++ic == ic_end) {
+            const GemvDesc &D = P.d[icur.id];
+            istart += min(D.cpp, D.nchunk - icur.kp * D.cpp);
+            if (istart < b1) {
                 cursor_next(P, icur);
                 set_issue_item();
             }
         }
+    };
+    auto issue = [&](int slot) {
+        if (istart < b1) {
+            copy_codes(slot);
+            copy_x_and_advance(slot);
+        }
         cp_async_commit();
     };
-#pragma unroll
-    for (int s = 0; s < kDotRing - 1; s++) issue(s);
+    static_assert(kDotRing == 2, "the prologue fills one stage");
+    const bool first_copy = istart < b1;
+    if (first_copy) copy_codes(0);
+    pdl_wait();
+    if (first_copy) copy_x_and_advance(0);
+    cp_async_commit();
 
     // ---- consumer side ----
     int slot = 0;
-    ItemCursor cur = cursor_at(P, it_begin);
-    for (int item = it_begin; item < it_end; item++, cursor_next(P, cur)) {
+    int v[NBX];
+    bool own_cut = false;  // the last item continues in later warps of the CTA
+    while (start < b1) {
         const GemvDesc &D = P.d[cur.id];
-        const int N = D.N;
-        const int unit = cur.unit;
-        const int c_begin = cur.kp * D.cpp, c_end = min(D.nchunk, c_begin + D.cpp);
+        const int first = cur.kp * D.cpp;
+        const int nreal = min(D.cpp, D.nchunk - first);
+        const int c_begin = first + max(b0 - start, 0);
+        const int c_end = first + min(b1 - start, nreal);
         int acc[NBX][2];
 #pragma unroll
         for (int b = 0; b < NBX; b++) acc[b][0] = acc[b][1] = 0;
@@ -859,9 +986,7 @@ __global__ void __launch_bounds__(kDotThreads, DotShape<NBX>::kMinBlocks)
                     for (int beta = 0; beta < 4; beta++) {
                         const uint32_t sl = d.sel(C, i, beta);
                         const int lo = (int)prmt(C.tlo[i], C.thi[i], sl);
-                        // high half of the selector: beta 0, 2 on the ALU, beta 1, 3 on the FMA pipe
-                        const int hi = (int)prmt(C.tlo[i], C.thi[i],
-                                                 (beta & 1) ? imulhi(sl, C.hi16) : (sl >> 16));
+                        const int hi = (int)prmt(C.tlo[i], C.thi[i], hi_half(C, sl));
 #pragma unroll
                         for (int b = 0; b < NBX; b++) {
                             const uint4 &xv = beta < 2 ? xa[b] : xb[b];
@@ -873,62 +998,44 @@ __global__ void __launch_bounds__(kDotThreads, DotShape<NBX>::kMinBlocks)
                 }
             }
         }
-        // epilogue: lane = row of the unit
-        const int row = unit * kUnitRows + lane;
-        const bool rv = row < N;
-        int v[NBX];
 #pragma unroll
         for (int b = 0; b < NBX; b++) v[b] = acc[b][0] + acc[b][1];
-        bool finish = true;
-        if (D.kparts > 1) {
-            if (rv) {
+        if (start < b0) {
+            // a later piece of an item cut at b0: hand the sums to its first warp
 #pragma unroll
-                for (int b = 0; b < NBX; b++)
-                    if (b < B) atomicAdd(D.part_acc + (size_t)b * N + row, v[b]);
-            }
-            __threadfence();
-            __syncwarp();
-            uint32_t done = 0;
-            if (lane == 0) done = atomicAdd(D.part_cnt + unit, 1u);
-            finish = __shfl_sync(0xFFFFFFFFu, done, 0) == (uint32_t)(D.kparts - 1);
-            if (finish) {
-                __threadfence();
-                if (rv) {
-#pragma unroll
-                    for (int b = 0; b < NBX; b++) {
-                        if (b < B) {
-                            int32_t *pa = D.part_acc + (size_t)b * N + row;
-                            v[b] = __ldcg(pa);
-                            *pa = 0;
-                        }
-                    }
-                }
-                if (lane == 0) D.part_cnt[unit] = 0u;
-            }
+            for (int b = 0; b < NBX; b++) cut_sum[(warp * NBX + b) * 32 + lane] = v[b];
+            if (lane == 0) cut_start[warp] = start;
+        } else if (b1 - start < nreal) {
+            own_cut = true;  // first piece of an item cut at b1: finished after the barrier
+        } else {
+            dot_finish<NBX, ACC_OUT>(D, cur.unit, B, lane, v);
         }
-        if (finish && rv) {
-            if (ACC_OUT) {
-#pragma unroll
-                for (int b = 0; b < NBX; b++)
-                    if (b < B) static_cast<int32_t *>(D.out)[(size_t)b * N + row] = v[b];
-            } else {
-#pragma unroll
-                for (int b = 0; b < NBX; b++)
-                    if (b < B)
-                        static_cast<float *>(D.out)[(size_t)b * N + row] = out_scale(D, row, b) * (float)v[b];
-            }
-        }
+        start += nreal;
+        if (start < b1) cursor_next(P, cur);
     }
     cp_async_wait<0>();
+    __syncthreads();  // the later pieces' sums are in shared memory
+    if (own_cut) {
+        int mine;  // first chunk of the cut item
+        cursor_at_chunk(P, b1 - 1, mine);
+        for (int w = warp + 1; w < kDotWarps; w++) {
+            const int cs = cut_start[w];
+            if (cs == -2) continue;
+            if (cs != mine) break;
+#pragma unroll
+            for (int b = 0; b < NBX; b++) v[b] += cut_sum[(w * NBX + b) * 32 + lane];
+        }
+        dot_finish<NBX, ACC_OUT>(P.d[cur.id], cur.unit, B, lane, v);
+    }
 }
 
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
 // Launch with the programmatic-stream-serialization attribute (see pdl_wait).
-template <typename KernelT>
+template <typename KernelT, typename ParamsT>
 void launch_pdl(KernelT kernel, int grid, int threads, size_t smem, cudaStream_t stream,
-                const GemvParams &gp) {
+                const ParamsT &gp) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3((unsigned)threads);
@@ -971,7 +1078,9 @@ template <int NBX, bool ACC>
 void launch_dot(const GemvParams &gp, cudaStream_t stream) {
     static int cache[64] = {0};
     const size_t smem = DotShape<NBX>::kSmem;
-    const int want = (gp.total_chunks + kDotWarps * 4 - 1) / (kDotWarps * 4);
+    // one chunk per warp at most: a small GEMV spreads over as many SMs as it
+    // has chunks (items cut between warps are summed in shared memory)
+    const int want = (gp.total_chunks + kDotWarps - 1) / kDotWarps;
     const int grid = grid_for(gemv_dot_kernel<NBX, ACC>, kDotThreads, smem, want, cache);
     launch_pdl(gemv_dot_kernel<NBX, ACC>, grid, kDotThreads, smem, stream, gp);
 }
@@ -1024,7 +1133,7 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
         const int64_t nchunk = padded_tiles(c.K) / kChunkTiles;
         const int64_t kparts = kparts_for(c.K);
         items += (c.N + kUnitRows - 1) / kUnitRows * kparts;
-        chunks += (c.N + kUnitRows - 1) / kUnitRows * kparts * ((nchunk + kparts - 1) / kparts);
+        chunks += (c.N + kUnitRows - 1) / kUnitRows * nchunk;
     }
     if (workspace_bytes < (size_t)words * 4) return SHERRY_ERR_WORKSPACE;
     if (words > 0x7FFFFFFF || units16 > 0x7FFFFFFF || items > 0x7FFFFFFF || chunks > 0x7FFFFFFF)
@@ -1045,9 +1154,8 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
     xp.B = gp.B = B;
     gp.mul4 = 4u;
     gp.mul2 = 2u;
-    gp.hi1 = 0x80000000u;
-    gp.hi2 = 0x40000000u;
-    gp.hi16 = 0x10000u;
+    gp.f16one = 0x3C003C00u;
+    gp.f16negz = 0x80008000u;
     gp.m33 = 0x33333333u;
     gp.m55 = 0x55555555u;
     gp.m44 = 0x44444444u;
@@ -1107,7 +1215,7 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
         wb += X.xunits + (X.zero_words + 31) / 32;
         ub16 += (int)((c.N + 15) / 16);
         ib += units * kparts;
-        cb += units * kparts * cpp;
+        cb += units * nchunk;
     }
     xp.total_units = wb;
     gp.total_units16 = ub16;
@@ -1115,7 +1223,7 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
     gp.total_chunks = cb;
     if (phase & kPrepare) {
         const int blocks = std::max(1, std::min((wb + 7) / 8, sm_count() * 8));
-        xprep_kernel<<<blocks, 256, 0, stream>>>(xp);
+        launch_pdl(xprep_kernel, blocks, 256, 0, stream, xp);
         const sherry_status st = launch_status("sherry_gemv (activation re-order)");
         if (st != SHERRY_OK) return st;
     }

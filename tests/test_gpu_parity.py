@@ -67,7 +67,9 @@ def test_pack_full_size_1b_layers(layer):
 GEMV_CASES = [(256, 1024, 1), (1, 128, 1), (17, 384, 3), (33, 640, 5), (40, 1152, 8),
               (19, 256, 9), (64, 512, 16), (2048, 2048, 1), (512, 2048, 4), (100, 3072, 2),
               (31, 8192, 1), (48, 8192, 16), (50, 1536, 2), (23, 512, 1), (70, 2560, 9),
-              (129, 4096, 8), (37, 8192, 2), (130, 2048, 3)]
+              (129, 4096, 8), (37, 8192, 2), (130, 2048, 3),
+              # B <= 2 with short last K-parts (5, 7 and 10 chunks per row)
+              (70, 2560, 1), (33, 3584, 2), (300, 5120, 1)]
 
 
 @pytest.mark.parametrize("N,K,B", GEMV_CASES)
@@ -139,6 +141,29 @@ def test_gemv_grouped_1b_stack_layer():
     S.gemv_grouped(items, B=1)
     for (_, _, _, y), ref in zip(items, refs):
         assert_y_matches(y.cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("B", [1, 2])
+def test_gemv_grouped_cut_items(B):
+    # many small GEMVs of mixed K (short last K-parts included) in one launch:
+    # warp ranges cut items at many places, inside and across GEMVs
+    shapes = [(33, 640), (96, 8192), (1, 128), (70, 2560), (200, 2048), (45, 3584),
+              (64, 5120), (7, 384), (130, 4096), (31, 1152)] * 3
+    items, refs = [], []
+    for li, (N, K) in enumerate(shapes):
+        codes, scales = oracle.pack(synth.latent_weights(N, K, seed=200 + li))
+        x = synth.int8_uniform((B, K), seed=300 + li)
+        y = torch.zeros((B, N), dtype=torch.float32, device="cuda")
+        items.append((dev_codes(codes), dev(scales), dev(x), y))
+        refs.append(oracle.gemv(codes, scales, x, K))
+    g = S.GroupedGemv(items, B=B)
+    g.prepare()
+    for _ in range(2):
+        for it in items:
+            it[3].zero_()
+        g.run()
+        for (_, _, _, y), ref in zip(items, refs):
+            assert_y_matches(y.cpu().numpy(), ref)
 
 
 def test_gemv_on_gpu_packed_codes():
