@@ -269,8 +269,63 @@ def time_gemm(S, torch, dev, flush, reps=5):
     return out
 
 
-def time_layers(layers, xs, S, torch, dev, flush, reps=20):
-    """Single-projection GEMVs of layer 0 with the L2 flushed before each launch."""
+HBM_SPEC_GBS = 8000.0  # the B200 HBM3e figure the workload description names (~8 TB/s)
+
+
+def read_stream_gbs(torch, dev, reps=10):
+    """Read-only HBM bandwidth: a 4 GiB fp32 sum, best of `reps`."""
+    buf = torch.ones(1 << 30, dtype=torch.float32, device=dev)
+    out = torch.empty((), dtype=torch.float32, device=dev)
+    for _ in range(2):
+        torch.sum(buf, dim=0, out=out)
+    best = None
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        torch.sum(buf, dim=0, out=out)
+        e1.record()
+        e1.synchronize()
+        t = e0.elapsed_time(e1) / 1e3
+        best = t if best is None else min(best, t)
+    del buf
+    return 4 * (1 << 30) / best / 1e9
+
+
+def graph_time(torch, calls, reps):
+    """Seconds per replay of a CUDA graph holding calls() (warmed up first),
+    timed with events around `reps` replays."""
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        calls()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        calls()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        g.replay()
+    e1.record()
+    e1.synchronize()
+    del g
+    return e0.elapsed_time(e1) / 1e3 / reps
+
+
+def replicas_for(nbytes):
+    """Copies of a weight set that together exceed twice the L2, so that each
+    call of a rotation reads its codes from HBM."""
+    return max(2, -(-2 * L2_BYTES // nbytes))
+
+
+def time_layers(layers, xs, S, torch, dev, reps=20):
+    """Single-projection sherry_gemv calls of layer 0, B = 1: each projection
+    is called on rotated copies of its codes (> 2x L2 in all) inside one CUDA
+    graph, so every call reads cold codes and launch cost is the GPU's only."""
     res = {}
     for layer, name, n, k, codes, scales in layers:
         if layer != 0:
@@ -278,27 +333,38 @@ def time_layers(layers, xs, S, torch, dev, flush, reps=20):
         x = xs[k]
         y = torch.empty((1, n), dtype=torch.float32, device=dev)
         ws = S.workspace(S.gemv_workspace_bytes(n, k, 1), dev)
-        for _ in range(3):
-            S.gemv(codes, scales, x, y, ws)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        ts = []
-        for _ in range(reps):
-            flush()
-            e0.record()
-            S.gemv(codes, scales, x, y, ws)
-            e1.record()
-            e1.synchronize()
-            ts.append(e0.elapsed_time(e1) / 1e3)
-        t = statistics.median(ts)
+        R = replicas_for(codes.numel() * 4)
+        reps_codes = [codes.clone() for _ in range(R)]
+
+        def calls():
+            for c in reps_codes:
+                S.gemv(c, scales, x, y, ws)
+        t = graph_time(torch, calls, reps) / R
+        del reps_codes
         cb = n * k * 5 // 32
-        res[name] = {"N": n, "K": k, "us": t * 1e6, "weight_gbs": cb / t / 1e9}
+        res[name] = {"N": n, "K": k, "us": t * 1e6, "weight_gbs": cb / t / 1e9, "copies": R}
     return res
 
 
-def time_3b_layer(S, torch, dev, flush, reps=10):
+def time_stack_single_calls(layers, xs, ys, S, torch, dev, reps=50):
+    """The stack as 112 separate sherry_gemv calls (one per projection, one
+    shared workspace), captured in one CUDA graph: time per step."""
+    ws = S.workspace(max(S.gemv_workspace_bytes(n, k, 1) for _, _, n, k, _, _ in layers), dev)
+
+    def calls():
+        for (_, _, n, k, codes, scales), y in zip(layers, ys):
+            S.gemv(codes, scales, xs[k], y, ws)
+    t = graph_time(torch, calls, reps)
+    code_bytes = sum(codes.numel() * 4 for _, _, _, _, codes, _ in layers)
+    return {"us_per_step": t * 1e6, "weight_gbs": code_bytes / t / 1e9, "calls": len(layers),
+            "steps": reps}
+
+
+def time_3b_layer(S, torch, dev, reps=10):
     """One LLaMA-3.2-3B-shaped layer (7 projections, one grouped call) at
-    B = 1, 4, 16 with int8 activations (seeds 1, 2, 3), L2 flushed before each
-    call."""
+    B = 1, 4, 16 with int8 activations (seeds 1, 2, 3): rotated copies of the
+    layer's codes (> 2x L2 in all), one grouped call per copy, in one CUDA
+    graph."""
     items_w = []
     for pi, (name, n, k) in enumerate(synth.LLAMA_3B_LAYERS):
         w = torch.from_numpy(synth.latent_weights(n, k, seed=synth.layer_seed(0, pi))).to(dev)
@@ -306,27 +372,23 @@ def time_3b_layer(S, torch, dev, flush, reps=10):
         del w
         items_w.append((n, k, codes, scales))
     code_bytes = sum(c.numel() * 4 for _, _, c, _ in items_w)
+    R = replicas_for(code_bytes)
+    copies = [[c.clone() for _, _, c, _ in items_w] for _ in range(R)]
     out = {}
     for B, seed in ((1, 1), (4, 2), (16, 3)):
         xs = {k: torch.from_numpy(synth.int8_uniform((B, k), seed=seed)).to(dev)
               for k in {k for _, k, _, _ in items_w}}
         ys = [torch.empty((B, n), dtype=torch.float32, device=dev) for n, _, _, _ in items_w]
-        step = S.GroupedGemv([(c, s, xs[k], y) for (n, k, c, s), y in zip(items_w, ys)], B=B)
-        for _ in range(3):
-            step()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        ts = []
-        for _ in range(reps):
-            flush()
-            e0.record()
-            step()
-            e1.record()
-            e1.synchronize()
-            ts.append(e0.elapsed_time(e1) / 1e3)
-        t = statistics.median(ts)
+        steps = [S.GroupedGemv([(c, s, xs[k], y) for (n, k, _, s), c, y in zip(items_w, cs, ys)], B=B)
+                 for cs in copies]
+
+        def calls():
+            for st in steps:
+                st()
+        t = graph_time(torch, calls, reps) / R
         out["B%d" % B] = {"us": t * 1e6, "weight_gbs": code_bytes / t / 1e9}
     out["code_bytes"] = code_bytes
+    out["copies"] = R
     return out
 
 
@@ -556,9 +618,15 @@ def main():
         del latents
         torch.cuda.empty_cache()
         line["gemm"] = time_gemm(S, torch, dev, flush)
-        line["gemv_layers_l2_flushed"] = time_layers(layers, xs, S, torch, dev, flush)
+        line["gemv_layers_rotated"] = time_layers(layers, xs, S, torch, dev)
         line["gemv_bf16_stack"] = time_bf16_stack(layers, S, torch, dev)
-        line["gemv_3b_layer_l2_flushed"] = time_3b_layer(S, torch, dev, flush)
+        line["gemv_stack_112_calls_graph"] = time_stack_single_calls(layers, xs, ys, S, torch, dev)
+        rs = read_stream_gbs(torch, dev)
+        line["roofline"]["other_denominators"] = {
+            "read_only_stream_gbs": rs, "frac_of_read_only_stream": achieved / rs,
+            "hbm_spec_gbs": HBM_SPEC_GBS, "frac_of_spec": achieved / HBM_SPEC_GBS,
+            "note": "read-only stream: torch.sum over 4 GiB of fp32 (a library kernel), best of 10"}
+        line["gemv_3b_layer_rotated"] = time_3b_layer(S, torch, dev)
         if world == 1:
             line["cpu_baseline"] = cpu_baseline(layers, xs_host, args.cpu_seconds)
     err = S.device_error()

@@ -785,7 +785,7 @@ __global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
 //     conflict-free shared loads and each lane ends with its row's sum (no
 //     reduction across lanes);
 //   * work is split by chunk count.  Each CTA takes a run of whole items
-//     (unit, K-part) holding about 1/gridDim of the chunks, and its 8 warps
+//     (unit, K-part) holding about 1/gridDim of the chunks, and its warps
 //     split the run into equal chunk ranges, so no warp ends the launch with a
 //     whole extra item to do.  An item cut by a warp boundary is summed by the
 //     warps holding its pieces: later pieces leave their row sums in shared
@@ -801,18 +801,22 @@ __global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
 //     than an m16n8k32 MMA whose 8 columns would mostly be empty.
 // K-parts and the split-K completion are those of the pipelined kernel.
 // ---------------------------------------------------------------------------
-constexpr int kDotThreads = 256;
-constexpr int kDotWarps = kDotThreads / 32;
-constexpr int kDotRing = 2;  // 2 stages x 8 warps: 50 KB per CTA, 4 CTAs (32 warps) per SM
+constexpr int kDotRing = 2;  // stages per warp: one chunk in flight while one is consumed
 constexpr int kDotCodeWords = kChunkTiles * kTileWords;  // 640
+// 8 warps per CTA: B = 1, 4 CTAs (32 warps) per SM at 64 registers (50 KB of
+// shared memory per CTA); B = 2, 2 CTAs per SM.  (One CTA of 32 warps per SM
+// balances the CTAs' item runs better but was measured slower: a CTA slot frees
+// only when all 32 warps are done.)
 template <int NBX>
 struct DotShape {
+    static constexpr int kWarps = 8;
+    static constexpr int kThreads = kWarps * 32;
+    static constexpr int kMinBlocks = NBX == 1 ? 4 : 2;
     static constexpr int kStageWords = kDotCodeWords + NBX * kChunkTiles * 32;
-    static constexpr int kRingWords = kDotWarps * kDotRing * kStageWords;
+    static constexpr int kRingWords = kWarps * kDotRing * kStageWords;
     // after the rings: per warp, the row sums of a later piece of a cut item
     // [warp][NBX][32] and the first chunk of that item [warp]
-    static constexpr size_t kSmem = ((size_t)kRingWords + kDotWarps * (NBX * 32 + 1)) * 4;
-    static constexpr int kMinBlocks = NBX == 1 ? 4 : 2;
+    static constexpr size_t kSmem = ((size_t)kRingWords + kWarps * (NBX * 32 + 1)) * 4;
 };
 
 // Finishes an item: lane = row of the unit, v = the item's row sums.  A K-part
@@ -866,21 +870,26 @@ __device__ __forceinline__ void dot_finish(const GemvDesc &D, int unit, int B, i
 }
 
 template <int NBX, bool ACC_OUT>
-__global__ void __launch_bounds__(kDotThreads, DotShape<NBX>::kMinBlocks)
+__global__ void __launch_bounds__(DotShape<NBX>::kThreads, DotShape<NBX>::kMinBlocks)
     gemv_dot_kernel(const __grid_constant__ GemvParams P) {
     pdl_allow_dependents();
     constexpr int SW = DotShape<NBX>::kStageWords;
     extern __shared__ __align__(16) uint32_t dot_smem[];
     int *cut_sum = reinterpret_cast<int *>(dot_smem + DotShape<NBX>::kRingWords);
-    int *cut_start = cut_sum + kDotWarps * NBX * 32;
+    constexpr int kWarps = DotShape<NBX>::kWarps;
+    int *cut_start = cut_sum + kWarps * NBX * 32;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    // chunk range [b0, b1) of this warp
-    const long long tc = P.total_chunks, nb = gridDim.x;
-    const int cta_lo = item_start_at_or_before(P, (int)(blockIdx.x * tc / nb));
-    const int cta_hi = item_start_at_or_before(P, (int)((blockIdx.x + 1) * tc / nb));
+    // chunk range [b0, b1) of this warp; threads 0 and 1 find the CTA's bounds
+    __shared__ int cta_bound[2];
+    if (threadIdx.x < 2) {
+        const long long tc = P.total_chunks, nb = gridDim.x;
+        cta_bound[threadIdx.x] = item_start_at_or_before(P, (int)((blockIdx.x + threadIdx.x) * tc / nb));
+    }
+    __syncthreads();
+    const int cta_lo = cta_bound[0], cta_hi = cta_bound[1];
     const long long len = cta_hi - cta_lo;
-    const int b0 = cta_lo + (int)(warp * len / kDotWarps);
-    const int b1 = cta_lo + (int)((warp + 1) * len / kDotWarps);
+    const int b0 = cta_lo + (int)(warp * len / kWarps);
+    const int b1 = cta_lo + (int)((warp + 1) * len / kWarps);
     // -1: no cut item starts before b0; -2: empty range (skipped when summing)
     if (lane == 0) cut_start[warp] = b0 < b1 ? -1 : -2;
     uint32_t *ring = dot_smem + (size_t)warp * kDotRing * SW;
@@ -1016,9 +1025,9 @@ __global__ void __launch_bounds__(kDotThreads, DotShape<NBX>::kMinBlocks)
     cp_async_wait<0>();
     __syncthreads();  // the later pieces' sums are in shared memory
     if (own_cut) {
-        int mine;  // first chunk of the cut item
-        cursor_at_chunk(P, b1 - 1, mine);
-        for (int w = warp + 1; w < kDotWarps; w++) {
+        const GemvDesc &D = P.d[cur.id];
+        const int mine = D.chunk_begin + cur.unit * D.nchunk + cur.kp * D.cpp;  // the cut item
+        for (int w = warp + 1; w < kWarps; w++) {
             const int cs = cut_start[w];
             if (cs == -2) continue;
             if (cs != mine) break;
@@ -1080,9 +1089,10 @@ void launch_dot(const GemvParams &gp, cudaStream_t stream) {
     const size_t smem = DotShape<NBX>::kSmem;
     // one chunk per warp at most: a small GEMV spreads over as many SMs as it
     // has chunks (items cut between warps are summed in shared memory)
-    const int want = (gp.total_chunks + kDotWarps - 1) / kDotWarps;
-    const int grid = grid_for(gemv_dot_kernel<NBX, ACC>, kDotThreads, smem, want, cache);
-    launch_pdl(gemv_dot_kernel<NBX, ACC>, grid, kDotThreads, smem, stream, gp);
+    constexpr int threads = DotShape<NBX>::kThreads, warps = DotShape<NBX>::kWarps;
+    const int want = (gp.total_chunks + warps - 1) / warps;
+    const int grid = grid_for(gemv_dot_kernel<NBX, ACC>, threads, smem, want, cache);
+    launch_pdl(gemv_dot_kernel<NBX, ACC>, grid, threads, smem, stream, gp);
 }
 
 template <int NB, bool ACC>
