@@ -52,7 +52,6 @@ struct GemvDesc {
     int nchunk;           // pipelined kernel: 4-tile chunks per row
     int kparts;           // pipelined kernel: K-parts per unit
     int cpp;              // pipelined kernel: chunks per K-part
-    int item_begin;       // pipelined kernel: first (unit, K-part) item in the group
     int chunk_begin;      // pipelined kernel: first 4-tile chunk of the group (all groups' rows
                           // in order, each row's K-parts in order)
 };
@@ -61,7 +60,6 @@ struct GemvParams {
     int count;
     int B;
     int total_units16;    // register kernel
-    int total_items;      // pipelined kernel
     int total_chunks;     // pipelined kernel: chunks of all groups (the balancing space)
     // Constants passed at run time so that they live in registers instead of
     // being re-created per use, and so that left shifts by a power of two stay
@@ -507,8 +505,10 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const __grid_constan
 //     private ring of kRing shared-memory stages filled by cp.async with
 //     consecutive lanes on consecutive 16 bytes, so an SM keeps ~100 KB of
 //     fully coalesced HBM reads in flight;
-//   * items are split into contiguous ranges of equal chunk count, one range
-//     per warp, in GEMV order, so no warp carries much more than the average;
+//   * each CTA takes a run of whole items (in GEMV order) of about 1/gridDim
+//     of the chunks and its warps split the run into equal chunk ranges; an
+//     item cut by a warp boundary is summed in shared memory by the warp that
+//     holds its first chunk, after one CTA barrier;
 //   * a unit with several K-parts adds its partial int32 sums into part_acc
 //     with atomics; the warp that completes the last part (per-unit counter)
 //     scales, writes y and clears its part_acc entries and the counter, so
@@ -527,14 +527,6 @@ __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
-__device__ __forceinline__ int find_desc_by_item(const GemvParams &P, int item) {
-    int lo = 0, hi = P.count - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (P.d[mid].item_begin <= item) lo = mid; else hi = mid - 1;
-    }
-    return lo;
-}
 
 // Chunk space: the 4-tile chunks of all groups, group by group, each group's
 // 32-row units in order and each unit's chunks in K order.  An item (unit,
@@ -548,18 +540,6 @@ __device__ __forceinline__ int desc_by_chunk(const GemvParams &P, int c) {
     return lo;
 }
 
-// First item that starts at chunk c or later (total_items if none).
-__device__ __forceinline__ int first_item_at_or_after(const GemvParams &P, int c) {
-    if (c >= P.total_chunks) return P.total_items;
-    const int id = desc_by_chunk(P, c);
-    const GemvDesc &D = P.d[id];
-    const int rc = c - D.chunk_begin;
-    const int unit = rc / D.nchunk;
-    const int kp = (rc - unit * D.nchunk + D.cpp - 1) / D.cpp;  // kparts: the next unit
-    const int k = unit * D.kparts + kp;
-    return k < D.units * D.kparts ? D.item_begin + k
-                                  : (id + 1 < P.count ? P.d[id + 1].item_begin : P.total_items);
-}
 
 // (GEMV, unit, K-part) of an item, advanced item by item without searches or
 // divisions.
@@ -597,38 +577,126 @@ __device__ __forceinline__ void cursor_next(const GemvParams &P, ItemCursor &c) 
 #ifndef SHERRY_PIPE_MIN_BLOCKS
 #define SHERRY_PIPE_MIN_BLOCKS 2
 #endif
+// Shared memory of the MMA kernel: the warps' rings, then per warp the
+// fragments of a later piece of a cut item [warp][2 * NB * 4][32] (the
+// chunk split and the cut items are those of the small-batch kernel below).
+template <int NB>
+struct PipeShape {
+    static constexpr int kCutWords = 2 * NB * 4 * 32;
+    static constexpr size_t kSmem = kPipeSmem + (size_t)kPipeWarps * kCutWords * 4;
+};
+
+// Finishes an item of the MMA kernel: per row block rb, fragment e holds
+// (row g + 8 [e >= 2], batch column 2t + (e & 1)) of the unit.
+template <int NB, bool ACC_OUT>
+__device__ __forceinline__ void pipe_finish(const GemvDesc &D, int unit, int B, int lane,
+                                            int (&acc)[2][NB][4]) {
+    const int g = lane >> 2, t = lane & 3;
+    const int N = D.N;
+    const int rbase = unit * kUnitRows;
+    bool finish = true;
+    if (D.kparts > 1) {
+#pragma unroll
+        for (int rb = 0; rb < 2; rb++)
+#pragma unroll
+            for (int nb = 0; nb < NB; nb++)
+#pragma unroll
+                for (int e = 0; e < 4; e++) {
+                    const int row = rbase + rb * 16 + g + ((e & 2) ? 8 : 0);
+                    const int b = nb * 8 + 2 * t + (e & 1);
+                    if (row < N && b < B) atomicAdd(D.part_acc + (size_t)b * N + row, acc[rb][nb][e]);
+                }
+        __threadfence();
+        __syncwarp();
+        uint32_t done = 0;
+        if (lane == 0) done = atomicAdd(D.part_cnt + unit, 1u);
+        finish = __shfl_sync(0xFFFFFFFFu, done, 0) == (uint32_t)(D.kparts - 1);
+        if (finish) {
+            __threadfence();
+#pragma unroll
+            for (int rb = 0; rb < 2; rb++)
+#pragma unroll
+                for (int nb = 0; nb < NB; nb++)
+#pragma unroll
+                    for (int e = 0; e < 4; e++) {
+                        const int row = rbase + rb * 16 + g + ((e & 2) ? 8 : 0);
+                        const int b = nb * 8 + 2 * t + (e & 1);
+                        if (row < N && b < B) {
+                            int32_t *pa = D.part_acc + (size_t)b * N + row;
+                            acc[rb][nb][e] = __ldcg(pa);
+                            *pa = 0;
+                        }
+                    }
+            if (lane == 0) D.part_cnt[unit] = 0u;
+        }
+    }
+    if (finish) {
+#pragma unroll
+        for (int rb = 0; rb < 2; rb++)
+#pragma unroll
+            for (int nb = 0; nb < NB; nb++)
+#pragma unroll
+                for (int e = 0; e < 4; e++) {
+                    const int row = rbase + rb * 16 + g + ((e & 2) ? 8 : 0);
+                    const int b = nb * 8 + 2 * t + (e & 1);
+                    if (row < N && b < B) {
+                        if (ACC_OUT)
+                            static_cast<int32_t *>(D.out)[(size_t)b * N + row] = acc[rb][nb][e];
+                        else
+                            static_cast<float *>(D.out)[(size_t)b * N + row] =
+                                out_scale(D, row, b) * (float)acc[rb][nb][e];
+                    }
+                }
+    }
+}
+
 template <int NB, bool ACC_OUT>
 __global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
     gemv_pipe_kernel(const __grid_constant__ GemvParams P) {
     pdl_allow_dependents();
-    pdl_wait();
     extern __shared__ __align__(16) uint32_t pipe_smem[];
+    int *cut_sum = reinterpret_cast<int *>(pipe_smem + kPipeSmem / 4);
+    __shared__ int cut_start[kPipeWarps];
+    __shared__ int cta_bound[2];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
-    const long long nw = (long long)gridDim.x * kPipeWarps;
-    const long long wg = (long long)blockIdx.x * kPipeWarps + warp;
-    const int it_begin = first_item_at_or_after(P, (int)(wg * P.total_chunks / nw));
-    const int it_end = first_item_at_or_after(P, (int)((wg + 1) * P.total_chunks / nw));
-    if (it_begin >= it_end) return;
+    // chunk range [b0, b1) of this warp: the CTA takes whole items of about
+    // 1/gridDim of the chunks, its warps equal chunk shares of them
+    if (threadIdx.x < 2) {
+        const long long tc = P.total_chunks, nb = gridDim.x;
+        cta_bound[threadIdx.x] = item_start_at_or_before(P, (int)((blockIdx.x + threadIdx.x) * tc / nb));
+    }
+    __syncthreads();
+    const int cta_lo = cta_bound[0];
+    const long long len = cta_bound[1] - cta_lo;
+    const int b0 = cta_lo + (int)(warp * len / kPipeWarps);
+    const int b1 = cta_lo + (int)((warp + 1) * len / kPipeWarps);
+    // -1: no cut item starts before b0; -2: empty range (skipped when summing)
+    if (lane == 0) cut_start[warp] = b0 < b1 ? -1 : -2;
     uint32_t *ring = pipe_smem + (size_t)warp * kRing * kStageWords;
     Consts C;
     load_consts(P, C);
+    const int B = P.B;
+
+    int start = b1;
+    ItemCursor cur = {0, 0, 0};
+    if (b0 < b1) cur = cursor_at_chunk(P, b0, start);
 
     // ---- producer side: the issue cursor runs kRing-1 stages ahead ----
     // lane l copies 16-byte pieces l + 32 j (j = 0..4) of the 2560-byte chunk;
-    // piece words 4i..4i+3 belong to tile block 4i / 160
-    int iitem = it_begin, id = find_desc_by_item(P, it_begin);
-    int ic = 0, ic_end = 0;          // chunk cursor within the current item
+    // piece words 4i..4i+3 belong to tile block 4i / 160.  Codes only: the
+    // activations are read from global memory after pdl_wait().
+    ItemCursor icur = cur;
+    int istart = start, ic = 0, ic_end = 0;
     const uint32_t *isrc = nullptr;  // first word of the current unit's group
     auto set_issue_item = [&]() {
-        const GemvDesc &D = P.d[id];
-        const int local = iitem - D.item_begin;
-        const int unit = local / D.kparts, kp = local - unit * D.kparts;
-        isrc = D.codes + (size_t)unit * D.T * kTileWords + 4 * lane;
-        ic = kp * D.cpp;
-        ic_end = min(D.nchunk, ic + D.cpp);
+        const GemvDesc &D = P.d[icur.id];
+        isrc = D.codes + (size_t)icur.unit * D.T * kTileWords + 4 * lane;
+        const int first = icur.kp * D.cpp;
+        ic = first + max(b0 - istart, 0);
+        ic_end = first + min(b1 - istart, min(D.cpp, D.nchunk - first));
     };
-    set_issue_item();
+    if (istart < b1) set_issue_item();
     uint32_t dst_piece[5];
 #pragma unroll
     for (int j = 0; j < 5; j++) {
@@ -637,37 +705,42 @@ __global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
         dst_piece[j] = smem_u32(ring) + 4u * (uint32_t)(tb * kTileWordsPadded + (wd - tb * kTileWords));
     }
     auto issue = [&](int slot) {
-        if (iitem < it_end) {
+        if (istart < b1) {
             const uint32_t *src = isrc + (size_t)ic * kChunkTiles * kTileWords;
             const uint32_t sofs = (uint32_t)slot * kStageWords * 4;
 #pragma unroll
             for (int j = 0; j < 5; j++) cp_async16(dst_piece[j] + sofs, src + 128 * j, 16u);
-            if (++ic == ic_end && ++iitem < it_end) {
-                if (iitem >= P.d[id].item_begin + P.d[id].units * P.d[id].kparts) id++;
-                set_issue_item();
+            if (++ic == ic_end) {
+                const GemvDesc &D = P.d[icur.id];
+                istart += min(D.cpp, D.nchunk - icur.kp * D.cpp);
+                if (istart < b1) {
+                    cursor_next(P, icur);
+                    set_issue_item();
+                }
             }
         }
         cp_async_commit();
     };
 #pragma unroll
     for (int s = 0; s < kRing - 1; s++) issue(s);
+    pdl_wait();
 
     // ---- consumer side ----
     int slot = 0;
-    for (int item = it_begin; item < it_end; item++) {
-        const GemvDesc &D = P.d[find_desc_by_item(P, item)];
-        const int N = D.N;
-        const int local = item - D.item_begin;
-        const int unit = local / D.kparts, kp = local - unit * D.kparts;
-        const int rbase = unit * kUnitRows;
-        const int c_begin = kp * D.cpp, c_end = min(D.nchunk, c_begin + D.cpp);
+    int acc[2][NB][4];  // [row block][batch group][fragment]
+    bool own_cut = false;  // the last item continues in later warps of the CTA
+    while (start < b1) {
+        const GemvDesc &D = P.d[cur.id];
+        const int first = cur.kp * D.cpp;
+        const int nreal = min(D.cpp, D.nchunk - first);
+        const int c_begin = first + max(b0 - start, 0);
+        const int c_end = first + min(b1 - start, nreal);
         const uint4 *xrow[NB];
 #pragma unroll
         for (int nb = 0; nb < NB; nb++) {
-            const int b = min(nb * 8 + g, P.B - 1);  // lanes past the batch: never stored
+            const int b = min(nb * 8 + g, B - 1);  // lanes past the batch: never stored
             xrow[nb] = D.xw + (size_t)b * D.Tp * 8 + (size_t)t * 8;
         }
-        int acc[2][NB][4];  // [row block][batch group][fragment]
 #pragma unroll
         for (int a = 0; a < 2; a++)
 #pragma unroll
@@ -719,64 +792,43 @@ __global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
                 }
             }
         }
-        // epilogue: per row block, c0/c1 = (row g, cols 2t, 2t+1), c2/c3 = row g+8
-        bool finish = true;
-        if (D.kparts > 1) {
+        if (start < b0) {
+            // a later piece of an item cut at b0: hand the fragments to its first warp
+            int *cs = cut_sum + warp * PipeShape<NB>::kCutWords + lane;
 #pragma unroll
             for (int rb = 0; rb < 2; rb++)
 #pragma unroll
                 for (int nb = 0; nb < NB; nb++)
 #pragma unroll
-                    for (int e = 0; e < 4; e++) {
-                        const int row = rbase + rb * 16 + g + ((e & 2) ? 8 : 0);
-                        const int b = nb * 8 + 2 * t + (e & 1);
-                        if (row < N && b < P.B)
-                            atomicAdd(D.part_acc + (size_t)b * N + row, acc[rb][nb][e]);
-                    }
-            __threadfence();
-            __syncwarp();
-            uint32_t done = 0;
-            if (lane == 0) done = atomicAdd(D.part_cnt + unit, 1u);
-            finish = __shfl_sync(0xFFFFFFFFu, done, 0) == (uint32_t)(D.kparts - 1);
-            if (finish) {
-                __threadfence();
-#pragma unroll
-                for (int rb = 0; rb < 2; rb++)
-#pragma unroll
-                    for (int nb = 0; nb < NB; nb++)
-#pragma unroll
-                        for (int e = 0; e < 4; e++) {
-                            const int row = rbase + rb * 16 + g + ((e & 2) ? 8 : 0);
-                            const int b = nb * 8 + 2 * t + (e & 1);
-                            if (row < N && b < P.B) {
-                                int32_t *pa = D.part_acc + (size_t)b * N + row;
-                                acc[rb][nb][e] = __ldcg(pa);
-                                *pa = 0;
-                            }
-                        }
-                if (lane == 0) D.part_cnt[unit] = 0u;
-            }
+                    for (int e = 0; e < 4; e++) cs[((rb * NB + nb) * 4 + e) * 32] = acc[rb][nb][e];
+            if (lane == 0) cut_start[warp] = start;
+        } else if (b1 - start < nreal) {
+            own_cut = true;  // first piece of an item cut at b1: finished after the barrier
+        } else {
+            pipe_finish<NB, ACC_OUT>(D, cur.unit, B, lane, acc);
         }
-        if (finish) {
-#pragma unroll
-            for (int rb = 0; rb < 2; rb++)
-#pragma unroll
-                for (int nb = 0; nb < NB; nb++)
-#pragma unroll
-                    for (int e = 0; e < 4; e++) {
-                        const int row = rbase + rb * 16 + g + ((e & 2) ? 8 : 0);
-                        const int b = nb * 8 + 2 * t + (e & 1);
-                        if (row < N && b < P.B) {
-                            if (ACC_OUT)
-                                static_cast<int32_t *>(D.out)[(size_t)b * N + row] = acc[rb][nb][e];
-                            else
-                                static_cast<float *>(D.out)[(size_t)b * N + row] =
-                                    out_scale(D, row, b) * (float)acc[rb][nb][e];
-                        }
-                    }
-        }
+        start += nreal;
+        if (start < b1) cursor_next(P, cur);
     }
     cp_async_wait<0>();
+    __syncthreads();  // the later pieces' fragments are in shared memory
+    if (own_cut) {
+        const GemvDesc &D = P.d[cur.id];
+        const int mine = D.chunk_begin + cur.unit * D.nchunk + cur.kp * D.cpp;  // the cut item
+        for (int w = warp + 1; w < kPipeWarps; w++) {
+            const int cs = cut_start[w];
+            if (cs == -2) continue;
+            if (cs != mine) break;
+            const int *src = cut_sum + w * PipeShape<NB>::kCutWords + lane;
+#pragma unroll
+            for (int rb = 0; rb < 2; rb++)
+#pragma unroll
+                for (int nb = 0; nb < NB; nb++)
+#pragma unroll
+                    for (int e = 0; e < 4; e++) acc[rb][nb][e] += src[((rb * NB + nb) * 4 + e) * 32];
+        }
+        pipe_finish<NB, ACC_OUT>(D, cur.unit, B, lane, acc);
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -1078,9 +1130,11 @@ int grid_for(KernelT kernel, int threads, size_t smem, int want, int *cache) {
 template <int NB, bool ACC>
 void launch_pipe(const GemvParams &gp, cudaStream_t stream) {
     static int cache[64] = {0};
-    const int want = (gp.total_chunks + kPipeWarps * 4 - 1) / (kPipeWarps * 4);
-    const int grid = grid_for(gemv_pipe_kernel<NB, ACC>, kPipeThreads, kPipeSmem, want, cache);
-    launch_pdl(gemv_pipe_kernel<NB, ACC>, grid, kPipeThreads, kPipeSmem, stream, gp);
+    // one chunk per warp at most (items cut between warps are summed in shared memory)
+    const size_t smem = PipeShape<NB>::kSmem;
+    const int want = (gp.total_chunks + kPipeWarps - 1) / kPipeWarps;
+    const int grid = grid_for(gemv_pipe_kernel<NB, ACC>, kPipeThreads, smem, want, cache);
+    launch_pdl(gemv_pipe_kernel<NB, ACC>, grid, kPipeThreads, smem, stream, gp);
 }
 
 template <int NBX, bool ACC>
@@ -1178,7 +1232,7 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
         }
     }
     int64_t off = 0;
-    int wb = 0, ub16 = 0, ib = 0, cb = 0;
+    int wb = 0, ub16 = 0, cb = 0;
     for (int i = 0; i < count; i++) {
         const GemvCall &c = calls[i];
         uint32_t *region = static_cast<uint32_t *>(workspace) + off;
@@ -1219,17 +1273,14 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
         D.nchunk = nchunk;
         D.kparts = kparts;
         D.cpp = cpp;
-        D.item_begin = ib;
         D.chunk_begin = cb;
         off += ws_words(c.N, c.K, B) + (bf ? kActScaleWords : 0);
         wb += X.xunits + (X.zero_words + 31) / 32;
         ub16 += (int)((c.N + 15) / 16);
-        ib += units * kparts;
         cb += units * nchunk;
     }
     xp.total_units = wb;
     gp.total_units16 = ub16;
-    gp.total_items = ib;
     gp.total_chunks = cb;
     if (phase & kPrepare) {
         const int blocks = std::max(1, std::min((wb + 7) / 8, sm_count() * 8));
