@@ -208,29 +208,39 @@ def build_stack(spec, dev, S, torch, keep_latents=False):
     return layers, latents
 
 
-def time_pack(latents, layers, S, torch, reps=3):
-    """sherry_pack over every latent matrix of the stack (3.9 GB fp32 read)."""
+def time_pack(latents, layers, S, torch, peak_gbs, reps=3):
+    """Packing every latent matrix of the stack (3.9 GB fp32 read): one
+    sherry_pack_grouped launch (the model-load path), and one sherry_pack call
+    per matrix for comparison."""
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     outs = [(torch.empty_like(l[4]), torch.empty_like(l[5])) for l in layers]
+    grouped = S.GroupedPack([(w, c, s) for w, (c, s) in zip(latents, outs)])
 
-    def one():
+    def per_matrix():
         for w, (c, s) in zip(latents, outs):
             S.pack(w, c, s)
-    one()
-    torch.cuda.synchronize()
-    times = []
-    for _ in range(reps):
-        start.record()
-        one()
-        end.record()
-        end.synchronize()
-        times.append(start.elapsed_time(end) / 1e3)
-    t = min(times)
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        times = []
+        for _ in range(reps):
+            start.record()
+            fn()
+            end.record()
+            end.synchronize()
+            times.append(start.elapsed_time(end) / 1e3)
+        return min(times)
+    t = timed(grouped)
+    t1 = timed(per_matrix)
     n_w = sum(l.numel() for l in latents)
     read = 4 * n_w
     written = sum(o[0].numel() * 4 + o[1].numel() * 4 for o in outs)
     return {"weights": n_w, "ms": t * 1e3, "gweights_per_s": n_w / t / 1e9,
-            "gbs": (read + written) / t / 1e9, "launches": len(latents),
+            "gbs": (read + written) / t / 1e9, "launches": 1, "call": "sherry_pack_grouped",
+            "frac_of_hbm_peak": (read + written) / t / 1e9 / peak_gbs,
+            "per_matrix_calls": {"launches": len(latents), "ms": t1 * 1e3,
+                                 "gbs": (read + written) / t1 / 1e9},
             "bytes_read": read, "bytes_written": written}
 
 
@@ -614,7 +624,7 @@ def main():
     }
     if extras:
         flush = l2_flusher(torch, dev)
-        line["pack"] = time_pack(latents, layers, S, torch)
+        line["pack"] = time_pack(latents, layers, S, torch, hbm_peak)
         del latents
         torch.cuda.empty_cache()
         line["gemm"] = time_gemm(S, torch, dev, flush)

@@ -8,8 +8,13 @@
 // ballot is block j, which is exactly the bit-sliced sign layout.  A warp
 // takes a run of tiles of one row and keeps eight tile loads in flight.  Kept
 // |w| are summed in double per lane, reduced over the warp once, then over the
-// warps of the row in a fixed order, so the scale is deterministic.
-// HBM-bound: 4 bytes read and 0.16 bytes written per weight.
+// warps of the row in a fixed order, so the scale is deterministic.  One
+// launch serves one matrix (sherry_pack) or a group of matrices
+// (sherry_pack_grouped: a model's projections at load time, without a launch
+// per matrix).  HBM-bound: 4 bytes read and 0.16 bytes written per weight.
+#include <algorithm>
+#include <cstring>
+
 #include "common.cuh"
 
 namespace sherry {
@@ -73,21 +78,45 @@ __device__ __forceinline__ void store_words(uint32_t *tile_out, const TileBits &
     if (lane < 5) tile_out[lane * SHERRY_ROW_GROUP] = word;
 }
 
-// CTA = 8 warps; `wpr` warps share one row, warp `sub` of a row takes the
-// `tpw` consecutive tiles sub * tpw .. and loads them kPackBatch at a time
-// (all loads of a batch in flight before the first tile is packed).  Each
-// lane sums its kept |w| in double over all its tiles; the lanes are reduced
-// once per warp and the warps of a row in a fixed order, so the scale is
-// deterministic.  Rows N..Npad-1 (padding of the last 32-row group) are
-// written as zero words.
-__global__ void __launch_bounds__(kPackThreads) pack_kernel(const float *__restrict__ w, int64_t N,
-                                                            int64_t Npad, int64_t K, int wpr,
-                                                            int64_t tpw, uint32_t *__restrict__ codes,
-                                                            float *__restrict__ scales) {
+// One launch packs a group of matrices; matrix i owns CTAs cta_begin[i] ..
+// cta_begin[i+1]-1.  CTA = 8 warps; `wpr` warps share one row, warp `sub` of
+// a row takes the `tpw` consecutive tiles sub * tpw .. and loads them
+// kPackBatch at a time (all loads of a batch in flight before the first tile
+// is packed).  Each lane sums its kept |w| in double over all its tiles; the
+// lanes are reduced once per warp and the warps of a row in a fixed order, so
+// the scale is deterministic.  Rows N..Npad-1 (padding of the last 32-row
+// group) are written as zero words.
+struct PackDesc {
+    const float *w;
+    uint32_t *codes;
+    float *scales;
+    int64_t N, Npad, K, tpw;
+    int wpr;
+    int cta_begin;
+};
+struct PackParams {
+    int count;
+    int pad;
+    PackDesc d[SHERRY_MAX_GROUP];
+};
+
+__global__ void __launch_bounds__(kPackThreads) pack_kernel(const __grid_constant__ PackParams P) {
     __shared__ double partial[kPackWarps];
+    int lo = 0, hi = P.count - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (P.d[mid].cta_begin <= (int)blockIdx.x) lo = mid; else hi = mid - 1;
+    }
+    const PackDesc &D = P.d[lo];
+    const float *__restrict__ w = D.w;
+    uint32_t *__restrict__ codes = D.codes;
+    float *__restrict__ scales = D.scales;
+    const int64_t N = D.N, Npad = D.Npad, K = D.K, tpw = D.tpw;
+    const int wpr = D.wpr;
+    const int64_t cta = (int64_t)blockIdx.x - D.cta_begin;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int rpc = kPackWarps / wpr;
-    const int64_t n = (int64_t)blockIdx.x * rpc + warp / wpr;
+    const int64_t n = cta * rpc + warp / wpr;
     const int sub = warp % wpr;
     const int64_t T = K / SHERRY_TILE_K;
     const int64_t t_begin = sub * tpw;
@@ -123,7 +152,7 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(const float *__restr
     if (lane == 0) partial[warp] = kept;
     __syncthreads();
     if (threadIdx.x < rpc) {
-        const int64_t rn = (int64_t)blockIdx.x * rpc + threadIdx.x;
+        const int64_t rn = cta * rpc + threadIdx.x;
         if (rn < N) {
             double s = 0.0;
             for (int k = 0; k < wpr; k++) s += partial[threadIdx.x * wpr + k];
@@ -133,24 +162,73 @@ __global__ void __launch_bounds__(kPackThreads) pack_kernel(const float *__restr
 }
 
 }  // namespace
+
+// Checks one matrix of a pack call.
+sherry_status pack_check(const float *w, int64_t N, int64_t K, const uint32_t *codes,
+                         const float *scales) {
+    if (!w || !codes || !scales) return SHERRY_ERR_NULL;
+    if (N < 1 || !valid_k(K)) return SHERRY_ERR_SHAPE;
+    if (!aligned(w, 16) || !aligned(codes, 16) || !aligned(scales, 4)) return SHERRY_ERR_ALIGN;
+    return SHERRY_OK;
+}
+
+// One launch over `count` checked matrices (w, codes, scales, N, K filled in).
+sherry_status pack_launch(PackDesc *descs, int count, cudaStream_t stream) {
+    static thread_local PackParams pp;
+    std::memset(&pp, 0, sizeof(pp));
+    pp.count = count;
+    int64_t ctas = 0;
+    for (int i = 0; i < count; i++) {
+        PackDesc &d = descs[i];
+        const int64_t T = d.K / SHERRY_TILE_K;
+        d.Npad = (d.N + SHERRY_ROW_GROUP - 1) / SHERRY_ROW_GROUP * SHERRY_ROW_GROUP;
+        // warps per row: as many as keep at least kPackMinTiles tiles each (up to 8)
+        int wpr = 1;
+        while (wpr < kPackWarps && (int64_t)wpr * 2 * kPackMinTiles <= T) wpr *= 2;
+        d.wpr = wpr;
+        d.tpw = (T + wpr - 1) / wpr;
+        const int rpc = kPackWarps / wpr;
+        d.cta_begin = (int)ctas;
+        ctas += (d.Npad + rpc - 1) / rpc;
+        if (ctas > 0x7FFFFFFF) return SHERRY_ERR_UNSUPPORTED;
+        pp.d[i] = d;
+    }
+    pack_kernel<<<(unsigned)ctas, kPackThreads, 0, stream>>>(pp);
+    return launch_status("sherry_pack");
+}
+
 }  // namespace sherry
 
 extern "C" sherry_status sherry_pack(const float *w, int64_t N, int64_t K, uint32_t *codes,
                                      float *scales, sherry_stream_t stream) {
     using namespace sherry;
-    if (!w || !codes || !scales) return SHERRY_ERR_NULL;
-    if (N < 1 || !valid_k(K)) return SHERRY_ERR_SHAPE;
-    if (!aligned(w, 16) || !aligned(codes, 16) || !aligned(scales, 4)) return SHERRY_ERR_ALIGN;
-    const int64_t T = K / SHERRY_TILE_K;
-    const int64_t Npad = (N + SHERRY_ROW_GROUP - 1) / SHERRY_ROW_GROUP * SHERRY_ROW_GROUP;
-    // warps per row: as many as keep at least kPackMinTiles tiles each (up to 8)
-    int wpr = 1;
-    while (wpr < kPackWarps && (int64_t)wpr * 2 * kPackMinTiles <= T) wpr *= 2;
-    const int64_t tpw = (T + wpr - 1) / wpr;
-    const int rpc = kPackWarps / wpr;
-    const int64_t grid = (Npad + rpc - 1) / rpc;
-    if (grid > 0x7FFFFFFF) return SHERRY_ERR_UNSUPPORTED;
-    pack_kernel<<<(unsigned)grid, kPackThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-        w, N, Npad, K, wpr, tpw, codes, scales);
-    return launch_status("sherry_pack");
+    const sherry_status st = pack_check(w, N, K, codes, scales);
+    if (st != SHERRY_OK) return st;
+    PackDesc d = {};
+    d.w = w;
+    d.codes = codes;
+    d.scales = scales;
+    d.N = N;
+    d.K = K;
+    return pack_launch(&d, 1, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" sherry_status sherry_pack_grouped(const sherry_pack_desc *descs, int count,
+                                             sherry_stream_t stream) {
+    using namespace sherry;
+    if (!descs) return SHERRY_ERR_NULL;
+    if (count < 1) return SHERRY_ERR_SHAPE;
+    if (count > SHERRY_MAX_GROUP) return SHERRY_ERR_UNSUPPORTED;
+    PackDesc d[SHERRY_MAX_GROUP] = {};
+    for (int i = 0; i < count; i++) {
+        const sherry_status st = pack_check(descs[i].w, descs[i].N, descs[i].K, descs[i].codes,
+                                            descs[i].scales);
+        if (st != SHERRY_OK) return st;
+        d[i].w = descs[i].w;
+        d[i].codes = descs[i].codes;
+        d[i].scales = descs[i].scales;
+        d[i].N = descs[i].N;
+        d[i].K = descs[i].K;
+    }
+    return pack_launch(d, count, reinterpret_cast<cudaStream_t>(stream));
 }

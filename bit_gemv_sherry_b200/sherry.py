@@ -35,6 +35,11 @@ class SherryError(RuntimeError):
         super().__init__(msg)
 
 
+class PackDesc(ctypes.Structure):
+    _fields_ = [("w", ctypes.c_void_p), ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("N", ctypes.c_int64), ("K", ctypes.c_int64)]
+
+
 class GemvDesc(ctypes.Structure):
     _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("x", ctypes.c_void_p),
                 ("y", ctypes.c_void_p), ("N", ctypes.c_int64), ("K", ctypes.c_int64)]
@@ -58,6 +63,7 @@ def lib():
     sig = {
         "sherry_packed_bytes": ([i64, i64], sz),
         "sherry_pack": ([p, i64, i64, p, p, p], i32),
+        "sherry_pack_grouped": ([p, i32, p], i32),
         "sherry_gemv_workspace_bytes": ([i64, i64, i32], sz),
         "sherry_gemv": ([p, p, p, p, i64, i64, i32, p, sz, p], i32),
         "sherry_gemv_acc": ([p, p, p, i64, i64, i32, p, sz, p], i32),
@@ -147,6 +153,41 @@ def pack(w, codes=None, scales=None):
         scales = torch.empty(N, dtype=torch.float32, device=w.device)
     _check(lib().sherry_pack(_ptr(w), N, K, _ptr(codes), _ptr(scales), _stream(w)), "sherry_pack")
     return codes, scales
+
+
+class GroupedPack:
+    """Pre-marshalled grouped pack (sherry_pack_grouped): items are
+    (w float32 [N, K], codes, scales) with codes/scales shaped as pack() makes them."""
+
+    def __init__(self, items):
+        n = len(items)
+        self.descs = (PackDesc * n)()
+        for i, (w, codes, scales) in enumerate(items):
+            _need(w, torch.float32, "w")
+            N, K = w.shape
+            _need(scales, torch.float32, "scales")
+            if tuple(codes.shape) != codes_shape(N, max(K, TILE_K)) or scales.numel() != N:
+                raise ValueError("codes/scales do not match w of shape %s" % (tuple(w.shape),))
+            self.descs[i] = PackDesc(w.data_ptr(), codes.data_ptr(), scales.data_ptr(), N, K)
+        self.items = items
+        self.n = n
+        self.device = items[0][0].device
+
+    def __call__(self, stream=None):
+        s = ctypes.c_void_p(stream if stream is not None
+                            else torch.cuda.current_stream(self.device).cuda_stream)
+        _check(lib().sherry_pack_grouped(ctypes.cast(self.descs, ctypes.c_void_p), self.n, s),
+               "sherry_pack_grouped")
+
+
+def pack_grouped(ws):
+    """Packs a list of float32 [N, K] CUDA matrices in one launch; returns
+    [(codes, scales)] as pack() would."""
+    outs = [(torch.empty(codes_shape(w.shape[0], max(w.shape[1], TILE_K)), dtype=torch.int32,
+                         device=w.device),
+             torch.empty(w.shape[0], dtype=torch.float32, device=w.device)) for w in ws]
+    GroupedPack([(w, c, s) for w, (c, s) in zip(ws, outs)])()
+    return outs
 
 
 def _codes_shape(codes, N):

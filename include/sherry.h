@@ -107,6 +107,28 @@ size_t sherry_packed_bytes(int64_t N, int64_t K);
 sherry_status sherry_pack(const float *w, int64_t N, int64_t K, uint32_t *codes,
                           float *scales, sherry_stream_t stream);
 
+/* One matrix of a grouped pack call (pointers and rules as for sherry_pack). */
+typedef struct {
+    const float *w;    /* [N][K] fp32, 16-byte aligned */
+    uint32_t *codes;   /* sherry_packed_bytes(N, K) bytes, 16-byte aligned */
+    float *scales;     /* [N] */
+    int64_t N;
+    int64_t K;
+} sherry_pack_desc;
+
+/*
+ * sherry_pack_grouped -- sherry_pack of `count` matrices (count <=
+ * SHERRY_MAX_GROUP) in one launch, e.g. every projection of a model at load
+ * time.  The results are those of one sherry_pack call per matrix, bit for bit.
+ *   descs  HOST array of `count` descriptors (copied into the launch
+ *          parameters; may be reused as soon as the call returns).
+ * Errors: NULL (descs or a pointer), SHAPE (count < 1 or a matrix's N, K),
+ * UNSUPPORTED (count > SHERRY_MAX_GROUP), ALIGN, CUDA.  Every descriptor is
+ * checked before anything is launched.
+ */
+sherry_status sherry_pack_grouped(const sherry_pack_desc *descs, int count,
+                                  sherry_stream_t stream);
+
 /*
  * Workspace of the GEMV calls.  Each call re-orders its activations once into
  * the order in which the decoded weights meet the tensor-core fragments, and

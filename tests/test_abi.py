@@ -61,6 +61,22 @@ def test_pack_argument_checks():
     assert L.sherry_pack(ctypes.c_void_p(0x100004), 4, 128, FAKE, FAKE, None) == 3
 
 
+def test_pack_grouped_argument_checks():
+    L = S.lib()
+    d = (S.PackDesc * 2)()
+    d[0] = S.PackDesc(0x100000, 0x100000, 0x100000, 4, 128)
+    d[1] = S.PackDesc(0x100000, 0x100000, None, 4, 128)
+    p = ctypes.cast(d, ctypes.c_void_p)
+    assert L.sherry_pack_grouped(None, 1, None) == 1
+    assert L.sherry_pack_grouped(p, 0, None) == 2
+    assert L.sherry_pack_grouped(p, 129, None) == 4
+    assert L.sherry_pack_grouped(p, 2, None) == 1      # desc 1 has no scales
+    d[1] = S.PackDesc(0x100000, 0x100000, 0x100000, 4, 200)
+    assert L.sherry_pack_grouped(p, 2, None) == 2      # K not a multiple of 128
+    d[1] = S.PackDesc(0x100008, 0x100000, 0x100000, 4, 128)
+    assert L.sherry_pack_grouped(p, 2, None) == 3      # w not 16-byte aligned
+
+
 def test_gemv_argument_checks():
     L = S.lib()
     ws = 1 << 20

@@ -63,6 +63,22 @@ def test_pack_full_size_1b_layers(layer):
     assert d.max() <= 1 and (d > 0).sum() <= max(1, N // 1000), name
 
 
+def test_pack_grouped_matches_single_calls_and_oracle():
+    # one launch over matrices of mixed shapes (ragged rows, K from 128 to 8192),
+    # bit for bit the codes and scales of one sherry_pack call per matrix
+    shapes = [(33, 640), (1, 128), (256, 1024), (7, 8192), (300, 2048), (64, 384), (5, 1152)]
+    ws = [synth.latent_weights(N, K, seed=30 + i) for i, (N, K) in enumerate(shapes)]
+    outs = S.pack_grouped([dev(w) for w in ws])
+    torch.cuda.synchronize()
+    for (N, K), w, (codes, scales) in zip(shapes, ws, outs):
+        c1, s1 = S.pack(dev(w))
+        assert np.array_equal(host_codes(codes), host_codes(c1)), (N, K)
+        assert np.array_equal(scales.cpu().numpy(), s1.cpu().numpy()), (N, K)
+        codes_ref, scales_ref = oracle.pack(w)
+        assert np.array_equal(host_codes(codes), codes_ref), (N, K)
+        assert ulp_diff_f32(scales.cpu().numpy(), scales_ref).max() <= 1, (N, K)
+
+
 # ----------------------------------------------------------------------------- gemv
 GEMV_CASES = [(256, 1024, 1), (1, 128, 1), (17, 384, 3), (33, 640, 5), (40, 1152, 8),
               (19, 256, 9), (64, 512, 16), (2048, 2048, 1), (512, 2048, 4), (100, 3072, 2),
