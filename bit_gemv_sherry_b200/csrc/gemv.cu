@@ -98,7 +98,14 @@ constexpr int kGemvWarps = kGemvThreads / 32;
 
 constexpr int kUnitRows = 32;      // pipelined kernel: rows per unit (two m16 blocks)
 constexpr int kChunkTiles = 4;     // tiles per K-chunk = per ring stage
-constexpr int kMaxPartChunks = 4;  // longest K-part: 4 chunks = 2048 weights per row
+// longest K-part: 16 chunks = 8192 weights per row, so rows up to K = 8192 are
+// never split.  A split row's K-parts meet through integer atomics and a
+// memory fence per part, which cost far more than the balance they buy:
+// measured on the 16-layer stacks, 4-chunk parts ran the 3B stack at B = 4 in
+// 245 us and the 1B stack in 54.4 us, 16-chunk parts in 107 us and 52.4 us.
+// Long rows (K > 8192) still split; an item cut between the warps of a CTA
+// is summed in shared memory instead.
+constexpr int kMaxPartChunks = 16;
 constexpr int kRing = 3;           // stages per warp
 // A stage holds one chunk: 4 tile blocks of 5 planes x 32 rows (160 words, a
 // contiguous 2560 bytes in global memory), each block padded to 168 words in
@@ -752,32 +759,41 @@ __global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
             const uint32_t *st = ring + slot * kStageWords + t * kTileWordsPadded + g;
             // padded tiles hold zero activations, so no load is predicated
             const size_t xoff = (size_t)c * kChunkTiles * 8;
+            // the four rows of this lane (g, g + 8 of row block 0, g + 16, g + 24 of row
+            // block 1) are decoded together, so each activation fragment is loaded once
+            // for both row blocks, and the next position's fragments are loaded while
+            // the current position's MMAs run
+            TileDecoder6 d[4];
 #pragma unroll
-            for (int rb = 0; rb < 2; rb++) {  // row block rb: rows g + 16 rb, g + 8 + 16 rb
-                TileDecoder6 d0, d1;
-                d0.load(C, st[0 * 32 + 16 * rb], st[1 * 32 + 16 * rb], st[2 * 32 + 16 * rb],
-                        st[3 * 32 + 16 * rb], st[4 * 32 + 16 * rb]);
-                d1.load(C, st[0 * 32 + 16 * rb + 8], st[1 * 32 + 16 * rb + 8],
-                        st[2 * 32 + 16 * rb + 8], st[3 * 32 + 16 * rb + 8], st[4 * 32 + 16 * rb + 8]);
-                if (rb == 1) {
-                    __syncwarp();  // every lane has its words: the stage can be refilled
-                    issue(slot == 0 ? kRing - 1 : slot - 1);
-                    slot = (slot + 1 == kRing) ? 0 : slot + 1;
-                }
+            for (int r = 0; r < 4; r++)
+                d[r].load(C, st[0 * 32 + 8 * r], st[1 * 32 + 8 * r], st[2 * 32 + 8 * r],
+                          st[3 * 32 + 8 * r], st[4 * 32 + 8 * r]);
+            __syncwarp();  // every lane has its words: the stage can be refilled
+            issue(slot == 0 ? kRing - 1 : slot - 1);
+            slot = (slot + 1 == kRing) ? 0 : slot + 1;
+            uint4 xq[NB][2], xn[NB][2];
 #pragma unroll
-                for (int i = 0; i < 4; i++) {
-                    uint4 xq[NB][2];
+            for (int nb = 0; nb < NB; nb++) {
+                xq[nb][0] = ld_x(xrow[nb] + xoff);
+                xq[nb][1] = ld_x(xrow[nb] + xoff + 1);
+            }
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                if (i < 3) {
 #pragma unroll
                     for (int nb = 0; nb < NB; nb++) {
-                        xq[nb][0] = ld_x(xrow[nb] + xoff + 2 * i);
-                        xq[nb][1] = ld_x(xrow[nb] + xoff + 2 * i + 1);
+                        xn[nb][0] = ld_x(xrow[nb] + xoff + 2 * i + 2);
+                        xn[nb][1] = ld_x(xrow[nb] + xoff + 2 * i + 3);
                     }
-                    const uint32_t tlo = C.tlo[i], thi = C.thi[i];
+                }
+                const uint32_t tlo = C.tlo[i], thi = C.thi[i];
 #pragma unroll
-                    for (int beta = 0; beta < 4; beta++) {
-                        const int m = 4 * i + beta;  // MMA index: activation words 2m, 2m+1
-                        const uint32_t s0 = d0.sel(C, i, beta);
-                        const uint32_t s1 = d1.sel(C, i, beta);
+                for (int beta = 0; beta < 4; beta++) {
+                    const int m = 4 * i + beta;  // MMA index: activation words 2m, 2m+1
+#pragma unroll
+                    for (int rb = 0; rb < 2; rb++) {  // row block rb: rows g + 16 rb, g + 8 + 16 rb
+                        const uint32_t s0 = d[2 * rb].sel(C, i, beta);
+                        const uint32_t s1 = d[2 * rb + 1].sel(C, i, beta);
                         const uint32_t a0 = prmt(tlo, thi, s0);
                         const uint32_t a2 = prmt(tlo, thi, hi_half(C, s0));
                         const uint32_t a1 = prmt(tlo, thi, s1);
@@ -788,6 +804,13 @@ __global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
                             mma_s8(acc[rb][nb], a0, a1, a2, a3, pick(xx, (m & 1) * 2),
                                    pick(xx, (m & 1) * 2 + 1));
                         }
+                    }
+                }
+                if (i < 3) {
+#pragma unroll
+                    for (int nb = 0; nb < NB; nb++) {
+                        xq[nb][0] = xn[nb][0];
+                        xq[nb][1] = xn[nb][1];
                     }
                 }
             }

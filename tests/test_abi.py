@@ -46,9 +46,13 @@ def test_packed_and_workspace_sizes():
     assert S.gemv_workspace_bytes(100, 384, 3) == 3 * 512
     assert S.gemv_workspace_bytes(40, 1024, 2) == 2 * 8 * 128
     assert S.gemv_workspace_bytes(2048, 2048, 1) == 2048
-    # 16 chunks per row -> 4 K-parts: activations, then partial sums [B][N] and 64 unit counters
-    assert S.gemv_workspace_bytes(2048, 8192, 1) == 4 * 64 * 32 + 4 * (2048 + 64)
-    assert S.gemv_workspace_bytes(100, 8192, 3) == 3 * 4 * 64 * 32 + 256 * ((4 * (300 + 4) + 255) // 256)
+    # up to 16 chunks per row: one K-part, re-ordered activations only
+    assert S.gemv_workspace_bytes(2048, 8192, 1) == 4 * 64 * 32
+    assert S.gemv_workspace_bytes(100, 8192, 3) == 3 * 4 * 64 * 32
+    # 34 chunks per row -> 3 K-parts: activations, then partial sums [B][N] and one
+    # counter per 32-row unit, rounded to 256 bytes
+    assert S.gemv_workspace_bytes(2048, 17408, 1) == 4 * 136 * 32 + 256 * ((4 * (2048 + 64) + 255) // 256)
+    assert S.gemv_workspace_bytes(100, 17408, 3) == 3 * 4 * 136 * 32 + 256 * ((4 * (300 + 4) + 255) // 256)
     assert S.gemv_workspace_bytes(16, 128, 0) == 0
 
 
@@ -103,7 +107,8 @@ def test_gemv_static_argument_checks():
     assert L.sherry_gemv_static(FAKE, FAKE, FAKE, FAKE, 4, 130, 1, None) == 2
     assert L.sherry_gemv_static(FAKE, FAKE, FAKE, FAKE, 4, 128, 17, None) == 4
     # beyond the 4 MiB static scratch: rejected on the host with both sizes in the message
-    assert L.sherry_gemv_static(FAKE, FAKE, FAKE, FAKE, 100000, 8192, 16, None) == 7
+    # 2 MiB of activations plus 6.4 MB of K-part sums: beyond the 4 MiB array
+    assert L.sherry_gemv_static(FAKE, FAKE, FAKE, FAKE, 100000, 131072, 16, None) == 7
     assert b"4194304" in L.sherry_last_error()
 
 

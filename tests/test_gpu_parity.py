@@ -84,8 +84,9 @@ GEMV_CASES = [(256, 1024, 1), (1, 128, 1), (17, 384, 3), (33, 640, 5), (40, 1152
               (19, 256, 9), (64, 512, 16), (2048, 2048, 1), (512, 2048, 4), (100, 3072, 2),
               (31, 8192, 1), (48, 8192, 16), (50, 1536, 2), (23, 512, 1), (70, 2560, 9),
               (129, 4096, 8), (37, 8192, 2), (130, 2048, 3),
-              # B <= 2 with short last K-parts (5, 7 and 10 chunks per row)
-              (70, 2560, 1), (33, 3584, 2), (300, 5120, 1)]
+              # rows split into K-parts (K > 8192), short last parts included:
+              # 21 chunks = 11 + 10, 34 = 12 + 12 + 10, 40 = 3 x 14 - 2, 128 = 8 x 16
+              (70, 10752, 1), (33, 17408, 2), (40, 20480, 9), (20, 65536, 1), (65, 17408, 16)]
 
 
 @pytest.mark.parametrize("N,K,B", GEMV_CASES)
@@ -164,7 +165,7 @@ def test_gemv_grouped_cut_items(B):
     # many small GEMVs of mixed K (short last K-parts included) in one launch:
     # warp ranges cut items at many places, inside and across GEMVs
     shapes = [(33, 640), (96, 8192), (1, 128), (70, 2560), (200, 2048), (45, 3584),
-              (64, 5120), (7, 384), (130, 4096), (31, 1152)] * 3
+              (64, 5120), (7, 384), (130, 4096), (31, 1152), (40, 10752), (9, 17408)] * 3
     items, refs = [], []
     for li, (N, K) in enumerate(shapes):
         codes, scales = oracle.pack(synth.latent_weights(N, K, seed=200 + li))
@@ -264,7 +265,7 @@ def test_gemv_prepare_then_run_equals_grouped():
 def test_gemv_run_repeats_after_one_prepare():
     # K-parts meet in the workspace; every run must leave it ready for the next
     items, refs = [], []
-    for li, (N, K) in enumerate([(96, 8192), (70, 3072), (33, 2048)]):
+    for li, (N, K) in enumerate([(96, 8192), (70, 3072), (33, 2048), (48, 12288), (40, 17408)]):
         codes, scales = oracle.pack(synth.latent_weights(N, K, seed=60 + li))
         x = synth.int8_uniform((2, K), seed=70 + li)
         y = torch.zeros((2, N), dtype=torch.float32, device="cuda")

@@ -59,7 +59,7 @@ def test_static_binding_and_repeat_after_other_shapes():
 
 
 def test_static_rejects_sizes_beyond_the_scratch():
-    N, K, B = 100000, 8192, 16
+    N, K, B = 100000, 131072, 16  # K-part sums of rows split past K = 8192
     assert S.gemv_workspace_bytes(N, K, B) > S.STATIC_SCRATCH_BYTES
     fake = ctypes.c_void_p(0x100000)
     L = S.lib()
