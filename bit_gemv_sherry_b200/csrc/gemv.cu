@@ -199,6 +199,9 @@ __device__ __forceinline__ uint32_t quant_word(uint2 v, float inv) {
 __device__ __forceinline__ float row_absmax_bf16(const uint16_t *row, int K, int lane) {
     float m = 0.0f;
     const uint4 *r4 = reinterpret_cast<const uint4 *>(row);  // 8 values per uint4
+    // eight loads in flight per lane: the row comes from L2, one load at a time
+    // would expose its latency K / 256 times
+#pragma unroll 8
     for (int i = lane; i < K / 8; i += 32) {
         const uint4 v = __ldg(r4 + i);
         m = fmaxf(m, fmaxf(fmaxf(fabsf(bf16_lo(v.x)), fabsf(bf16_hi(v.x))),
