@@ -38,8 +38,8 @@ METRIC = "W1.25A8 GEMV weight GB/s at batch 1 (LLaMA-3.2-1B decode stack)"
 UNIT = "GB/s"
 L2_BYTES = 126 * 2 ** 20
 # ncu capture of gemv_dot_kernel<1,false> on the 16-layer stack, B = 1:
-# dram read 154,045,696 + write 4,195,840 bytes per launch
-NCU_TRAFFIC_BYTES = 154045696 + 4195840
+# dram read 153,907,200 + write 5,125,376 bytes per launch
+NCU_TRAFFIC_BYTES = 153907200 + 5125376
 
 
 def parse_args():
