@@ -14,6 +14,8 @@ from .oracle import (  # noqa: F401
     pack,
     unpack,
     quantize_act,
+    quantize_f32,
+    swiglu,
     gemv_act,
     bf16_bits,
     gemv_acc,

@@ -45,8 +45,11 @@ def _load(path=None):
     lib.oracle_gemm.argtypes = [p, p, p, i64, i64, i64, p]
     lib.oracle_quantize_act.argtypes = [p, i64, i64, p, p]
     lib.oracle_gemv_act.argtypes = [p, p, p, p, i64, i64, i64, p]
+    lib.oracle_quantize_f32.argtypes = [p, i64, i64, p, p]
+    lib.oracle_swiglu.argtypes = [p, p, i64, p]
     for f in ("oracle_pack", "oracle_unpack", "oracle_gemv_acc", "oracle_gemv",
-              "oracle_gemm_acc", "oracle_gemm", "oracle_quantize_act", "oracle_gemv_act"):
+              "oracle_gemm_acc", "oracle_gemm", "oracle_quantize_act", "oracle_gemv_act",
+              "oracle_quantize_f32", "oracle_swiglu"):
         getattr(lib, f).restype = ctypes.c_int
     lib.oracle_num_threads.argtypes = []
     lib.oracle_num_threads.restype = ctypes.c_int
@@ -188,6 +191,30 @@ def quantize_act(x_bf16):
     s = np.zeros(B, np.float32)
     _check(_load().oracle_quantize_act(_ptr(x), B, K, _ptr(q), _ptr(s)), "oracle_quantize_act")
     return q, s
+
+
+def quantize_f32(x):
+    """Per-token absmax int8 quantization of fp32 activations [B][K] -> (q int8
+    [B][K], s float32 [B]); the rule of quantize_act, read from fp32 values."""
+    x = np.ascontiguousarray(x, dtype=np.float32)
+    if x.ndim == 1:
+        x = x.reshape(1, -1)
+    B, K = x.shape
+    q = np.zeros((B, K), np.int8)
+    s = np.zeros(B, np.float32)
+    _check(_load().oracle_quantize_f32(_ptr(x), B, K, _ptr(q), _ptr(s)), "oracle_quantize_f32")
+    return q, s
+
+
+def swiglu(g, u):
+    """h = silu(g) * u elementwise (fp32 in, double evaluation, fp32 out)."""
+    g = np.ascontiguousarray(g, dtype=np.float32)
+    u = np.ascontiguousarray(u, dtype=np.float32)
+    if g.shape != u.shape:
+        raise ValueError("g and u differ in shape")
+    h = np.zeros(g.shape, np.float32)
+    _check(_load().oracle_swiglu(_ptr(g), _ptr(u), g.size, _ptr(h)), "oracle_swiglu")
+    return h
 
 
 def gemv_act(codes, scales, q, sx, K):

@@ -275,30 +275,67 @@ static float orc_bf16(uint16_t h)
     return f;
 }
 
+/* The rule above on one token row of fp32 values. */
+static void orc_quantize_row(const float *xr, int64_t K, int8_t *q, float *s)
+{
+    float amax = 0.0f;
+    for (int64_t k = 0; k < K; k++) {
+        const float a = fabsf(xr[k]);
+        if (a > amax) amax = a;
+    }
+    if (amax == 0.0f) {
+        *s = 0.0f;
+        memset(q, 0, (size_t)K);
+        return;
+    }
+    const float inv = 127.0f / amax;
+    *s = amax / 127.0f;
+    for (int64_t k = 0; k < K; k++) {
+        const float v = xr[k] * inv;
+        float r = nearbyintf(v);
+        if (r > 127.0f) r = 127.0f;
+        if (r < -127.0f) r = -127.0f;
+        q[k] = (int8_t)r;
+    }
+}
+
 int oracle_quantize_act(const uint16_t *x, int64_t B, int64_t K, int8_t *q, float *s)
 {
     if (!x || !q || !s || B < 1 || K < 1) return ORC_BAD_ARG;
+    float *row = (float *)malloc(sizeof(float) * (size_t)K);
+    if (!row) return ORC_NO_MEM;
     for (int64_t b = 0; b < B; b++) {
-        const uint16_t *xr = x + b * K;
-        float amax = 0.0f;
-        for (int64_t k = 0; k < K; k++) {
-            const float a = fabsf(orc_bf16(xr[k]));
-            if (a > amax) amax = a;
-        }
-        if (amax == 0.0f) {
-            s[b] = 0.0f;
-            memset(q + b * K, 0, (size_t)K);
-            continue;
-        }
-        const float inv = 127.0f / amax;
-        s[b] = amax / 127.0f;
-        for (int64_t k = 0; k < K; k++) {
-            const float v = orc_bf16(xr[k]) * inv;
-            float r = nearbyintf(v);
-            if (r > 127.0f) r = 127.0f;
-            if (r < -127.0f) r = -127.0f;
-            q[b * K + k] = (int8_t)r;
-        }
+        for (int64_t k = 0; k < K; k++) row[k] = orc_bf16(x[b * K + k]);
+        orc_quantize_row(row, K, q + b * K, s + b);
+    }
+    free(row);
+    return ORC_OK;
+}
+
+/*
+ * Re-quantization of fp32 activations (for example the y of a previous GEMV,
+ * feeding the next layer): the same per-token rule, read from fp32 values.
+ */
+int oracle_quantize_f32(const float *x, int64_t B, int64_t K, int8_t *q, float *s)
+{
+    if (!x || !q || !s || B < 1 || K < 1) return ORC_BAD_ARG;
+    for (int64_t b = 0; b < B; b++) orc_quantize_row(x + b * K, K, q + b * K, s + b);
+    return ORC_OK;
+}
+
+/*
+ * SwiGLU, the gated activation of the LLaMA MLP (the models the method is
+ * evaluated on are LLaMA-3.2 1B and 3B): the down projection's input is
+ *     h = silu(g) * u,   silu(g) = g / (1 + e^(-g)),
+ * with g and u the gate and up projections' outputs.  Evaluated in double
+ * and rounded once to fp32.
+ */
+int oracle_swiglu(const float *g, const float *u, int64_t n, float *h)
+{
+    if (!g || !u || !h || n < 1) return ORC_BAD_ARG;
+    for (int64_t i = 0; i < n; i++) {
+        const double gd = (double)g[i];
+        h[i] = (float)(gd / (1.0 + exp(-gd)) * (double)u[i]);
     }
     return ORC_OK;
 }

@@ -266,3 +266,80 @@ def test_gemv_act_equals_scaled_bruteforce():
     acc = q.astype(np.int64) @ wt.T
     ref = scales.astype(np.float64)[None, :] * sx.astype(np.float64)[:, None] * acc
     assert np.array_equal(oracle.gemv_act(codes, scales, q, sx, K), ref)
+
+
+# ---------------------------------------------------------------------------
+# Front-end on fp32 activations (re-quantization of a GEMV's y for the next
+# layer): the per-token rule above, read from fp32 values.  Expected values
+# are derived by hand.
+# ---------------------------------------------------------------------------
+def test_quantize_f32_hand_cases():
+    # amax = 1: 127 / 1 = 127 and s = fl32(1 / 127).  -0.5 -> -63.5 -> -64
+    # (ties to even); 0.25 -> 31.75 -> 32; fl32(0.3) * 127 = 38.100002 -> 38;
+    # 0.99999994 (the float below 1) -> 126.99999 -> 127.  0.7441181 is read
+    # as fp32: 0.7441181 * 127 = 94.503 -> 95, where a bf16 copy of it
+    # (0.7421875, rounded or truncated) would give 94.26 -> 94.
+    x = np.array([[1.0, 0.99999994, -0.5, 0.25, 0.0, -1.0, 0.3, 0.7441181]], np.float32)
+    q, s = oracle.quantize_f32(x)
+    assert s[0] == np.float32(1.0) / np.float32(127.0)
+    assert q.tolist() == [[127, 127, -64, 32, 0, -127, 38, 95]]
+    # amax = 254 (second row): 127 / 254 = 0.5 exactly; 3.0 -> 1.5 -> 2,
+    # 5.0 -> 2.5 -> 2, -7.0 -> -3.5 -> -4; s = 2
+    q, s = oracle.quantize_f32(np.array([[3.0, 5.0, -7.0, 254.0], [0.0, 0.0, 0.0, 0.0]], np.float32))
+    assert s.tolist() == [2.0, 0.0]
+    assert q.tolist() == [[2, 2, -4, 127], [0, 0, 0, 0]]
+
+
+def test_quantize_f32_bounds_on_random_rows():
+    rng = np.random.default_rng(15)
+    x = rng.standard_normal((6, 384)).astype(np.float32) * np.array([1, 1e-3, 10, 1e4, 0.5, 3],
+                                                                    np.float32)[:, None]
+    q, s = oracle.quantize_f32(x)
+    amax = np.abs(x).max(axis=1)
+    assert np.array_equal(s, (amax / np.float32(127.0)).astype(np.float32))
+    assert np.abs(q.astype(np.int32)).max() <= 127
+    for b in range(6):
+        k = np.argmax(np.abs(x[b]))
+        assert abs(int(q[b, k])) == 127 and np.sign(q[b, k]) == np.sign(x[b, k])
+        err = np.abs(q[b].astype(np.float64) * float(s[b]) - x[b].astype(np.float64))
+        assert err.max() <= 0.5 * float(s[b]) * (1 + 1e-5)
+
+
+# ---------------------------------------------------------------------------
+# SwiGLU h = silu(g) * u, silu(g) = g / (1 + e^-g): closed forms of the
+# logistic function and the known minimum of silu.
+# ---------------------------------------------------------------------------
+def test_swiglu_closed_forms():
+    # silu(0) = 0; e^-ln3 = 1/3, so silu(ln 3) = (3/4) ln 3 (to fp32 rounding of
+    # ln 3, whose effect on the logistic factor is below 2e-8)
+    ln3 = np.float32(np.log(3.0))
+    g = np.array([0.0, ln3, ln3, -ln3, 40.0, -40.0, 2.0], np.float32)
+    u = np.array([5.0, 1.0, -2.0, 1.0, -3.0, 1.0, 0.0], np.float32)
+    h = oracle.swiglu(g, u).astype(np.float64)
+    assert h[0] == 0.0 and h[6] == 0.0
+    assert abs(h[1] - 0.75 * float(ln3)) <= 2e-7 * abs(h[1])
+    assert abs(h[2] + 1.5 * float(ln3)) <= 2e-7 * abs(h[2])
+    # silu(-g) = -g * e^-g / (1 + e^-g): at -ln 3 the factor is 1/4
+    assert abs(h[3] + 0.25 * float(ln3)) <= 2e-7 * abs(h[3])
+    # far tails: silu(40) = 40 to fp32; silu(-40) = -40 e^-40 / (1 + e^-40)
+    assert h[4] == -120.0
+    assert abs(h[5] + 40.0 * np.exp(-40.0)) <= 1e-6 * 40.0 * np.exp(-40.0)
+    # odd part: silu(g) - silu(-g) = g, since the logistic function satisfies
+    # sigma(g) + sigma(-g) = 1
+    rng = np.random.default_rng(21)
+    gr = (rng.standard_normal(4096) * 4).astype(np.float32)
+    one = np.ones_like(gr)
+    d = oracle.swiglu(gr, one).astype(np.float64) - oracle.swiglu(-gr, one).astype(np.float64)
+    assert np.all(np.abs(d - gr.astype(np.float64)) <= 2.4e-7 * np.maximum(np.abs(gr), 1.0))
+
+
+def test_swiglu_minimum_is_lambert_w():
+    # d/dg [g sigma(g)] = 0  <=>  e^g (g + 1) = -1  <=>  g* = -1 - W(1/e), and
+    # there silu(g*) = g* + 1 = -W(1/e)  (W: Lambert's W, principal branch)
+    from scipy.special import lambertw
+    w = float(lambertw(np.exp(-1.0)).real)
+    gs = np.float32(-1.0 - w)
+    g = np.array([gs, gs - np.float32(0.05), gs + np.float32(0.05)], np.float32)
+    h = oracle.swiglu(g, np.ones(3, np.float32)).astype(np.float64)
+    assert abs(h[0] + w) <= 1e-6
+    assert h[1] > h[0] and h[2] > h[0]

@@ -45,8 +45,13 @@ MUTANTS = {
                           "return ((n / ORC_GROUP) * T + t) * (ORC_NPLANE * ORC_GROUP) + (n % ORC_GROUP) * ORC_NPLANE + plane;"),
     "quantize_truncates": ("float r = nearbyintf(v);", "float r = truncf(v);"),
     "quantize_ties_away": ("float r = nearbyintf(v);", "float r = roundf(v);"),
-    "quantize_scale_over_128": ("s[b] = amax / 127.0f;", "s[b] = amax / 128.0f;"),
+    "quantize_scale_over_128": ("*s = amax / 127.0f;", "*s = amax / 128.0f;"),
     "quantize_inverse_scale_128": ("const float inv = 127.0f / amax;", "const float inv = 128.0f / amax;"),
+    "quantize_f32_reads_row_0": ("orc_quantize_row(x + b * K, K, q + b * K, s + b);",
+                                 "orc_quantize_row(x, K, q + b * K, s + b);"),
+    "swiglu_exp_of_plus_g": ("gd / (1.0 + exp(-gd))", "gd / (1.0 + exp(gd))"),
+    "swiglu_drops_up": ("gd / (1.0 + exp(-gd)) * (double)u[i]", "gd / (1.0 + exp(-gd))"),
+    "swiglu_sigmoid_only": ("gd / (1.0 + exp(-gd)) * (double)u[i]", "1.0 / (1.0 + exp(-gd)) * (double)u[i]"),
     "act_scale_dropped": ("y[b * N + n] = (double)scales[n] * (double)sx[b] * (double)acc[b * N + n];",
                           "y[b * N + n] = (double)scales[n] * (double)acc[b * N + n];"),
 }
@@ -67,6 +72,10 @@ def _run_pins(golden_dir):
         pins.test_quantize_act_hand_cases,
         pins.test_quantize_act_bounds_on_random_rows,
         pins.test_gemv_act_equals_scaled_bruteforce,
+        pins.test_quantize_f32_hand_cases,
+        pins.test_quantize_f32_bounds_on_random_rows,
+        pins.test_swiglu_closed_forms,
+        pins.test_swiglu_minimum_is_lambert_w,
     ]
     for c in checks:
         try:
