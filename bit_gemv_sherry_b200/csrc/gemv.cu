@@ -28,6 +28,8 @@
 #include <cstring>
 #include <mutex>
 
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 
 namespace sherry {
@@ -91,6 +93,29 @@ struct XprepParams {
     int total_units;
     int pad;
     XprepDesc d[SHERRY_MAX_GROUP];
+};
+
+// Front-end on fp32 activations: the y of a previous GEMV, or (u set) the
+// SwiGLU h = silu(g) * u of a gate and an up projection.
+struct XprepF32Desc {
+    const float *x;       // [B][K] activations; SwiGLU: the gate outputs g
+    const float *u;       // SwiGLU: the up outputs [B][K]; null for plain fp32
+    float *xscale;        // per batch row activation scales written here
+    uint32_t *xw;         // re-ordered activations [B][Tp][32 words], or null
+    int8_t *q;            // natural-order int8 output [B][K] (front-end alone), or null
+    uint32_t *zero;       // split-K partial sums and counters to clear
+    int K;
+    int Tp;
+    int cluster_begin;    // first cluster (= token row) of this GEMV
+    int zero_words;
+};
+
+struct XprepF32Params {
+    int count;
+    int B;
+    int total_clusters;
+    int pad;
+    XprepF32Desc d[SHERRY_MAX_GROUP];
 };
 
 constexpr int kGemvThreads = 256;
@@ -261,6 +286,105 @@ __global__ void __launch_bounds__(256) xprep_kernel(const __grid_constant__ Xpre
             if (w < D.zero_words) D.zero[w] = 0u;
         }
     }
+}
+
+// SwiGLU of the LLaMA MLP: silu(g) * u = g / (1 + e^-g) * u, each operation
+// rounded once (IEEE single precision; expf is CUDA's, within 2 ulp).  A g so
+// negative that e^-g overflows gives g / inf = -0.
+__device__ __forceinline__ float swiglu_f32(float g, float u) {
+    return __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, expf(-g))), u);
+}
+
+// Four consecutive activations of a token row from offset `off`.
+__device__ __forceinline__ float4 act4(const XprepF32Desc &D, size_t off) {
+    float4 a = __ldg(reinterpret_cast<const float4 *>(D.x + off));
+    if (D.u) {
+        const float4 v = __ldg(reinterpret_cast<const float4 *>(D.u + off));
+        a.x = swiglu_f32(a.x, v.x);
+        a.y = swiglu_f32(a.y, v.y);
+        a.z = swiglu_f32(a.z, v.z);
+        a.w = swiglu_f32(a.w, v.w);
+    }
+    return a;
+}
+
+constexpr int kF32Cluster = 8;                  // CTAs per token row (one cluster)
+constexpr int kF32Threads = 256;
+constexpr int kF32Warps = kF32Threads / 32;
+constexpr int kF32ClusterWarps = kF32Cluster * kF32Warps;
+
+// One thread-block cluster per (GEMV, token row).  Its 64 warps take the
+// row's 128-element tiles in turn: the first pass forms the activations and
+// their absolute maximum, the CTAs exchange their maxima through distributed
+// shared memory at a cluster barrier, and the second pass forms them again,
+// quantizes them with the per-token rule of the bf16 front-end and re-orders
+// them (or writes them in natural order).  Forming an activation twice costs
+// less than keeping the row: a 8192-element row is 1024 elements per CTA.
+__global__ void __launch_bounds__(kF32Threads) xprep_f32_kernel(const __grid_constant__ XprepF32Params P) {
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    __shared__ float warp_max[kF32Warps];
+    __shared__ float cta_max, row_max;
+    pdl_allow_dependents();
+    pdl_wait();  // x and u may come from the kernel before; the last GEMV may still read xw
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int rank = (int)cluster.block_rank();
+    const int ci = (int)(blockIdx.x / kF32Cluster);
+    int lo = 0, hi = P.count - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (P.d[mid].cluster_begin <= ci) lo = mid; else hi = mid - 1;
+    }
+    const XprepF32Desc &D = P.d[lo];
+    const int b = ci - D.cluster_begin;
+    const int T = D.K / SHERRY_TILE_K;
+    const int cw = rank * kF32Warps + warp;  // warp index within the cluster
+    const size_t row = (size_t)b * D.K;
+
+    float m = 0.0f;
+    for (int t = cw; t < T; t += kF32ClusterWarps) {
+        const float4 a = act4(D, row + (size_t)t * SHERRY_TILE_K + 4 * lane);
+        m = fmaxf(m, fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w))));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if (lane == 0) warp_max[warp] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float c = 0.0f;
+        for (int w = 0; w < kF32Warps; w++) c = fmaxf(c, warp_max[w]);
+        cta_max = c;
+    }
+    cluster.sync();  // every CTA's maximum is in its shared memory
+    if (warp == 0) {
+        float r = lane < kF32Cluster ? *cluster.map_shared_rank(&cta_max, (unsigned)lane) : 0.0f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) r = fmaxf(r, __shfl_xor_sync(0xFFFFFFFFu, r, o));
+        if (lane == 0) row_max = r;
+    }
+    __syncthreads();
+    const float amax = row_max;
+    const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+    if (rank == 0 && threadIdx.x == 0) D.xscale[b] = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
+
+    const int t_end = D.q ? T : D.Tp;
+    for (int t = cw; t < t_end; t += kF32ClusterWarps) {
+        uint32_t raw = 0u;
+        if (t < T) {
+            const float4 a = act4(D, row + (size_t)t * SHERRY_TILE_K + 4 * lane);
+            raw = quant_byte(a.x, inv) | (quant_byte(a.y, inv) << 8) | (quant_byte(a.z, inv) << 16) |
+                  (quant_byte(a.w, inv) << 24);
+        }
+        if (D.q)
+            reinterpret_cast<uint32_t *>(D.q + row + (size_t)t * SHERRY_TILE_K)[lane] = raw;
+        else
+            D.xw[((size_t)b * D.Tp + t) * 32 + lane] = reorder_word(raw, lane);
+    }
+    // the GEMV's split-K words, cleared by its clusters together
+    const int stride = P.B * kF32Cluster * kF32Threads;
+    for (int w = (b * kF32Cluster + rank) * kF32Threads + (int)threadIdx.x; w < D.zero_words; w += stride)
+        D.zero[w] = 0u;
+    cluster.sync();  // no CTA leaves while another may still read its maximum
 }
 
 // ---------------------------------------------------------------------------
@@ -1136,6 +1260,26 @@ void launch_pdl(KernelT kernel, int grid, int threads, size_t smem, cudaStream_t
     cudaLaunchKernelEx(&cfg, kernel, gp);
 }
 
+// The fp32 front-end: one cluster of kF32Cluster CTAs per (GEMV, token row),
+// launched like the others with programmatic stream serialization.
+void launch_xprep_f32(const XprepF32Params &p, cudaStream_t stream) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(p.total_clusters * kF32Cluster));
+    cfg.blockDim = dim3((unsigned)kF32Threads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kF32Cluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    cudaLaunchKernelEx(&cfg, xprep_f32_kernel, p);
+}
+
 template <typename KernelT>
 int grid_for(KernelT kernel, int threads, size_t smem, int want, int *cache) {
     int dev = 0;
@@ -1190,6 +1334,8 @@ struct GemvCall {
     void *out;
     int64_t N, K;
     const uint16_t *xbf;    // bf16 activations (quantized per token), or null
+    const float *xf = nullptr;  // fp32 activations (quantized per token), or null
+    const float *xu = nullptr;  // with xf: SwiGLU up outputs, the activations being silu(xf) * xu
 };
 
 // Words after a GEMV's region for the activation scales of the bf16 front-end.
@@ -1209,16 +1355,17 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
     for (int i = 0; i < count; i++) {
         const GemvCall &c = calls[i];
         const bool need_x = (phase & kPrepare) != 0, need_out = (phase & kRun) != 0;
-        if ((need_x && !c.x && !c.xbf) ||
+        if ((need_x && !c.x && !c.xbf && !c.xf) ||
             (need_out && (!c.codes || !c.out || (!acc_out && !c.scales))))
             return SHERRY_ERR_NULL;
         if (c.N < 1 || !valid_k(c.K)) return SHERRY_ERR_SHAPE;
         if ((need_x && c.x && !aligned(c.x, 4)) || (need_x && c.xbf && !aligned(c.xbf, 16)) ||
+            (need_x && c.xf && !aligned(c.xf, 16)) || (need_x && c.xu && !aligned(c.xu, 16)) ||
             (need_out && (!aligned(c.codes, 4) || !aligned(c.out, 4) ||
                           (c.scales && !aligned(c.scales, 4)))))
             return SHERRY_ERR_ALIGN;
         if (c.N > (int64_t)1 << 28) return SHERRY_ERR_UNSUPPORTED;
-        words += ws_words(c.N, c.K, B) + (c.xbf ? kActScaleWords : 0);
+        words += ws_words(c.N, c.K, B) + ((c.xbf || c.xf) ? kActScaleWords : 0);
         units16 += (c.N + 15) / 16;
         const int64_t nchunk = padded_tiles(c.K) / kChunkTiles;
         const int64_t kparts = kparts_for(c.K);
@@ -1236,12 +1383,21 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
             ((phase & kRun) && !aligned(calls[i].codes, 16)))
             pipelined = false;
 
+    // one front-end per call: the fp32 one runs as its own cluster launch
+    int nf32 = 0;
+    for (int i = 0; i < count; i++) nf32 += calls[i].xf != nullptr;
+    if (nf32 != 0 && nf32 != count) return SHERRY_ERR_UNSUPPORTED;
+    const bool f32 = nf32 == count;
+
     static thread_local XprepParams xp;
+    static thread_local XprepF32Params fp;
     static thread_local GemvParams gp;
     std::memset(&xp, 0, sizeof(xp));
     std::memset(&gp, 0, sizeof(gp));
-    xp.count = gp.count = count;
-    xp.B = gp.B = B;
+    if (f32) std::memset(&fp, 0, sizeof(fp));
+    xp.count = gp.count = fp.count = count;
+    xp.B = gp.B = fp.B = B;
+    fp.total_clusters = count * B;
     gp.mul4 = 4u;
     gp.mul2 = 2u;
     gp.f16one = 0x3C003C00u;
@@ -1268,8 +1424,8 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
         const int nchunk = Tp / kChunkTiles;
         const int kparts = (int)kparts_for(c.K);
         const int cpp = (nchunk + kparts - 1) / kparts;
-        const bool bf = c.xbf != nullptr;
-        // activation scales of the bf16 front-end follow the GEMV's regular words
+        const bool bf = c.xbf != nullptr || c.xf != nullptr;
+        // activation scales of the bf16 or fp32 front-end follow the GEMV's regular words
         float *act_scale = bf ? reinterpret_cast<float *>(region + ws_words(c.N, c.K, B)) : nullptr;
         XprepDesc &X = xp.d[i];
         X.x = c.x;
@@ -1283,6 +1439,19 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
         X.xunits = bf ? B * ((Tp + kXqTiles - 1) / kXqTiles) : B * Tp;
         X.zero_words = (int)split_words(c.N, c.K, B);
         X.kind = bf ? 1 : 0;
+        if (f32) {
+            XprepF32Desc &F = fp.d[i];
+            F.x = c.xf;
+            F.u = c.xu;
+            F.xscale = act_scale;
+            F.xw = region;
+            F.q = nullptr;
+            F.zero = X.zero;
+            F.K = (int)c.K;
+            F.Tp = Tp;
+            F.cluster_begin = i * B;
+            F.zero_words = X.zero_words;
+        }
         GemvDesc &D = gp.d[i];
         D.codes = c.codes;
         D.scales = c.scales;
@@ -1309,8 +1478,12 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
     gp.total_units16 = ub16;
     gp.total_chunks = cb;
     if (phase & kPrepare) {
-        const int blocks = std::max(1, std::min((wb + 7) / 8, sm_count() * 8));
-        launch_pdl(xprep_kernel, blocks, 256, 0, stream, xp);
+        if (f32) {
+            launch_xprep_f32(fp, stream);
+        } else {
+            const int blocks = std::max(1, std::min((wb + 7) / 8, sm_count() * 8));
+            launch_pdl(xprep_kernel, blocks, 256, 0, stream, xp);
+        }
         const sherry_status st = launch_status("sherry_gemv (activation re-order)");
         if (st != SHERRY_OK) return st;
     }
@@ -1363,6 +1536,44 @@ sherry_status grouped_bf16(const sherry_gemv_bf16_desc *descs, int count, int B,
                             descs[i].K, descs[i].x};
     }
     return gemv_launch(calls, count, B, false, workspace, workspace_bytes, stream, kBoth);
+}
+
+sherry_status grouped_f32(const sherry_gemv_f32_desc *descs, int count, int B, void *workspace,
+                          size_t workspace_bytes, cudaStream_t stream) {
+    if (!descs) return SHERRY_ERR_NULL;
+    if (count < 1) return SHERRY_ERR_SHAPE;
+    if (count > SHERRY_MAX_GROUP) return SHERRY_ERR_UNSUPPORTED;
+    GemvCall calls[SHERRY_MAX_GROUP];
+    for (int i = 0; i < count; i++) {
+        if (!descs[i].x) return SHERRY_ERR_NULL;
+        calls[i] = GemvCall{descs[i].codes, descs[i].scales, nullptr, descs[i].y, descs[i].N,
+                            descs[i].K, nullptr, descs[i].x, descs[i].u};
+    }
+    return gemv_launch(calls, count, B, false, workspace, workspace_bytes, stream, kBoth);
+}
+
+// The fp32 front-end alone: q and s in natural order (one cluster per row).
+sherry_status quantize_f32(const float *x, const float *u, int64_t B, int64_t K, int8_t *q, float *s,
+                           cudaStream_t stream) {
+    if (!x || !q || !s) return SHERRY_ERR_NULL;
+    if (B < 1 || !valid_k(K)) return SHERRY_ERR_SHAPE;
+    if (B > 65536) return SHERRY_ERR_UNSUPPORTED;
+    if (!aligned(x, 16) || (u && !aligned(u, 16)) || !aligned(q, 4) || !aligned(s, 4))
+        return SHERRY_ERR_ALIGN;
+    static thread_local XprepF32Params fp;
+    std::memset(&fp, 0, sizeof(fp));
+    fp.count = 1;
+    fp.B = (int)B;
+    fp.total_clusters = (int)B;
+    XprepF32Desc &F = fp.d[0];
+    F.x = x;
+    F.u = u;
+    F.xscale = s;
+    F.q = q;
+    F.K = (int)K;
+    F.Tp = (int)(K / SHERRY_TILE_K);
+    launch_xprep_f32(fp, stream);
+    return launch_status(u ? "sherry_quantize_swiglu" : "sherry_quantize_f32");
 }
 
 // Per-token quantization of bf16 activations, natural order (one warp per row).
@@ -1459,6 +1670,47 @@ extern "C" sherry_status sherry_quantize_act(const uint16_t *x, int64_t B, int64
     quantize_act_kernel<<<blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(x, (int)B, (int)K,
                                                                                     q, s);
     return launch_status("sherry_quantize_act");
+}
+
+extern "C" size_t sherry_gemv_f32_workspace_bytes(int64_t N, int64_t K, int B) {
+    return sherry_gemv_bf16_workspace_bytes(N, K, B);
+}
+
+extern "C" sherry_status sherry_gemv_f32(const uint32_t *codes, const float *scales, const float *x,
+                                         float *y, int64_t N, int64_t K, int B, void *workspace,
+                                         size_t workspace_bytes, sherry_stream_t stream) {
+    if (!scales || !x) return SHERRY_ERR_NULL;
+    const sherry::GemvCall c{codes, scales, nullptr, y, N, K, nullptr, x, nullptr};
+    return sherry::gemv_launch(&c, 1, B, false, workspace, workspace_bytes,
+                               reinterpret_cast<cudaStream_t>(stream), sherry::kBoth);
+}
+
+extern "C" sherry_status sherry_gemv_swiglu(const uint32_t *codes, const float *scales,
+                                            const float *g, const float *u, float *y, int64_t N,
+                                            int64_t K, int B, void *workspace,
+                                            size_t workspace_bytes, sherry_stream_t stream) {
+    if (!scales || !g || !u) return SHERRY_ERR_NULL;
+    const sherry::GemvCall c{codes, scales, nullptr, y, N, K, nullptr, g, u};
+    return sherry::gemv_launch(&c, 1, B, false, workspace, workspace_bytes,
+                               reinterpret_cast<cudaStream_t>(stream), sherry::kBoth);
+}
+
+extern "C" sherry_status sherry_gemv_f32_grouped(const sherry_gemv_f32_desc *descs, int count, int B,
+                                                 void *workspace, size_t workspace_bytes,
+                                                 sherry_stream_t stream) {
+    return sherry::grouped_f32(descs, count, B, workspace, workspace_bytes,
+                               reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" sherry_status sherry_quantize_f32(const float *x, int64_t B, int64_t K, int8_t *q, float *s,
+                                             sherry_stream_t stream) {
+    return sherry::quantize_f32(x, nullptr, B, K, q, s, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" sherry_status sherry_quantize_swiglu(const float *g, const float *u, int64_t B, int64_t K,
+                                                int8_t *q, float *s, sherry_stream_t stream) {
+    if (!u) return SHERRY_ERR_NULL;
+    return sherry::quantize_f32(g, u, B, K, q, s, reinterpret_cast<cudaStream_t>(stream));
 }
 
 // ---------------------------------------------------------------------------

@@ -45,6 +45,12 @@ class GemvDesc(ctypes.Structure):
                 ("y", ctypes.c_void_p), ("N", ctypes.c_int64), ("K", ctypes.c_int64)]
 
 
+class F32Desc(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("x", ctypes.c_void_p),
+                ("u", ctypes.c_void_p), ("y", ctypes.c_void_p), ("N", ctypes.c_int64),
+                ("K", ctypes.c_int64)]
+
+
 def library_path():
     return _build.LIB
 
@@ -72,6 +78,12 @@ def lib():
         "sherry_gemv_bf16_workspace_bytes": ([i64, i64, i32], sz),
         "sherry_gemv_bf16": ([p, p, p, p, i64, i64, i32, p, sz, p], i32),
         "sherry_gemv_bf16_grouped": ([p, i32, i32, p, sz, p], i32),
+        "sherry_quantize_f32": ([p, i64, i64, p, p, p], i32),
+        "sherry_quantize_swiglu": ([p, p, i64, i64, p, p, p], i32),
+        "sherry_gemv_f32_workspace_bytes": ([i64, i64, i32], sz),
+        "sherry_gemv_f32": ([p, p, p, p, i64, i64, i32, p, sz, p], i32),
+        "sherry_gemv_swiglu": ([p, p, p, p, p, i64, i64, i32, p, sz, p], i32),
+        "sherry_gemv_f32_grouped": ([p, i32, i32, p, sz, p], i32),
         "sherry_gemv_grouped": ([p, i32, i32, p, sz, p], i32),
         "sherry_gemv_prepare": ([p, i32, i32, p, sz, p], i32),
         "sherry_gemv_run": ([p, i32, i32, p, sz, p], i32),
@@ -322,6 +334,104 @@ def gemv_bf16_grouped(items, B, ws=None):
     _check(lib().sherry_gemv_bf16_grouped(ctypes.cast(descs, ctypes.c_void_p), n, B, _ptr(ws),
                                           ws.numel(), _stream(items[0][2])),
            "sherry_gemv_bf16_grouped")
+
+
+def _rows(t, name):
+    _need(t, torch.float32, name)
+    return t.view(1, -1) if t.dim() == 1 else t
+
+
+def quantize_f32(x, q=None, s=None):
+    """Per-token absmax int8 quantization of fp32 activations x [B, K]
+    (K a multiple of 128): returns (q int8 [B, K], s fp32 [B])."""
+    x2 = _rows(x, "x")
+    B, K = x2.shape
+    q = torch.empty((B, K), dtype=torch.int8, device=x.device) if q is None else q
+    s = torch.empty((B,), dtype=torch.float32, device=x.device) if s is None else s
+    _check(lib().sherry_quantize_f32(_ptr(x2), B, K, _ptr(q), _ptr(s), _stream(x)),
+           "sherry_quantize_f32")
+    return q, s
+
+
+def quantize_swiglu(g, u, q=None, s=None):
+    """quantize_f32 of h = silu(g) * u, formed inside the front-end."""
+    g2, u2 = _rows(g, "g"), _rows(u, "u")
+    if g2.shape != u2.shape:
+        raise ValueError("g and u differ in shape")
+    B, K = g2.shape
+    q = torch.empty((B, K), dtype=torch.int8, device=g.device) if q is None else q
+    s = torch.empty((B,), dtype=torch.float32, device=g.device) if s is None else s
+    _check(lib().sherry_quantize_swiglu(_ptr(g2), _ptr(u2), B, K, _ptr(q), _ptr(s), _stream(g)),
+           "sherry_quantize_swiglu")
+    return q, s
+
+
+def gemv_f32_workspace_bytes(N, K, B):
+    return int(lib().sherry_gemv_f32_workspace_bytes(N, K, B))
+
+
+def gemv_f32(codes, scales, x, y=None, ws=None):
+    """y[B, N] = scales * s_x * (W . q^T) for fp32 activations x [B, K] quantized per token."""
+    _need(scales, torch.float32, "scales")
+    N, K = _codes_shape(codes, scales.numel())
+    x2 = _rows(x, "x")
+    B = x2.shape[0]
+    y = torch.empty((B, N), dtype=torch.float32, device=x.device) if y is None else y
+    ws = workspace(gemv_f32_workspace_bytes(N, K, B), x.device) if ws is None else ws
+    _check(lib().sherry_gemv_f32(_ptr(codes), _ptr(scales), _ptr(x2), _ptr(y), N, K, B, _ptr(ws),
+                                 ws.numel(), _stream(x)), "sherry_gemv_f32")
+    return y
+
+
+def gemv_swiglu(codes, scales, g, u, y=None, ws=None):
+    """gemv_f32 on h = silu(g) * u (the down projection of a gated MLP); g, u fp32 [B, K]."""
+    _need(scales, torch.float32, "scales")
+    N, K = _codes_shape(codes, scales.numel())
+    g2, u2 = _rows(g, "g"), _rows(u, "u")
+    if g2.shape != u2.shape:
+        raise ValueError("g and u differ in shape")
+    B = g2.shape[0]
+    y = torch.empty((B, N), dtype=torch.float32, device=g.device) if y is None else y
+    ws = workspace(gemv_f32_workspace_bytes(N, K, B), g.device) if ws is None else ws
+    _check(lib().sherry_gemv_swiglu(_ptr(codes), _ptr(scales), _ptr(g2), _ptr(u2), _ptr(y), N, K, B,
+                                    _ptr(ws), ws.numel(), _stream(g)), "sherry_gemv_swiglu")
+    return y
+
+
+class GroupedGemvF32:
+    """Pre-marshalled grouped GEMV on fp32 activations (sherry_gemv_f32_grouped):
+    items are (codes, scales, x fp32 [B, K], u fp32 [B, K] or None, y [B, N])."""
+
+    def __init__(self, items, B, ws=None):
+        n = len(items)
+        self.descs = (F32Desc * n)()
+        total = 0
+        for i, (codes, scales, x, u, y) in enumerate(items):
+            _need(scales, torch.float32, "scales")
+            N, K = _codes_shape(codes, scales.numel())
+            _need(x, torch.float32, "x")
+            if u is not None:
+                _need(u, torch.float32, "u")
+            _need(y, torch.float32, "y")
+            self.descs[i] = F32Desc(codes.data_ptr(), scales.data_ptr(), x.data_ptr(),
+                                    u.data_ptr() if u is not None else None, y.data_ptr(), N, K)
+            total += gemv_f32_workspace_bytes(N, K, B)
+        self.items = items
+        dev = items[0][2].device
+        self.ws = torch.empty(max(total, 256), dtype=torch.uint8, device=dev) if ws is None else ws
+        self.args = (ctypes.cast(self.descs, ctypes.c_void_p), n, B, _ptr(self.ws),
+                     self.ws.numel())
+        self.device = dev
+
+    def __call__(self, stream=None):
+        s = ctypes.c_void_p(stream if stream is not None
+                            else torch.cuda.current_stream(self.device).cuda_stream)
+        _check(lib().sherry_gemv_f32_grouped(*self.args, s), "sherry_gemv_f32_grouped")
+
+
+def gemv_f32_grouped(items, B, ws=None):
+    """items: list of (codes, scales, x fp32 [B, K], u fp32 [B, K] or None, y [B, N])."""
+    GroupedGemvF32(items, B, ws)()
 
 
 class GroupedGemv:

@@ -215,6 +215,71 @@ sherry_status sherry_gemv_bf16_grouped(const sherry_gemv_bf16_desc *descs, int c
                                        sherry_stream_t stream);
 
 /*
+ * Front-end on fp32 activations, for chaining layers: the fp32 y of one GEMV
+ * becomes the next GEMV's input without leaving the library.  Two forms:
+ *   plain   the activations are x itself (e.g. the y of the previous layer);
+ *   SwiGLU  the activations are h = silu(g) * u, silu(g) = g / (1 + e^-g),
+ *           with g and u the outputs of the gate and up projections: the
+ *           gated MLP of the LLaMA models the method is evaluated on
+ *           (LLaMA-3.2 1B and 3B, arXiv 2601.07892, abstract).  h is formed in
+ *           fp32, each operation rounded once, e^-g by CUDA's expf (within
+ *           2 ulp); a g so negative that e^-g overflows gives h = -0 * u.
+ * Each token row is then quantized by the rule of sherry_quantize_act, read
+ * from the fp32 values.  The plain form is exact; in the SwiGLU form h differs
+ * from the exactly rounded silu(g) * u by a few ulp, so a q whose scaled value
+ * lies within ~1e-4 of a rounding tie may differ by one.
+ * The rows are handled by one cluster of 8 CTAs each, which exchange their
+ * maxima through distributed shared memory; NaN and Inf inputs are not
+ * supported (the result is unspecified).
+ *
+ * sherry_quantize_f32 / sherry_quantize_swiglu -- the front-end alone.
+ *   x, g, u  [B][K] fp32, row-major, device, 16-byte aligned; K a positive
+ *            multiple of 128, at most SHERRY_MAX_K; B at most 65536.
+ *   q  [B][K] int8 output, natural order, 4-byte aligned.   s  [B] fp32 output.
+ * Errors: NULL, SHAPE, ALIGN, UNSUPPORTED, CUDA.
+ */
+sherry_status sherry_quantize_f32(const float *x, int64_t B, int64_t K, int8_t *q, float *s,
+                                  sherry_stream_t stream);
+sherry_status sherry_quantize_swiglu(const float *g, const float *u, int64_t B, int64_t K, int8_t *q,
+                                     float *s, sherry_stream_t stream);
+
+/*
+ * sherry_gemv_f32 / sherry_gemv_swiglu -- the decode GEMV on fp32 activations
+ * (plain, or the SwiGLU h of g and u), quantized per token in the re-order
+ * launch as above, and scaled by both scales as sherry_gemv_bf16 is:
+ *   y[b][n] = fl32(fl32(s[n] * s_b) * acc[b][n]),  acc = W . q^T exactly.
+ *   x, g, u  [B][K] fp32, 16-byte aligned; other arguments as sherry_gemv.
+ *   workspace: sherry_gemv_f32_workspace_bytes(N, K, B) bytes (equal to the
+ *   bf16 size; a grouped call: the sum over its GEMVs, in descriptor order),
+ *   256-byte aligned.
+ * Errors: as sherry_gemv.
+ */
+size_t sherry_gemv_f32_workspace_bytes(int64_t N, int64_t K, int B);
+sherry_status sherry_gemv_f32(const uint32_t *codes, const float *scales, const float *x, float *y,
+                              int64_t N, int64_t K, int B, void *workspace, size_t workspace_bytes,
+                              sherry_stream_t stream);
+sherry_status sherry_gemv_swiglu(const uint32_t *codes, const float *scales, const float *g,
+                                 const float *u, float *y, int64_t N, int64_t K, int B,
+                                 void *workspace, size_t workspace_bytes, sherry_stream_t stream);
+
+/* One GEMV of a grouped fp32 call (device pointers); u NULL: plain, else SwiGLU. */
+typedef struct {
+    const uint32_t *codes;
+    const float *scales;
+    const float *x;  /* [B][K] fp32 activations; SwiGLU: the gate outputs g */
+    const float *u;  /* [B][K] up outputs (SwiGLU), or NULL */
+    float *y;        /* [B][N] */
+    int64_t N;
+    int64_t K;
+} sherry_gemv_f32_desc;
+
+/* sherry_gemv_f32 / _swiglu over `count` GEMVs with the same B in one pass
+ * (one front-end launch and one GEMV launch), as sherry_gemv_grouped. */
+sherry_status sherry_gemv_f32_grouped(const sherry_gemv_f32_desc *descs, int count, int B,
+                                      void *workspace, size_t workspace_bytes,
+                                      sherry_stream_t stream);
+
+/*
  * sherry_gemv_static -- sherry_gemv without a caller workspace: the call
  * allocates nothing.  The paper has no counterpart; this entry point exists
  * for callers that may not allocate device memory on their decode path.

@@ -129,6 +129,39 @@ def test_activation_front_end_argument_checks():
                               S.gemv_workspace_bytes(4, 1024, 2), None) == 7
 
 
+def test_fp32_front_end_argument_checks():
+    L = S.lib()
+    odd = ctypes.c_void_p(0x100008)
+    assert L.sherry_quantize_f32(None, 1, 128, FAKE, FAKE, None) == 1
+    assert L.sherry_quantize_f32(FAKE, 1, 136, FAKE, FAKE, None) == 2        # K % 128
+    assert L.sherry_quantize_f32(FAKE, 0, 128, FAKE, FAKE, None) == 2
+    assert L.sherry_quantize_f32(FAKE, 65537, 128, FAKE, FAKE, None) == 4
+    assert L.sherry_quantize_f32(odd, 1, 128, FAKE, FAKE, None) == 3
+    assert L.sherry_quantize_swiglu(FAKE, None, 1, 128, FAKE, FAKE, None) == 1
+    assert L.sherry_quantize_swiglu(FAKE, odd, 1, 128, FAKE, FAKE, None) == 3
+    ws = 1 << 20
+    assert L.sherry_gemv_f32(FAKE, FAKE, None, FAKE, 4, 128, 1, FAKE_WS, ws, None) == 1
+    assert L.sherry_gemv_f32(FAKE, FAKE, odd, FAKE, 4, 128, 1, FAKE_WS, ws, None) == 3
+    assert L.sherry_gemv_f32(FAKE, FAKE, FAKE, FAKE, 4, 128, 17, FAKE_WS, ws, None) == 4
+    assert L.sherry_gemv_swiglu(FAKE, FAKE, FAKE, None, FAKE, 4, 128, 1, FAKE_WS, ws, None) == 1
+    assert L.sherry_gemv_swiglu(FAKE, FAKE, FAKE, odd, FAKE, 4, 128, 1, FAKE_WS, ws, None) == 3
+    assert L.sherry_gemv_swiglu(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 100, 1, FAKE_WS, ws, None) == 2
+    # the activation scales take 64 more words than the int8 workspace, as for bf16
+    assert S.gemv_f32_workspace_bytes(2048, 8192, 1) == S.gemv_workspace_bytes(2048, 8192, 1) + 256
+    assert L.sherry_gemv_f32(FAKE, FAKE, FAKE, FAKE, 4, 1024, 2, FAKE_WS,
+                             S.gemv_workspace_bytes(4, 1024, 2), None) == 7
+    d = (S.F32Desc * 2)()
+    d[0] = S.F32Desc(0x100000, 0x100000, 0x100000, None, 0x100000, 16, 128)
+    d[1] = S.F32Desc(0x100000, 0x100000, None, 0x100000, 0x100000, 16, 128)
+    p = ctypes.cast(d, ctypes.c_void_p)
+    assert L.sherry_gemv_f32_grouped(None, 1, 1, FAKE_WS, ws, None) == 1
+    assert L.sherry_gemv_f32_grouped(p, 0, 1, FAKE_WS, ws, None) == 2
+    assert L.sherry_gemv_f32_grouped(p, 129, 1, FAKE_WS, ws, None) == 4
+    assert L.sherry_gemv_f32_grouped(p, 2, 1, FAKE_WS, ws, None) == 1    # desc 1 has no x
+    d[1] = S.F32Desc(0x100000, 0x100000, 0x100000, 0x100008, 0x100000, 16, 128)
+    assert L.sherry_gemv_f32_grouped(p, 2, 1, FAKE_WS, ws, None) == 3    # desc 1's u unaligned
+
+
 def test_grouped_argument_checks():
     L = S.lib()
     d = (S.GemvDesc * 2)()
