@@ -425,6 +425,52 @@ def time_bf16_stack(layers, S, torch, dev, reps=200):
             "note": "bf16 activations quantized per token inside the step (x seed 3)"}
 
 
+def time_mlp_chain(layers, S, torch, dev, reps=200):
+    """The 16 MLP blocks of the stack chained as a decoder runs them: per layer
+    one grouped bf16 GEMV over gate and up, then the down projection on
+    h = silu(g) * u, formed and quantized per token inside its re-order launch
+    (4 launches per layer, 64 per step; one bf16 input x for every layer)."""
+    gen = torch.Generator(device="cpu").manual_seed(4)
+    x = torch.randn((1, 2048), generator=gen).to(torch.bfloat16).to(dev)
+    by_layer = {}
+    for layer, name, n, k, codes, scales in layers:
+        by_layer.setdefault(layer, {})[name] = (n, k, codes, scales)
+    blocks, code_bytes = [], 0
+    for layer in sorted(by_layer):
+        p = by_layer[layer]
+        ni = p["gate"][0]
+        g = torch.empty((1, ni), dtype=torch.float32, device=dev)
+        u = torch.empty((1, ni), dtype=torch.float32, device=dev)
+        y = torch.empty((1, p["down"][0]), dtype=torch.float32, device=dev)
+        gu = S.GroupedGemvBf16([(p["gate"][2], p["gate"][3], x, g), (p["up"][2], p["up"][3], x, u)],
+                               B=1)
+        dn = S.GroupedGemvF32([(p["down"][2], p["down"][3], g, u, y)], B=1)
+        blocks.append((gu, dn))
+        code_bytes += sum(p[m][2].numel() * 4 for m in ("gate", "up", "down"))
+
+    def step():
+        for gu, dn in blocks:
+            gu()
+            dn()
+    for _ in range(5):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        step()
+    e1.record()
+    e1.synchronize()
+    t = e0.elapsed_time(e1) / 1e3 / reps
+    tg = graph_time(torch, step, reps)
+    return {"us_per_step": t * 1e6, "us_per_layer": t * 1e6 / len(blocks),
+            "weight_gbs": code_bytes / t / 1e9, "code_bytes": code_bytes, "steps": reps,
+            "graph_us_per_step": tg * 1e6, "graph_weight_gbs": code_bytes / tg / 1e9,
+            "launches_per_step": 4 * len(blocks),
+            "note": "x (bf16, seed 4) -> gate, up (sherry_gemv_bf16_grouped) -> down on "
+                    "silu(g) * u (sherry_gemv_f32_grouped), 16 layers chained"}
+
+
 def cpu_baseline(layers, xs_host, seconds):
     """The oracle, as it stands, on a bounded sample of the stack (host cores)."""
     import oracle
@@ -638,6 +684,7 @@ def main():
         line["gemm"] = time_gemm(S, torch, dev, flush)
         line["gemv_layers_rotated"] = time_layers(layers, xs, S, torch, dev)
         line["gemv_bf16_stack"] = time_bf16_stack(layers, S, torch, dev)
+        line["mlp_chain"] = time_mlp_chain(layers, S, torch, dev)
         line["gemv_stack_112_calls_graph"] = time_stack_single_calls(layers, xs, ys, S, torch, dev)
         rs = read_stream_gbs(torch, dev)
         line["roofline"]["other_denominators"] = {
