@@ -43,6 +43,7 @@ struct GemvDesc {
     const float *scales;
     const float *xscale;  // per batch row activation scales (bf16 front-end), else null
     const uint4 *xw;      // re-ordered activations [B][Tp][32 words]
+    const int8_t *x;      // raw int8 activations [B][K] (re-ordered inside the dot kernel)
     void *out;            // float y[B][N] or int32 acc[B][N]
     int32_t *part_acc;    // K-part partial sums [B][N] (pipelined kernel, kparts > 1)
     uint32_t *part_cnt;   // K-parts finished per unit (pipelined kernel, kparts > 1)
@@ -1004,6 +1005,7 @@ __global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
 // K-parts and the split-K completion are those of the pipelined kernel.
 // ---------------------------------------------------------------------------
 constexpr int kDotRing = 2;  // stages per warp: one chunk in flight while one is consumed
+constexpr int kRawXMaxChunksPerSM = 64;  // calls up to this many chunks per SM re-order x in the dot kernel
 constexpr int kDotCodeWords = kChunkTiles * kTileWords;  // 640
 // 8 warps per CTA: B = 1, 4 CTAs (32 warps) per SM at 64 registers (50 KB of
 // shared memory per CTA); B = 2, 2 CTAs per SM.  (One CTA of 32 warps per SM
@@ -1071,7 +1073,12 @@ __device__ __forceinline__ void dot_finish(const GemvDesc &D, int unit, int B, i
     }
 }
 
-template <int NBX, bool ACC_OUT>
+// XRAW: the activations are read raw from D.x (16-byte aligned rows) and each
+// warp re-orders its chunk's 4 tiles in shared memory (four shuffles and three
+// byte permutes per word, as the re-order launch does), so that a small call
+// needs no re-order launch.  Used for calls of few chunks, where that launch
+// and its wait cost more than re-ordering x once per chunk.
+template <int NBX, bool ACC_OUT, bool XRAW>
 __global__ void __launch_bounds__(DotShape<NBX>::kThreads, DotShape<NBX>::kMinBlocks)
     gemv_dot_kernel(const __grid_constant__ GemvParams P) {
     pdl_allow_dependents();
@@ -1113,11 +1120,17 @@ __global__ void __launch_bounds__(DotShape<NBX>::kThreads, DotShape<NBX>::kMinBl
     ItemCursor icur = cur;
     int istart = start, ic = 0, ic_end = 0, iTp = 0;
     const uint32_t *isrc = nullptr, *ixw = nullptr;
+    const int8_t *ixr = nullptr;
     auto set_issue_item = [&]() {
         const GemvDesc &D = P.d[icur.id];
         isrc = D.codes + (size_t)icur.unit * D.T * kTileWords + 4 * lane;
-        ixw = reinterpret_cast<const uint32_t *>(D.xw) + 4 * lane;
-        iTp = D.Tp;
+        if (XRAW) {
+            ixr = D.x + 16 * lane;
+            iTp = D.T * SHERRY_TILE_K;  // row stride of x in bytes
+        } else {
+            ixw = reinterpret_cast<const uint32_t *>(D.xw) + 4 * lane;
+            iTp = D.Tp;
+        }
         const int first = icur.kp * D.cpp;
         ic = first + max(b0 - istart, 0);
         ic_end = first + min(b1 - istart, min(D.cpp, D.nchunk - first));
@@ -1132,10 +1145,16 @@ __global__ void __launch_bounds__(DotShape<NBX>::kThreads, DotShape<NBX>::kMinBl
     auto copy_x_and_advance = [&](int slot) {
         const uint32_t dst = ring_addr + (uint32_t)slot * SW * 4 + 16u * lane;
 #pragma unroll
-        for (int b = 0; b < NBX; b++)
-            if (b < B)
-                cp_async16(dst + 4u * kDotCodeWords + 512u * b,
-                           ixw + ((size_t)b * iTp + (size_t)kChunkTiles * ic) * 32, 16u);
+        for (int b = 0; b < NBX; b++) {
+            if (b < B) {
+                if (XRAW)
+                    cp_async16(dst + 4u * kDotCodeWords + 512u * b,
+                               ixr + (size_t)b * iTp + (size_t)kChunkTiles * SHERRY_TILE_K * ic, 16u);
+                else
+                    cp_async16(dst + 4u * kDotCodeWords + 512u * b,
+                               ixw + ((size_t)b * iTp + (size_t)kChunkTiles * ic) * 32, 16u);
+            }
+        }
         if (++ic == ic_end) {
             const GemvDesc &D = P.d[icur.id];
             istart += min(D.cpp, D.nchunk - icur.kp * D.cpp);
@@ -1176,8 +1195,24 @@ __global__ void __launch_bounds__(DotShape<NBX>::kThreads, DotShape<NBX>::kMinBl
             cp_async_wait<kDotRing - 2>();
             __syncwarp();  // every lane is done with the previous stage: refill it
             issue(slot == 0 ? kDotRing - 1 : slot - 1);
-            const uint32_t *st = ring + slot * SW;
+            uint32_t *st = ring + slot * SW;
             slot = (slot + 1 == kDotRing) ? 0 : slot + 1;
+            if (XRAW) {  // raw words of the chunk's tiles -> the decode order, in place
+                uint32_t *xr = st + kDotCodeWords;
+                uint32_t w[NBX][kChunkTiles];
+#pragma unroll
+                for (int b = 0; b < NBX; b++)
+#pragma unroll
+                    for (int tt = 0; tt < kChunkTiles; tt++)
+                        w[b][tt] = b < B ? reorder_word(xr[(b * kChunkTiles + tt) * 32 + lane], lane) : 0u;
+                __syncwarp();
+#pragma unroll
+                for (int b = 0; b < NBX; b++)
+#pragma unroll
+                    for (int tt = 0; tt < kChunkTiles; tt++)
+                        if (b < B) xr[(b * kChunkTiles + tt) * 32 + lane] = w[b][tt];
+                __syncwarp();
+            }
 #pragma unroll
             for (int tt = 0; tt < kChunkTiles; tt++) {
                 const uint32_t *cw = st + tt * kTileWords + lane;
@@ -1307,7 +1342,7 @@ void launch_pipe(const GemvParams &gp, cudaStream_t stream) {
     launch_pdl(gemv_pipe_kernel<NB, ACC>, grid, kPipeThreads, smem, stream, gp);
 }
 
-template <int NBX, bool ACC>
+template <int NBX, bool ACC, bool XRAW>
 void launch_dot(const GemvParams &gp, cudaStream_t stream) {
     static int cache[64] = {0};
     const size_t smem = DotShape<NBX>::kSmem;
@@ -1315,8 +1350,8 @@ void launch_dot(const GemvParams &gp, cudaStream_t stream) {
     // has chunks (items cut between warps are summed in shared memory)
     constexpr int threads = DotShape<NBX>::kThreads, warps = DotShape<NBX>::kWarps;
     const int want = (gp.total_chunks + warps - 1) / warps;
-    const int grid = grid_for(gemv_dot_kernel<NBX, ACC>, threads, smem, want, cache);
-    launch_pdl(gemv_dot_kernel<NBX, ACC>, grid, threads, smem, stream, gp);
+    const int grid = grid_for(gemv_dot_kernel<NBX, ACC, XRAW>, threads, smem, want, cache);
+    launch_pdl(gemv_dot_kernel<NBX, ACC, XRAW>, grid, threads, smem, stream, gp);
 }
 
 template <int NB, bool ACC>
@@ -1457,6 +1492,7 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
         D.scales = c.scales;
         D.xscale = act_scale;
         D.xw = reinterpret_cast<const uint4 *>(region);
+        D.x = c.x;
         D.out = c.out;
         D.part_acc = kparts > 1 ? reinterpret_cast<int32_t *>(region + xw_words) : nullptr;
         D.part_cnt = kparts > 1 ? region + xw_words + (int64_t)B * c.N : nullptr;
@@ -1477,7 +1513,15 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
     xp.total_units = wb;
     gp.total_units16 = ub16;
     gp.total_chunks = cb;
-    if (phase & kPrepare) {
+    // A small int8 call skips the re-order launch: the dot kernel re-orders each
+    // chunk's activations itself (at most ~2 chunks per warp of a full GPU, so
+    // x is re-ordered at most twice per chunk position; rows are not split, so
+    // there are no K-part sums to clear).
+    bool raw_x = phase == kBoth && pipelined && B <= 2 && cb <= kRawXMaxChunksPerSM * sm_count();
+    for (int i = 0; i < count && raw_x; i++)
+        raw_x = calls[i].x && !calls[i].xbf && !calls[i].xf && aligned(calls[i].x, 16) &&
+                kparts_for(calls[i].K) == 1;
+    if ((phase & kPrepare) && !raw_x) {
         if (f32) {
             launch_xprep_f32(fp, stream);
         } else {
@@ -1491,10 +1535,16 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
     // B <= 2: dp4a kernel; B >= 3: the MMA kernel (its 8 batch columns cost the
     // same as one, while dp4a work grows with B) -- measured on the decode stack
     if (pipelined && B <= 2) {
-        if (B == 1) {
-            if (acc_out) launch_dot<1, true>(gp, stream); else launch_dot<1, false>(gp, stream);
+        if (raw_x) {
+            if (B == 1) {
+                if (acc_out) launch_dot<1, true, true>(gp, stream); else launch_dot<1, false, true>(gp, stream);
+            } else {
+                if (acc_out) launch_dot<2, true, true>(gp, stream); else launch_dot<2, false, true>(gp, stream);
+            }
+        } else if (B == 1) {
+            if (acc_out) launch_dot<1, true, false>(gp, stream); else launch_dot<1, false, false>(gp, stream);
         } else {
-            if (acc_out) launch_dot<2, true>(gp, stream); else launch_dot<2, false>(gp, stream);
+            if (acc_out) launch_dot<2, true, false>(gp, stream); else launch_dot<2, false, false>(gp, stream);
         }
     } else if (pipelined) {
         if (B <= 8) {
