@@ -53,6 +53,9 @@ def parse_args():
                     help="skip the pack/GEMM/per-layer/CPU-baseline sub-measurements")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--mlp-chain-only", action="store_true",
+                    help="only time the chained MLP blocks of --layers layers for --steps steps "
+                         "(a small case for profiling); prints their JSON")
     return ap.parse_args()
 
 
@@ -523,6 +526,10 @@ def main():
     S.lib()
 
     spec = stack_spec(args.layers)
+    if args.mlp_chain_only:
+        layers, _ = build_stack(spec, dev, S, torch)
+        print(json.dumps(time_mlp_chain(layers, S, torch, dev, reps=args.steps)))
+        return 0
     codes_bytes, alg_bytes = algorithmic_bytes(spec)
     extras = (rank == 0) and not args.no_extras
     layers, latents = build_stack(spec, dev, S, torch, keep_latents=extras)

@@ -317,10 +317,11 @@ constexpr int kF32ClusterWarps = kF32Cluster * kF32Warps;
 // One thread-block cluster per (GEMV, token row).  Its 64 warps take the
 // row's 128-element tiles in turn: the first pass forms the activations and
 // their absolute maximum, the CTAs exchange their maxima through distributed
-// shared memory at a cluster barrier, and the second pass forms them again,
-// quantizes them with the per-token rule of the bf16 front-end and re-orders
-// them (or writes them in natural order).  Forming an activation twice costs
-// less than keeping the row: a 8192-element row is 1024 elements per CTA.
+// shared memory at a cluster barrier, and the second pass quantizes them with
+// the per-token rule of the bf16 front-end and re-orders them (or writes them
+// in natural order).  A warp keeps the activations of its first two tiles in
+// registers between the passes (every tile of rows up to K = 16384) and forms
+// those of later tiles again.
 __global__ void __launch_bounds__(kF32Threads) xprep_f32_kernel(const __grid_constant__ XprepF32Params P) {
     namespace cg = cooperative_groups;
     cg::cluster_group cluster = cg::this_cluster();
@@ -342,11 +343,17 @@ __global__ void __launch_bounds__(kF32Threads) xprep_f32_kernel(const __grid_con
     const int cw = rank * kF32Warps + warp;  // warp index within the cluster
     const size_t row = (size_t)b * D.K;
 
+    auto absmax4 = [](float m, const float4 &a) {
+        return fmaxf(m, fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w))));
+    };
     float m = 0.0f;
-    for (int t = cw; t < T; t += kF32ClusterWarps) {
-        const float4 a = act4(D, row + (size_t)t * SHERRY_TILE_K + 4 * lane);
-        m = fmaxf(m, fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w))));
-    }
+    float4 h0 = make_float4(0.0f, 0.0f, 0.0f, 0.0f), h1 = h0;  // tiles cw and cw + 64
+    if (cw < T) h0 = act4(D, row + (size_t)cw * SHERRY_TILE_K + 4 * lane);
+    if (cw + kF32ClusterWarps < T)
+        h1 = act4(D, row + (size_t)(cw + kF32ClusterWarps) * SHERRY_TILE_K + 4 * lane);
+    m = absmax4(absmax4(m, h0), h1);
+    for (int t = cw + 2 * kF32ClusterWarps; t < T; t += kF32ClusterWarps)
+        m = absmax4(m, act4(D, row + (size_t)t * SHERRY_TILE_K + 4 * lane));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
     if (lane == 0) warp_max[warp] = m;
@@ -369,10 +376,10 @@ __global__ void __launch_bounds__(kF32Threads) xprep_f32_kernel(const __grid_con
     if (rank == 0 && threadIdx.x == 0) D.xscale[b] = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
 
     const int t_end = D.q ? T : D.Tp;
-    for (int t = cw; t < t_end; t += kF32ClusterWarps) {
+    for (int t = cw, j = 0; t < t_end; t += kF32ClusterWarps, j++) {
         uint32_t raw = 0u;
         if (t < T) {
-            const float4 a = act4(D, row + (size_t)t * SHERRY_TILE_K + 4 * lane);
+            const float4 a = j == 0 ? h0 : j == 1 ? h1 : act4(D, row + (size_t)t * SHERRY_TILE_K + 4 * lane);
             raw = quant_byte(a.x, inv) | (quant_byte(a.y, inv) << 8) | (quant_byte(a.z, inv) << 16) |
                   (quant_byte(a.w, inv) << 24);
         }

@@ -279,3 +279,26 @@ def test_gemv_run_repeats_after_one_prepare():
         g.run()
         for (_, _, _, y), ref in zip(items, refs):
             assert_y_matches(y.cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("B", [1, 2])
+def test_gemv_in_kernel_reorder_equals_reorder_launch(B):
+    """Small int8 calls re-order x inside the dot kernel (no re-order launch);
+    the split prepare/run calls and an x that is only 4-byte aligned take the
+    re-order launch.  All three give the oracle's y bit for bit."""
+    for li, (N, K) in enumerate([(2048, 2048), (512, 2048), (33, 8192), (100, 1024), (1, 512)]):
+        codes, scales = oracle.pack(synth.latent_weights(N, K, seed=80 + li))
+        x = synth.int8_uniform((B, K), seed=90 + li)
+        ref = oracle.gemv(codes, scales, x, K)
+        tc, ts = dev_codes(codes), dev(scales)
+        tx = dev(x)
+        assert_y_matches(S.gemv(tc, ts, tx).cpu().numpy(), ref)            # in-kernel re-order
+        y = torch.zeros((B, N), dtype=torch.float32, device="cuda")
+        g = S.GroupedGemv([(tc, ts, tx, y)], B=B)
+        g.prepare()
+        g.run()                                                             # re-order launch
+        assert_y_matches(y.cpu().numpy(), ref)
+        buf = torch.zeros(B * K + 4, dtype=torch.int8, device="cuda")
+        xo = buf[4:].view(B, K)                                             # 4-byte aligned only
+        xo.copy_(tx)
+        assert_y_matches(S.gemv(tc, ts, xo).cpu().numpy(), ref)
