@@ -1,28 +1,40 @@
-// gemv.cu -- decode GEMV on Sherry codes: y = s (.) (W_ternary . x_int8), B <= 16.
+// gemv.cu -- decode GEMV on Sherry codes: y = s (.) (W_ternary . x_int8), B <= 16,
+// and the activation front-ends that feed it.
 //
 // The product is the one the pages state for ternary weights with 3:4 blocks
 // coded in five bits (arXiv 2601.07892, abstract; Figure 2 caption: "SIMD-
 // friendly 4-way patterns").  On B200 a batch-1 GEMV is bound by HBM reads of
 // the codes (0.15625 bytes per weight) only if the decode costs a few
-// instructions per 4-weight block, so:
+// instructions per 4-weight block.  Every kernel here decodes the same way:
 //
-//   * the int8 MMA m16n8k32 does the multiply-accumulate: the decoded weights
-//     are its A fragment straight from registers (16 rows x 32 K per MMA), the
-//     activations its B fragment (one batch row per column, so batches up to 8
-//     cost the same MMA count as batch 1), int32 accumulation is exact;
 //   * a thread decodes whole 128-weight tiles with 32-bit SWAR logic: for a
 //     (position i, block group beta) pair one selector word holds, per nibble,
 //     (zero position | sign << 2) of one block, and one byte permute (PRMT)
 //     against an 8-byte table per position turns four nibbles into four
 //     ternary bytes; shifts that move left run as IMAD on the FMA pipe, so the
 //     ALU pipe carries only the permutes, the selector merges and a few shifts;
-//   * the activations are re-ordered once per call (xprep_kernel) into the
-//     order in which the decoded bytes meet the MMA fragments.
+//   * the activations are re-ordered into the order in which the decoded
+//     bytes meet the multiply-accumulate.
 //
-// Two kernels share this scheme.  The pipelined kernel (K a multiple of 512,
-// codes 16-byte aligned) streams codes through per-warp shared-memory rings
-// filled by cp.async and splits long rows into K-parts that are summed exactly
-// with integer atomics; the register kernel is the general fallback.
+// Kernels:
+//   gemv_dot_kernel   B <= 2 (the decode path): per-warp cp.async rings of
+//                     4-tile chunks, dp4a against broadcast activation words,
+//                     chunk-balanced warp ranges, items cut between warps
+//                     summed in shared memory.  Small int8 calls copy raw x
+//                     and re-order it in the kernel (no re-order launch).
+//   gemv_pipe_kernel  B >= 3: the same rings; the int8 MMA m16n8k32 takes the
+//                     decoded weights as its A fragment from registers and one
+//                     batch row per column, so batches up to 8 cost the same
+//                     MMA count as one.
+//   gemv_kernel       the general fallback (K not a multiple of 512, or code
+//                     rows not 16-byte aligned), MMA from registers.
+//   xprep_kernel      re-orders int8 activations, or quantizes bf16 ones per
+//                     token first; clears the K-part sums of split rows.
+//   xprep_f32_kernel  the fp32 / SwiGLU front-end: one thread-block cluster
+//                     per token row, maxima exchanged through distributed
+//                     shared memory.
+// Rows longer than 8192 are split into K-parts, summed exactly with integer
+// atomics.  Consecutive launches use programmatic dependent launch.
 #include <algorithm>
 #include <cstdio>
 #include <cstring>
