@@ -429,10 +429,10 @@ def time_bf16_stack(layers, S, torch, dev, reps=200):
 
 
 def time_mlp_chain(layers, S, torch, dev, reps=200):
-    """The 16 MLP blocks of the stack chained as a decoder runs them: per layer
-    one grouped bf16 GEMV over gate and up, then the down projection on
-    h = silu(g) * u, formed and quantized per token inside its re-order launch
-    (4 launches per layer, 64 per step; one bf16 input x for every layer)."""
+    """The MLP blocks of the stack chained as a decoder runs them: per layer
+    one grouped bf16 GEMV over gate and up (its kernel quantizes x), then the
+    down projection on h = silu(g) * u, formed and quantized per token in its
+    re-order launch (3 launches per layer; one bf16 input x for every layer)."""
     gen = torch.Generator(device="cpu").manual_seed(4)
     x = torch.randn((1, 2048), generator=gen).to(torch.bfloat16).to(dev)
     by_layer = {}
@@ -469,9 +469,10 @@ def time_mlp_chain(layers, S, torch, dev, reps=200):
     return {"us_per_step": t * 1e6, "us_per_layer": t * 1e6 / len(blocks),
             "weight_gbs": code_bytes / t / 1e9, "code_bytes": code_bytes, "steps": reps,
             "graph_us_per_step": tg * 1e6, "graph_weight_gbs": code_bytes / tg / 1e9,
-            "launches_per_step": 4 * len(blocks),
-            "note": "x (bf16, seed 4) -> gate, up (sherry_gemv_bf16_grouped) -> down on "
-                    "silu(g) * u (sherry_gemv_f32_grouped), 16 layers chained"}
+            "launches_per_step": 3 * len(blocks),
+            "note": "x (bf16, seed 4) -> gate, up (sherry_gemv_bf16_grouped: one launch, the "
+                    "GEMV quantizes x) -> down on silu(g) * u (sherry_gemv_f32_grouped: front-end "
+                    "+ GEMV), layers chained"}
 
 
 def cpu_baseline(layers, xs_host, seconds):

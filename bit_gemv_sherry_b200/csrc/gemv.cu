@@ -56,6 +56,7 @@ struct GemvDesc {
     const float *xscale;  // per batch row activation scales (bf16 front-end), else null
     const uint4 *xw;      // re-ordered activations [B][Tp][32 words]
     const int8_t *x;      // raw int8 activations [B][K] (re-ordered inside the dot kernel)
+    const uint16_t *xbf;  // raw bf16 activations [B][K] (quantized inside the dot kernel)
     void *out;            // float y[B][N] or int32 acc[B][N]
     int32_t *part_acc;    // K-part partial sums [B][N] (pipelined kernel, kparts > 1)
     uint32_t *part_cnt;   // K-parts finished per unit (pipelined kernel, kparts > 1)
@@ -1030,12 +1031,16 @@ constexpr int kDotCodeWords = kChunkTiles * kTileWords;  // 640
 // shared memory per CTA); B = 2, 2 CTAs per SM.  (One CTA of 32 warps per SM
 // balances the CTAs' item runs better but was measured slower: a CTA slot frees
 // only when all 32 warps are done.)
-template <int NBX>
+// XMODE 2 adds to each stage the chunk's raw bf16 activations (1 KB per batch
+// row), so that B = 1 fits 3 CTAs per SM.
+template <int NBX, int XMODE = 0>
 struct DotShape {
     static constexpr int kWarps = 8;
     static constexpr int kThreads = kWarps * 32;
-    static constexpr int kMinBlocks = NBX == 1 ? 4 : 2;
-    static constexpr int kStageWords = kDotCodeWords + NBX * kChunkTiles * 32;
+    static constexpr int kMinBlocks = NBX == 1 ? (XMODE == 2 ? 3 : 4) : 2;
+    static constexpr int kXWords = NBX * kChunkTiles * 32;           // int8, decode order
+    static constexpr int kBfWords = XMODE == 2 ? NBX * kChunkTiles * 64 : 0;
+    static constexpr int kStageWords = kDotCodeWords + kXWords + kBfWords;
     static constexpr int kRingWords = kWarps * kDotRing * kStageWords;
     // after the rings: per warp, the row sums of a later piece of a cut item
     // [warp][NBX][32] and the first chunk of that item [warp]
@@ -1045,9 +1050,10 @@ struct DotShape {
 // Finishes an item: lane = row of the unit, v = the item's row sums.  A K-part
 // of a split row adds into the K-part sums; the last K-part to finish scales,
 // stores and clears them.
-template <int NBX, bool ACC_OUT>
+// sx: the activation scales, when the kernel quantized the activations itself.
+template <int NBX, bool ACC_OUT, bool SX_REG>
 __device__ __forceinline__ void dot_finish(const GemvDesc &D, int unit, int B, int lane,
-                                           int (&v)[NBX]) {
+                                           int (&v)[NBX], const float (&sx)[NBX]) {
     const int N = D.N;
     const int row = unit * kUnitRows + lane;
     const bool rv = row < N;
@@ -1085,26 +1091,37 @@ __device__ __forceinline__ void dot_finish(const GemvDesc &D, int unit, int B, i
                 if (b < B) static_cast<int32_t *>(D.out)[(size_t)b * N + row] = v[b];
         } else {
 #pragma unroll
-            for (int b = 0; b < NBX; b++)
-                if (b < B)
-                    static_cast<float *>(D.out)[(size_t)b * N + row] = out_scale(D, row, b) * (float)v[b];
+            for (int b = 0; b < NBX; b++) {
+                if (b < B) {
+                    const float sc = SX_REG ? __fmul_rn(__ldg(D.scales + row), sx[b]) : out_scale(D, row, b);
+                    static_cast<float *>(D.out)[(size_t)b * N + row] = sc * (float)v[b];
+                }
+            }
         }
     }
 }
 
-// XRAW: the activations are read raw from D.x (16-byte aligned rows) and each
-// warp re-orders its chunk's 4 tiles in shared memory (four shuffles and three
-// byte permutes per word, as the re-order launch does), so that a small call
-// needs no re-order launch.  Used for calls of few chunks, where that launch
-// and its wait cost more than re-ordering x once per chunk.
-template <int NBX, bool ACC_OUT, bool XRAW>
-__global__ void __launch_bounds__(DotShape<NBX>::kThreads, DotShape<NBX>::kMinBlocks)
+// XMODE: where the activations come from.
+//   0  re-ordered words in the workspace (written by the re-order launch);
+//   1  raw int8 from D.x (16-byte aligned rows): each warp re-orders its
+//      chunk's 4 tiles in shared memory (four shuffles and three byte permutes
+//      per word, as the re-order launch does);
+//   2  raw bf16 from D.xbf: each warp takes the token's absmax from the row
+//      (once per activation pointer), then quantizes and re-orders its chunk's
+//      tiles by the rule of the bf16 front-end.
+// Modes 1 and 2 need no re-order launch.  They are used for calls of few
+// chunks, where that launch and its wait cost more than the per-chunk work.
+template <int NBX, bool ACC_OUT, int XMODE>
+__global__ void __launch_bounds__(DotShape<NBX, XMODE>::kThreads, DotShape<NBX, XMODE>::kMinBlocks)
     gemv_dot_kernel(const __grid_constant__ GemvParams P) {
+    constexpr bool XRAW = XMODE == 1;
+    constexpr bool XBF = XMODE == 2;
+    using Shape = DotShape<NBX, XMODE>;
     pdl_allow_dependents();
-    constexpr int SW = DotShape<NBX>::kStageWords;
+    constexpr int SW = Shape::kStageWords;
     extern __shared__ __align__(16) uint32_t dot_smem[];
-    int *cut_sum = reinterpret_cast<int *>(dot_smem + DotShape<NBX>::kRingWords);
-    constexpr int kWarps = DotShape<NBX>::kWarps;
+    int *cut_sum = reinterpret_cast<int *>(dot_smem + Shape::kRingWords);
+    constexpr int kWarps = Shape::kWarps;
     int *cut_start = cut_sum + kWarps * NBX * 32;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     // chunk range [b0, b1) of this warp; threads 0 and 1 find the CTA's bounds
@@ -1146,6 +1163,9 @@ __global__ void __launch_bounds__(DotShape<NBX>::kThreads, DotShape<NBX>::kMinBl
         if (XRAW) {
             ixr = D.x + 16 * lane;
             iTp = D.T * SHERRY_TILE_K;  // row stride of x in bytes
+        } else if (XBF) {
+            ixr = reinterpret_cast<const int8_t *>(D.xbf) + 16 * lane;
+            iTp = D.T * SHERRY_TILE_K * 2;  // row stride of x in bytes
         } else {
             ixw = reinterpret_cast<const uint32_t *>(D.xw) + 4 * lane;
             iTp = D.Tp;
@@ -1166,7 +1186,12 @@ __global__ void __launch_bounds__(DotShape<NBX>::kThreads, DotShape<NBX>::kMinBl
 #pragma unroll
         for (int b = 0; b < NBX; b++) {
             if (b < B) {
-                if (XRAW)
+                if (XBF) {  // 1 KB of bf16 per batch row: pieces l and l + 32
+                    const int8_t *src = ixr + (size_t)b * iTp + (size_t)kChunkTiles * SHERRY_TILE_K * 2 * ic;
+                    const uint32_t d0 = dst + 4u * (kDotCodeWords + Shape::kXWords) + 1024u * b;
+                    cp_async16(d0, src, 16u);
+                    cp_async16(d0 + 512u, src + 512, 16u);
+                } else if (XRAW)
                     cp_async16(dst + 4u * kDotCodeWords + 512u * b,
                                ixr + (size_t)b * iTp + (size_t)kChunkTiles * SHERRY_TILE_K * ic, 16u);
                 else
@@ -1201,8 +1226,27 @@ __global__ void __launch_bounds__(DotShape<NBX>::kThreads, DotShape<NBX>::kMinBl
     int slot = 0;
     int v[NBX];
     bool own_cut = false;  // the last item continues in later warps of the CTA
+    // XMODE 2: per-token quantization of the activations the warp works on
+    const uint16_t *sx_of = nullptr;  // the activations (and row length) sx belongs to
+    int sx_T = 0;
+    float sx[NBX], sx_inv[NBX];
+#pragma unroll
+    for (int b = 0; b < NBX; b++) sx[b] = sx_inv[b] = 0.0f;
     while (start < b1) {
         const GemvDesc &D = P.d[cur.id];
+        if (XBF && (D.xbf != sx_of || D.T != sx_T)) {  // after pdl_wait(): x may come from the kernel before
+            sx_of = D.xbf;
+            sx_T = D.T;
+#pragma unroll
+            for (int b = 0; b < NBX; b++) {
+                if (b < B) {
+                    const float amax = row_absmax_bf16(D.xbf + (size_t)b * D.T * SHERRY_TILE_K,
+                                                       D.T * SHERRY_TILE_K, lane);
+                    sx_inv[b] = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+                    sx[b] = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
+                }
+            }
+        }
         const int first = cur.kp * D.cpp;
         const int nreal = min(D.cpp, D.nchunk - first);
         const int c_begin = first + max(b0 - start, 0);
@@ -1230,6 +1274,18 @@ __global__ void __launch_bounds__(DotShape<NBX>::kThreads, DotShape<NBX>::kMinBl
 #pragma unroll
                     for (int tt = 0; tt < kChunkTiles; tt++)
                         if (b < B) xr[(b * kChunkTiles + tt) * 32 + lane] = w[b][tt];
+                __syncwarp();
+            }
+            if (XBF) {  // bf16 of the chunk's tiles -> quantized words in the decode order
+                uint32_t *xq = st + kDotCodeWords;
+                const uint2 *xb = reinterpret_cast<const uint2 *>(st + kDotCodeWords + Shape::kXWords);
+#pragma unroll
+                for (int b = 0; b < NBX; b++)
+#pragma unroll
+                    for (int tt = 0; tt < kChunkTiles; tt++)
+                        if (b < B)
+                            xq[(b * kChunkTiles + tt) * 32 + lane] =
+                                reorder_word(quant_word(xb[(b * kChunkTiles + tt) * 32 + lane], sx_inv[b]), lane);
                 __syncwarp();
             }
 #pragma unroll
@@ -1273,7 +1329,7 @@ __global__ void __launch_bounds__(DotShape<NBX>::kThreads, DotShape<NBX>::kMinBl
         } else if (b1 - start < nreal) {
             own_cut = true;  // first piece of an item cut at b1: finished after the barrier
         } else {
-            dot_finish<NBX, ACC_OUT>(D, cur.unit, B, lane, v);
+            dot_finish<NBX, ACC_OUT, XBF>(D, cur.unit, B, lane, v, sx);
         }
         start += nreal;
         if (start < b1) cursor_next(P, cur);
@@ -1290,7 +1346,7 @@ __global__ void __launch_bounds__(DotShape<NBX>::kThreads, DotShape<NBX>::kMinBl
 #pragma unroll
             for (int b = 0; b < NBX; b++) v[b] += cut_sum[(w * NBX + b) * 32 + lane];
         }
-        dot_finish<NBX, ACC_OUT>(P.d[cur.id], cur.unit, B, lane, v);
+        dot_finish<NBX, ACC_OUT, XBF>(P.d[cur.id], cur.unit, B, lane, v, sx);
     }
 }
 
@@ -1361,16 +1417,16 @@ void launch_pipe(const GemvParams &gp, cudaStream_t stream) {
     launch_pdl(gemv_pipe_kernel<NB, ACC>, grid, kPipeThreads, smem, stream, gp);
 }
 
-template <int NBX, bool ACC, bool XRAW>
+template <int NBX, bool ACC, int XMODE>
 void launch_dot(const GemvParams &gp, cudaStream_t stream) {
     static int cache[64] = {0};
-    const size_t smem = DotShape<NBX>::kSmem;
+    const size_t smem = DotShape<NBX, XMODE>::kSmem;
     // one chunk per warp at most: a small GEMV spreads over as many SMs as it
     // has chunks (items cut between warps are summed in shared memory)
-    constexpr int threads = DotShape<NBX>::kThreads, warps = DotShape<NBX>::kWarps;
+    constexpr int threads = DotShape<NBX, XMODE>::kThreads, warps = DotShape<NBX, XMODE>::kWarps;
     const int want = (gp.total_chunks + warps - 1) / warps;
-    const int grid = grid_for(gemv_dot_kernel<NBX, ACC, XRAW>, threads, smem, want, cache);
-    launch_pdl(gemv_dot_kernel<NBX, ACC, XRAW>, grid, threads, smem, stream, gp);
+    const int grid = grid_for(gemv_dot_kernel<NBX, ACC, XMODE>, threads, smem, want, cache);
+    launch_pdl(gemv_dot_kernel<NBX, ACC, XMODE>, grid, threads, smem, stream, gp);
 }
 
 template <int NB, bool ACC>
@@ -1512,6 +1568,7 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
         D.xscale = act_scale;
         D.xw = reinterpret_cast<const uint4 *>(region);
         D.x = c.x;
+        D.xbf = c.xbf;
         D.out = c.out;
         D.part_acc = kparts > 1 ? reinterpret_cast<int32_t *>(region + xw_words) : nullptr;
         D.part_cnt = kparts > 1 ? region + xw_words + (int64_t)B * c.N : nullptr;
@@ -1537,10 +1594,14 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
     // x is re-ordered at most twice per chunk position; rows are not split, so
     // there are no K-part sums to clear).
     bool raw_x = phase == kBoth && pipelined && B <= 2 && cb <= kRawXMaxChunksPerSM * sm_count();
+    bool raw_bf = raw_x && !acc_out;
     for (int i = 0; i < count && raw_x; i++)
         raw_x = calls[i].x && !calls[i].xbf && !calls[i].xf && aligned(calls[i].x, 16) &&
                 kparts_for(calls[i].K) == 1;
-    if ((phase & kPrepare) && !raw_x) {
+    // likewise a small bf16 call: each warp quantizes the tokens it reads
+    for (int i = 0; i < count && raw_bf; i++)
+        raw_bf = calls[i].xbf && kparts_for(calls[i].K) == 1;
+    if ((phase & kPrepare) && !raw_x && !raw_bf) {
         if (f32) {
             launch_xprep_f32(fp, stream);
         } else {
@@ -1554,16 +1615,18 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
     // B <= 2: dp4a kernel; B >= 3: the MMA kernel (its 8 batch columns cost the
     // same as one, while dp4a work grows with B) -- measured on the decode stack
     if (pipelined && B <= 2) {
-        if (raw_x) {
+        if (raw_bf) {  // bf16 calls have no accumulator form
+            if (B == 1) launch_dot<1, false, 2>(gp, stream); else launch_dot<2, false, 2>(gp, stream);
+        } else if (raw_x) {
             if (B == 1) {
-                if (acc_out) launch_dot<1, true, true>(gp, stream); else launch_dot<1, false, true>(gp, stream);
+                if (acc_out) launch_dot<1, true, 1>(gp, stream); else launch_dot<1, false, 1>(gp, stream);
             } else {
-                if (acc_out) launch_dot<2, true, true>(gp, stream); else launch_dot<2, false, true>(gp, stream);
+                if (acc_out) launch_dot<2, true, 1>(gp, stream); else launch_dot<2, false, 1>(gp, stream);
             }
         } else if (B == 1) {
-            if (acc_out) launch_dot<1, true, false>(gp, stream); else launch_dot<1, false, false>(gp, stream);
+            if (acc_out) launch_dot<1, true, 0>(gp, stream); else launch_dot<1, false, 0>(gp, stream);
         } else {
-            if (acc_out) launch_dot<2, true, false>(gp, stream); else launch_dot<2, false, false>(gp, stream);
+            if (acc_out) launch_dot<2, true, 0>(gp, stream); else launch_dot<2, false, 0>(gp, stream);
         }
     } else if (pipelined) {
         if (B <= 8) {

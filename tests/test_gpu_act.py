@@ -72,3 +72,31 @@ def test_gemv_bf16_grouped_equals_single_calls():
     for (_, _, _, y), ref in zip(items, singles):
         assert torch.equal(y, ref)
     assert S.device_error() == 0
+
+
+@pytest.mark.parametrize("B", [1, 2])
+def test_gemv_bf16_small_calls_quantize_in_the_gemv(B):
+    """Small bf16 calls (B <= 2) skip the re-order launch: each warp takes the
+    token's absmax and quantizes its chunks itself.  One activation buffer read
+    as two row lengths (a 2048-value prefix of an 8192-value token) in one
+    grouped call must give two different scales; y is the oracle's bit for bit."""
+    cuda = torch.device("cuda")
+    bits = bf16_rows(B, 8192, seed=170 + B)
+    xfull = to_bf16(bits)
+    cases = [(64, 8192, xfull, bits)]
+    if B == 1:
+        cases.append((96, 2048, xfull[:, :2048], bits[:, :2048]))
+    items, refs = [], []
+    for i, (n, k, xt, xb) in enumerate(cases):
+        codes, scales = oracle.pack(synth.latent_weights(n, k, seed=180 + i))
+        q_ref, s_ref = oracle.quantize_act(np.ascontiguousarray(xb))
+        acc = oracle.gemv_acc(codes, q_ref, n, k)
+        refs.append((scales[None, :] * s_ref[:, None]).astype(np.float32) * acc.astype(np.float32))
+        y = torch.empty((B, n), dtype=torch.float32, device=cuda)
+        items.append((dev_codes(codes), dev(scales), xt, y))
+        assert np.array_equal(S.gemv_bf16(items[-1][0], items[-1][1], xt).cpu().numpy(), refs[-1])
+    S.gemv_bf16_grouped(items, B)
+    torch.cuda.synchronize()
+    for (_, _, _, y), ref in zip(items, refs):
+        assert np.array_equal(y.cpu().numpy(), ref)
+    assert S.device_error() == 0
