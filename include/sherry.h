@@ -130,16 +130,19 @@ sherry_status sherry_pack_grouped(const sherry_pack_desc *descs, int count,
                                   sherry_stream_t stream);
 
 /*
- * Workspace of the GEMV calls.  Each call re-orders its activations once into
- * the order in which the decoded weights meet the tensor-core fragments, and
+ * Workspace of the GEMV calls.  A call re-orders its activations once into
+ * the order in which the decoded weights meet the multiply-accumulate, and
  * long rows are processed as several K-parts whose int32 partial sums meet in
  * the workspace.  sherry_gemv_workspace_bytes(N, K, B) is the size one GEMV
  * needs; a grouped call needs the sum over its GEMVs, laid out in descriptor
- * order.  The workspace is a device buffer, 256-byte aligned, owned by the
- * caller; its contents are scratch: every call that prepares activations
- * (sherry_gemv, sherry_gemv_acc, sherry_gemv_grouped, sherry_gemv_prepare)
- * rewrites it, and a run leaves its partial-sum area cleared.  Calls that
- * overlap on the GPU must not share a workspace.
+ * order.  Small calls (B <= 2, K a multiple of 512, at most 64 chunks of
+ * 4 x 128 weights per SM, rows not split, activations 16-byte aligned) re-order (and for bf16,
+ * quantize) inside the GEMV kernel and leave the workspace untouched; the
+ * size asked is the same.  The workspace is a device buffer, 256-byte
+ * aligned, owned by the caller; its contents are scratch: every call that
+ * prepares activations (sherry_gemv, sherry_gemv_acc, sherry_gemv_grouped,
+ * sherry_gemv_prepare) may rewrite it, and a run leaves its partial-sum area
+ * cleared.  Calls that overlap on the GPU must not share a workspace.
  */
 size_t sherry_gemv_workspace_bytes(int64_t N, int64_t K, int B);
 
@@ -184,9 +187,10 @@ sherry_status sherry_quantize_act(const uint16_t *x, int64_t B, int64_t K, int8_
                                   sherry_stream_t stream);
 
 /*
- * sherry_gemv_bf16 -- the decode GEMV on bf16 activations: the re-order launch
- * quantizes each token as sherry_quantize_act does (keeping s_b in the
- * workspace) and the GEMV scales by both the weight and the activation scale:
+ * sherry_gemv_bf16 -- the decode GEMV on bf16 activations: each token is
+ * quantized as sherry_quantize_act does (in the re-order launch, keeping s_b in
+ * the workspace; for small calls inside the GEMV kernel) and the GEMV scales
+ * by both the weight and the activation scale:
  *   y[b][n] = fl32(fl32(s[n] * s_b) * acc[b][n]),  acc = W . q^T exactly.
  *   x  [B][K] bf16, 16-byte aligned; other arguments as sherry_gemv.
  *   workspace: sherry_gemv_bf16_workspace_bytes(N, K, B) bytes (a grouped call:
