@@ -1,0 +1,49 @@
+"""bench.py's contract pieces that run without a GPU: the reference arm (the
+oracle on the host cores) prints its one JSON line, a second rank of it exits
+without work, and the algorithmic bytes of the decode stack match the closed
+forms of the workload."""
+import json
+import os
+import subprocess
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def _run(extra_env, *args):
+    env = dict(os.environ, **extra_env)
+    return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *args], env=env,
+                          capture_output=True, text=True, timeout=300, cwd=ROOT)
+
+
+def test_reference_arm_prints_one_json_line():
+    r = _run({}, "--impl", "reference", "--layers", "1", "--steps", "2", "--warmup", "0")
+    assert r.returncode == 0, r.stderr
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "GB/s" and d["higher_is_better"] is True
+    assert d["metric"] == bench.METRIC and d["value"] > 0 and 1 <= d["steps"] <= 2
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["cpu_baseline"]["cores"] >= 1 and "7 GEMVs" in d["cpu_baseline"]["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_other_ranks_exit_without_work():
+    r = _run({"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"}, "--impl", "reference",
+             "--layers", "1", "--steps", "1")
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.strip() == ""
+
+
+def test_stack_algorithmic_bytes_closed_forms():
+    codes, total = bench.algorithmic_bytes(bench.stack_spec(16))
+    # 973,078,528 weights at 5 bits per 4 weights
+    assert codes == 973078528 * 5 // 32 == 152043520
+    # + fp32 scales (4 B per row), int8 x (K per GEMV) and fp32 y (4 B per row)
+    rows = 16 * (2048 + 512 + 512 + 2048 + 8192 + 8192 + 2048)
+    ks = 16 * (6 * 2048 + 8192)
+    assert total == codes + 4 * rows + ks + 4 * rows == 155385856
