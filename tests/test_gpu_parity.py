@@ -160,12 +160,19 @@ def test_gemv_grouped_1b_stack_layer():
         assert_y_matches(y.cpu().numpy(), ref)
 
 
-@pytest.mark.parametrize("B", [1, 2])
-def test_gemv_grouped_cut_items(B):
-    # many small GEMVs of mixed K (short last K-parts included) in one launch:
-    # warp ranges cut items at many places, inside and across GEMVs
-    shapes = [(33, 640), (96, 8192), (1, 128), (70, 2560), (200, 2048), (45, 3584),
-              (64, 5120), (7, 384), (130, 4096), (31, 1152), (40, 10752), (9, 17408)] * 3
+GROUPED_PIPELINED = [(33, 1536), (96, 8192), (1, 512), (70, 2560), (200, 2048), (45, 3584),
+                     (64, 5120), (7, 1024), (130, 4096), (31, 2560), (40, 10752), (9, 17408)] * 3
+# one K with T mod 4 != 0 sends the whole group to the register kernel
+GROUPED_REGISTER = [(33, 640), (96, 8192), (1, 128), (70, 2560), (200, 2048), (45, 3584),
+                    (64, 5120), (7, 384), (130, 4096), (31, 1152), (40, 10752), (9, 17408)] * 3
+
+
+@pytest.mark.parametrize("B", [1, 2, 5])
+@pytest.mark.parametrize("shapes", [GROUPED_PIPELINED, GROUPED_REGISTER], ids=["pipelined", "register"])
+def test_gemv_grouped_cut_items(B, shapes):
+    # many small GEMVs of mixed K (short last K-parts included) in one launch,
+    # through prepare + run (the re-order launch): warp ranges cut items at many
+    # places, inside and across GEMVs (dot kernel at B <= 2, MMA kernel at B = 5)
     items, refs = [], []
     for li, (N, K) in enumerate(shapes):
         codes, scales = oracle.pack(synth.latent_weights(N, K, seed=200 + li))
@@ -181,6 +188,33 @@ def test_gemv_grouped_cut_items(B):
         g.run()
         for (_, _, _, y), ref in zip(items, refs):
             assert_y_matches(y.cpu().numpy(), ref)
+
+
+def test_gemv_full_size_decode_stack_as_benched():
+    """The benchmark's launch: the 16-layer 1B stack, 112 GEMVs at B = 1, one
+    re-order launch and one GEMV launch (prepare + run), on random code words
+    (every word pattern is a valid code) and random scales; 64 sampled rows of
+    every GEMV against the oracle, bit for bit."""
+    rng = np.random.default_rng(2024)
+    xs = {2048: synth.int8_uniform((1, 2048), seed=1), 8192: synth.int8_uniform((1, 8192), seed=2)}
+    xd = {k: dev(v) for k, v in xs.items()}
+    items, host = [], []
+    for _, _, N, K, _ in synth.decode_stack(16):
+        codes = rng.integers(0, 2 ** 32, size=((N + 31) // 32, K // 128, 5, 32),
+                             dtype=np.uint64).astype(np.uint32)
+        scales = (rng.random(N) * 0.05 + 1e-3).astype(np.float32)
+        y = torch.empty((1, N), dtype=torch.float32, device="cuda")
+        items.append((dev_codes(codes), dev(scales), xd[K], y))
+        host.append((codes, scales, K))
+    g = S.GroupedGemv(items, B=1)
+    g.prepare()
+    g.run()
+    torch.cuda.synchronize()
+    for i, ((codes, scales, K), it) in enumerate(zip(host, items)):
+        rows = np.random.default_rng(i).choice(scales.shape[0], size=64, replace=False)
+        ref = oracle.gemv(rows_subset(codes, rows), scales[rows], xs[K], K)
+        assert_y_matches(it[3].cpu().numpy()[:, rows], ref)
+    assert S.device_error() == 0
 
 
 def test_gemv_on_gpu_packed_codes():
