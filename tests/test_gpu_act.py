@@ -100,3 +100,34 @@ def test_gemv_bf16_small_calls_quantize_in_the_gemv(B):
     for (_, _, _, y), ref in zip(items, refs):
         assert np.array_equal(y.cpu().numpy(), ref)
     assert S.device_error() == 0
+
+
+@pytest.mark.parametrize("B", [1, 2])
+def test_gemv_bf16_large_group_through_the_reorder_launch(B):
+    """A bf16 call too large for the in-kernel quantization (3 layers of the 1B
+    stack, 21 GEMVs, 11,136 chunks) quantizes in the re-order launch and the dot
+    kernel reads the scales from the workspace; sampled rows of every GEMV
+    against the oracle, bit for bit."""
+    from tests.gpu_helpers import rows_subset
+    cuda = torch.device("cuda")
+    rng = np.random.default_rng(190 + B)
+    xb = {k: bf16_rows(B, k, seed=200 + k + B) for k in (2048, 8192)}
+    xt = {k: to_bf16(v) for k, v in xb.items()}
+    q_s = {k: oracle.quantize_act(v) for k, v in xb.items()}
+    items, host = [], []
+    for _, _, n, k, _ in synth.decode_stack(3):
+        codes = rng.integers(0, 2 ** 32, size=((n + 31) // 32, k // 128, 5, 32),
+                             dtype=np.uint64).astype(np.uint32)
+        scales = (rng.random(n) * 0.05 + 1e-3).astype(np.float32)
+        y = torch.empty((B, n), dtype=torch.float32, device=cuda)
+        items.append((dev_codes(codes), dev(scales), xt[k], y))
+        host.append((codes, scales, k))
+    S.gemv_bf16_grouped(items, B)
+    torch.cuda.synchronize()
+    for i, ((codes, scales, k), it) in enumerate(zip(host, items)):
+        rows = np.random.default_rng(i).choice(scales.shape[0], size=48, replace=False)
+        q_ref, s_ref = q_s[k]
+        acc = oracle.gemv_acc(rows_subset(codes, rows), q_ref, len(rows), k)
+        ref = (scales[rows][None, :] * s_ref[:, None]).astype(np.float32) * acc.astype(np.float32)
+        assert np.array_equal(it[3].cpu().numpy()[:, rows], ref)
+    assert S.device_error() == 0
