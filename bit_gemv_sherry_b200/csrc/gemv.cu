@@ -2,8 +2,8 @@
 // and the activation front-ends that feed it.
 //
 // The product is the one the pages state for ternary weights with 3:4 blocks
-// coded in five bits (arXiv 2601.07892, abstract; Figure 2 caption: "SIMD-
-// friendly 4-way patterns").  On B200 a batch-1 GEMV is bound by HBM reads of
+// coded in five bits (arXiv 2601.07892, abstract; Figure 2 caption, which
+// presents the block patterns as suited to SIMD).  On B200 a batch-1 GEMV is bound by HBM reads of
 // the codes (0.15625 bytes per weight) only if the decode costs a few
 // instructions per 4-weight block.  Every kernel here decodes the same way:
 //

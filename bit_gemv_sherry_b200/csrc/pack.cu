@@ -1,7 +1,7 @@
 // pack.cu -- sherry_pack: fp32 latent weights -> Sherry 1.25-bit codes + row scales.
 //
-// The step the pages call "packing blocks of four weights into five bits" under
-// "3:4 fine-grained sparsity" (arXiv 2601.07892, abstract).  One warp handles a
+// The format's packing step: every block of four weights keeps one zero (3:4
+// sparsity) and is coded in five bits (arXiv 2601.07892, abstract).  One warp handles a
 // 128-weight tile at a time: lane j loads block j as a float4 (one coalesced
 // 512-byte row segment per warp), picks its zero (smallest |w|, lowest index
 // on ties), and the warp assembles the five words with ballots -- bit j of a

@@ -4,7 +4,7 @@
  *
  * The method ("Sherry: Hardware-Efficient 1.25-Bit Ternary Quantization via
  * Fine-grained Sparsification", arXiv 2601.07892, abstract; Figure 2 caption)
- * keeps weights in {-1, 0, +1} with 3:4 fine-grained sparsity -- every block of
+ * keeps weights in {-1, 0, +1} with 3:4 sparsity -- every block of
  * four consecutive weights along K holds exactly one zero -- and codes each
  * block in five bits (4 zero positions x 2^3 signs = 32 states), a regular
  * 1.25 bits per weight.  The product it serves is
@@ -12,7 +12,7 @@
  *     y[b][n] = s[n] * sum_k W[n][k] * x[b][k],    W ternary, x int8, s fp32.
  *
  * ---------------------------------------------------------------------------
- * Packed layout (the pages fix only "four weights in five bits"; this layout is
+ * Packed layout (the pages fix only the code size, five bits per four weights; this layout is
  * the library's reading, chosen so that 32 blocks decode with 32-bit SWAR
  * logic and a GEMV work chunk is one contiguous block of memory):
  *   - a row of K weights (K a multiple of 128) is cut into T = K / 128 tiles of
@@ -95,7 +95,7 @@ size_t sherry_packed_bytes(int64_t N, int64_t K);
 
 /*
  * sherry_pack -- 3:4 prune, ternarise, encode and scale (arXiv 2601.07892,
- * abstract: "packing blocks of four weights into five bits").
+ * abstract: blocks of four weights, five bits each).
  *   w       [N][K] fp32, row-major, finite values (NaN/Inf give an unspecified
  *           but deterministic code); 16-byte aligned.
  *   codes   output, sherry_packed_bytes(N, K) bytes, layout above (padding rows
