@@ -73,23 +73,49 @@ def algorithmic_bytes(spec, B=1):
 
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi samples of the GPU this process uses (timestamps on the host)."""
+    """nvidia-smi samples of the GPU this process uses (timestamps on the host).
+
+    The GPU is matched by UUID (case and the "GPU-" prefix ignored) or by PCI
+    domain/bus/device, whichever torch reports; a listing of a single GPU is
+    taken as that GPU."""
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, uuid):
-        self.uuid = uuid
+    def __init__(self, uuid=None, pci=None):
+        self.uuid = self.norm_uuid(uuid) if uuid else None
+        self.pci = pci
         self.samples = []
+        self.seen = {}
         self.proc = None
         self.thread = None
+
+    @staticmethod
+    def norm_uuid(u):
+        u = str(u).strip().lower()
+        return u[4:] if u.startswith("gpu-") else u
+
+    @staticmethod
+    def parse_pci(bus_id):
+        """'00000000:1B:00.0' -> (domain, bus, device)."""
+        try:
+            dom, bus, rest = bus_id.strip().split(":")
+            return int(dom, 16), int(bus, 16), int(rest.split(".")[0], 16)
+        except ValueError:
+            return None
+
+    def matches(self, uuid, bus_id):
+        if self.uuid and self.norm_uuid(uuid) == self.uuid:
+            return True
+        return self.pci is not None and self.parse_pci(bus_id) == self.pci
 
     def start(self):
         try:
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "--query-gpu=uuid," + self.FIELDS, "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                ["nvidia-smi", "--query-gpu=uuid,pci.bus_id," + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except (OSError, ValueError):
             self.proc = None
             return
@@ -99,9 +125,10 @@ class ClockSampler:
     def _read(self):
         for line in self.proc.stdout:
             parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9 or (self.uuid and parts[0] != self.uuid):
+            if len(parts) < 10:
                 continue
-            self.samples.append((time.time(), parts[1:]))
+            self.seen[parts[0]] = parts[1]
+            self.samples.append((time.time(), parts[0], parts[1], parts[2:]))
 
     def stop(self):
         if self.proc is not None:
@@ -111,10 +138,18 @@ class ClockSampler:
             except subprocess.TimeoutExpired:
                 self.proc.kill()
 
+    def select(self, samples):
+        mine = [s for _, u, b, s in samples if self.matches(u, b)]
+        if mine:
+            return mine, "matched"
+        if len(self.seen) == 1:
+            return [s for _, _, _, s in samples], "only gpu listed"
+        return [], "no match among %d gpus" % len(self.seen)
+
     def summary(self, t0, t1):
-        sel = [s for ts, s in self.samples if t0 <= ts <= t1]
+        sel, how = self.select([x for x in self.samples if t0 <= x[0] <= t1])
         if not sel:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "gpu": how}
 
         def num(v):
             try:
@@ -129,7 +164,18 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(smax) if smax else None,
                 "power_w_max": max(pw) if pw else None,
-                "reasons": reasons, "samples": len(sel)}
+                "reasons": reasons, "samples": len(sel), "gpu": how}
+
+
+def device_keys(torch, dev):
+    """(uuid, (pci domain, bus, device)) of a torch CUDA device, each None if unknown."""
+    props = torch.cuda.get_device_properties(dev)
+    uuid = getattr(props, "uuid", None)
+    try:
+        pci = (int(props.pci_domain_id), int(props.pci_bus_id), int(props.pci_device_id))
+    except (AttributeError, TypeError, ValueError):
+        pci = None
+    return (str(uuid) if uuid is not None else None), pci
 
 
 # ----------------------------------------------------------------------------- reference arm
@@ -551,17 +597,10 @@ def main():
     sptr = stream.cuda_stream
 
     for _ in range(args.warmup):
-        step.prepare(sptr)
-        step.run(sptr)
+        step(sptr)
     torch.cuda.synchronize(dev)
 
-    uuid = None
-    try:
-        uuid = str(torch.cuda.get_device_properties(dev).uuid)
-        uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
-    except Exception:
-        uuid = None
-    clocks = ClockSampler(uuid)
+    clocks = ClockSampler(*device_keys(torch, dev))
     clocks.start()
     time.sleep(0.3)
 
@@ -577,8 +616,7 @@ def main():
     t_host0 = time.time()
     e_start.record(stream)
     for i in range(K):
-        step.prepare(sptr)
-        step.run(sptr)
+        step(sptr)
     e_end.record(stream)
     torch.cuda.synchronize(dev)
     t_host1 = time.time()
@@ -667,8 +705,8 @@ def main():
             "code_bytes": codes_bytes, "batch": 1,
             "l2": "inputs larger than L2: %.0f MB of codes per step > 126 MB L2, no flush" % (
                 codes_bytes / 1e6),
-            "launch": "sherry_gemv_prepare + sherry_gemv_run (one activation re-order launch and "
-                      "one GEMV launch per step)",
+            "launch": "sherry_gemv_grouped (one activation re-order launch and one GEMV launch "
+                      "per step)",
             "parallelism": "replicas x%d" % world,
         },
         "gpu_launches": 2 * K,

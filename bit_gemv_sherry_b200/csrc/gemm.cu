@@ -30,6 +30,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 
 #include "common.cuh"
 
@@ -54,6 +55,13 @@ constexpr uint32_t kIdesc = (2u << 4)                  // D = s32
                             | (1u << 7) | (1u << 10)   // A, B = signed int8
                             | ((uint32_t)(kBN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
 constexpr size_t kSmemBytes = (size_t)kStages * kStageBytes + 1024 + 512;
+constexpr int kMaxDevices = 64;  // devices whose kernel attributes are tracked
+// Bounded waits, in SM clock cycles: the operand and accumulator barriers
+// (settable through sherry_set_wait_limit) and the drains of copies and MMAs
+// already in flight, which keep their own long limit.
+constexpr long long kDefaultWaitLimit = 4000000000LL;  // ~2 s at 1.9 GHz
+constexpr long long kDrainWaitLimit = 1000000000LL;
+std::atomic<long long> g_wait_limit{0};  // 0: kDefaultWaitLimit
 
 struct __align__(8) Barriers {
     uint64_t full_a[kStages];         // A tile written: 128 decoder threads
@@ -85,7 +93,8 @@ __device__ __forceinline__ void transpose4(const uint32_t (&in)[4], uint32_t (&o
 template <bool ACC_OUT>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const uint32_t *__restrict__ codes,
-                const float *__restrict__ scales, void *__restrict__ out, int M, int N, int T) {
+                const float *__restrict__ scales, void *__restrict__ out, int M, int N, int T,
+                long long wait_limit) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + ((1024 - (raw_addr & 1023)) & 1023);
@@ -128,20 +137,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int kt = 0; kt < T; kt++, it++) {
                     const int s = it % kStages;
                     const uint32_t ph = (it / kStages) & 1;
-                    if (!mbar_wait(&bar->empty[s >> 1], ph ^ 1, abort, err)) break;
+                    if (!mbar_wait(&bar->empty[s >> 1], ph ^ 1, abort, err, wait_limit)) break;
                     uint8_t *b_smem = smem + (size_t)s * kStageBytes + kABytes;
                     mbar_arrive_expect_tx(&bar->full_b[s], kBBytes);
                     tma_load_2d(b_smem, &tmap_x, &bar->full_b[s], kt * kBK, xb * kBN);
                 }
             }
-            if (*abort) {  // let issued copies land before the CTA's memory is released
-                const uint32_t n = it < (uint32_t)kStages ? it : (uint32_t)kStages;
-                for (uint32_t j = 1; j <= n; j++) {
-                    const uint32_t k = it - j;
-                    volatile int no_abort = 0;
-                    mbar_wait(&bar->full_b[k % kStages], (k / kStages) & 1, &no_abort, err,
-                              1000000000LL);
-                }
+            // Let every issued copy land before the CTA's shared memory is released,
+            // whether or not a role gave up later: the last copy of each stage
+            // (earlier ones were consumed through the stage's barrier phases).
+            const uint32_t n = it < (uint32_t)kStages ? it : (uint32_t)kStages;
+            for (uint32_t j = 1; j <= n; j++) {
+                const uint32_t k = it - j;
+                volatile int no_abort = 0;
+                mbar_wait(&bar->full_b[k % kStages], (k / kStages) & 1, &no_abort, err,
+                          kDrainWaitLimit);
             }
         }
     } else if (warp == 1) {
@@ -151,15 +161,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool issued = false;
             for (int tile = blockIdx.x; tile < num_tiles && !*abort; tile += gridDim.x, acc_it++) {
                 const uint32_t a = acc_it & 1, aph = (acc_it >> 1) & 1;
-                if (!mbar_wait(&bar->tmem_empty[a], aph ^ 1, abort, err)) break;
+                if (!mbar_wait(&bar->tmem_empty[a], aph ^ 1, abort, err, wait_limit)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + a * kBN;
                 bool ok = true;
                 for (int kt = 0; kt < T; kt++, it++) {
                     const int s = it % kStages;
                     const uint32_t ph = (it / kStages) & 1;
-                    if (!mbar_wait(&bar->full_a[s], ph, abort, err) ||
-                        !mbar_wait(&bar->full_b[s], ph, abort, err)) {
+                    if (!mbar_wait(&bar->full_a[s], ph, abort, err, wait_limit) ||
+                        !mbar_wait(&bar->full_b[s], ph, abort, err, wait_limit)) {
                         ok = false;
                         break;
                     }
@@ -178,10 +188,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!ok) break;
                 umma_commit(&bar->tmem_full[a]);
             }
-            if (*abort && issued) {  // wait for MMAs in flight before TMEM is released
+            // Wait for every issued MMA before TMEM and the operand stages are
+            // released, whether or not a role gave up after this loop ended.
+            if (issued) {
                 umma_commit(&bar->drain);
                 volatile int no_abort = 0;
-                mbar_wait(&bar->drain, 0, &no_abort, err, 1000000000LL);
+                mbar_wait(&bar->drain, 0, &no_abort, err, kDrainWaitLimit);
             }
         }
     } else if (warp < 2 + 4 * kDecGroups) {
@@ -221,7 +233,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int s = j % kStages;
             const uint32_t ph = (j / kStages) & 1;
             // the A slot's previous tile has been consumed by the MMAs
-            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&bar->empty[s >> 1], ph ^ 1, abort, err))) break;
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&bar->empty[s >> 1], ph ^ 1, abort, err, wait_limit)))
+                break;
             const int tile = (int)blockIdx.x + (int)(j / T) * (int)gridDim.x;
             const bool valid = (tile % tiles_n) * kBM + r < N;
             TileDecoder dec;
@@ -258,7 +271,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int wb = tile % tiles_n, xb = tile / tiles_n;
             const uint32_t a = acc_it & 1, aph = (acc_it >> 1) & 1;
             // every lane waits; the warp leaves together if any lane's wait gave up
-            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&bar->tmem_full[a], aph, abort, err))) break;
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&bar->tmem_full[a], aph, abort, err, wait_limit)))
+                break;
             tc_fence_after();
             const int row = wb * kBM + q * 32 + lane;
             const bool rv = row < N;
@@ -333,8 +347,19 @@ sherry_status gemm_launch(const uint32_t *codes, const float *scales, const int8
         set_last_error("cuTensorMapEncodeTiled", cudaErrorInvalidValue);
         return SHERRY_ERR_CUDA;
     }
-    static bool attr_set[2] = {false, false};
-    if (!attr_set[ACC]) {
+    // the shared-memory attribute is per device: set it once on each device
+    // this kernel runs on
+    static std::atomic<bool> attr_set[kMaxDevices];
+    int dev = 0;
+    {
+        const cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) {
+            set_last_error("sherry_gemm (cudaGetDevice)", e);
+            return SHERRY_ERR_CUDA;
+        }
+    }
+    if (dev < 0 || dev >= kMaxDevices) return SHERRY_ERR_UNSUPPORTED;
+    if (!attr_set[dev].load(std::memory_order_acquire)) {
         const cudaError_t e = cudaFuncSetAttribute(gemm_kernel<ACC>,
                                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                    (int)kSmemBytes);
@@ -342,13 +367,15 @@ sherry_status gemm_launch(const uint32_t *codes, const float *scales, const int8
             set_last_error("sherry_gemm (shared memory attribute)", e);
             return SHERRY_ERR_CUDA;
         }
-        attr_set[ACC] = true;
+        attr_set[dev].store(true, std::memory_order_release);
     }
     const int64_t tiles = ((N + kBM - 1) / kBM) * ((M + kBN - 1) / kBN);
     if (tiles > 0x7FFFFFFF) return SHERRY_ERR_UNSUPPORTED;
     const int grid = (int)std::min<int64_t>(tiles, sm_count());
+    const long long lim = g_wait_limit.load(std::memory_order_relaxed);
     gemm_kernel<ACC><<<grid, kThreads, kSmemBytes, stream>>>(tmap, codes, scales, out, (int)M,
-                                                             (int)N, (int)(K / kBK));
+                                                             (int)N, (int)(K / kBK),
+                                                             lim > 0 ? lim : kDefaultWaitLimit);
     return launch_status("sherry_gemm");
 }
 
@@ -366,6 +393,12 @@ extern "C" sherry_status sherry_gemm_acc(const uint32_t *codes, const int8_t *x,
                                          int64_t M, int64_t N, int64_t K, sherry_stream_t stream) {
     return sherry::gemm_launch<true>(codes, nullptr, x, acc, M, N, K,
                                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" sherry_status sherry_set_wait_limit(int64_t cycles) {
+    if (cycles < 0) return SHERRY_ERR_SHAPE;
+    sherry::g_wait_limit.store((long long)cycles, std::memory_order_relaxed);
+    return SHERRY_OK;
 }
 
 extern "C" sherry_status sherry_device_error(void) {

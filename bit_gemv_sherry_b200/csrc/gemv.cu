@@ -75,6 +75,13 @@ struct GemvDesc {
 struct GemvParams {
     int count;
     int B;
+    // 1: this launch follows the call's own re-order launch, whose grid writes
+    // no codes and started only after every earlier ordinary launch completed,
+    // so the first code copies may be issued before griddepcontrol.wait.  0:
+    // the kernel before may be the caller's (e.g. the one that wrote the
+    // codes), so nothing is read before the wait.
+    int prefetch_codes;
+    int pad0;
     int total_units16;    // register kernel
     int total_chunks;     // pipelined kernel: chunks of all groups (the balancing space)
     // Constants passed at run time so that they live in registers instead of
@@ -839,8 +846,9 @@ __global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
 
     // ---- producer side: the issue cursor runs kRing-1 stages ahead ----
     // lane l copies 16-byte pieces l + 32 j (j = 0..4) of the 2560-byte chunk;
-    // piece words 4i..4i+3 belong to tile block 4i / 160.  Codes only: the
-    // activations are read from global memory after pdl_wait().
+    // piece words 4i..4i+3 belong to tile block 4i / 160.  Codes only (and
+    // only when P.prefetch_codes allows it before pdl_wait()): the activations
+    // are read from global memory after pdl_wait().
     ItemCursor icur = cur;
     int istart = start, ic = 0, ic_end = 0;
     const uint32_t *isrc = nullptr;  // first word of the current unit's group
@@ -876,9 +884,10 @@ __global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
         }
         cp_async_commit();
     };
+    if (!P.prefetch_codes) pdl_wait();
 #pragma unroll
     for (int s = 0; s < kRing - 1; s++) issue(s);
-    pdl_wait();
+    if (P.prefetch_codes) pdl_wait();
 
     // ---- consumer side ----
     int slot = 0;
@@ -1151,8 +1160,9 @@ __global__ void __launch_bounds__(DotShape<NBX, XMODE>::kThreads, DotShape<NBX, 
     // ---- producer side: the issue cursor runs kDotRing-1 stages ahead ----
     // lane l copies 16-byte pieces l + 32 j (j = 0..4) of the chunk's codes and
     // piece l of each batch row's 128 activation words.  Until pdl_wait() only
-    // codes are read: the activation words and the K-part sums belong to the
-    // re-order kernel before this one.
+    // codes are read, and only when P.prefetch_codes says the kernel before is
+    // this call's re-order launch: the activation words and the K-part sums
+    // belong to that kernel.
     ItemCursor icur = cur;
     int istart = start, ic = 0, ic_end = 0, iTp = 0;
     const uint32_t *isrc = nullptr, *ixw = nullptr;
@@ -1217,8 +1227,9 @@ __global__ void __launch_bounds__(DotShape<NBX, XMODE>::kThreads, DotShape<NBX, 
     };
     static_assert(kDotRing == 2, "the prologue fills one stage");
     const bool first_copy = istart < b1;
-    if (first_copy) copy_codes(0);
+    if (first_copy && P.prefetch_codes) copy_codes(0);
     pdl_wait();
+    if (first_copy && !P.prefetch_codes) copy_codes(0);
     if (first_copy) copy_x_and_advance(0);
     cp_async_commit();
 
@@ -1601,6 +1612,7 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
     // likewise a small bf16 call: each warp quantizes the tokens it reads
     for (int i = 0; i < count && raw_bf; i++)
         raw_bf = calls[i].xbf && kparts_for(calls[i].K) == 1;
+    gp.prefetch_codes = (phase & kPrepare) && !raw_x && !raw_bf;
     if ((phase & kPrepare) && !raw_x && !raw_bf) {
         if (f32) {
             launch_xprep_f32(fp, stream);

@@ -90,6 +90,7 @@ def lib():
         "sherry_gemm": ([p, p, p, p, i64, i64, i64, p], i32),
         "sherry_gemm_acc": ([p, p, p, i64, i64, i64, p], i32),
         "sherry_device_error": ([], i32),
+        "sherry_set_wait_limit": ([i64], i32),
         "sherry_status_string": ([i32], ctypes.c_char_p),
         "sherry_last_error": ([], ctypes.c_char_p),
         "sherry_version": ([], i32),
@@ -532,3 +533,9 @@ def gemm_acc(codes, x, N, acc=None):
 def device_error():
     """Synchronise and return (and clear) the device-side error word (0 = none)."""
     return int(lib().sherry_device_error())
+
+
+def set_wait_limit(cycles):
+    """Limit (SM clock cycles) of the kernels' bounded barrier waits, for
+    kernels launched afterwards by this process; 0 restores the default."""
+    _check(lib().sherry_set_wait_limit(int(cycles)), "sherry_set_wait_limit")

@@ -89,7 +89,10 @@ typedef enum {
 #define SHERRY_STATIC_SCRATCH_BYTES (4u << 20)  /* scratch of sherry_gemv_static */
 
 /* Bytes of packed codes for an N x K matrix: ceil(N/32)*32 * K * 5 / 32
- * (N * K * 5 / 32 when N is a multiple of 32; scales excluded).
+ * (N * K * 5 / 32 when N is a multiple of 32; scales excluded).  The count
+ * is the abstract's five bits per block of four weights, 1.25 bits per weight
+ * (arXiv 2601.07892, abstract); the rounding of N up to whole 32-row groups
+ * is this layout's own.
  * Returns 0 when K is not a positive multiple of 128 or N < 1. */
 size_t sherry_packed_bytes(int64_t N, int64_t K);
 
@@ -324,7 +327,10 @@ typedef struct {
  * sherry_gemv_grouped -- `count` independent GEMVs (count <= SHERRY_MAX_GROUP),
  * all with the same batch B, in one pass: one activation re-ordering launch
  * and one GEMV launch whose warps stream the codes of every GEMV.  This is the
- * decode step of a whole stack of layers whose inputs are already known.
+ * decode step of a whole stack of layers whose inputs are already known.  The
+ * pages define no grouping; each GEMV is the product of sherry_gemv, and the
+ * stack is the batch-1 decode workload of LLaMA-3.2-1B-shaped layers that the
+ * method is evaluated on (arXiv 2601.07892, abstract: LLaMA-3.2 1B and 3B).
  *   descs  HOST array of `count` descriptors (copied into the launch
  *          parameters; may be reused as soon as the call returns).
  *   workspace: at least the sum over the group of
@@ -357,6 +363,10 @@ sherry_status sherry_gemv_run(const sherry_gemv_desc *descs, int count, int B,
 /*
  * sherry_gemm -- prefill GEMM, Y = X . W^T scaled per output column,
  *   Y[m][n] = s[n] * sum_k X[m][k] * W[n][k]   (the same product for M tokens).
+ * The pages define no GEMM: this is the product the abstract serves
+ * (arXiv 2601.07892, abstract: ternary weights with int8 activations) taken
+ * over M tokens at once, the prefill step of the same decoder layers; at
+ * M >= 64 it is a dense contraction and runs on the tensor cores.
  * The kernel decodes weight tiles to int8 in shared memory and runs them on
  * the tcgen05 int8 tensor-core path with int32 accumulators in tensor memory.
  *   codes   [ceil(N/32)][K/128][5][32] uint32; 4-byte aligned.
@@ -380,6 +390,19 @@ sherry_status sherry_gemm_acc(const uint32_t *codes, const int8_t *x, int32_t *a
  * clears it.
  */
 sherry_status sherry_device_error(void);
+
+/*
+ * sherry_set_wait_limit -- limit, in SM clock cycles, of the bounded waits of
+ * kernels launched after this call by any thread of the process (the GEMM's
+ * operand and accumulator barriers).  0 restores the default of 4e9 cycles
+ * (about 2 s at 1.9 GHz).  Meant for tests and failure drills: with a small
+ * limit the waits give up, the kernel records SHERRY_ERR_TIMEOUT (read and
+ * cleared by sherry_device_error), lets the copies and MMAs it already issued
+ * finish (those drains keep their own long limit), releases its tensor memory
+ * and returns; its output is then undefined.  The setting is process-wide.
+ * Errors: SHAPE if cycles < 0.
+ */
+sherry_status sherry_set_wait_limit(int64_t cycles);
 
 /* Text of a status code (static string). */
 const char *sherry_status_string(sherry_status status);

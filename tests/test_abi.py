@@ -189,3 +189,10 @@ def test_python_binding_rejects_cpu_tensors():
     import torch
     with pytest.raises(TypeError):
         S.pack(torch.zeros(4, 128))
+
+
+def test_wait_limit_setting_is_checked_and_restorable():
+    L = S.lib()
+    assert L.sherry_set_wait_limit(-1) == 2
+    assert L.sherry_set_wait_limit(1000) == 0
+    assert L.sherry_set_wait_limit(0) == 0

@@ -47,3 +47,31 @@ def test_stack_algorithmic_bytes_closed_forms():
     rows = 16 * (2048 + 512 + 512 + 2048 + 8192 + 8192 + 2048)
     ks = 16 * (6 * 2048 + 8192)
     assert total == codes + 4 * rows + ks + 4 * rows == 155385856
+
+
+def _sample(uuid, bus, mhz, power_cap="Not Active"):
+    return (1.0, uuid, bus, [str(mhz), "1965", "700", "0x0", "Not Active", "Not Active",
+                             "Not Active", power_cap])
+
+
+def test_clock_sampler_matches_the_gpu_by_uuid_or_pci_bus():
+    rows = [_sample("GPU-AbCd-0001", "00000000:1B:00.0", 1965),
+            _sample("GPU-ffff-0002", "00000009:2C:00.0", 1200, "Active")]
+    # torch prints the UUID without the prefix and in lower case
+    by_uuid = bench.ClockSampler("abcd-0001", None)
+    by_uuid.samples, by_uuid.seen = rows, {r[1]: r[2] for r in rows}
+    s = by_uuid.summary(0.0, 2.0)
+    assert s["samples"] == 1 and s["sm_mhz"] == 1965.0 and s["reasons"] == []
+    # no usable UUID: the PCI domain, bus and device decide
+    by_pci = bench.ClockSampler(None, (9, 0x2C, 0))
+    by_pci.samples, by_pci.seen = rows, {r[1]: r[2] for r in rows}
+    s = by_pci.summary(0.0, 2.0)
+    assert s["samples"] == 1 and s["sm_mhz"] == 1200.0 and s["reasons"] == ["sw_power_cap"]
+    # nothing matches among several GPUs: no samples rather than another GPU's
+    none = bench.ClockSampler("0000", (1, 2, 3))
+    none.samples, none.seen = rows, {r[1]: r[2] for r in rows}
+    assert none.summary(0.0, 2.0)["samples"] == 0
+    # a listing of one GPU is that GPU
+    one = bench.ClockSampler("0000", None)
+    one.samples, one.seen = rows[:1], {rows[0][1]: rows[0][2]}
+    assert one.summary(0.0, 2.0)["samples"] == 1

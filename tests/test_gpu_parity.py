@@ -268,6 +268,34 @@ def test_gemm_full_size_prefill(case):
     assert_y_matches(y[:, rows], oracle.gemm(sub, scales[rows], x, K))
 
 
+@pytest.mark.parametrize("N,K,B", [(256, 1024, 1), (96, 2048, 2), (320, 4096, 3)])
+def test_pack_then_gemv_back_to_back_on_one_stream(N, K, B):
+    """The GEMV right after the kernel that wrote its codes, with no host
+    synchronisation: small calls (the first two shapes) skip the re-order
+    launch, so the pack kernel is the GEMV launch's direct predecessor and the
+    GEMV must read the codes only after its grid-dependency wait."""
+    w1, w2 = synth.latent_weights(N, K, seed=41), synth.latent_weights(N, K, seed=42)
+    x = synth.int8_uniform((B, K), seed=43)
+    c1, _ = oracle.pack(w1)
+    c2, _ = oracle.pack(w2)
+    tw1, tw2, tx = dev(w1), dev(w2), dev(x)
+    codes = torch.zeros(S.codes_shape(N, K), dtype=torch.int32, device="cuda")
+    sc1 = torch.zeros(N, dtype=torch.float32, device="cuda")
+    sc2 = torch.zeros_like(sc1)
+    ws = S.workspace(S.gemv_workspace_bytes(N, K, B), torch.device("cuda"))
+    y1 = torch.empty((B, N), dtype=torch.float32, device="cuda")
+    y2 = torch.empty_like(y1)
+    torch.cuda.synchronize()
+    for tw, sc, y in ((tw1, sc1, y1), (tw2, sc2, y2)):   # the second pack overwrites the codes
+        S.pack(tw, codes, sc)
+        S.gemv(codes, sc, tx, y, ws)
+    torch.cuda.synchronize()
+    for c, sc, y in ((c1, sc1, y1), (c2, sc2, y2)):
+        # y against the oracle's dot products with the scales the GPU wrote, so
+        # that only the codes each GEMV read decide the comparison
+        assert_y_matches(y.cpu().numpy(), oracle.gemv(c, sc.cpu().numpy(), x, K))
+
+
 def test_gemm_m1_equals_gemv():
     N, K = 384, 1024
     codes, scales = oracle.pack(synth.latent_weights(N, K, seed=5))

@@ -26,8 +26,11 @@ def _x(B, K, seed):
     return torch.from_numpy(synth.int8_uniform((B, K), seed=seed)).cuda()
 
 
+# (2048, 16384, 4): rows longer than 8192 are split into K-parts, so the static
+# array also holds the int32 partial sums and the per-unit counters, which each
+# call must find cleared by the call before it.
 @pytest.mark.parametrize("N,K,B", [(2048, 8192, 1), (1000, 2048, 5), (4096, 4096, 16),
-                                   (33, 384, 3)])
+                                   (33, 384, 3), (2048, 16384, 4), (70, 17408, 1)])
 def test_static_matches_workspace_gemv_two_calls_in_a_row(N, K, B):
     codes, scales = _layer(N, K, seed=900 + N % 97)
     x1, x2 = _x(B, K, seed=901), _x(B, K, seed=902)
