@@ -24,4 +24,13 @@ from .oracle import (  # noqa: F401
     gemm,
     num_threads,
     set_num_threads,
+    FMT_I2,
+    FMT_T3,
+    cmp_tiles,
+    cmp_packed_bytes,
+    t3_code,
+    t3_weights,
+    cmp_encode,
+    cmp_unpack,
+    cmp_gemv_acc,
 )

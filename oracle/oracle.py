@@ -47,9 +47,22 @@ def _load(path=None):
     lib.oracle_gemv_act.argtypes = [p, p, p, p, i64, i64, i64, p]
     lib.oracle_quantize_f32.argtypes = [p, i64, i64, p, p]
     lib.oracle_swiglu.argtypes = [p, p, i64, p]
+    i32 = ctypes.c_int32
+    lib.oracle_cmp_tiles.argtypes = [i32, i64]
+    lib.oracle_cmp_tiles.restype = i64
+    lib.oracle_cmp_packed_bytes.argtypes = [i32, i64, i64]
+    lib.oracle_cmp_packed_bytes.restype = i64
+    lib.oracle_t3_code.argtypes = [p]
+    lib.oracle_t3_code.restype = i32
+    lib.oracle_t3_weights.argtypes = [i32, p]
+    lib.oracle_t3_weights.restype = None
+    lib.oracle_cmp_encode.argtypes = [i32, p, i64, i64, p]
+    lib.oracle_cmp_unpack.argtypes = [i32, p, i64, i64, p]
+    lib.oracle_cmp_gemv_acc.argtypes = [i32, p, p, i64, i64, i64, p]
     for f in ("oracle_pack", "oracle_unpack", "oracle_gemv_acc", "oracle_gemv",
               "oracle_gemm_acc", "oracle_gemm", "oracle_quantize_act", "oracle_gemv_act",
-              "oracle_quantize_f32", "oracle_swiglu"):
+              "oracle_quantize_f32", "oracle_swiglu", "oracle_cmp_encode", "oracle_cmp_unpack",
+              "oracle_cmp_gemv_acc"):
         getattr(lib, f).restype = ctypes.c_int
     lib.oracle_num_threads.argtypes = []
     lib.oracle_num_threads.restype = ctypes.c_int
@@ -237,3 +250,57 @@ def bf16_bits(values):
     if np.any(u & 0xFFFF):
         raise ValueError("value not representable in bf16")
     return (u >> 16).astype(np.uint16)
+
+
+# ----------------------------------------------------------------------------- comparison formats
+FMT_I2 = 1  # 2 bits per weight, aligned
+FMT_T3 = 2  # three weights in five bits (base 3)
+_TILE_WORDS = {FMT_I2: 8, FMT_T3: 5}
+
+
+def cmp_tiles(fmt, K):
+    return int(_load().oracle_cmp_tiles(fmt, K))
+
+
+def cmp_packed_bytes(fmt, N, K):
+    return int(_load().oracle_cmp_packed_bytes(fmt, N, K))
+
+
+def t3_code(tri):
+    t = np.ascontiguousarray(tri, dtype=np.int8)
+    assert t.shape == (3,)
+    return int(_load().oracle_t3_code(_ptr(t)))
+
+
+def t3_weights(code):
+    w = np.zeros(3, np.int8)
+    _load().oracle_t3_weights(int(code), _ptr(w))
+    return w
+
+
+def cmp_encode(fmt, wt):
+    """Ternary int8 [N, K] -> codes uint32 [ceil(N/32), tiles, words, 32] of format fmt."""
+    wt = np.ascontiguousarray(wt, dtype=np.int8)
+    N, K = wt.shape
+    T = cmp_tiles(fmt, K)
+    if T == 0:
+        raise ValueError("bad format or K")
+    codes = np.zeros(((N + GROUP - 1) // GROUP, T, _TILE_WORDS[fmt], GROUP), np.uint32)
+    _check(_load().oracle_cmp_encode(fmt, _ptr(wt), N, K, _ptr(codes)), "oracle_cmp_encode")
+    return codes
+
+
+def cmp_unpack(fmt, codes, N, K):
+    codes = np.ascontiguousarray(codes, dtype=np.uint32)
+    wt = np.zeros((N, K), np.int8)
+    _check(_load().oracle_cmp_unpack(fmt, _ptr(codes), N, K, _ptr(wt)), "oracle_cmp_unpack")
+    return wt
+
+
+def cmp_gemv_acc(fmt, codes, x, N, K):
+    codes = np.ascontiguousarray(codes, dtype=np.uint32)
+    x = _x2(x, K)
+    acc = np.zeros((x.shape[0], N), np.int64)
+    _check(_load().oracle_cmp_gemv_acc(fmt, _ptr(codes), _ptr(x), N, K, x.shape[0], _ptr(acc)),
+           "oracle_cmp_gemv_acc")
+    return acc

@@ -355,3 +355,188 @@ int oracle_gemv_act(const uint32_t *codes, const float *scales, const int8_t *q,
     free(acc);
     return rc;
 }
+
+/*
+ * Comparison formats.  The pages set Sherry's 1.25 bits per weight against
+ * the two ternary packings they call the state of the art (arXiv 2601.07892,
+ * abstract; Figure 2 caption): a 2-bit aligned packing, which wastes a quarter
+ * of its code space, and a 1.67-bit packing of three weights in five bits,
+ * whose 3-way grouping does not match power-of-two lanes.  Neither layout is
+ * printed; the readings below are this build's own (restated in the design
+ * notes).  Both hold any ternary matrix; for comparison they are filled from
+ * the same ternary values as a Sherry matrix (via oracle_unpack).
+ *
+ * Format 1, "I2" (2 bits per weight, aligned):
+ *   - code of one weight: 0 -> 0, 1 -> +1, 3 -> -1 (bit 0 = nonzero, bit 1 =
+ *     negative); the unused code 2 decodes to 0;
+ *   - a tile is 128 weights of a row in eight 32-bit words; word q holds
+ *     weights k = 128 t + 16 q + m (m = 0..15): weight m sits at bits
+ *     [4 (m mod 8) + 2 (m / 8), +1], so nibble n of the word holds weights n
+ *     (low two bits) and n + 8 (high two bits);
+ *   - rows in groups of 32 as for Sherry: word(q, n, t) =
+ *     codes[((n / 32) * T + t) * 256 + 32 q + n % 32], T = K / 128, K a
+ *     multiple of 128; rows past N are zero.
+ * Format 2, "T3" (three weights in five bits, 1.67 bits per weight):
+ *   - code of a triple (w0, w1, w2): c = (w0 + 1) + 3 (w1 + 1) + 9 (w2 + 1),
+ *     0..26; codes 27..31 are never written and decode to three zeros;
+ *   - a tile is 32 triples = 96 weights of a row in five 32-bit words: triple
+ *     j covers k = 96 t + 3 j + {0, 1, 2} and its code is bits [5 j, 5 j + 4]
+ *     of the 160-bit little-endian string of words 0..4 (string bit b is bit
+ *     b mod 32 of word b / 32), so triples 6, 12, 19 and 25 straddle words;
+ *   - a row of K weights (K a multiple of 128) is padded with zero weights to
+ *     an even number of tiles, T3 = 2 * ceil(K / 192) (the GPU streams tiles
+ *     in pairs); rows in groups of 32: word(p, n, t) =
+ *     codes[((n / 32) * T3 + t) * 160 + 32 p + n % 32].
+ */
+enum { ORC_FMT_I2 = 1, ORC_FMT_T3 = 2 };
+
+/* Tiles per row of a comparison format (0 for a bad format or K). */
+int64_t oracle_cmp_tiles(int32_t fmt, int64_t K)
+{
+    if (K < ORC_TILE || K % ORC_TILE) return 0;
+    if (fmt == ORC_FMT_I2) return K / ORC_TILE;
+    if (fmt == ORC_FMT_T3) return 2 * ((K + 191) / 192);
+    return 0;
+}
+
+/* Words per tile per row of a comparison format. */
+static int64_t orc_cmp_tile_words(int32_t fmt) { return fmt == ORC_FMT_I2 ? 8 : 5; }
+
+/* Bytes of codes of an N x K matrix in a comparison format (-1 if invalid). */
+int64_t oracle_cmp_packed_bytes(int32_t fmt, int64_t N, int64_t K)
+{
+    const int64_t T = oracle_cmp_tiles(fmt, K);
+    if (T == 0 || N < 1) return -1;
+    return orc_padded_rows(N) * T * orc_cmp_tile_words(fmt) * 4;
+}
+
+static int64_t orc_cmp_word(int32_t fmt, int64_t q, int64_t n, int64_t t, int64_t T)
+{
+    const int64_t tw = orc_cmp_tile_words(fmt);
+    return ((n / ORC_GROUP) * T + t) * (tw * ORC_GROUP) + q * ORC_GROUP + n % ORC_GROUP;
+}
+
+/* 2-bit code of one ternary value, and back. */
+static uint32_t orc_i2_code(int8_t w) { return w == 0 ? 0u : (w > 0 ? 1u : 3u); }
+static int8_t orc_i2_weight(uint32_t c) { return (c & 1u) ? ((c & 2u) ? -1 : 1) : 0; }
+
+/* Base-3 code of a triple, and back (codes past 26 give zeros). */
+int32_t oracle_t3_code(const int8_t *w)
+{
+    return (w[0] + 1) + 3 * (w[1] + 1) + 9 * (w[2] + 1);
+}
+
+void oracle_t3_weights(int32_t code, int8_t *w)
+{
+    if (code < 0 || code > 26) {
+        w[0] = w[1] = w[2] = 0;
+        return;
+    }
+    w[0] = (int8_t)(code % 3 - 1);
+    w[1] = (int8_t)((code / 3) % 3 - 1);
+    w[2] = (int8_t)(code / 9 - 1);
+}
+
+/* Ternary weight k of row `row` (K values), zero past K. */
+static int8_t orc_row_at(const int8_t *row, int64_t K, int64_t k) { return k < K ? row[k] : 0; }
+
+/* Encode a ternary matrix Wt[N][K] (values in {-1, 0, +1}) in format fmt. */
+int oracle_cmp_encode(int32_t fmt, const int8_t *wt, int64_t N, int64_t K, uint32_t *codes)
+{
+    const int64_t T = oracle_cmp_tiles(fmt, K);
+    if (!wt || !codes || N < 1 || T == 0) return ORC_BAD_ARG;
+    const int64_t tw = orc_cmp_tile_words(fmt);
+    memset(codes, 0, (size_t)oracle_cmp_packed_bytes(fmt, N, K));
+    for (int64_t n = 0; n < N; n++) {
+        const int8_t *row = wt + n * K;
+        for (int64_t t = 0; t < T; t++) {
+            uint32_t w[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+            if (fmt == ORC_FMT_I2) {
+                for (int q = 0; q < 8; q++)
+                    for (int m = 0; m < 16; m++) {
+                        const uint32_t c = orc_i2_code(row[t * ORC_TILE + 16 * q + m]);
+                        w[q] |= c << (4 * (m % 8) + 2 * (m / 8));
+                    }
+            } else {
+                for (int j = 0; j < 32; j++) {
+                    int8_t tri[3];
+                    for (int i = 0; i < 3; i++) tri[i] = orc_row_at(row, K, 96 * t + 3 * j + i);
+                    const uint32_t c = (uint32_t)oracle_t3_code(tri);
+                    for (int b = 0; b < 5; b++) {
+                        const int bit = 5 * j + b;
+                        w[bit / 32] |= ((c >> b) & 1u) << (bit % 32);
+                    }
+                }
+            }
+            for (int q = 0; q < tw; q++) codes[orc_cmp_word(fmt, q, n, t, T)] = w[q];
+        }
+    }
+    return ORC_OK;
+}
+
+/* Ternary row n (K values) of a comparison-format matrix. */
+static void orc_cmp_unpack_row(int32_t fmt, const uint32_t *codes, int64_t n, int64_t K, int8_t *row)
+{
+    const int64_t T = oracle_cmp_tiles(fmt, K);
+    const int64_t tw = orc_cmp_tile_words(fmt);
+    for (int64_t t = 0; t < T; t++) {
+        uint32_t w[8];
+        for (int q = 0; q < tw; q++) w[q] = codes[orc_cmp_word(fmt, q, n, t, T)];
+        if (fmt == ORC_FMT_I2) {
+            for (int q = 0; q < 8; q++)
+                for (int m = 0; m < 16; m++)
+                    row[t * ORC_TILE + 16 * q + m] =
+                        orc_i2_weight(w[q] >> (4 * (m % 8) + 2 * (m / 8)));
+        } else {
+            for (int j = 0; j < 32; j++) {
+                uint32_t c = 0;
+                for (int b = 0; b < 5; b++) {
+                    const int bit = 5 * j + b;
+                    c |= ((w[bit / 32] >> (bit % 32)) & 1u) << b;
+                }
+                int8_t tri[3];
+                oracle_t3_weights((int32_t)c, tri);
+                for (int i = 0; i < 3; i++) {
+                    const int64_t k = 96 * t + 3 * j + i;
+                    if (k < K) row[k] = tri[i];
+                }
+            }
+        }
+    }
+}
+
+int oracle_cmp_unpack(int32_t fmt, const uint32_t *codes, int64_t N, int64_t K, int8_t *wt)
+{
+    if (!codes || !wt || N < 1 || oracle_cmp_tiles(fmt, K) == 0) return ORC_BAD_ARG;
+    #pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; n++) orc_cmp_unpack_row(fmt, codes, n, K, wt + n * K);
+    return ORC_OK;
+}
+
+/* acc[b][n] = sum_k Wt[n][k] * x[b][k] in int64 for a comparison-format matrix. */
+int oracle_cmp_gemv_acc(int32_t fmt, const uint32_t *codes, const int8_t *x, int64_t N, int64_t K,
+                        int64_t B, int64_t *acc)
+{
+    if (!codes || !x || !acc || N < 1 || B < 1 || oracle_cmp_tiles(fmt, K) == 0) return ORC_BAD_ARG;
+    int err = 0;
+    #pragma omp parallel
+    {
+        int8_t *row = (int8_t *)malloc((size_t)K);
+        if (!row) {
+            #pragma omp atomic write
+            err = 1;
+        }
+        #pragma omp for schedule(static)
+        for (int64_t n = 0; n < N; n++) {
+            if (!row) continue;
+            orc_cmp_unpack_row(fmt, codes, n, K, row);
+            for (int64_t b = 0; b < B; b++) {
+                int64_t a = 0;
+                for (int64_t k = 0; k < K; k++) a += (int64_t)row[k] * (int64_t)x[b * K + k];
+                acc[b * N + n] = a;
+            }
+        }
+        free(row);
+    }
+    return err ? ORC_NO_MEM : ORC_OK;
+}
