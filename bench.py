@@ -331,6 +331,27 @@ def time_gemm(S, torch, dev, flush, reps=5):
 HBM_SPEC_GBS = 8000.0  # the B200 HBM3e figure the workload description names (~8 TB/s)
 
 
+def probe_int8_tops(S, torch, iters=20000, reps=3):
+    """Measured int8 tensor-core rate: sherry_probe_mma_i8 (one CTA per SM
+    issuing back-to-back tcgen05 kind::i8 MMAs of the GEMM's 128 x 256 x 32
+    shape, operands in shared memory), best of `reps`, in TOPS (2 ops/MAC)."""
+    S.probe_mma_i8(100)
+    torch.cuda.synchronize()
+    best = None
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        ctas = S.probe_mma_i8(iters)
+        e1.record()
+        e1.synchronize()
+        t = e0.elapsed_time(e1) / 1e3
+        best = t if best is None else min(best, t)
+    macs = ctas * iters * 4 * 128 * 256 * 32
+    return {"tops": 2.0 * macs / best / 1e12, "ctas": ctas, "iters": iters, "ms": best * 1e3,
+            "how": "sherry_probe_mma_i8: %d CTAs x %d x 4 tcgen05.mma kind::i8 M=128 N=256 K=32, "
+                   "A and B in shared memory, back to back; best of %d" % (ctas, iters, reps)}
+
+
 def read_stream_gbs(torch, dev, reps=10):
     """Read-only HBM bandwidth: a 4 GiB fp32 sum, best of `reps`."""
     buf = torch.ones(1 << 30, dtype=torch.float32, device=dev)
@@ -521,13 +542,51 @@ def time_mlp_chain(layers, S, torch, dev, reps=200):
                     "+ GEMV), layers chained"}
 
 
-def cpu_baseline(layers, xs_host, seconds):
-    """The oracle, as it stands, on a bounded sample of the stack (host cores)."""
+def time_cmp_stack(layers, xs, S, torch, dev, sherry_us, reps=500):
+    """The decode stack in the two formats the pages compare Sherry against
+    (2 bits per weight aligned; three weights in five bits), holding the same
+    ternary matrices (transcoded on the GPU from the Sherry codes) and run by
+    the same decode kernel at B = 1: one grouped call per step, back to back
+    between one event pair.  The codes of each format exceed L2."""
+    n_w = sum(n * k for _, _, n, k, _, _ in layers)
+    sherry_bytes = sum(codes.numel() * 4 for _, _, _, _, codes, _ in layers)
+    out = {"sherry": {"bits_per_weight": 8.0 * sherry_bytes / n_w, "code_bytes": sherry_bytes,
+                      "us_per_step": sherry_us, "gweights_per_s": n_w / sherry_us / 1e3,
+                      "weight_gbs": sherry_bytes / sherry_us / 1e3}}
+    for name, fmt in (("i2_2bit", S.CMP_I2), ("t3_3in5", S.CMP_T3)):
+        items, code_bytes = [], 0
+        for _, _, n, k, codes, scales in layers:
+            cc = S.cmp_transcode(fmt, codes, n)
+            code_bytes += cc.numel() * 4
+            items.append((cc, scales, xs[k], torch.empty((1, n), dtype=torch.float32, device=dev), k))
+        step = S.GroupedCmpGemv(fmt, items, B=1)
+        for _ in range(5):
+            step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            step()
+        e1.record()
+        e1.synchronize()
+        t = e0.elapsed_time(e1) / 1e3 / reps
+        out[name] = {"bits_per_weight": 8.0 * code_bytes / n_w, "code_bytes": code_bytes,
+                     "us_per_step": t * 1e6, "gweights_per_s": n_w / t / 1e9,
+                     "weight_gbs": code_bytes / t / 1e9,
+                     "sherry_speedup": t * 1e6 / sherry_us}
+        del items, step
+        torch.cuda.empty_cache()
+    out["note"] = ("same ternary matrices in each format; one grouped decode GEMV per step "
+                   "(T3 adds one activation-expansion launch, Sherry one re-order launch); "
+                   "sherry_speedup = format's step time / Sherry's step time")
+    return out
+
+
+def _oracle_gemv_rate(host, xs_host, seconds):
+    """Oracle GEMVs of the stack in stack order, repeated for ~`seconds` of
+    oracle time: (GB/s of codes, GEMVs, passes started, weights, code bytes, s)."""
     import oracle
-    host = [(n, k, codes.cpu().numpy().view(np.uint32), scales.cpu().numpy())
-            for _, _, n, k, codes, scales in layers]
-    done_bytes, done_w, n_gemv, passes = 0, 0, 0, 0
-    t_compute = 0.0
+    done_bytes, done_w, n_gemv, passes, t_compute = 0, 0, 0, 0, 0.0
     while t_compute < seconds:
         for n, k, c, s in host:
             t0 = time.perf_counter()
@@ -539,11 +598,71 @@ def cpu_baseline(layers, xs_host, seconds):
             if t_compute >= seconds:
                 break
         passes += 1
-    return {"value": done_bytes / t_compute / 1e9, "unit": UNIT, "cores": oracle.num_threads(),
-            "kind": "oracle", "seconds": t_compute,
-            "sample": "%d GEMVs of the stack in stack order (%d passes started; %d weights, %d "
-                      "code bytes), %.1f s of oracle time" % (n_gemv, passes, done_w, done_bytes,
-                                                              t_compute)}
+    return done_bytes / t_compute / 1e9, n_gemv, passes, done_w, done_bytes, t_compute
+
+
+def cpu_baseline(layers, xs_host, seconds):
+    """The oracle, as it stands, on bounded samples of the workloads (host
+    cores).  The line's value is the decode stack on all cores; the legs add
+    the stack on one thread, the pack of one layer's latents and a row slice
+    of the gate/up-shaped prefill GEMM (each extrapolated to its full workload
+    and labelled so)."""
+    import oracle
+    host = [(n, k, codes.cpu().numpy().view(np.uint32), scales.cpu().numpy())
+            for _, _, n, k, codes, scales in layers]
+    all_cores = oracle.num_threads()
+    n_w = sum(n * k for n, k, _, _ in host)
+    code_bytes = sum(c.nbytes for _, _, c, _ in host)
+    v, n_gemv, passes, done_w, done_bytes, t_all = _oracle_gemv_rate(host, xs_host, 0.5 * seconds)
+    legs = {"gemv_stack_all_cores": {
+        "gbs": v, "cores": all_cores, "seconds": t_all,
+        "stack_ms_extrapolated": code_bytes / v / 1e6,
+        "sample": "%d GEMVs of the stack in stack order (%d passes started; %d weights)" % (
+            n_gemv, passes, done_w)}}
+    try:
+        oracle.set_num_threads(1)
+        v1, g1, _, w1, _, t1 = _oracle_gemv_rate(host, xs_host, 0.2 * seconds)
+        legs["gemv_stack_1_thread"] = {
+            "gbs": v1, "cores": 1, "seconds": t1, "stack_ms_extrapolated": code_bytes / v1 / 1e6,
+            "sample": "%d GEMVs of the stack in stack order (%d weights)" % (g1, w1)}
+    finally:
+        oracle.set_num_threads(all_cores)
+    # pack: the seven latent matrices of layer 0, best of 3
+    lat = [synth.latent_weights(n, k, seed=synth.layer_seed(0, pi))
+           for pi, (_, n, k) in enumerate(synth.LLAMA_1B_LAYERS)]
+    best = None
+    for _ in range(3):
+        t0 = time.perf_counter()
+        for w in lat:
+            oracle.pack(w)
+        t = time.perf_counter() - t0
+        best = t if best is None else min(best, t)
+    lw = sum(w.size for w in lat)
+    legs["pack_all_cores"] = {
+        "gweights_per_s": lw / best / 1e9, "gbs_read_write": (4 * lw + lw * 5 / 32) / best / 1e9,
+        "cores": all_cores, "seconds": best,
+        "stack_ms_extrapolated": 973078528 / (lw / best) * 1e3,
+        "sample": "oracle_pack of layer 0's 7 latent matrices (%d weights), best of 3; "
+                  "extrapolated to the stack's 973,078,528" % lw}
+    # prefill GEMM 2048 x 8192 x 2048: a slice of 64 output rows, best of 3
+    name, M, N, K = synth.PREFILL_GEMMS[0]
+    rows = 64
+    codes, scales = oracle.pack(synth.latent_weights(rows, K, seed=0))
+    x = synth.int8_clipped_normal((M, K), seed=1)
+    best = None
+    for _ in range(3):
+        t0 = time.perf_counter()
+        oracle.gemm(codes, scales, x, K)
+        t = time.perf_counter() - t0
+        best = t if best is None else min(best, t)
+    legs["gemm_all_cores"] = {
+        "tops": 2.0 * M * rows * K / best / 1e12, "cores": all_cores, "seconds": best,
+        "full_ms_extrapolated": best * (N / rows) * 1e3,
+        "sample": "oracle_gemm of %d of the %d output rows of the %s GEMM (M=%d, K=%d), best of 3; "
+                  "extrapolated to all rows" % (rows, N, name, M, K)}
+    return {"value": v, "unit": UNIT, "cores": all_cores, "kind": "oracle", "seconds": t_all,
+            "sample": legs["gemv_stack_all_cores"]["sample"] + ", %.1f s of oracle time" % t_all,
+            "legs": legs}
 
 
 def main():
@@ -728,6 +847,19 @@ def main():
         del latents
         torch.cuda.empty_cache()
         line["gemm"] = time_gemm(S, torch, dev, flush)
+        probe = probe_int8_tops(S, torch)
+        bf16x2 = 2.0 * peaks.get("bf16_tflops", 1590.0)
+        gemm_rows = {}
+        for name, g in line["gemm"].items():
+            gemm_rows[name] = {"achieved": g["tops"], "frac": g["tops"] / probe["tops"],
+                               "frac_of_2x_bf16": g["tops"] / bf16x2, "ms": g["ms"]}
+        top = max(line["gemm"].values(), key=lambda g: g["ms"])
+        line["gemm_roofline"] = {
+            "bound": "tensor", "kernel": "gemm_kernel (sherry_gemm)", "unit": "TOPS",
+            "achieved": top["tops"], "peak": probe["tops"], "frac": top["tops"] / probe["tops"],
+            "peak_source": "measured tcgen05 kind::i8 probe (this run)",
+            "peak_2x_measured_bf16": bf16x2, "shapes": gemm_rows, "probe": probe,
+            "ops_per_launch": "2*M*N*K (dense-equivalent; 3/4 of the products are nonzero)"}
         line["gemv_layers_rotated"] = time_layers(layers, xs, S, torch, dev)
         line["gemv_bf16_stack"] = time_bf16_stack(layers, S, torch, dev)
         line["mlp_chain"] = time_mlp_chain(layers, S, torch, dev)
@@ -738,6 +870,7 @@ def main():
             "hbm_spec_gbs": HBM_SPEC_GBS, "frac_of_spec": achieved / HBM_SPEC_GBS,
             "note": "read-only stream: torch.sum over 4 GiB of fp32 (a library kernel), best of 10"}
         line["gemv_3b_layer_rotated"] = time_3b_layer(S, torch, dev)
+        line["formats_compared"] = time_cmp_stack(layers, xs, S, torch, dev, ms_per_step * 1e3)
         if world == 1:
             line["cpu_baseline"] = cpu_baseline(layers, xs_host, args.cpu_seconds)
     err = S.device_error()

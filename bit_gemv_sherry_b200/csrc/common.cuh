@@ -27,6 +27,9 @@ inline bool valid_k(int64_t K) { return K >= SHERRY_TILE_K && K % SHERRY_TILE_K 
 // Number of SMs of the current device (cached per device).
 int sm_count();
 
+// Reads and clears the error word of the GEMV kernels (after a device sync).
+sherry_status gemv_device_error();
+
 // ---------------------------------------------------------------------------
 // Tile decode
 // ---------------------------------------------------------------------------

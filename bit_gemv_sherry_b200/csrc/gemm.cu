@@ -308,6 +308,54 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+// Tensor-core peak probe: one CTA per SM issues back-to-back
+// tcgen05.mma.cta_group::1.kind::i8 of the GEMM's shape (M = 128, N = 256,
+// K = 32, A and B from 128-byte-swizzled shared memory, int32 accumulator in
+// tensor memory) on zeroed operands, with no data movement and no barrier
+// between them: the int8 rate the GEMM's MMAs can reach on this device.
+constexpr int kProbeThreads = 128;
+constexpr size_t kProbeSmem = (size_t)kABytes + kBBytes + 1024;
+
+__global__ void __launch_bounds__(kProbeThreads, 1) mma_probe_kernel(int iters) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + ((1024 - (raw_addr & 1023)) & 1023);
+    __shared__ __align__(8) uint64_t done;
+    __shared__ uint32_t tmem_base;
+    for (int i = threadIdx.x; i < (kABytes + kBBytes) / 16; i += blockDim.x)
+        reinterpret_cast<uint4 *>(smem)[i] = make_uint4(0u, 0u, 0u, 0u);
+    fence_proxy_async_smem();  // the zeroed operands, to the tensor core's view
+    if (threadIdx.x == 0) {
+        mbar_init(&done, 1);
+        fence_mbar_init();
+    }
+    if (threadIdx.x < 32) {
+        tmem_alloc(&tmem_base, kBN);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (threadIdx.x == 0) {
+        const uint32_t a_addr = smem_u32(smem), b_addr = a_addr + kABytes;
+        for (int it = 0; it < iters; it++) {
+#pragma unroll
+            for (int k = 0; k < kBK / 32; k++)
+                umma_i8(tmem_base, smem_desc_sw128(a_addr + 32 * k), smem_desc_sw128(b_addr + 32 * k),
+                        kIdesc, (it | k) != 0);
+        }
+        umma_commit(&done);
+        volatile int no_abort = 0;
+        mbar_wait(&done, 0, &no_abort, &g_gemm_device_error, kDrainWaitLimit);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, kBN);
+    }
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     if (!fn) {
@@ -395,6 +443,32 @@ extern "C" sherry_status sherry_gemm_acc(const uint32_t *codes, const int8_t *x,
                                      reinterpret_cast<cudaStream_t>(stream));
 }
 
+extern "C" sherry_status sherry_probe_mma_i8(int iters, int *ctas, sherry_stream_t stream) {
+    using namespace sherry;
+    if (!ctas) return SHERRY_ERR_NULL;
+    if (iters < 1) return SHERRY_ERR_SHAPE;
+    static std::atomic<bool> attr_set[kMaxDevices];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        set_last_error("sherry_probe_mma_i8 (cudaGetDevice)", e);
+        return SHERRY_ERR_CUDA;
+    }
+    if (dev < 0 || dev >= kMaxDevices) return SHERRY_ERR_UNSUPPORTED;
+    if (!attr_set[dev].load(std::memory_order_acquire)) {
+        e = cudaFuncSetAttribute(mma_probe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kProbeSmem);
+        if (e != cudaSuccess) {
+            set_last_error("sherry_probe_mma_i8 (shared memory attribute)", e);
+            return SHERRY_ERR_CUDA;
+        }
+        attr_set[dev].store(true, std::memory_order_release);
+    }
+    *ctas = sm_count();
+    mma_probe_kernel<<<*ctas, kProbeThreads, kProbeSmem, reinterpret_cast<cudaStream_t>(stream)>>>(iters);
+    return launch_status("sherry_probe_mma_i8");
+}
+
 extern "C" sherry_status sherry_set_wait_limit(int64_t cycles) {
     if (cycles < 0) return SHERRY_ERR_SHAPE;
     sherry::g_wait_limit.store((long long)cycles, std::memory_order_relaxed);
@@ -421,5 +495,8 @@ extern "C" sherry_status sherry_device_error(void) {
             return SHERRY_ERR_CUDA;
         }
     }
+    // the GEMV kernels keep their own word; both are read and cleared
+    const sherry_status g = sherry::gemv_device_error();
+    if (v == 0) return g;
     return static_cast<sherry_status>(v);
 }

@@ -64,7 +64,9 @@ struct GemvDesc {
     int T;                // tiles per row (K / 128)
     int Tp;               // tile stride of xw (T rounded up to a whole chunk)
     int unit_begin16;     // register kernel: first 16-row unit in the group
-    int units;            // pipelined kernel: 32-row units
+    int units;            // pipelined kernels: items per K-part column (32-row units, or
+                          // groups of kDotUnits units for the dot kernel)
+    int units32;          // 32-row units of the GEMV (ceil(N / 32))
     int nchunk;           // pipelined kernel: 4-tile chunks per row
     int kparts;           // pipelined kernel: K-parts per unit
     int cpp;              // pipelined kernel: chunks per K-part
@@ -1013,97 +1015,244 @@ __global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
 
 // ---------------------------------------------------------------------------
 // Small-batch kernel (B <= 2): dot products on the ALU/FMA pipes, no MMA.
-//   * lane l owns row l of a 32-row unit, so a tile's five words are five
-//     conflict-free shared loads and each lane ends with its row's sum (no
-//     reduction across lanes);
-//   * work is split by chunk count.  Each CTA takes a run of whole items
-//     (unit, K-part) holding about 1/gridDim of the chunks, and its warps
-//     split the run into equal chunk ranges, so no warp ends the launch with a
-//     whole extra item to do.  An item cut by a warp boundary is summed by the
-//     warps holding its pieces: later pieces leave their row sums in shared
-//     memory, and after one CTA barrier the warp holding the item's first
-//     chunk adds them and finishes the item;
-//   * the unit's chunks (2560 contiguous bytes) and the chunk's re-ordered
-//     activations (128 words per batch row) stream through a private 2-stage
-//     cp.async ring per warp (one chunk in flight while one is consumed, 32
-//     warps per SM); the activation words are the same for all lanes
-//     (broadcast reads);
+//   * an item is (unit group, K-part), a unit group being kDotUnits
+//     consecutive 32-row units.  Lane l owns row l of each unit of the group,
+//     so a tile's five words of one unit are five conflict-free shared loads,
+//     each lane ends with its rows' sums (no reduction across lanes), and the
+//     activation words of a tile, read once per warp (broadcast loads), feed
+//     kDotUnits rows per lane;
+//   * work is split by chunk count, a chunk being 4 tiles of every unit of a
+//     group.  Each CTA takes a run of whole items holding about 1/gridDim of
+//     the chunks and its warps split the run into equal chunk ranges, so no
+//     warp ends the launch with a whole extra item to do.  An item cut by a
+//     warp boundary is summed by the warps holding its pieces: later pieces
+//     leave their row sums in shared memory, and after one CTA barrier the
+//     warp holding the item's first chunk adds them and finishes the item;
+//   * each warp streams its chunks through a private 2-stage ring in shared
+//     memory.  One lane fills a stage with bulk copies (cp.async.bulk): one
+//     per unit of the group (a unit's chunk is a contiguous 2,560 bytes of the
+//     code layout) and one per batch row for the chunk's activations, all
+//     completing on the stage's mbarrier.  The next chunk is requested before
+//     the current one is waited for, so a warp has two chunks in flight;
 //   * each decoded word (four ternary bytes) meets its activation word in one
-//     dp4a, so a batch row costs 32 dp4a per tile: for B <= 2 this is cheaper
-//     than an m16n8k32 MMA whose 8 columns would mostly be empty.
-// K-parts and the split-K completion are those of the pipelined kernel.
+//     dp4a: for B <= 2 this is cheaper than an m16n8k32 MMA whose 8 columns
+//     would mostly be empty.
+// K-parts and the split-K completion are those of the pipelined kernel, with
+// one counter per unit group.
 // ---------------------------------------------------------------------------
-constexpr int kDotRing = 2;  // stages per warp: one chunk in flight while one is consumed
-constexpr int kRawXMaxChunksPerSM = 64;  // calls up to this many chunks per SM re-order x in the dot kernel
-constexpr int kDotCodeWords = kChunkTiles * kTileWords;  // 640
-// 8 warps per CTA: B = 1, 4 CTAs (32 warps) per SM at 64 registers (50 KB of
-// shared memory per CTA); B = 2, 2 CTAs per SM.  (One CTA of 32 warps per SM
-// balances the CTAs' item runs better but was measured slower: a CTA slot frees
-// only when all 32 warps are done.)
-// XMODE 2 adds to each stage the chunk's raw bf16 activations (1 KB per batch
-// row), so that B = 1 fits 3 CTAs per SM.
-template <int NBX, int XMODE = 0>
-struct DotShape {
-    static constexpr int kWarps = 8;
-    static constexpr int kThreads = kWarps * 32;
-    static constexpr int kMinBlocks = NBX == 1 ? (XMODE == 2 ? 3 : 4) : 2;
-    static constexpr int kXWords = NBX * kChunkTiles * 32;           // int8, decode order
-    static constexpr int kBfWords = XMODE == 2 ? NBX * kChunkTiles * 64 : 0;
-    static constexpr int kStageWords = kDotCodeWords + kXWords + kBfWords;
-    static constexpr int kRingWords = kWarps * kDotRing * kStageWords;
-    // after the rings: per warp, the row sums of a later piece of a cut item
-    // [warp][NBX][32] and the first chunk of that item [warp]
-    static constexpr size_t kSmem = ((size_t)kRingWords + kWarps * (NBX * 32 + 1)) * 4;
+#ifndef SHERRY_DOT_UNITS
+#define SHERRY_DOT_UNITS 2
+#endif
+constexpr int kDotUnits = SHERRY_DOT_UNITS;  // 32-row units per item of the dot kernel
+constexpr int kDotRing = 2;                  // stages per warp
+constexpr int kRawXMaxChunksPerSM = 64;  // calls up to this many 32-row chunks per SM re-order x in the dot kernel
+constexpr int kDotCodeWords = kChunkTiles * kTileWords;  // 640 words: one unit's chunk
+// A stage's copies read ordinary device memory and always complete; the bound
+// only keeps a warp from spinning for good after a fault elsewhere.
+constexpr long long kStageWaitLimit = 4000000000LL;
+
+// First error recorded by a GEMV kernel (see sherry_device_error).
+__device__ unsigned int g_gemv_device_error = 0;
+
+// Weight formats the small-batch kernel streams: Sherry, and the two ternary
+// packings the pages compare it against (arXiv 2601.07892, abstract; Figure 2
+// caption): 2 bits per weight, aligned ("I2"), and three weights in five bits
+// ("T3").  Per format: 32-bit words per tile of one row, weights per tile,
+// tiles per chunk.  Every format's chunk carries 32 activation words per tile
+// and batch row.
+enum DotFormat { kFmtSherry = 0, kFmtI2 = 1, kFmtT3 = 2 };
+template <int FMT>
+struct FmtTraits {
+    static constexpr int kTileWords = FMT == kFmtI2 ? 8 : 5;
+    static constexpr int kTileK = FMT == kFmtT3 ? 96 : 128;
+    static constexpr int kChunkTiles = FMT == kFmtT3 ? 2 : 4;
+    static constexpr int kUnitChunkWords = kChunkTiles * kTileWords * kUnitRows;
 };
 
-// Finishes an item: lane = row of the unit, v = the item's row sums.  A K-part
-// of a split row adds into the K-part sums; the last K-part to finish scales,
-// stores and clears them.
+// 8 warps per CTA.  B = 1 with two units per item: 2 CTAs (16 warps) per SM,
+// 90 KB of shared memory per CTA, up to 128 registers per thread.
+// XMODE 2 adds to each stage the chunk's raw bf16 activations (1 KB per batch row).
+template <int NBX, int XMODE = 0, int FMT = kFmtSherry>
+struct DotShape {
+    static constexpr int NU = kDotUnits;
+    static constexpr int kWarps = 8;
+    static constexpr int kThreads = kWarps * 32;
+    static constexpr int kChunkTilesF = FmtTraits<FMT>::kChunkTiles;
+    static constexpr int kCodeWords = NU * FmtTraits<FMT>::kUnitChunkWords;
+    static constexpr int kXWords = NBX * kChunkTilesF * 32;                     // int8, decode order
+    static constexpr int kBfWords = XMODE == 2 ? NBX * kChunkTiles * 64 : 0;    // raw bf16
+    static constexpr int kStageWords = kCodeWords + kXWords + kBfWords;
+    static constexpr int kRingWords = kWarps * kDotRing * kStageWords;
+    static constexpr int kCutWords = NU * NBX * 32;
+    // after the rings: the stages' mbarriers [warp][stage], then per warp the
+    // row sums of a later piece of a cut item [NU][NBX][32] and that item's
+    // first chunk
+    static constexpr size_t kBarOffset = (size_t)kRingWords * 4;
+    static constexpr size_t kCutOffset = kBarOffset + (size_t)kWarps * kDotRing * 8;
+    static constexpr size_t kSmem = kCutOffset + ((size_t)kWarps * kCutWords + kWarps) * 4;
+    // CTAs per SM that fit the 227 KB of shared memory (1 KB reserved per CTA)
+    static constexpr int kFit = (int)((227u * 1024u) / (kSmem + 1024u));
+    static constexpr int kMinBlocks = kFit < 1 ? 1 : (kFit > 4 ? 4 : kFit);
+    static_assert(kStageWords % 4 == 0, "stages must stay 16-byte aligned for bulk copies");
+};
+
+// Finishes an item: lane = row of each unit of the group, v = the item's row
+// sums.  A K-part of a split row adds into the K-part sums; the last K-part to
+// finish scales, stores and clears them.
 // sx: the activation scales, when the kernel quantized the activations itself.
 template <int NBX, bool ACC_OUT, bool SX_REG>
-__device__ __forceinline__ void dot_finish(const GemvDesc &D, int unit, int B, int lane,
-                                           int (&v)[NBX], const float (&sx)[NBX]) {
+__device__ __forceinline__ void dot_finish(const GemvDesc &D, int group, int B, int lane,
+                                           int (&v)[kDotUnits][NBX], const float (&sx)[NBX]) {
+    constexpr int NU = kDotUnits;
     const int N = D.N;
-    const int row = unit * kUnitRows + lane;
-    const bool rv = row < N;
     bool finish = true;
     if (D.kparts > 1) {
-        if (rv) {
 #pragma unroll
-            for (int b = 0; b < NBX; b++)
-                if (b < B) atomicAdd(D.part_acc + (size_t)b * N + row, v[b]);
+        for (int u = 0; u < NU; u++) {
+            const int row = (group * NU + u) * kUnitRows + lane;
+            if (row < N) {
+#pragma unroll
+                for (int b = 0; b < NBX; b++)
+                    if (b < B) atomicAdd(D.part_acc + (size_t)b * N + row, v[u][b]);
+            }
         }
         __threadfence();
         __syncwarp();
         uint32_t done = 0;
-        if (lane == 0) done = atomicAdd(D.part_cnt + unit, 1u);
+        if (lane == 0) done = atomicAdd(D.part_cnt + group, 1u);
         finish = __shfl_sync(0xFFFFFFFFu, done, 0) == (uint32_t)(D.kparts - 1);
         if (finish) {
             __threadfence();
-            if (rv) {
 #pragma unroll
-                for (int b = 0; b < NBX; b++) {
-                    if (b < B) {
-                        int32_t *pa = D.part_acc + (size_t)b * N + row;
-                        v[b] = __ldcg(pa);
-                        *pa = 0;
+            for (int u = 0; u < NU; u++) {
+                const int row = (group * NU + u) * kUnitRows + lane;
+                if (row < N) {
+#pragma unroll
+                    for (int b = 0; b < NBX; b++) {
+                        if (b < B) {
+                            int32_t *pa = D.part_acc + (size_t)b * N + row;
+                            v[u][b] = __ldcg(pa);
+                            *pa = 0;
+                        }
                     }
                 }
             }
-            if (lane == 0) D.part_cnt[unit] = 0u;
+            if (lane == 0) D.part_cnt[group] = 0u;
         }
     }
-    if (finish && rv) {
-        if (ACC_OUT) {
+    if (!finish) return;
 #pragma unroll
-            for (int b = 0; b < NBX; b++)
-                if (b < B) static_cast<int32_t *>(D.out)[(size_t)b * N + row] = v[b];
-        } else {
+    for (int u = 0; u < NU; u++) {
+        const int row = (group * NU + u) * kUnitRows + lane;
+        if (row >= N) continue;
 #pragma unroll
-            for (int b = 0; b < NBX; b++) {
-                if (b < B) {
-                    const float sc = SX_REG ? __fmul_rn(__ldg(D.scales + row), sx[b]) : out_scale(D, row, b);
-                    static_cast<float *>(D.out)[(size_t)b * N + row] = sc * (float)v[b];
+        for (int b = 0; b < NBX; b++) {
+            if (b >= B) continue;
+            if (ACC_OUT) {
+                static_cast<int32_t *>(D.out)[(size_t)b * N + row] = v[u][b];
+            } else {
+                const float sc = SX_REG ? __fmul_rn(__ldg(D.scales + row), sx[b]) : out_scale(D, row, b);
+                static_cast<float *>(D.out)[(size_t)b * N + row] = sc * (float)v[u][b];
+            }
+        }
+    }
+}
+
+// Bounded wait of all lanes on a stage's mbarrier phase; false (on every lane)
+// if it did not complete within kStageWaitLimit cycles on some lane.
+__device__ __forceinline__ bool stage_wait(uint64_t *bar, uint32_t parity) {
+    bool ok = mbar_try_wait(bar, parity);
+    if (!ok) {
+        const long long t0 = clock64();
+        while (!(ok = mbar_try_wait(bar, parity)))
+            if (clock64() - t0 > kStageWaitLimit) break;
+    }
+    return __all_sync(0xFFFFFFFFu, ok);
+}
+
+// One chunk of the 2-bit format: 4 tiles x 8 words per unit.  Word q of a
+// tile holds weights 16 q + n (low two bits of nibble n) and 16 q + 8 + n
+// (high two bits); code 1 is +1, 3 is -1, 0 and 2 are 0.  Masking the low (or,
+// after a shift, the high) two bits of every nibble gives a PRMT selector
+// whose halves decode four consecutive weights each, so the activations stay
+// in natural order: x word 4 q + r of the tile meets decoded word r.
+template <int NBX, int NU>
+__device__ __forceinline__ void dot_chunk_i2(const uint32_t *st, int code_words, int lane,
+                                             const Consts &C, int (&acc)[kDotUnits][NBX][2]) {
+    // table: byte c = weight of code c (0, +1, 0, -1)
+    const uint32_t tab = 0xFF000100u;
+#pragma unroll
+    for (int tt = 0; tt < 4; tt++) {
+        const uint4 *xs = reinterpret_cast<const uint4 *>(st + code_words + tt * 32);
+#pragma unroll
+        for (int q = 0; q < 8; q++) {
+            uint4 xv[NBX];
+#pragma unroll
+            for (int b = 0; b < NBX; b++) xv[b] = xs[b * 32 + q];
+#pragma unroll
+            for (int u = 0; u < NU; u++) {
+                const uint32_t w = st[u * FmtTraits<kFmtI2>::kUnitChunkWords + tt * 256 + q * 32 + lane];
+                const uint32_t s0 = w & C.m33, s1 = (w >> 2) & C.m33;
+                const int d0 = (int)prmt(tab, 0u, s0), d1 = (int)prmt(tab, 0u, hi_half(C, s0));
+                const int d2 = (int)prmt(tab, 0u, s1), d3 = (int)prmt(tab, 0u, hi_half(C, s1));
+#pragma unroll
+                for (int b = 0; b < NBX; b++) {
+                    acc[u][b][0] = __dp4a(d0, (int)xv[b].x, acc[u][b][0]);
+                    acc[u][b][1] = __dp4a(d1, (int)xv[b].y, acc[u][b][1]);
+                    acc[u][b][0] = __dp4a(d2, (int)xv[b].z, acc[u][b][0]);
+                    acc[u][b][1] = __dp4a(d3, (int)xv[b].w, acc[u][b][1]);
+                }
+            }
+        }
+    }
+}
+
+// Field j (bits 5 j .. 5 j + 4) of a T3 tile's 160-bit string, times 4 (its
+// table entry's byte offset).  j is a constant after unrolling, so only one
+// branch remains: one shift (or funnel shift, for the fields that straddle
+// two words) and one mask.
+__device__ __forceinline__ uint32_t t3_field_x4(const uint32_t (&w)[5], int j) {
+    const int b = 5 * j, wi = b >> 5, sh = b & 31;
+    if (sh >= 2 && sh <= 27) return (w[wi] >> (sh - 2)) & 0x7Cu;
+    if (sh < 2) return (w[wi] << (2 - sh)) & 0x7Cu;
+    return __funnelshift_r(w[wi], w[wi + 1], sh - 2) & 0x7Cu;
+}
+
+// One chunk of the three-in-five format: 2 tiles x 5 words per unit; triple
+// j's code indexes a 32-entry table of packed ternary bytes in shared memory
+// (lane = row, so a lookup of 32 rows is one conflict-free access), and the
+// entry meets activation word j = (x[3j], x[3j+1], x[3j+2], 0) in one dp4a.
+template <int NBX, int NU>
+__device__ __forceinline__ void dot_chunk_t3(const uint32_t *st, int code_words, int lane,
+                                             const uint32_t *lut, int (&acc)[kDotUnits][NBX][2]) {
+    const uint8_t *lut_b = reinterpret_cast<const uint8_t *>(lut);
+#pragma unroll
+    for (int tt = 0; tt < 2; tt++) {
+        uint32_t w[NU][5];
+#pragma unroll
+        for (int u = 0; u < NU; u++)
+#pragma unroll
+            for (int p = 0; p < 5; p++)
+                w[u][p] = st[u * FmtTraits<kFmtT3>::kUnitChunkWords + tt * 160 + p * 32 + lane];
+        const uint4 *xs = reinterpret_cast<const uint4 *>(st + code_words + tt * 32);
+#pragma unroll
+        for (int q = 0; q < 8; q++) {
+            uint4 xv[NBX];
+#pragma unroll
+            for (int b = 0; b < NBX; b++) xv[b] = xs[b * 16 + q];  // 64 words per batch row
+#pragma unroll
+            for (int u = 0; u < NU; u++) {
+                int e[4];
+                e[0] = *reinterpret_cast<const int *>(lut_b + t3_field_x4(w[u], 4 * q + 0));
+                e[1] = *reinterpret_cast<const int *>(lut_b + t3_field_x4(w[u], 4 * q + 1));
+                e[2] = *reinterpret_cast<const int *>(lut_b + t3_field_x4(w[u], 4 * q + 2));
+                e[3] = *reinterpret_cast<const int *>(lut_b + t3_field_x4(w[u], 4 * q + 3));
+#pragma unroll
+                for (int b = 0; b < NBX; b++) {
+                    acc[u][b][0] = __dp4a(e[0], (int)xv[b].x, acc[u][b][0]);
+                    acc[u][b][1] = __dp4a(e[1], (int)xv[b].y, acc[u][b][1]);
+                    acc[u][b][0] = __dp4a(e[2], (int)xv[b].z, acc[u][b][0]);
+                    acc[u][b][1] = __dp4a(e[3], (int)xv[b].w, acc[u][b][1]);
                 }
             }
         }
@@ -1120,24 +1269,47 @@ __device__ __forceinline__ void dot_finish(const GemvDesc &D, int unit, int B, i
 //      tiles by the rule of the bf16 front-end.
 // Modes 1 and 2 need no re-order launch.  They are used for calls of few
 // chunks, where that launch and its wait cost more than the per-chunk work.
-template <int NBX, bool ACC_OUT, int XMODE>
-__global__ void __launch_bounds__(DotShape<NBX, XMODE>::kThreads, DotShape<NBX, XMODE>::kMinBlocks)
+// FMT: the weight format (Sherry, or a comparison format with XMODE 0).
+template <int NBX, bool ACC_OUT, int XMODE, int FMT = kFmtSherry>
+__global__ void __launch_bounds__(DotShape<NBX, XMODE, FMT>::kThreads,
+                                  DotShape<NBX, XMODE, FMT>::kMinBlocks)
     gemv_dot_kernel(const __grid_constant__ GemvParams P) {
     constexpr bool XRAW = XMODE == 1;
     constexpr bool XBF = XMODE == 2;
-    using Shape = DotShape<NBX, XMODE>;
-    pdl_allow_dependents();
+    static_assert(FMT == kFmtSherry || XMODE == 0, "comparison formats read prepared activations");
+    using Shape = DotShape<NBX, XMODE, FMT>;
+    using F = FmtTraits<FMT>;
+    constexpr int CT = F::kChunkTiles;
+    constexpr int UCW = F::kUnitChunkWords;
+    constexpr int NU = Shape::NU;
     constexpr int SW = Shape::kStageWords;
-    extern __shared__ __align__(16) uint32_t dot_smem[];
-    int *cut_sum = reinterpret_cast<int *>(dot_smem + Shape::kRingWords);
     constexpr int kWarps = Shape::kWarps;
-    int *cut_start = cut_sum + kWarps * NBX * 32;
+    pdl_allow_dependents();
+    extern __shared__ __align__(128) uint32_t dot_smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    uint8_t *smem_bytes = reinterpret_cast<uint8_t *>(dot_smem);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem_bytes + Shape::kBarOffset) + warp * kDotRing;
+    int *cut_sum = reinterpret_cast<int *>(smem_bytes + Shape::kCutOffset);
+    int *cut_start = cut_sum + kWarps * Shape::kCutWords;
     // chunk range [b0, b1) of this warp; threads 0 and 1 find the CTA's bounds
     __shared__ int cta_bound[2];
     if (threadIdx.x < 2) {
         const long long tc = P.total_chunks, nb = gridDim.x;
         cta_bound[threadIdx.x] = item_start_at_or_before(P, (int)((blockIdx.x + threadIdx.x) * tc / nb));
+    }
+    if (lane == 0) {
+#pragma unroll
+        for (int s = 0; s < kDotRing; s++) mbar_init(&bars[s], 1);
+        fence_mbar_init();
+    }
+    // T3: entry c of the table = the triple of code c as three ternary bytes
+    // (byte 3 zero), codes past 26 zero
+    __shared__ uint32_t t3_lut[32];
+    if (FMT == kFmtT3 && threadIdx.x < 32) {
+        const int c = (int)threadIdx.x;
+        t3_lut[c] = c > 26 ? 0u
+                           : ((uint32_t)(c % 3 - 1) & 0xFFu) | (((uint32_t)((c / 3) % 3 - 1) & 0xFFu) << 8) |
+                                 (((uint32_t)(c / 9 - 1) & 0xFFu) << 16);
     }
     __syncthreads();
     const int cta_lo = cta_bound[0], cta_hi = cta_bound[1];
@@ -1157,60 +1329,63 @@ __global__ void __launch_bounds__(DotShape<NBX, XMODE>::kThreads, DotShape<NBX, 
     ItemCursor cur = {0, 0, 0};
     if (b0 < b1) cur = cursor_at_chunk(P, b0, start);
 
-    // ---- producer side: the issue cursor runs kDotRing-1 stages ahead ----
-    // lane l copies 16-byte pieces l + 32 j (j = 0..4) of the chunk's codes and
-    // piece l of each batch row's 128 activation words.  Until pdl_wait() only
-    // codes are read, and only when P.prefetch_codes says the kernel before is
-    // this call's re-order launch: the activation words and the K-part sums
-    // belong to that kernel.
+    // ---- producer side: runs one chunk ahead of the consumer ----
+    // Lane 0 arms the stage's mbarrier with the byte count and issues the bulk
+    // copies; every lane advances the cursor.  Until pdl_wait() only codes are
+    // read, and only when P.prefetch_codes says the kernel before is this
+    // call's re-order launch: the activation words and the K-part sums belong
+    // to that kernel.
     ItemCursor icur = cur;
-    int istart = start, ic = 0, ic_end = 0, iTp = 0;
-    const uint32_t *isrc = nullptr, *ixw = nullptr;
-    const int8_t *ixr = nullptr;
+    int istart = start, ic = 0, ic_end = 0;
     auto set_issue_item = [&]() {
         const GemvDesc &D = P.d[icur.id];
-        isrc = D.codes + (size_t)icur.unit * D.T * kTileWords + 4 * lane;
-        if (XRAW) {
-            ixr = D.x + 16 * lane;
-            iTp = D.T * SHERRY_TILE_K;  // row stride of x in bytes
-        } else if (XBF) {
-            ixr = reinterpret_cast<const int8_t *>(D.xbf) + 16 * lane;
-            iTp = D.T * SHERRY_TILE_K * 2;  // row stride of x in bytes
-        } else {
-            ixw = reinterpret_cast<const uint32_t *>(D.xw) + 4 * lane;
-            iTp = D.Tp;
-        }
         const int first = icur.kp * D.cpp;
         ic = first + max(b0 - istart, 0);
         ic_end = first + min(b1 - istart, min(D.cpp, D.nchunk - first));
     };
     if (istart < b1) set_issue_item();
-    auto copy_codes = [&](int slot) {
-        const uint32_t *src = isrc + (size_t)ic * kChunkTiles * kTileWords;
-        const uint32_t dst = ring_addr + (uint32_t)slot * SW * 4 + 16u * lane;
+    // activation bytes per chunk and batch row: 32 words per tile (raw bf16: twice that)
+    constexpr uint32_t kXBytes = XBF ? CT * 128 * 2 : CT * 128;
+    auto issue_codes = [&](int slot) {
+        const GemvDesc &D = P.d[icur.id];
+        if (lane == 0) {
+            const int unit0 = icur.unit * NU;
+            const int present = min(NU, D.units32 - unit0);
+            const uint32_t dst = ring_addr + (uint32_t)slot * SW * 4;
+            fence_proxy_async_smem();  // the warp's reads of the stage's previous chunk come first
+            mbar_arrive_expect_tx(&bars[slot], (uint32_t)present * UCW * 4 + (uint32_t)B * kXBytes);
+            const uint32_t *src =
+                D.codes + ((size_t)unit0 * D.T + (size_t)ic * CT) * (F::kTileWords * kUnitRows);
 #pragma unroll
-        for (int j = 0; j < 5; j++) cp_async16(dst + 512u * j, src + 128 * j, 16u);
+            for (int u = 0; u < NU; u++)
+                if (u < present)
+                    bulk_load(dst + (uint32_t)u * UCW * 4,
+                              src + (size_t)u * D.T * (F::kTileWords * kUnitRows), UCW * 4, &bars[slot]);
+        }
     };
-    auto copy_x_and_advance = [&](int slot) {
-        const uint32_t dst = ring_addr + (uint32_t)slot * SW * 4 + 16u * lane;
+    auto issue_x_and_advance = [&](int slot) {
+        const GemvDesc &D = P.d[icur.id];
+        if (lane == 0) {
+            const uint32_t dst = ring_addr + (uint32_t)slot * SW * 4 + (uint32_t)Shape::kCodeWords * 4;
 #pragma unroll
-        for (int b = 0; b < NBX; b++) {
-            if (b < B) {
-                if (XBF) {  // 1 KB of bf16 per batch row: pieces l and l + 32
-                    const int8_t *src = ixr + (size_t)b * iTp + (size_t)kChunkTiles * SHERRY_TILE_K * 2 * ic;
-                    const uint32_t d0 = dst + 4u * (kDotCodeWords + Shape::kXWords) + 1024u * b;
-                    cp_async16(d0, src, 16u);
-                    cp_async16(d0 + 512u, src + 512, 16u);
-                } else if (XRAW)
-                    cp_async16(dst + 4u * kDotCodeWords + 512u * b,
-                               ixr + (size_t)b * iTp + (size_t)kChunkTiles * SHERRY_TILE_K * ic, 16u);
-                else
-                    cp_async16(dst + 4u * kDotCodeWords + 512u * b,
-                               ixw + ((size_t)b * iTp + (size_t)kChunkTiles * ic) * 32, 16u);
+            for (int b = 0; b < NBX; b++) {
+                if (b < B) {
+                    if (XBF)
+                        bulk_load(dst + (uint32_t)Shape::kXWords * 4 + (uint32_t)b * kXBytes,
+                                  D.xbf + ((size_t)b * D.T + (size_t)ic * CT) * SHERRY_TILE_K,
+                                  kXBytes, &bars[slot]);
+                    else if (XRAW)
+                        bulk_load(dst + (uint32_t)b * kXBytes,
+                                  D.x + ((size_t)b * D.T + (size_t)ic * CT) * SHERRY_TILE_K,
+                                  kXBytes, &bars[slot]);
+                    else  // 32 words (8 uint4) per tile
+                        bulk_load(dst + (uint32_t)b * kXBytes,
+                                  D.xw + ((size_t)b * D.Tp + (size_t)ic * CT) * 8, kXBytes,
+                                  &bars[slot]);
+                }
             }
         }
         if (++ic == ic_end) {
-            const GemvDesc &D = P.d[icur.id];
             istart += min(D.cpp, D.nchunk - icur.kp * D.cpp);
             if (istart < b1) {
                 cursor_next(P, icur);
@@ -1218,24 +1393,28 @@ __global__ void __launch_bounds__(DotShape<NBX, XMODE>::kThreads, DotShape<NBX, 
             }
         }
     };
+    uint32_t inflight = 0;  // stages whose copies were issued and not yet waited for
     auto issue = [&](int slot) {
         if (istart < b1) {
-            copy_codes(slot);
-            copy_x_and_advance(slot);
+            issue_codes(slot);
+            issue_x_and_advance(slot);
+            inflight |= 1u << slot;
         }
-        cp_async_commit();
     };
-    static_assert(kDotRing == 2, "the prologue fills one stage");
     const bool first_copy = istart < b1;
-    if (first_copy && P.prefetch_codes) copy_codes(0);
+    if (first_copy && P.prefetch_codes) issue_codes(0);
     pdl_wait();
-    if (first_copy && !P.prefetch_codes) copy_codes(0);
-    if (first_copy) copy_x_and_advance(0);
-    cp_async_commit();
+    if (first_copy && !P.prefetch_codes) issue_codes(0);
+    if (first_copy) {
+        issue_x_and_advance(0);
+        inflight = 1u;
+    }
 
     // ---- consumer side ----
     int slot = 0;
-    int v[NBX];
+    uint32_t phase = 0;  // bit s: parity of stage s's next phase
+    bool failed = false;
+    int v[NU][NBX];
     bool own_cut = false;  // the last item continues in later warps of the CTA
     // XMODE 2: per-token quantization of the activations the warp works on
     const uint16_t *sx_of = nullptr;  // the activations (and row length) sx belongs to
@@ -1262,17 +1441,22 @@ __global__ void __launch_bounds__(DotShape<NBX, XMODE>::kThreads, DotShape<NBX, 
         const int nreal = min(D.cpp, D.nchunk - first);
         const int c_begin = first + max(b0 - start, 0);
         const int c_end = first + min(b1 - start, nreal);
-        int acc[NBX][2];
+        int acc[NU][NBX][2];
 #pragma unroll
-        for (int b = 0; b < NBX; b++) acc[b][0] = acc[b][1] = 0;
+        for (int u = 0; u < NU; u++)
+#pragma unroll
+            for (int b = 0; b < NBX; b++) acc[u][b][0] = acc[u][b][1] = 0;
         for (int c = c_begin; c < c_end; c++) {
-            cp_async_wait<kDotRing - 2>();
-            __syncwarp();  // every lane is done with the previous stage: refill it
-            issue(slot == 0 ? kDotRing - 1 : slot - 1);
+            issue(slot ^ 1);  // the next chunk into the stage the previous chunk used
+            if (!stage_wait(&bars[slot], (phase >> slot) & 1u)) {
+                failed = true;
+                break;
+            }
+            inflight &= ~(1u << slot);
+            phase ^= 1u << slot;
             uint32_t *st = ring + slot * SW;
-            slot = (slot + 1 == kDotRing) ? 0 : slot + 1;
             if (XRAW) {  // raw words of the chunk's tiles -> the decode order, in place
-                uint32_t *xr = st + kDotCodeWords;
+                uint32_t *xr = st + Shape::kCodeWords;
                 uint32_t w[NBX][kChunkTiles];
 #pragma unroll
                 for (int b = 0; b < NBX; b++)
@@ -1288,8 +1472,8 @@ __global__ void __launch_bounds__(DotShape<NBX, XMODE>::kThreads, DotShape<NBX, 
                 __syncwarp();
             }
             if (XBF) {  // bf16 of the chunk's tiles -> quantized words in the decode order
-                uint32_t *xq = st + kDotCodeWords;
-                const uint2 *xb = reinterpret_cast<const uint2 *>(st + kDotCodeWords + Shape::kXWords);
+                uint32_t *xq = st + Shape::kCodeWords;
+                const uint2 *xb = reinterpret_cast<const uint2 *>(st + Shape::kCodeWords + Shape::kXWords);
 #pragma unroll
                 for (int b = 0; b < NBX; b++)
 #pragma unroll
@@ -1299,13 +1483,21 @@ __global__ void __launch_bounds__(DotShape<NBX, XMODE>::kThreads, DotShape<NBX, 
                                 reorder_word(quant_word(xb[(b * kChunkTiles + tt) * 32 + lane], sx_inv[b]), lane);
                 __syncwarp();
             }
+            if (FMT == kFmtI2) {
+                dot_chunk_i2<NBX, NU>(st, Shape::kCodeWords, lane, C, acc);
+            } else if (FMT == kFmtT3) {
+                dot_chunk_t3<NBX, NU>(st, Shape::kCodeWords, lane, t3_lut, acc);
+            } else {
 #pragma unroll
             for (int tt = 0; tt < kChunkTiles; tt++) {
-                const uint32_t *cw = st + tt * kTileWords + lane;
-                TileDecoder6 d;
-                d.load(C, cw[0], cw[32], cw[64], cw[96], cw[128]);
+                TileDecoder6 d[NU];
+#pragma unroll
+                for (int u = 0; u < NU; u++) {
+                    const uint32_t *cw = st + u * kDotCodeWords + tt * kTileWords + lane;
+                    d[u].load(C, cw[0], cw[32], cw[64], cw[96], cw[128]);
+                }
                 // activation words of tile tt: batch row b at b * 128, word q at q
-                const uint4 *xs = reinterpret_cast<const uint4 *>(st + kDotCodeWords + tt * 32);
+                const uint4 *xs = reinterpret_cast<const uint4 *>(st + Shape::kCodeWords + tt * 32);
 #pragma unroll
                 for (int i = 0; i < 4; i++) {
                     uint4 xa[NBX], xb[NBX];  // words 8i..8i+3 (beta 0, 1) and 8i+4..8i+7 (beta 2, 3)
@@ -1316,26 +1508,37 @@ __global__ void __launch_bounds__(DotShape<NBX, XMODE>::kThreads, DotShape<NBX, 
                     }
 #pragma unroll
                     for (int beta = 0; beta < 4; beta++) {
-                        const uint32_t sl = d.sel(C, i, beta);
-                        const int lo = (int)prmt(C.tlo[i], C.thi[i], sl);
-                        const int hi = (int)prmt(C.tlo[i], C.thi[i], hi_half(C, sl));
 #pragma unroll
-                        for (int b = 0; b < NBX; b++) {
-                            const uint4 &xv = beta < 2 ? xa[b] : xb[b];
-                            int &a = acc[b][beta & 1];
-                            a = __dp4a(lo, (int)pick(xv, 2 * (beta & 1)), a);
-                            a = __dp4a(hi, (int)pick(xv, 2 * (beta & 1) + 1), a);
+                        for (int u = 0; u < NU; u++) {
+                            const uint32_t sl = d[u].sel(C, i, beta);
+                            const int lo = (int)prmt(C.tlo[i], C.thi[i], sl);
+                            const int hi = (int)prmt(C.tlo[i], C.thi[i], hi_half(C, sl));
+#pragma unroll
+                            for (int b = 0; b < NBX; b++) {
+                                const uint4 &xv = beta < 2 ? xa[b] : xb[b];
+                                int &a = acc[u][b][beta & 1];
+                                a = __dp4a(lo, (int)pick(xv, 2 * (beta & 1)), a);
+                                a = __dp4a(hi, (int)pick(xv, 2 * (beta & 1) + 1), a);
+                            }
                         }
                     }
                 }
             }
+            }
+            __syncwarp();  // every lane is done with this stage before it is refilled
+            slot ^= 1;
         }
+        if (failed) break;
 #pragma unroll
-        for (int b = 0; b < NBX; b++) v[b] = acc[b][0] + acc[b][1];
+        for (int u = 0; u < NU; u++)
+#pragma unroll
+            for (int b = 0; b < NBX; b++) v[u][b] = acc[u][b][0] + acc[u][b][1];
         if (start < b0) {
             // a later piece of an item cut at b0: hand the sums to its first warp
 #pragma unroll
-            for (int b = 0; b < NBX; b++) cut_sum[(warp * NBX + b) * 32 + lane] = v[b];
+            for (int u = 0; u < NU; u++)
+#pragma unroll
+                for (int b = 0; b < NBX; b++) cut_sum[((warp * NU + u) * NBX + b) * 32 + lane] = v[u][b];
             if (lane == 0) cut_start[warp] = start;
         } else if (b1 - start < nreal) {
             own_cut = true;  // first piece of an item cut at b1: finished after the barrier
@@ -1345,7 +1548,15 @@ __global__ void __launch_bounds__(DotShape<NBX, XMODE>::kThreads, DotShape<NBX, 
         start += nreal;
         if (start < b1) cursor_next(P, cur);
     }
-    cp_async_wait<0>();
+    if (failed) {
+        // a stage never completed: record it, let the copies still in flight
+        // land (bounded) and leave the CTA's item summing alone
+        if (lane == 0) atomicCAS(&g_gemv_device_error, 0u, (unsigned int)SHERRY_ERR_TIMEOUT);
+#pragma unroll
+        for (int s = 0; s < kDotRing; s++)
+            if (inflight & (1u << s)) stage_wait(&bars[s], (phase >> s) & 1u);
+        own_cut = false;
+    }
     __syncthreads();  // the later pieces' sums are in shared memory
     if (own_cut) {
         const GemvDesc &D = P.d[cur.id];
@@ -1355,7 +1566,9 @@ __global__ void __launch_bounds__(DotShape<NBX, XMODE>::kThreads, DotShape<NBX, 
             if (cs == -2) continue;
             if (cs != mine) break;
 #pragma unroll
-            for (int b = 0; b < NBX; b++) v[b] += cut_sum[(w * NBX + b) * 32 + lane];
+            for (int u = 0; u < NU; u++)
+#pragma unroll
+                for (int b = 0; b < NBX; b++) v[u][b] += cut_sum[((w * NU + u) * NBX + b) * 32 + lane];
         }
         dot_finish<NBX, ACC_OUT, XBF>(P.d[cur.id], cur.unit, B, lane, v, sx);
     }
@@ -1432,8 +1645,8 @@ template <int NBX, bool ACC, int XMODE>
 void launch_dot(const GemvParams &gp, cudaStream_t stream) {
     static int cache[64] = {0};
     const size_t smem = DotShape<NBX, XMODE>::kSmem;
-    // one chunk per warp at most: a small GEMV spreads over as many SMs as it
-    // has chunks (items cut between warps are summed in shared memory)
+    // one chunk (of a unit group) per warp at most: a small GEMV spreads over as
+    // many SMs as it has chunks (items cut between warps are summed in shared memory)
     constexpr int threads = DotShape<NBX, XMODE>::kThreads, warps = DotShape<NBX, XMODE>::kWarps;
     const int want = (gp.total_chunks + warps - 1) / warps;
     const int grid = grid_for(gemv_dot_kernel<NBX, ACC, XMODE>, threads, smem, want, cache);
@@ -1534,14 +1747,18 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
             gp.thi[i] = hi[i];
         }
     }
+    // items of the dot kernel (B <= 2) hold kDotUnits 32-row units, the MMA kernel's one
+    const bool dot = pipelined && B <= 2;
+    const int nu = dot ? kDotUnits : 1;
     int64_t off = 0;
-    int wb = 0, ub16 = 0, cb = 0;
+    int wb = 0, ub16 = 0, cb = 0, cb32 = 0;
     for (int i = 0; i < count; i++) {
         const GemvCall &c = calls[i];
         uint32_t *region = static_cast<uint32_t *>(workspace) + off;
         const int Tp = (int)padded_tiles(c.K);
         const int xw_words = (int)round_words((int64_t)B * Tp * 32);
-        const int units = (int)((c.N + kUnitRows - 1) / kUnitRows);
+        const int units32 = (int)((c.N + kUnitRows - 1) / kUnitRows);
+        const int units = (units32 + nu - 1) / nu;
         const int nchunk = Tp / kChunkTiles;
         const int kparts = (int)kparts_for(c.K);
         const int cpp = (nchunk + kparts - 1) / kparts;
@@ -1588,6 +1805,7 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
         D.Tp = Tp;
         D.unit_begin16 = ub16;
         D.units = units;
+        D.units32 = units32;
         D.nchunk = nchunk;
         D.kparts = kparts;
         D.cpp = cpp;
@@ -1596,6 +1814,7 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
         wb += X.xunits + (X.zero_words + 31) / 32;
         ub16 += (int)((c.N + 15) / 16);
         cb += units * nchunk;
+        cb32 += units32 * nchunk;
     }
     xp.total_units = wb;
     gp.total_units16 = ub16;
@@ -1604,7 +1823,7 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
     // chunk's activations itself (at most ~2 chunks per warp of a full GPU, so
     // x is re-ordered at most twice per chunk position; rows are not split, so
     // there are no K-part sums to clear).
-    bool raw_x = phase == kBoth && pipelined && B <= 2 && cb <= kRawXMaxChunksPerSM * sm_count();
+    bool raw_x = phase == kBoth && dot && cb32 <= kRawXMaxChunksPerSM * sm_count();
     bool raw_bf = raw_x && !acc_out;
     for (int i = 0; i < count && raw_x; i++)
         raw_x = calls[i].x && !calls[i].xbf && !calls[i].xf && aligned(calls[i].x, 16) &&
@@ -1626,7 +1845,7 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
     if (!(phase & kRun)) return SHERRY_OK;
     // B <= 2: dp4a kernel; B >= 3: the MMA kernel (its 8 batch columns cost the
     // same as one, while dp4a work grows with B) -- measured on the decode stack
-    if (pipelined && B <= 2) {
+    if (dot) {
         if (raw_bf) {  // bf16 calls have no accumulator form
             if (B == 1) launch_dot<1, false, 2>(gp, stream); else launch_dot<2, false, 2>(gp, stream);
         } else if (raw_x) {
@@ -1720,6 +1939,214 @@ sherry_status quantize_f32(const float *x, const float *u, int64_t B, int64_t K,
     return launch_status(u ? "sherry_quantize_swiglu" : "sherry_quantize_f32");
 }
 
+// ---------------------------------------------------------------------------
+// Comparison formats: the 2-bit aligned and the three-in-five ternary
+// packings the pages set Sherry against, streamed by the same small-batch
+// kernel (gemv_dot_kernel with FMT = kFmtI2 / kFmtT3) for a like-for-like
+// measurement.  Their codes are made from Sherry codes (the same ternary
+// matrix) by a transcode kernel.
+// ---------------------------------------------------------------------------
+int64_t cmp_tiles(int fmt, int64_t K) {
+    if (!valid_k(K)) return 0;
+    if (fmt == kFmtI2) return K / SHERRY_TILE_K;
+    if (fmt == kFmtT3) return 2 * ((K + 191) / 192);
+    return 0;
+}
+int64_t cmp_tile_words(int fmt) { return fmt == kFmtI2 ? 8 : 5; }
+
+// Ternary weight k of row n from Sherry codes (T tiles per row).
+__device__ __forceinline__ int sherry_weight(const uint32_t *codes, int n, int k, int T) {
+    const int t = k >> 7, j = (k >> 2) & 31, i = k & 3;
+    const uint32_t *tile = codes + ((size_t)(n >> 5) * T + t) * kTileWords + (n & 31);
+    const int p = (int)((__ldg(tile + 32 * (j & 1)) >> (2 * (j >> 1))) & 3u);
+    if (i == p) return 0;
+    const int r = i - (i > p ? 1 : 0);
+    return ((__ldg(tile + 32 * (2 + r)) >> j) & 1u) ? -1 : 1;
+}
+
+// One thread per (row, comparison tile): decode the tile's weights from the
+// Sherry codes and write its words (rows past N: zero weights).
+__global__ void __launch_bounds__(256) transcode_kernel(const uint32_t *__restrict__ codes,
+                                                        uint32_t *__restrict__ out, int N, int K,
+                                                        int T, int Tc, int rows, int fmt) {
+    const long long id = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (id >= (long long)rows * Tc) return;
+    const int n = (int)(id % rows), t = (int)(id / rows);
+    const bool real = n < N;
+    if (fmt == kFmtI2) {
+        uint32_t *dst = out + ((size_t)(n >> 5) * Tc + t) * 256 + (n & 31);
+        for (int q = 0; q < 8; q++) {
+            uint32_t w = 0;
+            for (int m = 0; m < 16; m++) {
+                const int v = real ? sherry_weight(codes, n, 128 * t + 16 * q + m, T) : 0;
+                const uint32_t c = v == 0 ? 0u : (v > 0 ? 1u : 3u);
+                w |= c << (4 * (m & 7) + 2 * (m >> 3));
+            }
+            dst[32 * q] = w;
+        }
+    } else {
+        uint32_t w[5] = {0u, 0u, 0u, 0u, 0u};
+        for (int j = 0; j < 32; j++) {
+            int d[3];
+            for (int e = 0; e < 3; e++) {
+                const int k = 96 * t + 3 * j + e;
+                d[e] = (real && k < K) ? sherry_weight(codes, n, k, T) : 0;
+            }
+            const uint32_t c = (uint32_t)((d[0] + 1) + 3 * (d[1] + 1) + 9 * (d[2] + 1));
+            const int b = 5 * j;
+            w[b >> 5] |= c << (b & 31);
+            if ((b & 31) > 27) w[(b >> 5) + 1] |= c >> (32 - (b & 31));
+        }
+        uint32_t *dst = out + ((size_t)(n >> 5) * Tc + t) * 160 + (n & 31);
+        for (int p = 0; p < 5; p++) dst[32 * p] = w[p];
+    }
+}
+
+// T3 activations: word j of tile t = (x[96t+3j], x[96t+3j+1], x[96t+3j+2], 0)
+// (zero past K), [B][Tc][32] per GEMV.  One thread per word.
+struct CmpXDesc {
+    const int8_t *x;
+    uint32_t *xw;
+    int K, Tc, word_begin, words;
+};
+struct CmpXParams {
+    int count;
+    int total_words;
+    CmpXDesc d[SHERRY_MAX_GROUP];
+};
+
+__global__ void __launch_bounds__(256) t3_expand_kernel(const __grid_constant__ CmpXParams P) {
+    pdl_allow_dependents();
+    pdl_wait();  // x may come from the kernel before; the last GEMV may still read xw
+    for (int g = blockIdx.x * blockDim.x + threadIdx.x; g < P.total_words; g += gridDim.x * blockDim.x) {
+        int lo = 0, hi = P.count - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (P.d[mid].word_begin <= g) lo = mid; else hi = mid - 1;
+        }
+        const CmpXDesc &D = P.d[lo];
+        const int w = g - D.word_begin;
+        const int b = w / (D.Tc * 32), r = w - b * D.Tc * 32;  // r = tile * 32 + j
+        const int k0 = 3 * (r & 31) + 96 * (r >> 5);
+        const int8_t *xr = D.x + (size_t)b * D.K;
+        uint32_t v = 0;
+        for (int e = 0; e < 3; e++)
+            if (k0 + e < D.K) v |= (uint32_t)(uint8_t)xr[k0 + e] << (8 * e);
+        D.xw[w] = v;
+    }
+}
+
+int64_t cmp_ws_words(int fmt, int64_t K, int B) {
+    return fmt == kFmtT3 ? round_words((int64_t)B * cmp_tiles(fmt, K) * 32) : 0;
+}
+
+template <int NBX, bool ACC, int FMT>
+void launch_dot_fmt(const GemvParams &gp, cudaStream_t stream) {
+    static int cache[64] = {0};
+    using Shape = DotShape<NBX, 0, FMT>;
+    const size_t smem = Shape::kSmem;
+    const int want = (gp.total_chunks + Shape::kWarps - 1) / Shape::kWarps;
+    const int grid = grid_for(gemv_dot_kernel<NBX, ACC, 0, FMT>, Shape::kThreads, smem, want, cache);
+    launch_pdl(gemv_dot_kernel<NBX, ACC, 0, FMT>, grid, Shape::kThreads, smem, stream, gp);
+}
+
+sherry_status cmp_launch(int fmt, const GemvCall *calls, int count, int B, bool acc_out,
+                         void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    if (fmt != kFmtI2 && fmt != kFmtT3) return SHERRY_ERR_UNSUPPORTED;
+    if (count < 1) return SHERRY_ERR_SHAPE;
+    if (count > SHERRY_MAX_GROUP) return SHERRY_ERR_UNSUPPORTED;
+    if (B < 1) return SHERRY_ERR_SHAPE;
+    if (B > 2) return SHERRY_ERR_UNSUPPORTED;  // the comparison runs the decode kernel (B <= 2)
+    int64_t words = 0, chunks = 0;
+    for (int i = 0; i < count; i++) {
+        const GemvCall &c = calls[i];
+        if (!c.codes || !c.x || !c.out || (!acc_out && !c.scales)) return SHERRY_ERR_NULL;
+        if (c.N < 1 || !valid_k(c.K)) return SHERRY_ERR_SHAPE;
+        if (fmt == kFmtI2 && c.K % (4 * SHERRY_TILE_K) != 0) return SHERRY_ERR_SHAPE;
+        if (!aligned(c.codes, 16) || !aligned(c.out, 4) || (c.scales && !aligned(c.scales, 4)) ||
+            !aligned(c.x, fmt == kFmtI2 ? 16 : 1))
+            return SHERRY_ERR_ALIGN;
+        if (c.N > (int64_t)1 << 28) return SHERRY_ERR_UNSUPPORTED;
+        words += cmp_ws_words(fmt, c.K, B);
+        const int64_t groups = ((c.N + kUnitRows - 1) / kUnitRows + kDotUnits - 1) / kDotUnits;
+        chunks += groups * (cmp_tiles(fmt, c.K) / (fmt == kFmtT3 ? 2 : 4));
+    }
+    if (words > 0 && (!workspace || !aligned(workspace, 256))) return workspace ? SHERRY_ERR_ALIGN
+                                                                                : SHERRY_ERR_WORKSPACE;
+    if (workspace_bytes < (size_t)words * 4) return SHERRY_ERR_WORKSPACE;
+    if (words > 0x7FFFFFFF || chunks > 0x7FFFFFFF) return SHERRY_ERR_UNSUPPORTED;
+
+    static thread_local GemvParams gp;
+    static thread_local CmpXParams xp;
+    std::memset(&gp, 0, sizeof(gp));
+    std::memset(&xp, 0, sizeof(xp));
+    gp.count = xp.count = count;
+    gp.B = B;
+    gp.m33 = 0x33333333u;
+    gp.f16one = 0x3C003C00u;
+    gp.f16negz = 0x80008000u;
+    int64_t off = 0;
+    int cb = 0, xb = 0;
+    for (int i = 0; i < count; i++) {
+        const GemvCall &c = calls[i];
+        const int Tc = (int)cmp_tiles(fmt, c.K);
+        const int ct = fmt == kFmtT3 ? 2 : 4;
+        GemvDesc &D = gp.d[i];
+        D.codes = c.codes;
+        D.scales = c.scales;
+        D.out = c.out;
+        D.N = (int)c.N;
+        D.T = Tc;
+        D.units32 = (int)((c.N + kUnitRows - 1) / kUnitRows);
+        D.units = (D.units32 + kDotUnits - 1) / kDotUnits;
+        D.nchunk = Tc / ct;
+        D.kparts = 1;
+        D.cpp = D.nchunk;
+        D.chunk_begin = cb;
+        cb += D.units * D.nchunk;
+        if (fmt == kFmtI2) {  // natural-order activations, read in place
+            D.xw = reinterpret_cast<const uint4 *>(c.x);
+            D.Tp = Tc;
+        } else {
+            uint32_t *region = static_cast<uint32_t *>(workspace) + off;
+            D.xw = reinterpret_cast<const uint4 *>(region);
+            D.Tp = Tc;
+            CmpXDesc &X = xp.d[i];
+            X.x = c.x;
+            X.xw = region;
+            X.K = (int)c.K;
+            X.Tc = Tc;
+            X.word_begin = xb;
+            X.words = B * Tc * 32;
+            xb += X.words;
+            off += cmp_ws_words(fmt, c.K, B);
+        }
+    }
+    gp.total_chunks = cb;
+    xp.total_words = xb;
+    if (fmt == kFmtT3) {
+        const int blocks = std::max(1, std::min((xb + 255) / 256, sm_count() * 8));
+        launch_pdl(t3_expand_kernel, blocks, 256, 0, stream, xp);
+        const sherry_status st = launch_status("sherry_cmp_gemv (activation expansion)");
+        if (st != SHERRY_OK) return st;
+        gp.prefetch_codes = 1;  // follows this call's own expansion launch
+    }
+    if (fmt == kFmtI2) {
+        if (B == 1) {
+            if (acc_out) launch_dot_fmt<1, true, kFmtI2>(gp, stream); else launch_dot_fmt<1, false, kFmtI2>(gp, stream);
+        } else {
+            if (acc_out) launch_dot_fmt<2, true, kFmtI2>(gp, stream); else launch_dot_fmt<2, false, kFmtI2>(gp, stream);
+        }
+    } else {
+        if (B == 1) {
+            if (acc_out) launch_dot_fmt<1, true, kFmtT3>(gp, stream); else launch_dot_fmt<1, false, kFmtT3>(gp, stream);
+        } else {
+            if (acc_out) launch_dot_fmt<2, true, kFmtT3>(gp, stream); else launch_dot_fmt<2, false, kFmtT3>(gp, stream);
+        }
+    }
+    return launch_status("sherry_cmp_gemv");
+}
+
 // Per-token quantization of bf16 activations, natural order (one warp per row).
 __global__ void __launch_bounds__(256) quantize_act_kernel(const uint16_t *__restrict__ x, int B, int K,
                                                            int8_t *__restrict__ q, float *__restrict__ s) {
@@ -1736,6 +2163,27 @@ __global__ void __launch_bounds__(256) quantize_act_kernel(const uint16_t *__res
 }
 
 }  // namespace
+
+// Reads and clears the GEMV kernels' error word (SHERRY_OK if none); the
+// caller has synchronised the device.
+sherry_status gemv_device_error() {
+    unsigned int v = 0;
+    cudaError_t err = cudaMemcpyFromSymbol(&v, g_gemv_device_error, sizeof(v));
+    if (err != cudaSuccess) {
+        set_last_error("sherry_device_error (read)", err);
+        return SHERRY_ERR_CUDA;
+    }
+    if (v != 0) {
+        const unsigned int zero = 0;
+        err = cudaMemcpyToSymbol(g_gemv_device_error, &zero, sizeof(zero));
+        if (err != cudaSuccess) {
+            set_last_error("sherry_device_error (clear)", err);
+            return SHERRY_ERR_CUDA;
+        }
+    }
+    return static_cast<sherry_status>(v);
+}
+
 }  // namespace sherry
 
 extern "C" size_t sherry_gemv_workspace_bytes(int64_t N, int64_t K, int B) {
@@ -1855,6 +2303,59 @@ extern "C" sherry_status sherry_quantize_swiglu(const float *g, const float *u, 
                                                 int8_t *q, float *s, sherry_stream_t stream) {
     if (!u) return SHERRY_ERR_NULL;
     return sherry::quantize_f32(g, u, B, K, q, s, reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" size_t sherry_cmp_packed_bytes(int fmt, int64_t N, int64_t K) {
+    const int64_t T = sherry::cmp_tiles(fmt, K);
+    if (T == 0 || N < 1) return 0;
+    return (size_t)((N + SHERRY_ROW_GROUP - 1) / SHERRY_ROW_GROUP) * SHERRY_ROW_GROUP * (size_t)T *
+           (size_t)sherry::cmp_tile_words(fmt) * 4;
+}
+
+extern "C" size_t sherry_cmp_workspace_bytes(int fmt, int64_t N, int64_t K, int B) {
+    if (N < 1 || B < 1 || sherry::cmp_tiles(fmt, K) == 0) return 0;
+    return (size_t)sherry::cmp_ws_words(fmt, K, B) * 4;
+}
+
+extern "C" sherry_status sherry_cmp_transcode(int fmt, const uint32_t *codes, int64_t N, int64_t K,
+                                              uint32_t *out, sherry_stream_t stream) {
+    using namespace sherry;
+    if (fmt != kFmtI2 && fmt != kFmtT3) return SHERRY_ERR_UNSUPPORTED;
+    if (!codes || !out) return SHERRY_ERR_NULL;
+    if (N < 1 || !valid_k(K)) return SHERRY_ERR_SHAPE;
+    if (N > (int64_t)1 << 28) return SHERRY_ERR_UNSUPPORTED;
+    if (!aligned(codes, 4) || !aligned(out, 4)) return SHERRY_ERR_ALIGN;
+    const int64_t rows = (N + kUnitRows - 1) / kUnitRows * kUnitRows;
+    const int64_t Tc = cmp_tiles(fmt, K);
+    const int64_t threads = rows * Tc;
+    if (threads > 0x7FFFFFFFLL * 256) return SHERRY_ERR_UNSUPPORTED;
+    transcode_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        codes, out, (int)N, (int)K, (int)(K / SHERRY_TILE_K), (int)Tc, (int)rows, fmt);
+    return launch_status("sherry_cmp_transcode");
+}
+
+extern "C" sherry_status sherry_cmp_gemv_grouped(int fmt, const sherry_gemv_desc *descs, int count,
+                                                 int B, void *workspace, size_t workspace_bytes,
+                                                 sherry_stream_t stream) {
+    using namespace sherry;
+    if (!descs) return SHERRY_ERR_NULL;
+    if (count < 1) return SHERRY_ERR_SHAPE;
+    if (count > SHERRY_MAX_GROUP) return SHERRY_ERR_UNSUPPORTED;
+    GemvCall calls[SHERRY_MAX_GROUP];
+    for (int i = 0; i < count; i++)
+        calls[i] = GemvCall{descs[i].codes, descs[i].scales, descs[i].x, descs[i].y, descs[i].N,
+                            descs[i].K, nullptr};
+    return cmp_launch(fmt, calls, count, B, false, workspace, workspace_bytes,
+                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" sherry_status sherry_cmp_gemv_acc(int fmt, const uint32_t *codes, const int8_t *x,
+                                             int32_t *acc, int64_t N, int64_t K, int B,
+                                             void *workspace, size_t workspace_bytes,
+                                             sherry_stream_t stream) {
+    const sherry::GemvCall c{codes, nullptr, x, acc, N, K, nullptr};
+    return sherry::cmp_launch(fmt, &c, 1, B, true, workspace, workspace_bytes,
+                              reinterpret_cast<cudaStream_t>(stream));
 }
 
 // ---------------------------------------------------------------------------

@@ -89,6 +89,12 @@ def lib():
         "sherry_gemv_run": ([p, i32, i32, p, sz, p], i32),
         "sherry_gemm": ([p, p, p, p, i64, i64, i64, p], i32),
         "sherry_gemm_acc": ([p, p, p, i64, i64, i64, p], i32),
+        "sherry_cmp_packed_bytes": ([i32, i64, i64], sz),
+        "sherry_cmp_workspace_bytes": ([i32, i64, i64, i32], sz),
+        "sherry_cmp_transcode": ([i32, p, i64, i64, p, p], i32),
+        "sherry_cmp_gemv_grouped": ([i32, p, i32, i32, p, sz, p], i32),
+        "sherry_cmp_gemv_acc": ([i32, p, p, p, i64, i64, i32, p, sz, p], i32),
+        "sherry_probe_mma_i8": ([i32, p, p], i32),
         "sherry_device_error": ([], i32),
         "sherry_set_wait_limit": ([i64], i32),
         "sherry_status_string": ([i32], ctypes.c_char_p),
@@ -539,3 +545,79 @@ def set_wait_limit(cycles):
     """Limit (SM clock cycles) of the kernels' bounded barrier waits, for
     kernels launched afterwards by this process; 0 restores the default."""
     _check(lib().sherry_set_wait_limit(int(cycles)), "sherry_set_wait_limit")
+
+
+# ----------------------------------------------------------------------------- comparison formats
+CMP_I2 = 1  # 2 bits per weight, aligned
+CMP_T3 = 2  # three weights in five bits
+_CMP_TILE_WORDS = {CMP_I2: 8, CMP_T3: 5}
+
+
+def cmp_tiles(fmt, K):
+    if fmt == CMP_I2:
+        return K // TILE_K
+    return 2 * ((K + 191) // 192)
+
+
+def cmp_transcode(fmt, codes, N):
+    """Sherry codes of an N x K matrix -> the same matrix in comparison format
+    fmt, int32 [ceil(N/32), tiles, words, 32] holding the uint32 words."""
+    N, K = _codes_shape(codes, N)
+    shape = ((N + 31) // 32, cmp_tiles(fmt, K), _CMP_TILE_WORDS[fmt], 32)
+    out = torch.empty(shape, dtype=torch.int32, device=codes.device)
+    assert out.numel() * 4 == lib().sherry_cmp_packed_bytes(fmt, N, K)
+    _check(lib().sherry_cmp_transcode(fmt, _ptr(codes), N, K, _ptr(out), _stream(codes)),
+           "sherry_cmp_transcode")
+    return out
+
+
+def cmp_gemv_acc(fmt, codes, x, N, K, acc=None):
+    """Exact int32 acc[B, N] of a comparison-format matrix against int8 x [B, K]."""
+    _need(x, torch.int8, "x")
+    x2 = x.view(1, -1) if x.dim() == 1 else x
+    B = x2.shape[0]
+    if acc is None:
+        acc = torch.empty((B, N), dtype=torch.int32, device=x.device)
+    nb = lib().sherry_cmp_workspace_bytes(fmt, N, K, B)
+    ws = workspace(max(nb, 256), x.device)
+    _check(lib().sherry_cmp_gemv_acc(fmt, _ptr(codes), _ptr(x2), _ptr(acc), N, K, B, _ptr(ws),
+                                     ws.numel(), _stream(x)), "sherry_cmp_gemv_acc")
+    return acc
+
+
+class GroupedCmpGemv:
+    """Pre-marshalled grouped GEMV on comparison-format matrices: items are
+    (codes in format fmt, scales, x int8 [B, K], y [B, N], K)."""
+
+    def __init__(self, fmt, items, B):
+        n = len(items)
+        self.descs = (GemvDesc * n)()
+        total = 0
+        for i, (codes, scales, x, y, K) in enumerate(items):
+            _need(scales, torch.float32, "scales")
+            _need(x, torch.int8, "x")
+            _need(y, torch.float32, "y")
+            N = scales.numel()
+            self.descs[i] = GemvDesc(codes.data_ptr(), scales.data_ptr(), x.data_ptr(),
+                                     y.data_ptr(), N, K)
+            total += lib().sherry_cmp_workspace_bytes(fmt, N, K, B)
+        self.items = items
+        dev = items[0][2].device
+        self.ws = torch.empty(max(total, 256), dtype=torch.uint8, device=dev)
+        self.args = (fmt, ctypes.cast(self.descs, ctypes.c_void_p), n, B, _ptr(self.ws),
+                     self.ws.numel())
+        self.device = dev
+
+    def __call__(self, stream=None):
+        s = ctypes.c_void_p(stream if stream is not None
+                            else torch.cuda.current_stream(self.device).cuda_stream)
+        _check(lib().sherry_cmp_gemv_grouped(*self.args, s), "sherry_cmp_gemv_grouped")
+
+
+def probe_mma_i8(iters, stream=None):
+    """Launch the tensor-core int8 probe; returns the number of CTAs (one per
+    SM).  Each CTA runs iters * 4 MMAs of 128 x 256 x 32."""
+    ctas = ctypes.c_int(0)
+    s = ctypes.c_void_p(stream if stream is not None else torch.cuda.current_stream().cuda_stream)
+    _check(lib().sherry_probe_mma_i8(int(iters), ctypes.byref(ctas), s), "sherry_probe_mma_i8")
+    return ctas.value

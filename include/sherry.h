@@ -361,6 +361,65 @@ sherry_status sherry_gemv_run(const sherry_gemv_desc *descs, int count, int B,
                               sherry_stream_t stream);
 
 /*
+ * Comparison formats.  The pages set Sherry's 1.25 bits per weight against two
+ * ternary packings (arXiv 2601.07892, abstract; Figure 2 caption): a 2-bit
+ * aligned one and a 1.67-bit one of three weights in five bits.  These calls
+ * hold the same ternary matrix in those formats and run the same decode GEMV
+ * machinery on them, so that the three can be measured side by side.  Layouts
+ * (the pages print none; these are the library's readings):
+ *   SHERRY_CMP_I2  2 bits per weight: code 0 -> 0, 1 -> +1, 3 -> -1 (2 -> 0);
+ *                  a tile is 128 weights of a row in 8 words; word q holds
+ *                  weights 16 q + n at bits [4 n, 4 n + 1] and 16 q + 8 + n at
+ *                  bits [4 n + 2, 4 n + 3], n = 0..7; rows in groups of 32:
+ *                  codes[((n / 32) * T + t) * 256 + 32 q + n % 32], T = K / 128.
+ *   SHERRY_CMP_T3  three weights in five bits: triple (w0, w1, w2) has code
+ *                  (w0 + 1) + 3 (w1 + 1) + 9 (w2 + 1); a tile is 32 triples = 96
+ *                  weights in 5 words, triple j at bits [5 j, 5 j + 4] of the
+ *                  160-bit little-endian string of the words; a row is padded
+ *                  with zero weights to T3 = 2 * ceil(K / 192) tiles; rows in
+ *                  groups of 32: codes[((n / 32) * T3 + t) * 160 + 32 p + n % 32].
+ * The GEMV takes B <= 2 rows of int8 activations (row-major [B][K]) and writes
+ * y = s (.) (W . x^T) as sherry_gemv does; it is not tuned beyond the decode
+ * kernel it shares with Sherry.
+ */
+#define SHERRY_CMP_I2 1
+#define SHERRY_CMP_T3 2
+
+/* Bytes of codes of an N x K matrix in a comparison format (0 if invalid). */
+size_t sherry_cmp_packed_bytes(int fmt, int64_t N, int64_t K);
+
+/* Workspace of a comparison GEMV (the sum over a grouped call's GEMVs):
+ * T3 expands each activation triple to a 32-bit word; I2 reads x in place (0). */
+size_t sherry_cmp_workspace_bytes(int fmt, int64_t N, int64_t K, int B);
+
+/*
+ * sherry_cmp_transcode -- the matrix of Sherry `codes` (N x K, layout above)
+ * written in comparison format `fmt` to `out` (sherry_cmp_packed_bytes bytes;
+ * padding rows and padding weights are zero weights).  Device pointers,
+ * 4-byte aligned.
+ * Errors: NULL, SHAPE, ALIGN, UNSUPPORTED (unknown fmt), CUDA.
+ */
+sherry_status sherry_cmp_transcode(int fmt, const uint32_t *codes, int64_t N, int64_t K,
+                                   uint32_t *out, sherry_stream_t stream);
+
+/*
+ * sherry_cmp_gemv_grouped -- sherry_gemv_grouped on matrices in comparison
+ * format `fmt` (descs[i].codes in that format), B <= 2.  Codes 16-byte
+ * aligned; I2 also needs K a multiple of 512 and x 16-byte aligned.
+ *   workspace: at least the sum of sherry_cmp_workspace_bytes over the group,
+ *   256-byte aligned (may be NULL when that sum is 0).
+ * Errors: NULL, SHAPE, ALIGN, UNSUPPORTED (fmt, B > 2, count), WORKSPACE, CUDA.
+ */
+sherry_status sherry_cmp_gemv_grouped(int fmt, const sherry_gemv_desc *descs, int count, int B,
+                                      void *workspace, size_t workspace_bytes,
+                                      sherry_stream_t stream);
+
+/* One comparison GEMV writing the exact int32 accumulators acc[B][N]. */
+sherry_status sherry_cmp_gemv_acc(int fmt, const uint32_t *codes, const int8_t *x, int32_t *acc,
+                                  int64_t N, int64_t K, int B, void *workspace,
+                                  size_t workspace_bytes, sherry_stream_t stream);
+
+/*
  * sherry_gemm -- prefill GEMM, Y = X . W^T scaled per output column,
  *   Y[m][n] = s[n] * sum_k X[m][k] * W[n][k]   (the same product for M tokens).
  * The pages define no GEMM: this is the product the abstract serves
@@ -403,6 +462,18 @@ sherry_status sherry_device_error(void);
  * Errors: SHAPE if cycles < 0.
  */
 sherry_status sherry_set_wait_limit(int64_t cycles);
+
+/*
+ * sherry_probe_mma_i8 -- measurement aid, not part of the product: one CTA
+ * per SM (their number written to *ctas) issues `iters` x 4 back-to-back
+ * tcgen05.mma.cta_group::1.kind::i8 of the GEMM's shape (M = 128 weight rows,
+ * N = 256 tokens, K = 32, operands in 128-byte-swizzled shared memory) on
+ * zeroed operands.  Timing the launch gives the int8 tensor-core rate the
+ * GEMM's MMAs can reach on this device: *ctas * iters * 4 * 128 * 256 * 32
+ * multiply-accumulates (twice that in ops).  Asynchronous on `stream`.
+ * Errors: NULL, SHAPE (iters < 1), CUDA.
+ */
+sherry_status sherry_probe_mma_i8(int iters, int *ctas, sherry_stream_t stream);
 
 /* Text of a status code (static string). */
 const char *sherry_status_string(sherry_status status);

@@ -196,3 +196,22 @@ def test_wait_limit_setting_is_checked_and_restorable():
     assert L.sherry_set_wait_limit(-1) == 2
     assert L.sherry_set_wait_limit(1000) == 0
     assert L.sherry_set_wait_limit(0) == 0
+
+
+def test_cmp_argument_checks_on_the_host():
+    L = S.lib()
+    assert L.sherry_cmp_packed_bytes(1, 32, 1024) == 32 * 1024 * 2 // 8
+    assert L.sherry_cmp_packed_bytes(2, 32, 1920) == 32 * 1920 * 5 // 3 // 8
+    assert L.sherry_cmp_packed_bytes(3, 32, 1024) == 0 and L.sherry_cmp_packed_bytes(1, 32, 100) == 0
+    assert L.sherry_cmp_workspace_bytes(1, 64, 2048, 1) == 0          # I2 reads x in place
+    assert L.sherry_cmp_workspace_bytes(2, 64, 2048, 2) == 4 * 64 * ((2 * 22 * 32 + 63) // 64)
+    acc = FAKE
+    assert L.sherry_cmp_gemv_acc(3, FAKE, FAKE, acc, 32, 512, 1, FAKE_WS, 1 << 20, None) == 4
+    assert L.sherry_cmp_gemv_acc(1, FAKE, FAKE, acc, 32, 512, 3, FAKE_WS, 1 << 20, None) == 4
+    assert L.sherry_cmp_gemv_acc(1, FAKE, FAKE, acc, 32, 384, 1, FAKE_WS, 1 << 20, None) == 2
+    assert L.sherry_cmp_gemv_acc(1, None, FAKE, acc, 32, 512, 1, FAKE_WS, 1 << 20, None) == 1
+    assert L.sherry_cmp_gemv_acc(1, ctypes.c_void_p(0x100004), FAKE, acc, 32, 512, 1, FAKE_WS,
+                                 1 << 20, None) == 3
+    assert L.sherry_cmp_gemv_acc(2, FAKE, FAKE, acc, 32, 512, 1, FAKE_WS, 16, None) == 7
+    assert L.sherry_cmp_transcode(5, FAKE, 32, 512, FAKE, None) == 4
+    assert L.sherry_cmp_transcode(1, FAKE, 32, 500, FAKE, None) == 2

@@ -136,15 +136,21 @@ def test_gemv_extreme_and_zero_activations():
 
 @pytest.mark.parametrize("B", [1, 4, 16])
 def test_gemv_full_size_3b_layers(B):
+    """All seven LLaMA-3.2-3B-shaped projections at B = 1, 4, 16: every output
+    of every projection against the oracle, one call each and the seven as one
+    grouped call."""
+    x = {k: synth.int8_uniform((B, k), seed={1: 1, 4: 2, 16: 3}[B]) for k in (3072, 8192)}
+    items, refs = [], []
     for li, (name, N, K) in enumerate(synth.LLAMA_3B_LAYERS):
-        if name in ("k", "v", "o"):
-            continue  # same kernels and shapes as q and the K=3072 layers
         codes, scales = oracle.pack(synth.latent_weights(N, K, seed=synth.layer_seed(0, li)))
-        x = synth.int8_uniform((B, K), seed={1: 1, 4: 2, 16: 3}[B])
-        y = S.gemv(dev_codes(codes), dev(scales), dev(x)).cpu().numpy()
-        rows = np.random.default_rng(li).choice(N, size=min(N, 96), replace=False)
-        sub = rows_subset(codes, rows)
-        assert_y_matches(y[:, rows], oracle.gemv(sub, scales[rows], x, K))
+        ref = oracle.gemv(codes, scales, x[K], K)
+        tc, ts = dev_codes(codes), dev(scales)
+        assert_y_matches(S.gemv(tc, ts, dev(x[K])).cpu().numpy(), ref)
+        items.append((tc, ts, dev(x[K]), torch.empty((B, N), dtype=torch.float32, device="cuda")))
+        refs.append(ref)
+    S.gemv_grouped(items, B=B)
+    for (_, _, _, y), ref in zip(items, refs):
+        assert_y_matches(y.cpu().numpy(), ref)
 
 
 def test_gemv_grouped_1b_stack_layer():
@@ -192,9 +198,9 @@ def test_gemv_grouped_cut_items(B, shapes):
 
 def test_gemv_full_size_decode_stack_as_benched():
     """The benchmark's launch: the 16-layer 1B stack, 112 GEMVs at B = 1, one
-    re-order launch and one GEMV launch (prepare + run), on random code words
-    (every word pattern is a valid code) and random scales; 64 sampled rows of
-    every GEMV against the oracle, bit for bit."""
+    re-order launch and one GEMV launch (one grouped call, and prepare + run),
+    on random code words (every word pattern is a valid code) and random
+    scales; every output of every GEMV against the oracle, bit for bit."""
     rng = np.random.default_rng(2024)
     xs = {2048: synth.int8_uniform((1, 2048), seed=1), 8192: synth.int8_uniform((1, 8192), seed=2)}
     xd = {k: dev(v) for k, v in xs.items()}
@@ -207,13 +213,14 @@ def test_gemv_full_size_decode_stack_as_benched():
         items.append((dev_codes(codes), dev(scales), xd[K], y))
         host.append((codes, scales, K))
     g = S.GroupedGemv(items, B=1)
-    g.prepare()
-    g.run()
-    torch.cuda.synchronize()
-    for i, ((codes, scales, K), it) in enumerate(zip(host, items)):
-        rows = np.random.default_rng(i).choice(scales.shape[0], size=64, replace=False)
-        ref = oracle.gemv(rows_subset(codes, rows), scales[rows], xs[K], K)
-        assert_y_matches(it[3].cpu().numpy()[:, rows], ref)
+    refs = [oracle.gemv(codes, scales, xs[K], K) for codes, scales, K in host]
+    for run in (g, lambda: (g.prepare(), g.run())):
+        for it in items:
+            it[3].fill_(float("nan"))
+        run()
+        torch.cuda.synchronize()
+        for ref, it in zip(refs, items):
+            assert_y_matches(it[3].cpu().numpy(), ref)
     assert S.device_error() == 0
 
 
