@@ -1965,7 +1965,8 @@ __device__ __forceinline__ int sherry_weight(const uint32_t *codes, int n, int k
 }
 
 // One thread per (row, comparison tile): decode the tile's weights from the
-// Sherry codes and write its words (rows past N: zero weights).
+// Sherry codes and write its words; rows past N (the last group's padding)
+// hold zero words, as in the Sherry layout.
 __global__ void __launch_bounds__(256) transcode_kernel(const uint32_t *__restrict__ codes,
                                                         uint32_t *__restrict__ out, int N, int K,
                                                         int T, int Tc, int rows, int fmt) {
@@ -1998,7 +1999,7 @@ __global__ void __launch_bounds__(256) transcode_kernel(const uint32_t *__restri
             if ((b & 31) > 27) w[(b >> 5) + 1] |= c >> (32 - (b & 31));
         }
         uint32_t *dst = out + ((size_t)(n >> 5) * Tc + t) * 160 + (n & 31);
-        for (int p = 0; p < 5; p++) dst[32 * p] = w[p];
+        for (int p = 0; p < 5; p++) dst[32 * p] = real ? w[p] : 0u;
     }
 }
 

@@ -395,8 +395,8 @@ size_t sherry_cmp_workspace_bytes(int fmt, int64_t N, int64_t K, int B);
 /*
  * sherry_cmp_transcode -- the matrix of Sherry `codes` (N x K, layout above)
  * written in comparison format `fmt` to `out` (sherry_cmp_packed_bytes bytes;
- * padding rows and padding weights are zero weights).  Device pointers,
- * 4-byte aligned.
+ * T3's padding weights past K are zero weights; padding rows past N hold zero
+ * words).  Device pointers, 4-byte aligned.
  * Errors: NULL, SHAPE, ALIGN, UNSUPPORTED (unknown fmt), CUDA.
  */
 sherry_status sherry_cmp_transcode(int fmt, const uint32_t *codes, int64_t N, int64_t K,

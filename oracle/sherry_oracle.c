@@ -386,7 +386,8 @@ int oracle_gemv_act(const uint32_t *codes, const float *scales, const int8_t *q,
  *   - a row of K weights (K a multiple of 128) is padded with zero weights to
  *     an even number of tiles, T3 = 2 * ceil(K / 192) (the GPU streams tiles
  *     in pairs); rows in groups of 32: word(p, n, t) =
- *     codes[((n / 32) * T3 + t) * 160 + 32 p + n % 32].
+ *     codes[((n / 32) * T3 + t) * 160 + 32 p + n % 32]; rows past N hold
+ *     zero words (as in both other layouts).
  */
 enum { ORC_FMT_I2 = 1, ORC_FMT_T3 = 2 };
 
