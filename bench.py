@@ -472,6 +472,55 @@ def time_3b_layer(S, torch, dev, reps=10):
     return out
 
 
+def time_3b_stack(S, torch, dev, peak_gbs, n_layers=16, reps=200):
+    """A 16-layer LLaMA-3.2-3B-shaped stack (7 projections per layer, 252 MB of
+    codes > L2) at B = 1, 4, 16: one grouped call per step (re-order launch +
+    GEMV launch), back to back.  The codes are random words on the device
+    (every word is a valid code; the kernels' work does not depend on the
+    values), so no latents need to be made on the host."""
+    g = torch.Generator(device=dev).manual_seed(7)
+    mats = []
+    for layer in range(n_layers):
+        for name, n, k in synth.LLAMA_3B_LAYERS:
+            codes = torch.randint(-2 ** 31, 2 ** 31 - 1, ((n + 31) // 32, k // 128, 5, 32),
+                                  dtype=torch.int32, device=dev, generator=g)
+            scales = torch.rand(n, device=dev, generator=g) * 0.05 + 1e-3
+            mats.append((n, k, codes, scales))
+    code_bytes = sum(c.numel() * 4 for _, _, c, _ in mats)
+    out = {"layers": n_layers, "code_bytes": code_bytes, "codes": "random words on the device"}
+    for B, seed in ((1, 1), (4, 2), (16, 3)):
+        xs = {k: torch.from_numpy(synth.int8_uniform((B, k), seed=seed)).to(dev) for k in (3072, 8192)}
+        ys = [torch.empty((B, n), dtype=torch.float32, device=dev) for n, _, _, _ in mats]
+        step = S.GroupedGemv([(c, s, xs[k], y) for (n, k, c, s), y in zip(mats, ys)], B=B)
+        for _ in range(5):
+            step()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(reps):
+            step()
+        e1.record()
+        e1.synchronize()
+        t = e0.elapsed_time(e1) / 1e3 / reps
+        step.prepare()
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(reps):
+            step.run()
+        e1.record()
+        e1.synchronize()
+        tk = e0.elapsed_time(e1) / 1e3 / reps
+        alg = code_bytes + sum(4 * n + B * k + 4 * B * n for n, k, _, _ in mats)
+        out["B%d" % B] = {"us_per_step": t * 1e6, "weight_gbs": code_bytes / t / 1e9,
+                          "kernel_us": tk * 1e6, "kernel_gbs_algorithmic": alg / tk / 1e9,
+                          "frac_of_hbm": alg / tk / 1e9 / peak_gbs,
+                          "kernel": "gemv_dot_kernel" if B <= 2 else "gemv_pipe_kernel"}
+        del step, ys
+    del mats
+    torch.cuda.empty_cache()
+    return out
+
+
 def time_bf16_stack(layers, S, torch, dev, reps=200):
     """The same stack with bf16 activations: each step quantizes every GEMV's
     activations per token (fused into the re-order launch) and runs the GEMVs."""
@@ -798,6 +847,47 @@ def main():
         dist.barrier()
     e2e_value = whole_job_value(world, codes_bytes, K_e2e, e2e_s)
 
+    # ---------------- row-sharded step (N > 1 ranks): strong scaling of the same stack
+    sharded_line = None
+    if world > 1:
+        from bit_gemv_sherry_b200 import sharded as SH
+        parts = [SH.max_share_rows(n, world) for _, _, n, _, _, _ in layers]
+        y_part = torch.zeros((sum(parts),), dtype=torch.float32, device=dev)
+        y_gather = torch.empty((world * sum(parts),), dtype=torch.float32, device=dev)
+        sh_items, o = [], 0
+        for (_, _, n, k, codes, scales), part in zip(layers, parts):
+            c_r, s_r, (n0, n1) = SH.shard(codes, scales, rank, world)
+            if n1 > n0:
+                sh_items.append((c_r, s_r, xs[k], y_part[o:o + n1 - n0].view(1, n1 - n0)))
+            o += part
+        sh_step = S.GroupedGemv(sh_items, B=1)
+
+        def sharded_step():
+            sh_step(sptr)
+            dist.all_gather_into_tensor(y_gather, y_part)
+        for _ in range(args.warmup):
+            sharded_step()
+        torch.cuda.synchronize(dev)
+        dist.barrier()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        K_sh = max(3, min(K, 2000))
+        e0.record(stream)
+        for _ in range(K_sh):
+            sharded_step()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        dist.barrier()
+        t_sh = max_over_ranks(e0.elapsed_time(e1) / 1e3, dist, dev)
+        sharded_line = {
+            "us_per_step": t_sh / K_sh * 1e6, "steps": K_sh, "scaling": "strong",
+            "weight_gbs": codes_bytes * K_sh / t_sh / 1e9,
+            "gather_bytes_per_rank": 4 * sum(parts),
+            "note": "every projection's rows split over the %d ranks in whole 32-row groups; "
+                    "per step one grouped GEMV on the shards and one NCCL all-gather of all "
+                    "outputs; value = the whole stack's code bytes / max-over-ranks time" % world}
+        del sh_step
+
     peaks = {}
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -841,6 +931,8 @@ def main():
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": K_e2e, "ms_per_step": e2e_s / K_e2e * 1e3},
     }
+    if sharded_line is not None:
+        line["sharded_step"] = sharded_line
     if extras:
         flush = l2_flusher(torch, dev)
         line["pack"] = time_pack(latents, layers, S, torch, hbm_peak)
@@ -870,6 +962,7 @@ def main():
             "hbm_spec_gbs": HBM_SPEC_GBS, "frac_of_spec": achieved / HBM_SPEC_GBS,
             "note": "read-only stream: torch.sum over 4 GiB of fp32 (a library kernel), best of 10"}
         line["gemv_3b_layer_rotated"] = time_3b_layer(S, torch, dev)
+        line["gemv_3b_stack"] = time_3b_stack(S, torch, dev, hbm_peak)
         line["formats_compared"] = time_cmp_stack(layers, xs, S, torch, dev, ms_per_step * 1e3)
         if world == 1:
             line["cpu_baseline"] = cpu_baseline(layers, xs_host, args.cpu_seconds)
