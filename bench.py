@@ -37,9 +37,10 @@ import synth  # noqa: E402
 METRIC = "W1.25A8 GEMV weight GB/s at batch 1 (LLaMA-3.2-1B decode stack)"
 UNIT = "GB/s"
 L2_BYTES = 126 * 2 ** 20
-# ncu capture of gemv_dot_kernel<1,false> on the 16-layer stack, B = 1:
-# dram read 153,907,200 + write 5,125,376 bytes per launch
-NCU_TRAFFIC_BYTES = 153907200 + 5125376
+# dram__bytes_read.sum + dram__bytes_write.sum of one launch of the timed GEMV
+# kernel on the 16-layer stack, B = 1, from an ncu capture of this kernel
+# version (profiles/gemv_dot_decode_stack_b1.md); None until captured.
+NCU_TRAFFIC_BYTES = None
 
 
 def parse_args():
@@ -791,14 +792,16 @@ def main():
     if world > 1:
         dist.barrier()
     total_s = e_start.elapsed_time(e_end) / 1e3
-    # the GEMV launch alone (roofline): K2 back-to-back runs on one prepared
-    # workspace between one event pair (152 MB of codes > L2, so every run reads
-    # HBM); and, for reference, the same launch bracketed by its own events
+    # The GEMV launch alone (roofline).  At B = 1 the step is that one launch
+    # (the kernel re-orders each chunk's activations itself), so K2 steps back
+    # to back between one event pair give its average duration (152 MB of
+    # codes > L2: every launch reads HBM); for reference, the same launch
+    # bracketed by its own events, and the split path (one re-order launch,
+    # then GEMV launches on the prepared workspace).
     K2 = max(3, min(K, 2000))
-    step.prepare(sptr)
     e_start.record(stream)
     for i in range(K2):
-        step.run(sptr)
+        step(sptr)
     e_end.record(stream)
     torch.cuda.synchronize(dev)
     gemv_s = e_start.elapsed_time(e_end) / 1e3 / K2
@@ -808,10 +811,17 @@ def main():
     for i in range(K3):
         b, c = ev2[i]
         b.record(stream)
-        step.run(sptr)
+        step(sptr)
         c.record(stream)
     torch.cuda.synchronize(dev)
     gemv_bracketed_s = sum(b.elapsed_time(c) for b, c in ev2) / 1e3 / K3
+    step.prepare(sptr)
+    e_start.record(stream)
+    for i in range(K2):
+        step.run(sptr)
+    e_end.record(stream)
+    torch.cuda.synchronize(dev)
+    run_prepared_s = e_start.elapsed_time(e_end) / 1e3 / K2
     time.sleep(0.2)
     clocks.stop()
     clk = clocks.summary(t_host0, t_host1)
@@ -901,7 +911,7 @@ def main():
     achieved = alg_bytes / gemv_s / 1e9
     # dram__bytes_read.sum + dram__bytes_write.sum of one gemv_dot_kernel launch
     # on this workload (ncu --set full); valid only for that kernel version
-    ncu_traffic = NCU_TRAFFIC_BYTES if args.layers == 16 else None
+    ncu_traffic = NCU_TRAFFIC_BYTES if args.layers == 16 and NCU_TRAFFIC_BYTES else None
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
@@ -914,19 +924,21 @@ def main():
             "code_bytes": codes_bytes, "batch": 1,
             "l2": "inputs larger than L2: %.0f MB of codes per step > 126 MB L2, no flush" % (
                 codes_bytes / 1e6),
-            "launch": "sherry_gemv_grouped (one activation re-order launch and one GEMV launch "
-                      "per step)",
+            "launch": "sherry_gemv_grouped: one GEMV launch per step (the kernel re-orders the "
+                      "activations of each chunk itself)",
             "parallelism": "replicas x%d" % world,
         },
-        "gpu_launches": 2 * K,
+        "gpu_launches": K,
         "clocks": clk,
-        "roofline": {"bound": "hbm", "kernel": "gemv_dot_kernel (sherry_gemv_run)",
+        "roofline": {"bound": "hbm",
+                     "kernel": "gemv_dot_kernel<1,false,1> (sherry_gemv_grouped, in-kernel re-order)",
                      "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "peak_source": peak_src,
                      "bytes_per_launch": alg_bytes, "kernel_us": gemv_s * 1e6,
                      "kernel_launches_timed": K2,
                      "timing": "average over back-to-back launches between one event pair",
                      "kernel_us_each_bracketed_by_events": gemv_bracketed_s * 1e6,
+                     "kernel_us_prepared_run": run_prepared_s * 1e6,
                      "traffic": ncu_traffic, "traffic_unit": "bytes per launch"},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": K_e2e, "ms_per_step": e2e_s / K_e2e * 1e3},

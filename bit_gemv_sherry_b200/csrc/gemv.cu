@@ -757,31 +757,16 @@ __device__ __forceinline__ bool stage_wait(uint64_t *bar, uint32_t parity) {
     return __all_sync(0xFFFFFFFFu, ok);
 }
 
-// Shared memory of the MMA kernel.  Per warp a ring of kPipeRing stages; a
-// stage holds one chunk: the 4 tiles' code blocks (each 160 words padded to
-// 168, so that a read of (tile t, plane p, rows g + 8 rb) by lanes (g, t) hits
-// 32 distinct banks), then the chunk's activations as (batch row, tile)
-// pieces of 32 words padded to 36 (lane (g, t) reads piece (g, t): within a
-// quarter-warp the pieces start 4 banks apart, so the 16-byte fragment loads
-// are conflict-free).  After the rings: the stages' mbarriers [warp][stage],
-// then per warp the fragments of a later piece of a cut item [2 * NB * 4][32].
-constexpr int kPipeRing = 2;
-constexpr int kXPieceWords = 36;
+#ifndef SHERRY_PIPE_MIN_BLOCKS
+#define SHERRY_PIPE_MIN_BLOCKS 2
+#endif
+// Shared memory of the MMA kernel: the warps' rings, then per warp the
+// fragments of a later piece of a cut item [warp][2 * NB * 4][32] (the
+// chunk split and the cut items are those of the small-batch kernel below).
 template <int NB>
 struct PipeShape {
-    static constexpr int kWarps = 4;
-    static constexpr int kThreads = kWarps * 32;
-    static constexpr int kCodeWords = kChunkTiles * kTileWordsPadded;          // 672
-    static constexpr int kXPieces = 8 * NB * kChunkTiles;                      // batch rows x tiles
-    static constexpr int kStageWords = kCodeWords + kXPieces * kXPieceWords;
-    static constexpr int kRingWords = kWarps * kPipeRing * kStageWords;
     static constexpr int kCutWords = 2 * NB * 4 * 32;
-    static constexpr size_t kBarOffset = (size_t)kRingWords * 4;
-    static constexpr size_t kCutOffset = kBarOffset + (size_t)kWarps * kPipeRing * 8;
-    static constexpr size_t kSmem = kCutOffset + ((size_t)kWarps * kCutWords + kWarps) * 4;
-    static constexpr int kFit = (int)((227u * 1024u) / (kSmem + 1024u));
-    static constexpr int kMinBlocks = kFit < 1 ? 1 : (kFit > 4 ? 4 : kFit);
-    static_assert(kStageWords % 4 == 0 && kCodeWords % 4 == 0, "16-byte aligned stages");
+    static constexpr size_t kSmem = kPipeSmem + (size_t)kPipeWarps * kCutWords * 4;
 };
 
 // Finishes an item of the MMA kernel: per row block rb, fragment e holds
@@ -849,40 +834,29 @@ __device__ __forceinline__ void pipe_finish(const GemvDesc &D, int unit, int B, 
 }
 
 template <int NB, bool ACC_OUT>
-__global__ void __launch_bounds__(PipeShape<NB>::kThreads, PipeShape<NB>::kMinBlocks)
+__global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
     gemv_pipe_kernel(const __grid_constant__ GemvParams P) {
-    using Shape = PipeShape<NB>;
-    constexpr int kWarps = Shape::kWarps;
-    constexpr int SW = Shape::kStageWords;
     pdl_allow_dependents();
-    extern __shared__ __align__(128) uint32_t pipe_smem[];
-    uint8_t *smem_bytes = reinterpret_cast<uint8_t *>(pipe_smem);
+    extern __shared__ __align__(16) uint32_t pipe_smem[];
+    int *cut_sum = reinterpret_cast<int *>(pipe_smem + kPipeSmem / 4);
+    __shared__ int cut_start[kPipeWarps];
+    __shared__ int cta_bound[2];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem_bytes + Shape::kBarOffset) + warp * kPipeRing;
-    int *cut_sum = reinterpret_cast<int *>(smem_bytes + Shape::kCutOffset);
-    int *cut_start = cut_sum + kWarps * Shape::kCutWords;
-    __shared__ int cta_bound[2];
     // chunk range [b0, b1) of this warp: the CTA takes whole items of about
     // 1/gridDim of the chunks, its warps equal chunk shares of them
     if (threadIdx.x < 2) {
         const long long tc = P.total_chunks, nb = gridDim.x;
         cta_bound[threadIdx.x] = item_start_at_or_before(P, (int)((blockIdx.x + threadIdx.x) * tc / nb));
     }
-    if (lane == 0) {
-#pragma unroll
-        for (int s = 0; s < kPipeRing; s++) mbar_init(&bars[s], 1);
-        fence_mbar_init();
-    }
     __syncthreads();
     const int cta_lo = cta_bound[0];
     const long long len = cta_bound[1] - cta_lo;
-    const int b0 = cta_lo + (int)(warp * len / kWarps);
-    const int b1 = cta_lo + (int)((warp + 1) * len / kWarps);
+    const int b0 = cta_lo + (int)(warp * len / kPipeWarps);
+    const int b1 = cta_lo + (int)((warp + 1) * len / kPipeWarps);
     // -1: no cut item starts before b0; -2: empty range (skipped when summing)
     if (lane == 0) cut_start[warp] = b0 < b1 ? -1 : -2;
-    uint32_t *ring = pipe_smem + (size_t)warp * kPipeRing * SW;
-    const uint32_t ring_addr = smem_u32(ring);
+    uint32_t *ring = pipe_smem + (size_t)warp * kRing * kStageWords;
     Consts C;
     load_consts(P, C);
     const int B = P.B;
@@ -891,76 +865,53 @@ __global__ void __launch_bounds__(PipeShape<NB>::kThreads, PipeShape<NB>::kMinBl
     ItemCursor cur = {0, 0, 0};
     if (b0 < b1) cur = cursor_at_chunk(P, b0, start);
 
-    // ---- producer side: runs one chunk ahead of the consumer ----
-    // Lane 0 arms the stage's mbarrier with the chunk's bytes; lanes 0..3 copy
-    // the 4 tiles' code blocks (640 bytes each, contiguous in global memory)
-    // into their padded slots, and lanes l, l + 32 copy the activation pieces
-    // (batch row b, tile) = l, l + 32 (128 bytes each) of the B batch rows.
-    // Until pdl_wait() only codes are read, and only when P.prefetch_codes
-    // says the kernel before is this call's re-order launch.
+    // ---- producer side: the issue cursor runs kRing-1 stages ahead ----
+    // lane l copies 16-byte pieces l + 32 j (j = 0..4) of the 2560-byte chunk;
+    // piece words 4i..4i+3 belong to tile block 4i / 160.  Codes only (and
+    // only when P.prefetch_codes allows it before pdl_wait()): the activations
+    // are read from global memory after pdl_wait().
     ItemCursor icur = cur;
     int istart = start, ic = 0, ic_end = 0;
+    const uint32_t *isrc = nullptr;  // first word of the current unit's group
     auto set_issue_item = [&]() {
         const GemvDesc &D = P.d[icur.id];
+        isrc = D.codes + (size_t)icur.unit * D.T * kTileWords + 4 * lane;
         const int first = icur.kp * D.cpp;
         ic = first + max(b0 - istart, 0);
         ic_end = first + min(b1 - istart, min(D.cpp, D.nchunk - first));
     };
     if (istart < b1) set_issue_item();
-    const uint32_t chunk_bytes = (uint32_t)kChunkTiles * kTileWords * 4 + (uint32_t)B * kChunkTiles * 128;
-    auto issue_codes = [&](int slot) {
-        const GemvDesc &D = P.d[icur.id];
-        const uint32_t dst = ring_addr + (uint32_t)slot * SW * 4;
-        if (lane == 0) {
-            fence_proxy_async_smem();  // the warp's reads of the stage's previous chunk come first
-            mbar_arrive_expect_tx(&bars[slot], chunk_bytes);
-        }
-        __syncwarp();
-        if (lane < kChunkTiles)
-            bulk_load(dst + (uint32_t)lane * kTileWordsPadded * 4,
-                      D.codes + ((size_t)icur.unit * D.T + (size_t)ic * kChunkTiles + lane) * kTileWords,
-                      kTileWords * 4, &bars[slot]);
-    };
-    auto issue_x_and_advance = [&](int slot) {
-        const GemvDesc &D = P.d[icur.id];
-        const uint32_t dst = ring_addr + (uint32_t)slot * SW * 4 + (uint32_t)Shape::kCodeWords * 4;
+    uint32_t dst_piece[5];
 #pragma unroll
-        for (int j = 0; j < 2; j++) {
-            const int pc = lane + 32 * j;  // piece = (batch row pc / 4, tile pc % 4)
-            if (pc < B * kChunkTiles)
-                bulk_load(dst + (uint32_t)pc * kXPieceWords * 4,
-                          D.xw + ((size_t)(pc >> 2) * D.Tp + (size_t)ic * kChunkTiles + (pc & 3)) * 8, 128,
-                          &bars[slot]);
-        }
-        if (++ic == ic_end) {
-            istart += min(D.cpp, D.nchunk - icur.kp * D.cpp);
-            if (istart < b1) {
-                cursor_next(P, icur);
-                set_issue_item();
-            }
-        }
-    };
-    uint32_t inflight = 0;
+    for (int j = 0; j < 5; j++) {
+        const int wd = 4 * (lane + 32 * j);
+        const int tb = wd / kTileWords;
+        dst_piece[j] = smem_u32(ring) + 4u * (uint32_t)(tb * kTileWordsPadded + (wd - tb * kTileWords));
+    }
     auto issue = [&](int slot) {
         if (istart < b1) {
-            issue_codes(slot);
-            issue_x_and_advance(slot);
-            inflight |= 1u << slot;
+            const uint32_t *src = isrc + (size_t)ic * kChunkTiles * kTileWords;
+            const uint32_t sofs = (uint32_t)slot * kStageWords * 4;
+#pragma unroll
+            for (int j = 0; j < 5; j++) cp_async16(dst_piece[j] + sofs, src + 128 * j, 16u);
+            if (++ic == ic_end) {
+                const GemvDesc &D = P.d[icur.id];
+                istart += min(D.cpp, D.nchunk - icur.kp * D.cpp);
+                if (istart < b1) {
+                    cursor_next(P, icur);
+                    set_issue_item();
+                }
+            }
         }
+        cp_async_commit();
     };
-    const bool first_copy = istart < b1;
-    if (first_copy && P.prefetch_codes) issue_codes(0);
-    pdl_wait();
-    if (first_copy && !P.prefetch_codes) issue_codes(0);
-    if (first_copy) {
-        issue_x_and_advance(0);
-        inflight = 1u;
-    }
+    if (!P.prefetch_codes) pdl_wait();
+#pragma unroll
+    for (int s = 0; s < kRing - 1; s++) issue(s);
+    if (P.prefetch_codes) pdl_wait();
 
     // ---- consumer side ----
     int slot = 0;
-    uint32_t phase = 0;
-    bool failed = false;
     int acc[2][NB][4];  // [row block][batch group][fragment]
     bool own_cut = false;  // the last item continues in later warps of the CTA
     while (start < b1) {
@@ -969,42 +920,49 @@ __global__ void __launch_bounds__(PipeShape<NB>::kThreads, PipeShape<NB>::kMinBl
         const int nreal = min(D.cpp, D.nchunk - first);
         const int c_begin = first + max(b0 - start, 0);
         const int c_end = first + min(b1 - start, nreal);
+        const uint4 *xrow[NB];
+#pragma unroll
+        for (int nb = 0; nb < NB; nb++) {
+            const int b = min(nb * 8 + g, B - 1);  // lanes past the batch: never stored
+            xrow[nb] = D.xw + (size_t)b * D.Tp * 8 + (size_t)t * 8;
+        }
 #pragma unroll
         for (int a = 0; a < 2; a++)
 #pragma unroll
             for (int nb = 0; nb < NB; nb++) acc[a][nb][0] = acc[a][nb][1] = acc[a][nb][2] = acc[a][nb][3] = 0;
         for (int c = c_begin; c < c_end; c++) {
-            issue(slot ^ 1);  // the next chunk into the stage the previous chunk used
-            if (!stage_wait(&bars[slot], (phase >> slot) & 1u)) {
-                failed = true;
-                break;
-            }
-            inflight &= ~(1u << slot);
-            phase ^= 1u << slot;
+            cp_async_wait<kRing - 2>();
+            __syncwarp();
             // tile t of the chunk, plane p, row g + 8 r: word t * 168 + 32 p + g + 8 r
-            const uint32_t *st = ring + slot * SW + t * kTileWordsPadded + g;
-            // the activation piece (batch row nb * 8 + g, tile t): rows past B hold
-            // stale words, whose MMA columns are never stored
-            const uint4 *xp[NB];
-#pragma unroll
-            for (int nb = 0; nb < NB; nb++)
-                xp[nb] = reinterpret_cast<const uint4 *>(ring + slot * SW + Shape::kCodeWords +
-                                                         ((nb * 8 + g) * kChunkTiles + t) * kXPieceWords);
-            // the four rows of this lane (g, g + 8 of row block 0, g + 16, g + 24 of
-            // row block 1) are decoded together, so each activation fragment is
-            // loaded once for both row blocks
+            const uint32_t *st = ring + slot * kStageWords + t * kTileWordsPadded + g;
+            // padded tiles hold zero activations, so no load is predicated
+            const size_t xoff = (size_t)c * kChunkTiles * 8;
+            // the four rows of this lane (g, g + 8 of row block 0, g + 16, g + 24 of row
+            // block 1) are decoded together, so each activation fragment is loaded once
+            // for both row blocks, and the next position's fragments are loaded while
+            // the current position's MMAs run
             TileDecoder6 d[4];
 #pragma unroll
             for (int r = 0; r < 4; r++)
                 d[r].load(C, st[0 * 32 + 8 * r], st[1 * 32 + 8 * r], st[2 * 32 + 8 * r],
                           st[3 * 32 + 8 * r], st[4 * 32 + 8 * r]);
+            __syncwarp();  // every lane has its words: the stage can be refilled
+            issue(slot == 0 ? kRing - 1 : slot - 1);
+            slot = (slot + 1 == kRing) ? 0 : slot + 1;
+            uint4 xq[NB][2], xn[NB][2];
+#pragma unroll
+            for (int nb = 0; nb < NB; nb++) {
+                xq[nb][0] = ld_x(xrow[nb] + xoff);
+                xq[nb][1] = ld_x(xrow[nb] + xoff + 1);
+            }
 #pragma unroll
             for (int i = 0; i < 4; i++) {
-                uint4 xq[NB][2];
+                if (i < 3) {
 #pragma unroll
-                for (int nb = 0; nb < NB; nb++) {
-                    xq[nb][0] = xp[nb][2 * i];
-                    xq[nb][1] = xp[nb][2 * i + 1];
+                    for (int nb = 0; nb < NB; nb++) {
+                        xn[nb][0] = ld_x(xrow[nb] + xoff + 2 * i + 2);
+                        xn[nb][1] = ld_x(xrow[nb] + xoff + 2 * i + 3);
+                    }
                 }
                 const uint32_t tlo = C.tlo[i], thi = C.thi[i];
 #pragma unroll
@@ -1026,14 +984,18 @@ __global__ void __launch_bounds__(PipeShape<NB>::kThreads, PipeShape<NB>::kMinBl
                         }
                     }
                 }
+                if (i < 3) {
+#pragma unroll
+                    for (int nb = 0; nb < NB; nb++) {
+                        xq[nb][0] = xn[nb][0];
+                        xq[nb][1] = xn[nb][1];
+                    }
+                }
             }
-            __syncwarp();  // every lane is done with this stage before it is refilled
-            slot ^= 1;
         }
-        if (failed) break;
         if (start < b0) {
             // a later piece of an item cut at b0: hand the fragments to its first warp
-            int *cs = cut_sum + warp * Shape::kCutWords + lane;
+            int *cs = cut_sum + warp * PipeShape<NB>::kCutWords + lane;
 #pragma unroll
             for (int rb = 0; rb < 2; rb++)
 #pragma unroll
@@ -1049,22 +1011,16 @@ __global__ void __launch_bounds__(PipeShape<NB>::kThreads, PipeShape<NB>::kMinBl
         start += nreal;
         if (start < b1) cursor_next(P, cur);
     }
-    if (failed) {
-        if (lane == 0) atomicCAS(&g_gemv_device_error, 0u, (unsigned int)SHERRY_ERR_TIMEOUT);
-#pragma unroll
-        for (int s = 0; s < kPipeRing; s++)
-            if (inflight & (1u << s)) stage_wait(&bars[s], (phase >> s) & 1u);
-        own_cut = false;
-    }
+    cp_async_wait<0>();
     __syncthreads();  // the later pieces' fragments are in shared memory
     if (own_cut) {
         const GemvDesc &D = P.d[cur.id];
         const int mine = D.chunk_begin + cur.unit * D.nchunk + cur.kp * D.cpp;  // the cut item
-        for (int w = warp + 1; w < kWarps; w++) {
+        for (int w = warp + 1; w < kPipeWarps; w++) {
             const int cs = cut_start[w];
             if (cs == -2) continue;
             if (cs != mine) break;
-            const int *src = cut_sum + w * Shape::kCutWords + lane;
+            const int *src = cut_sum + w * PipeShape<NB>::kCutWords + lane;
 #pragma unroll
             for (int rb = 0; rb < 2; rb++)
 #pragma unroll
@@ -1112,23 +1068,23 @@ constexpr int kDotUnits = SHERRY_DOT_UNITS;  // 32-row units per item of the dot
 #endif
 constexpr int kDotWaves = SHERRY_DOT_WAVES;  // CTA waves of the dot kernel (see grid_for)
 constexpr int kDotRing = 2;                  // stages per warp
-#ifndef SHERRY_RAW_X_MAX_CHUNKS_PER_SM
-#define SHERRY_RAW_X_MAX_CHUNKS_PER_SM 64
-#endif
-// calls up to this many 32-row chunks per SM re-order x in the dot kernel
-constexpr int kRawXMaxChunksPerSM = SHERRY_RAW_X_MAX_CHUNKS_PER_SM;
+// bf16 calls up to this many 32-row chunks per SM quantize and re-order x in
+// the dot kernel (each warp takes the token's absmax from the row itself, so
+// large calls keep the front-end launch); int8 calls of any size re-order x
+// in the kernel (measured on the 16-layer 1B stack: 54.5 us per step against
+// 56.6 us with the re-order launch).
+constexpr int kRawBfMaxChunksPerSM = 64;
 constexpr int kDotCodeWords = kChunkTiles * kTileWords;  // 640 words: one unit's chunk
 // Weight formats the small-batch kernel streams: Sherry, and the two ternary
 // packings the pages compare it against (arXiv 2601.07892, abstract; Figure 2
 // caption): 2 bits per weight, aligned ("I2"), and three weights in five bits
-// ("T3").  Per format: 32-bit words per tile of one row, weights per tile,
-// tiles per chunk.  Every format's chunk carries 32 activation words per tile
-// and batch row.
+// ("T3").  Per format: 32-bit words per tile of one row (a tile is 128
+// weights, or 96 for T3) and tiles per chunk.  Every format's chunk carries
+// 32 activation words per tile and batch row.
 enum DotFormat { kFmtSherry = 0, kFmtI2 = 1, kFmtT3 = 2 };
 template <int FMT>
 struct FmtTraits {
     static constexpr int kTileWords = FMT == kFmtI2 ? 8 : 5;
-    static constexpr int kTileK = FMT == kFmtT3 ? 96 : 128;
     static constexpr int kChunkTiles = FMT == kFmtT3 ? 2 : 4;
     static constexpr int kUnitChunkWords = kChunkTiles * kTileWords * kUnitRows;
 };
@@ -1690,11 +1646,10 @@ template <int NB, bool ACC>
 void launch_pipe(const GemvParams &gp, cudaStream_t stream) {
     static int cache[64] = {0};
     // one chunk per warp at most (items cut between warps are summed in shared memory)
-    using Shape = PipeShape<NB>;
-    const size_t smem = Shape::kSmem;
-    const int want = (gp.total_chunks + Shape::kWarps - 1) / Shape::kWarps;
-    const int grid = grid_for(gemv_pipe_kernel<NB, ACC>, Shape::kThreads, smem, want, cache);
-    launch_pdl(gemv_pipe_kernel<NB, ACC>, grid, Shape::kThreads, smem, stream, gp);
+    const size_t smem = PipeShape<NB>::kSmem;
+    const int want = (gp.total_chunks + kPipeWarps - 1) / kPipeWarps;
+    const int grid = grid_for(gemv_pipe_kernel<NB, ACC>, kPipeThreads, smem, want, cache);
+    launch_pdl(gemv_pipe_kernel<NB, ACC>, grid, kPipeThreads, smem, stream, gp);
 }
 
 template <int NBX, bool ACC, int XMODE>
@@ -1875,12 +1830,12 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
     xp.total_units = wb;
     gp.total_units16 = ub16;
     gp.total_chunks = cb;
-    // A small int8 call skips the re-order launch: the dot kernel re-orders each
-    // chunk's activations itself (at most ~2 chunks per warp of a full GPU, so
-    // x is re-ordered at most twice per chunk position; rows are not split, so
-    // there are no K-part sums to clear).
-    bool raw_x = phase == kBoth && dot && cb32 <= kRawXMaxChunksPerSM * sm_count();
-    bool raw_bf = raw_x && !acc_out;
+    // An int8 call at B <= 2 skips the re-order launch: the dot kernel re-orders
+    // each chunk's activations itself (four shuffles and three byte permutes
+    // per word, shared by the unit group's rows; rows are not split, so there
+    // are no K-part sums to clear).
+    bool raw_x = phase == kBoth && dot;
+    bool raw_bf = raw_x && !acc_out && cb32 <= kRawBfMaxChunksPerSM * sm_count();
     for (int i = 0; i < count && raw_x; i++)
         raw_x = calls[i].x && !calls[i].xbf && !calls[i].xf && aligned(calls[i].x, 16) &&
                 kparts_for(calls[i].K) == 1;

@@ -138,10 +138,11 @@ sherry_status sherry_pack_grouped(const sherry_pack_desc *descs, int count,
  * long rows are processed as several K-parts whose int32 partial sums meet in
  * the workspace.  sherry_gemv_workspace_bytes(N, K, B) is the size one GEMV
  * needs; a grouped call needs the sum over its GEMVs, laid out in descriptor
- * order.  Small calls (B <= 2, K a multiple of 512, at most 64 chunks of
- * 4 x 128 weights per SM, rows not split, activations 16-byte aligned) re-order (and for bf16,
- * quantize) inside the GEMV kernel and leave the workspace untouched; the
- * size asked is the same.  The workspace is a device buffer, 256-byte
+ * order.  Int8 calls with B <= 2, K a multiple of 512 and at most 8192, and
+ * 16-byte aligned activations re-order inside the GEMV kernel and leave the
+ * workspace untouched, as do bf16 calls of that kind with at most 64 chunks
+ * of 32 rows x 512 weights per SM (which also quantize there); the size asked
+ * is the same.  The workspace is a device buffer, 256-byte
  * aligned, owned by the caller; its contents are scratch: every call that
  * prepares activations (sherry_gemv, sherry_gemv_acc, sherry_gemv_grouped,
  * sherry_gemv_prepare) may rewrite it, and a run leaves its partial-sum area
