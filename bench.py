@@ -54,6 +54,12 @@ def parse_args():
                     help="skip the pack/GEMM/per-layer/CPU-baseline sub-measurements")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--gemm-only", action="store_true",
+                    help="only run the two prefill GEMMs --steps times each (a small case for "
+                         "profiling); prints their timings as JSON")
+    ap.add_argument("--stack3b-only", type=int, default=0, metavar="B",
+                    help="only run the 16-layer 3B stack at batch B for --steps steps (a case for "
+                         "profiling); prints its timing as JSON")
     ap.add_argument("--mlp-chain-only", action="store_true",
                     help="only time the chained MLP blocks of --layers layers for --steps steps "
                          "(a small case for profiling); prints their JSON")
@@ -473,7 +479,7 @@ def time_3b_layer(S, torch, dev, reps=10):
     return out
 
 
-def time_3b_stack(S, torch, dev, peak_gbs, n_layers=16, reps=200):
+def time_3b_stack(S, torch, dev, peak_gbs, n_layers=16, reps=200, batches=(1, 4, 16)):
     """A 16-layer LLaMA-3.2-3B-shaped stack (7 projections per layer, 252 MB of
     codes > L2) at B = 1, 4, 16: one grouped call per step (re-order launch +
     GEMV launch), back to back.  The codes are random words on the device
@@ -489,7 +495,8 @@ def time_3b_stack(S, torch, dev, peak_gbs, n_layers=16, reps=200):
             mats.append((n, k, codes, scales))
     code_bytes = sum(c.numel() * 4 for _, _, c, _ in mats)
     out = {"layers": n_layers, "code_bytes": code_bytes, "codes": "random words on the device"}
-    for B, seed in ((1, 1), (4, 2), (16, 3)):
+    for B in batches:
+        seed = {1: 1, 4: 2, 16: 3}.get(B, B)
         xs = {k: torch.from_numpy(synth.int8_uniform((B, k), seed=seed)).to(dev) for k in (3072, 8192)}
         ys = [torch.empty((B, n), dtype=torch.float32, device=dev) for n, _, _, _ in mats]
         step = S.GroupedGemv([(c, s, xs[k], y) for (n, k, c, s), y in zip(mats, ys)], B=B)
@@ -742,6 +749,15 @@ def main():
     S.lib()
 
     spec = stack_spec(args.layers)
+    if args.gemm_only:
+        flush = l2_flusher(torch, dev)
+        print(json.dumps(time_gemm(S, torch, dev, flush, reps=max(1, args.steps))))
+        return 0
+    if args.stack3b_only:
+        B = args.stack3b_only
+        print(json.dumps(time_3b_stack(S, torch, dev, 6558.1, reps=max(1, args.steps),
+                                       batches=(B,))))
+        return 0
     if args.mlp_chain_only:
         layers, _ = build_stack(spec, dev, S, torch)
         print(json.dumps(time_mlp_chain(layers, S, torch, dev, reps=args.steps)))

@@ -227,6 +227,11 @@ __device__ __forceinline__ void bulk_load(uint32_t dst_smem, const void *src, ui
         "l"(src), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
 }
+// Warm L2 with `bytes` bytes from global `src` (16-byte aligned, a multiple of
+// 16 bytes).  Nothing reaches the CTA: a later copy reads the data from L2.
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 // Arrive on `bar` once all previously issued tcgen05.mma of this thread completed.
 __device__ __forceinline__ void umma_commit(uint64_t *bar) {
     asm volatile(

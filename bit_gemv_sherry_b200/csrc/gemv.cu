@@ -1410,7 +1410,19 @@ __global__ void __launch_bounds__(DotShape<NBX, XMODE, FMT>::kThreads,
         }
     };
     const bool first_copy = istart < b1;
-    if (first_copy && P.prefetch_codes) issue_codes(0);
+    if (first_copy && P.prefetch_codes) {
+        issue_codes(0);
+    } else if (first_copy && lane == 0) {
+        // the kernel before may have written the codes: only warm L2 with the
+        // first chunk's codes before the wait (L2 is where every write lands,
+        // so the copy after the wait reads the final data from it)
+        const GemvDesc &D = P.d[icur.id];
+        const int unit0 = icur.unit * NU;
+        const int present = min(NU, D.units32 - unit0);
+        const uint32_t *src = D.codes + ((size_t)unit0 * D.T + (size_t)ic * CT) * (F::kTileWords * kUnitRows);
+        for (int u = 0; u < present; u++)
+            bulk_prefetch_l2(src + (size_t)u * D.T * (F::kTileWords * kUnitRows), UCW * 4);
+    }
     pdl_wait();
     if (first_copy && !P.prefetch_codes) issue_codes(0);
     if (first_copy) {
