@@ -38,9 +38,10 @@ METRIC = "W1.25A8 GEMV weight GB/s at batch 1 (LLaMA-3.2-1B decode stack)"
 UNIT = "GB/s"
 L2_BYTES = 126 * 2 ** 20
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch of the timed GEMV
-# kernel on the 16-layer stack, B = 1, from an ncu capture of this kernel
-# version (profiles/gemv_dot_decode_stack_b1.md); None until captured.
-NCU_TRAFFIC_BYTES = None
+# kernel (gemv_dot_kernel<1,false,1>) on the 16-layer stack, B = 1, from an ncu
+# capture of this kernel version (profiles/gemv_dot_decode_stack_b1.md):
+# 153,650,432 read + 3,292,416 written.
+NCU_TRAFFIC_BYTES = 153650432 + 3292416
 
 
 def parse_args():
