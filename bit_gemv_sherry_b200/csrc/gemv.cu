@@ -1063,10 +1063,6 @@ __global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
 #define SHERRY_DOT_UNITS 2
 #endif
 constexpr int kDotUnits = SHERRY_DOT_UNITS;  // 32-row units per item of the dot kernel
-#ifndef SHERRY_DOT_WAVES
-#define SHERRY_DOT_WAVES 1
-#endif
-constexpr int kDotWaves = SHERRY_DOT_WAVES;  // CTA waves of the dot kernel (see grid_for)
 constexpr int kDotRing = 2;                  // stages per warp
 // bf16 calls up to this many 32-row chunks per SM quantize and re-order x in
 // the dot kernel (each warp takes the token's absmax from the row itself, so
@@ -1634,11 +1630,8 @@ void launch_xprep_f32(const XprepF32Params &p, cudaStream_t stream) {
     cudaLaunchKernelEx(&cfg, xprep_f32_kernel, p);
 }
 
-// Resident CTAs times `waves`: with several waves of smaller CTAs, SMs that
-// finish their CTAs early take later ones, so the launch does not wait for
-// the slowest SM's fixed share.
 template <typename KernelT>
-int grid_for(KernelT kernel, int threads, size_t smem, int want, int *cache, int waves = 1) {
+int grid_for(KernelT kernel, int threads, size_t smem, int want, int *cache) {
     int dev = 0;
     cudaGetDevice(&dev);
     int &bps = cache[dev & 63];
@@ -1651,7 +1644,7 @@ int grid_for(KernelT kernel, int threads, size_t smem, int want, int *cache, int
             n = 1;
         bps = n;
     }
-    return std::max(1, std::min(want, waves * bps * sm_count()));
+    return std::max(1, std::min(want, bps * sm_count()));
 }
 
 template <int NB, bool ACC>
@@ -1672,7 +1665,7 @@ void launch_dot(const GemvParams &gp, cudaStream_t stream) {
     // many SMs as it has chunks (items cut between warps are summed in shared memory)
     constexpr int threads = DotShape<NBX, XMODE>::kThreads, warps = DotShape<NBX, XMODE>::kWarps;
     const int want = (gp.total_chunks + warps - 1) / warps;
-    const int grid = grid_for(gemv_dot_kernel<NBX, ACC, XMODE>, threads, smem, want, cache, kDotWaves);
+    const int grid = grid_for(gemv_dot_kernel<NBX, ACC, XMODE>, threads, smem, want, cache);
     launch_pdl(gemv_dot_kernel<NBX, ACC, XMODE>, grid, threads, smem, stream, gp);
 }
 
