@@ -65,7 +65,7 @@ struct GemvDesc {
     int Tp;               // tile stride of xw (T rounded up to a whole chunk)
     int unit_begin16;     // register kernel: first 16-row unit in the group
     int units;            // pipelined kernels: items per K-part column (32-row units, or
-                          // groups of kDotUnits units for the dot kernel)
+                          // groups of 1 or 2 units for the dot kernel)
     int units32;          // 32-row units of the GEMV (ceil(N / 32))
     int nchunk;           // pipelined kernel: 4-tile chunks per row
     int kparts;           // pipelined kernel: K-parts per unit
@@ -1034,12 +1034,12 @@ __global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
 
 // ---------------------------------------------------------------------------
 // Small-batch kernel (B <= 2): dot products on the ALU/FMA pipes, no MMA.
-//   * an item is (unit group, K-part), a unit group being kDotUnits
+//   * an item is (unit group, K-part), a unit group being NU (1 or 2)
 //     consecutive 32-row units.  Lane l owns row l of each unit of the group,
 //     so a tile's five words of one unit are five conflict-free shared loads,
 //     each lane ends with its rows' sums (no reduction across lanes), and the
 //     activation words of a tile, read once per warp (broadcast loads), feed
-//     kDotUnits rows per lane;
+//     NU rows per lane;
 //   * work is split by chunk count, a chunk being 4 tiles of every unit of a
 //     group.  Each CTA takes a run of whole items holding about 1/gridDim of
 //     the chunks and its warps split the run into equal chunk ranges, so no
@@ -1059,10 +1059,14 @@ __global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
 // K-parts and the split-K completion are those of the pipelined kernel, with
 // one counter per unit group.
 // ---------------------------------------------------------------------------
-#ifndef SHERRY_DOT_UNITS
-#define SHERRY_DOT_UNITS 2
-#endif
-constexpr int kDotUnits = SHERRY_DOT_UNITS;  // 32-row units per item of the dot kernel
+// 32-row units per item of the dot kernel: 2 for calls of more than
+// kDotPairMinChunksPerSM 32-row chunks per SM (the broadcast activation loads
+// and the in-kernel re-order are shared by two rows per lane), else 1 (twice
+// the items, so a small call spreads over twice the SMs).  Measured on the
+// 16-layer 1B stack with in-kernel re-order: 54.5 us per step with 2, 58.9
+// with 1; a 2048 x 8192 GEMV: 7.3 us with 1, 9.1 with 2.
+constexpr int kDotMaxUnits = 2;
+constexpr int kDotPairMinChunksPerSM = 64;
 constexpr int kDotRing = 2;                  // stages per warp
 // bf16 calls up to this many 32-row chunks per SM quantize and re-order x in
 // the dot kernel (each warp takes the token's absmax from the row itself, so
@@ -1088,9 +1092,9 @@ struct FmtTraits {
 // 8 warps per CTA.  B = 1 with two units per item: 2 CTAs (16 warps) per SM,
 // 90 KB of shared memory per CTA, up to 128 registers per thread.
 // XMODE 2 adds to each stage the chunk's raw bf16 activations (1 KB per batch row).
-template <int NBX, int XMODE = 0, int FMT = kFmtSherry>
+template <int NBX, int XMODE = 0, int FMT = kFmtSherry, int NU_ = kDotMaxUnits>
 struct DotShape {
-    static constexpr int NU = kDotUnits;
+    static constexpr int NU = NU_;
     static constexpr int kWarps = 8;
     static constexpr int kThreads = kWarps * 32;
     static constexpr int kChunkTilesF = FmtTraits<FMT>::kChunkTiles;
@@ -1116,10 +1120,9 @@ struct DotShape {
 // sums.  A K-part of a split row adds into the K-part sums; the last K-part to
 // finish scales, stores and clears them.
 // sx: the activation scales, when the kernel quantized the activations itself.
-template <int NBX, bool ACC_OUT, bool SX_REG>
+template <int NBX, int NU, bool ACC_OUT, bool SX_REG>
 __device__ __forceinline__ void dot_finish(const GemvDesc &D, int group, int B, int lane,
-                                           int (&v)[kDotUnits][NBX], const float (&sx)[NBX]) {
-    constexpr int NU = kDotUnits;
+                                           int (&v)[NU][NBX], const float (&sx)[NBX]) {
     const int N = D.N;
     bool finish = true;
     if (D.kparts > 1) {
@@ -1182,7 +1185,7 @@ __device__ __forceinline__ void dot_finish(const GemvDesc &D, int group, int B, 
 // in natural order: x word 4 q + r of the tile meets decoded word r.
 template <int NBX, int NU>
 __device__ __forceinline__ void dot_chunk_i2(const uint32_t *st, int code_words, int lane,
-                                             const Consts &C, int (&acc)[kDotUnits][NBX][2]) {
+                                             const Consts &C, int (&acc)[NU][NBX][2]) {
     // table: byte c = weight of code c (0, +1, 0, -1)
     const uint32_t tab = 0xFF000100u;
 #pragma unroll
@@ -1228,7 +1231,7 @@ __device__ __forceinline__ uint32_t t3_field_x4(const uint32_t (&w)[5], int j) {
 // entry meets activation word j = (x[3j], x[3j+1], x[3j+2], 0) in one dp4a.
 template <int NBX, int NU>
 __device__ __forceinline__ void dot_chunk_t3(const uint32_t *st, int code_words, int lane,
-                                             const uint32_t *lut, int (&acc)[kDotUnits][NBX][2]) {
+                                             const uint32_t *lut, int (&acc)[NU][NBX][2]) {
     const uint8_t *lut_b = reinterpret_cast<const uint8_t *>(lut);
 #pragma unroll
     for (int tt = 0; tt < 2; tt++) {
@@ -1274,14 +1277,14 @@ __device__ __forceinline__ void dot_chunk_t3(const uint32_t *st, int code_words,
 // Modes 1 and 2 need no re-order launch.  They are used for calls of few
 // chunks, where that launch and its wait cost more than the per-chunk work.
 // FMT: the weight format (Sherry, or a comparison format with XMODE 0).
-template <int NBX, bool ACC_OUT, int XMODE, int FMT = kFmtSherry>
-__global__ void __launch_bounds__(DotShape<NBX, XMODE, FMT>::kThreads,
-                                  DotShape<NBX, XMODE, FMT>::kMinBlocks)
+template <int NBX, bool ACC_OUT, int XMODE, int FMT = kFmtSherry, int NU_ = kDotMaxUnits>
+__global__ void __launch_bounds__(DotShape<NBX, XMODE, FMT, NU_>::kThreads,
+                                  DotShape<NBX, XMODE, FMT, NU_>::kMinBlocks)
     gemv_dot_kernel(const __grid_constant__ GemvParams P) {
     constexpr bool XRAW = XMODE == 1;
     constexpr bool XBF = XMODE == 2;
     static_assert(FMT == kFmtSherry || XMODE == 0, "comparison formats read prepared activations");
-    using Shape = DotShape<NBX, XMODE, FMT>;
+    using Shape = DotShape<NBX, XMODE, FMT, NU_>;
     using F = FmtTraits<FMT>;
     constexpr int CT = F::kChunkTiles;
     constexpr int UCW = F::kUnitChunkWords;
@@ -1559,7 +1562,7 @@ __global__ void __launch_bounds__(DotShape<NBX, XMODE, FMT>::kThreads,
         } else if (b1 - start < nreal) {
             own_cut = true;  // first piece of an item cut at b1: finished after the barrier
         } else {
-            dot_finish<NBX, ACC_OUT, XBF>(D, cur.unit, B, lane, v, sx);
+            dot_finish<NBX, NU, ACC_OUT, XBF>(D, cur.unit, B, lane, v, sx);
         }
         start += nreal;
         if (start < b1) cursor_next(P, cur);
@@ -1586,7 +1589,7 @@ __global__ void __launch_bounds__(DotShape<NBX, XMODE, FMT>::kThreads,
 #pragma unroll
                 for (int b = 0; b < NBX; b++) v[u][b] += cut_sum[((w * NU + u) * NBX + b) * 32 + lane];
         }
-        dot_finish<NBX, ACC_OUT, XBF>(P.d[cur.id], cur.unit, B, lane, v, sx);
+        dot_finish<NBX, NU, ACC_OUT, XBF>(P.d[cur.id], cur.unit, B, lane, v, sx);
     }
 }
 
@@ -1657,16 +1660,22 @@ void launch_pipe(const GemvParams &gp, cudaStream_t stream) {
     launch_pdl(gemv_pipe_kernel<NB, ACC>, grid, kPipeThreads, smem, stream, gp);
 }
 
-template <int NBX, bool ACC, int XMODE>
-void launch_dot(const GemvParams &gp, cudaStream_t stream) {
+template <int NBX, bool ACC, int XMODE, int NU>
+void launch_dot_nu(const GemvParams &gp, cudaStream_t stream) {
     static int cache[64] = {0};
-    const size_t smem = DotShape<NBX, XMODE>::kSmem;
+    using Shape = DotShape<NBX, XMODE, kFmtSherry, NU>;
     // one chunk (of a unit group) per warp at most: a small GEMV spreads over as
     // many SMs as it has chunks (items cut between warps are summed in shared memory)
-    constexpr int threads = DotShape<NBX, XMODE>::kThreads, warps = DotShape<NBX, XMODE>::kWarps;
-    const int want = (gp.total_chunks + warps - 1) / warps;
-    const int grid = grid_for(gemv_dot_kernel<NBX, ACC, XMODE>, threads, smem, want, cache);
-    launch_pdl(gemv_dot_kernel<NBX, ACC, XMODE>, grid, threads, smem, stream, gp);
+    const int want = (gp.total_chunks + Shape::kWarps - 1) / Shape::kWarps;
+    const int grid = grid_for(gemv_dot_kernel<NBX, ACC, XMODE, kFmtSherry, NU>, Shape::kThreads,
+                              Shape::kSmem, want, cache);
+    launch_pdl(gemv_dot_kernel<NBX, ACC, XMODE, kFmtSherry, NU>, grid, Shape::kThreads, Shape::kSmem,
+               stream, gp);
+}
+template <int NBX, bool ACC, int XMODE>
+void launch_dot(const GemvParams &gp, int nu, cudaStream_t stream) {
+    if (nu == 2) launch_dot_nu<NBX, ACC, XMODE, 2>(gp, stream);
+    else launch_dot_nu<NBX, ACC, XMODE, 1>(gp, stream);
 }
 
 template <int NB, bool ACC>
@@ -1763,9 +1772,9 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
             gp.thi[i] = hi[i];
         }
     }
-    // items of the dot kernel (B <= 2) hold kDotUnits 32-row units, the MMA kernel's one
+    // items of the dot kernel (B <= 2) hold one or two 32-row units, the MMA kernel's one
     const bool dot = pipelined && B <= 2;
-    const int nu = dot ? kDotUnits : 1;
+    const int nu = dot && chunks > (int64_t)kDotPairMinChunksPerSM * sm_count() ? 2 : 1;
     int64_t off = 0;
     int wb = 0, ub16 = 0, cb = 0, cb32 = 0;
     for (int i = 0; i < count; i++) {
@@ -1863,17 +1872,17 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
     // same as one, while dp4a work grows with B) -- measured on the decode stack
     if (dot) {
         if (raw_bf) {  // bf16 calls have no accumulator form
-            if (B == 1) launch_dot<1, false, 2>(gp, stream); else launch_dot<2, false, 2>(gp, stream);
+            if (B == 1) launch_dot<1, false, 2>(gp, nu, stream); else launch_dot<2, false, 2>(gp, nu, stream);
         } else if (raw_x) {
             if (B == 1) {
-                if (acc_out) launch_dot<1, true, 1>(gp, stream); else launch_dot<1, false, 1>(gp, stream);
+                if (acc_out) launch_dot<1, true, 1>(gp, nu, stream); else launch_dot<1, false, 1>(gp, nu, stream);
             } else {
-                if (acc_out) launch_dot<2, true, 1>(gp, stream); else launch_dot<2, false, 1>(gp, stream);
+                if (acc_out) launch_dot<2, true, 1>(gp, nu, stream); else launch_dot<2, false, 1>(gp, nu, stream);
             }
         } else if (B == 1) {
-            if (acc_out) launch_dot<1, true, 0>(gp, stream); else launch_dot<1, false, 0>(gp, stream);
+            if (acc_out) launch_dot<1, true, 0>(gp, nu, stream); else launch_dot<1, false, 0>(gp, nu, stream);
         } else {
-            if (acc_out) launch_dot<2, true, 0>(gp, stream); else launch_dot<2, false, 0>(gp, stream);
+            if (acc_out) launch_dot<2, true, 0>(gp, nu, stream); else launch_dot<2, false, 0>(gp, nu, stream);
         }
     } else if (pipelined) {
         if (B <= 8) {
@@ -2057,14 +2066,19 @@ int64_t cmp_ws_words(int fmt, int64_t K, int B) {
     return fmt == kFmtT3 ? round_words((int64_t)B * cmp_tiles(fmt, K) * 32) : 0;
 }
 
-template <int NBX, bool ACC, int FMT>
-void launch_dot_fmt(const GemvParams &gp, cudaStream_t stream) {
+template <int NBX, bool ACC, int FMT, int NU>
+void launch_dot_fmt_nu(const GemvParams &gp, cudaStream_t stream) {
     static int cache[64] = {0};
-    using Shape = DotShape<NBX, 0, FMT>;
+    using Shape = DotShape<NBX, 0, FMT, NU>;
     const size_t smem = Shape::kSmem;
     const int want = (gp.total_chunks + Shape::kWarps - 1) / Shape::kWarps;
-    const int grid = grid_for(gemv_dot_kernel<NBX, ACC, 0, FMT>, Shape::kThreads, smem, want, cache);
-    launch_pdl(gemv_dot_kernel<NBX, ACC, 0, FMT>, grid, Shape::kThreads, smem, stream, gp);
+    const int grid = grid_for(gemv_dot_kernel<NBX, ACC, 0, FMT, NU>, Shape::kThreads, smem, want, cache);
+    launch_pdl(gemv_dot_kernel<NBX, ACC, 0, FMT, NU>, grid, Shape::kThreads, smem, stream, gp);
+}
+template <int NBX, bool ACC, int FMT>
+void launch_dot_fmt(const GemvParams &gp, int nu, cudaStream_t stream) {
+    if (nu == 2) launch_dot_fmt_nu<NBX, ACC, FMT, 2>(gp, stream);
+    else launch_dot_fmt_nu<NBX, ACC, FMT, 1>(gp, stream);
 }
 
 sherry_status cmp_launch(int fmt, const GemvCall *calls, int count, int B, bool acc_out,
@@ -2085,14 +2099,15 @@ sherry_status cmp_launch(int fmt, const GemvCall *calls, int count, int B, bool 
             return SHERRY_ERR_ALIGN;
         if (c.N > (int64_t)1 << 28) return SHERRY_ERR_UNSUPPORTED;
         words += cmp_ws_words(fmt, c.K, B);
-        const int64_t groups = ((c.N + kUnitRows - 1) / kUnitRows + kDotUnits - 1) / kDotUnits;
-        chunks += groups * (cmp_tiles(fmt, c.K) / (fmt == kFmtT3 ? 2 : 4));
+        chunks += (c.N + kUnitRows - 1) / kUnitRows * (cmp_tiles(fmt, c.K) / (fmt == kFmtT3 ? 2 : 4));
     }
     if (words > 0 && (!workspace || !aligned(workspace, 256))) return workspace ? SHERRY_ERR_ALIGN
                                                                                 : SHERRY_ERR_WORKSPACE;
     if (workspace_bytes < (size_t)words * 4) return SHERRY_ERR_WORKSPACE;
     if (words > 0x7FFFFFFF || chunks > 0x7FFFFFFF) return SHERRY_ERR_UNSUPPORTED;
 
+    // one or two 32-row units per item, as for Sherry calls
+    const int nu = chunks > (int64_t)kDotPairMinChunksPerSM * sm_count() ? 2 : 1;
     static thread_local GemvParams gp;
     static thread_local CmpXParams xp;
     std::memset(&gp, 0, sizeof(gp));
@@ -2115,7 +2130,7 @@ sherry_status cmp_launch(int fmt, const GemvCall *calls, int count, int B, bool 
         D.N = (int)c.N;
         D.T = Tc;
         D.units32 = (int)((c.N + kUnitRows - 1) / kUnitRows);
-        D.units = (D.units32 + kDotUnits - 1) / kDotUnits;
+        D.units = (D.units32 + nu - 1) / nu;
         D.nchunk = Tc / ct;
         D.kparts = 1;
         D.cpp = D.nchunk;
@@ -2150,15 +2165,15 @@ sherry_status cmp_launch(int fmt, const GemvCall *calls, int count, int B, bool 
     }
     if (fmt == kFmtI2) {
         if (B == 1) {
-            if (acc_out) launch_dot_fmt<1, true, kFmtI2>(gp, stream); else launch_dot_fmt<1, false, kFmtI2>(gp, stream);
+            if (acc_out) launch_dot_fmt<1, true, kFmtI2>(gp, nu, stream); else launch_dot_fmt<1, false, kFmtI2>(gp, nu, stream);
         } else {
-            if (acc_out) launch_dot_fmt<2, true, kFmtI2>(gp, stream); else launch_dot_fmt<2, false, kFmtI2>(gp, stream);
+            if (acc_out) launch_dot_fmt<2, true, kFmtI2>(gp, nu, stream); else launch_dot_fmt<2, false, kFmtI2>(gp, nu, stream);
         }
     } else {
         if (B == 1) {
-            if (acc_out) launch_dot_fmt<1, true, kFmtT3>(gp, stream); else launch_dot_fmt<1, false, kFmtT3>(gp, stream);
+            if (acc_out) launch_dot_fmt<1, true, kFmtT3>(gp, nu, stream); else launch_dot_fmt<1, false, kFmtT3>(gp, nu, stream);
         } else {
-            if (acc_out) launch_dot_fmt<2, true, kFmtT3>(gp, stream); else launch_dot_fmt<2, false, kFmtT3>(gp, stream);
+            if (acc_out) launch_dot_fmt<2, true, kFmtT3>(gp, nu, stream); else launch_dot_fmt<2, false, kFmtT3>(gp, nu, stream);
         }
     }
     return launch_status("sherry_cmp_gemv");

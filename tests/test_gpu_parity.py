@@ -196,6 +196,34 @@ def test_gemv_grouped_cut_items(B, shapes):
             assert_y_matches(y.cpu().numpy(), ref)
 
 
+@pytest.mark.parametrize("B", [1, 2])
+def test_gemv_grouped_two_unit_items_with_odd_units(B):
+    """A call large enough for items of two 32-row units (more than 64 chunks
+    of 32 rows x 512 weights per SM), whose GEMVs have an odd number of units
+    and ragged rows, so the last item of a GEMV holds one unit; items are cut
+    between warps at many places.  Every output against the oracle, through the
+    in-kernel re-order (one grouped call) and the re-order launch (prepare + run)."""
+    shapes = [(4000, 8192), (1000, 8192), (33, 8192), (4064, 4096), (1, 8192), (2100, 8192),
+              (4000, 8192), (999, 2048)] * 2
+    items, refs = [], []
+    for li, (N, K) in enumerate(shapes):
+        codes, scales = oracle.pack(synth.latent_weights(N, K, seed=500 + li))
+        x = synth.int8_uniform((B, K), seed=600 + li)
+        items.append((dev_codes(codes), dev(scales), dev(x),
+                      torch.zeros((B, N), dtype=torch.float32, device="cuda")))
+        refs.append(oracle.gemv(codes, scales, x, K))
+    chunks = sum((N + 31) // 32 * (K // 512) for N, K in shapes)
+    assert chunks > 64 * torch.cuda.get_device_properties(0).multi_processor_count
+    g = S.GroupedGemv(items, B=B)
+    for run in (g, lambda: (g.prepare(), g.run())):
+        for it in items:
+            it[3].fill_(float("nan"))
+        run()
+        torch.cuda.synchronize()
+        for (_, _, _, y), ref in zip(items, refs):
+            assert_y_matches(y.cpu().numpy(), ref)
+
+
 def test_gemv_full_size_decode_stack_as_benched():
     """The benchmark's launch: the 16-layer 1B stack, 112 GEMVs at B = 1, one
     re-order launch and one GEMV launch (one grouped call, and prepare + run),
