@@ -314,7 +314,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 // tensor memory) on zeroed operands, with no data movement and no barrier
 // between them: the int8 rate the GEMM's MMAs can reach on this device.
 constexpr int kProbeThreads = 128;
-constexpr size_t kProbeSmem = (size_t)kABytes + kBBytes + 1024;
+constexpr int kProbeN = 256;                                  // widest UMMA N
+constexpr size_t kProbeSmem = (size_t)kABytes + kProbeN * kBK + 1024;
+constexpr uint32_t kProbeIdesc = (2u << 4) | (1u << 7) | (1u << 10) |
+                                 ((uint32_t)(kProbeN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
 
 __global__ void __launch_bounds__(kProbeThreads, 1) mma_probe_kernel(int iters) {
     extern __shared__ uint8_t smem_raw[];
@@ -322,7 +325,7 @@ __global__ void __launch_bounds__(kProbeThreads, 1) mma_probe_kernel(int iters) 
     uint8_t *smem = smem_raw + ((1024 - (raw_addr & 1023)) & 1023);
     __shared__ __align__(8) uint64_t done;
     __shared__ uint32_t tmem_base;
-    for (int i = threadIdx.x; i < (kABytes + kBBytes) / 16; i += blockDim.x)
+    for (int i = threadIdx.x; i < (kABytes + kProbeN * kBK) / 16; i += blockDim.x)
         reinterpret_cast<uint4 *>(smem)[i] = make_uint4(0u, 0u, 0u, 0u);
     fence_proxy_async_smem();  // the zeroed operands, to the tensor core's view
     if (threadIdx.x == 0) {
@@ -330,7 +333,7 @@ __global__ void __launch_bounds__(kProbeThreads, 1) mma_probe_kernel(int iters) 
         fence_mbar_init();
     }
     if (threadIdx.x < 32) {
-        tmem_alloc(&tmem_base, kBN);
+        tmem_alloc(&tmem_base, kProbeN);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -342,7 +345,7 @@ __global__ void __launch_bounds__(kProbeThreads, 1) mma_probe_kernel(int iters) 
 #pragma unroll
             for (int k = 0; k < kBK / 32; k++)
                 umma_i8(tmem_base, smem_desc_sw128(a_addr + 32 * k), smem_desc_sw128(b_addr + 32 * k),
-                        kIdesc, (it | k) != 0);
+                        kProbeIdesc, (it | k) != 0);
         }
         umma_commit(&done);
         volatile int no_abort = 0;
@@ -352,7 +355,7 @@ __global__ void __launch_bounds__(kProbeThreads, 1) mma_probe_kernel(int iters) 
     __syncthreads();
     if (threadIdx.x < 32) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, kBN);
+        tmem_dealloc(tmem_base, kProbeN);
     }
 }
 
