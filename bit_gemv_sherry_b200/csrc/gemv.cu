@@ -25,7 +25,9 @@
 //   gemv_pipe_kernel  B >= 3: the same rings; the int8 MMA m16n8k32 takes the
 //                     decoded weights as its A fragment from registers and one
 //                     batch row per column, so batches up to 8 cost the same
-//                     MMA count as one.
+//                     MMA count as one.  Its activation fragments come from a
+//                     layout in fragment order (xw_word), so that each warp
+//                     load covers whole 128-byte lines.
 //   gemv_kernel       the general fallback (K not a multiple of 512, or code
 //                     rows not 16-byte aligned), MMA from registers.
 //   xprep_kernel      re-orders int8 activations, or quantizes bf16 ones per
@@ -54,7 +56,7 @@ struct GemvDesc {
     const uint32_t *codes;
     const float *scales;
     const float *xscale;  // per batch row activation scales (bf16 front-end), else null
-    const uint4 *xw;      // re-ordered activations [B][Tp][32 words]
+    const uint4 *xw;      // re-ordered activations (layout: see xw_word)
     const int8_t *x;      // raw int8 activations [B][K] (re-ordered inside the dot kernel)
     const uint16_t *xbf;  // raw bf16 activations [B][K] (quantized inside the dot kernel)
     void *out;            // float y[B][N] or int32 acc[B][N]
@@ -114,7 +116,7 @@ struct XprepParams {
     int count;
     int B;
     int total_units;
-    int pad;
+    int xrows;            // layout of the re-ordered activations (see xw_word)
     XprepDesc d[SHERRY_MAX_GROUP];
 };
 
@@ -124,7 +126,7 @@ struct XprepF32Desc {
     const float *x;       // [B][K] activations; SwiGLU: the gate outputs g
     const float *u;       // SwiGLU: the up outputs [B][K]; null for plain fp32
     float *xscale;        // per batch row activation scales written here
-    uint32_t *xw;         // re-ordered activations [B][Tp][32 words], or null
+    uint32_t *xw;         // re-ordered activations (see xw_word), or null
     int8_t *q;            // natural-order int8 output [B][K] (front-end alone), or null
     uint32_t *zero;       // split-K partial sums and counters to clear
     int K;
@@ -137,7 +139,7 @@ struct XprepF32Params {
     int count;
     int B;
     int total_clusters;
-    int pad;
+    int xrows;            // layout of the re-ordered activations (see xw_word)
     XprepF32Desc d[SHERRY_MAX_GROUP];
 };
 
@@ -172,6 +174,30 @@ int64_t padded_tiles(int64_t K) {
 }
 int64_t round_words(int64_t w) { return (w + 63) / 64 * 64; }  // 256-byte regions
 
+// Layout of a call's re-ordered activations, fixed by the batch B alone so
+// that a prepared workspace and the run that reads it always agree.
+//   B <= 2 (the small-batch kernel): [b][Tp][32 words], tile by tile.
+//   B >= 3 (the MMA kernels): batch rows in groups of R = xgroup_rows(B) rows
+//   (4 for B <= 4, else 8; the last group padded), laid out as
+//   [group][chunk c][uint4 j][row r][tile t of the chunk][word e]: uint4 j of
+//   tile 4c + t of row r holds the tile's re-ordered words 4j .. 4j+3.  A
+//   warp's fragment load j of a chunk (lane (g, t) reads row g of the group,
+//   tile t) then covers 64 R contiguous bytes, i.e. 2 or 4 whole 128-byte
+//   lines, where the tile-by-tile layout spread it over 16 or 32 lines.
+__host__ __device__ __forceinline__ int xgroup_rows(int B) { return B <= 2 ? 0 : (B <= 4 ? 4 : 8); }
+// rows of the region: B, or B padded to whole groups
+int64_t xw_rows(int B) {
+    const int R = xgroup_rows(B);
+    return R ? (int64_t)(B + R - 1) / R * R : (int64_t)B;
+}
+// word index of re-ordered word l (0..31) of tile t of batch row b; R =
+// xgroup_rows(B), Tp a multiple of 4
+__device__ __forceinline__ size_t xw_word(int R, int Tp, int b, int t, int l) {
+    if (R == 0) return ((size_t)b * Tp + t) * 32 + l;
+    const int grp = b / R, r = b - grp * R;
+    return (((((size_t)grp * (Tp >> 2) + (t >> 2)) * 8 + (l >> 2)) * R + r) * 4 + (t & 3)) * 4 + (l & 3);
+}
+
 // K-parts per 32-row unit in the pipelined kernel.
 int64_t kparts_for(int64_t K) {
     const int64_t nchunk = padded_tiles(K) / kChunkTiles;
@@ -187,13 +213,14 @@ int64_t split_words(int64_t N, int64_t K, int B) {
 
 // Workspace words of one GEMV: re-ordered activations, then the split-K words.
 int64_t ws_words(int64_t N, int64_t K, int B) {
-    return round_words((int64_t)B * padded_tiles(K) * 32) + split_words(N, K, B);
+    return round_words(xw_rows(B) * padded_tiles(K) * 32) + split_words(N, K, B);
 }
 
 // ---------------------------------------------------------------------------
 // Activation re-order
 // ---------------------------------------------------------------------------
-// xw[b][t][q] (t < Tp): word q = 2 (4 i + beta) + h holds the activations met
+// Word q (of 32) of tile t (t < Tp) of batch row b, stored at xw_word(b, t, q):
+// q = 2 (4 i + beta) + h holds the activations met
 // by char4(i, beta, h) of tile t: bytes x[b][128 t + 16 k' + 64 h + 4 beta + i],
 // k' = 0..3; tiles t >= K/128 are zero so that padded chunks contribute
 // nothing.  The split-K partial sums and counters are cleared.
@@ -294,7 +321,7 @@ __global__ void __launch_bounds__(256) xprep_kernel(const __grid_constant__ Xpre
                 if (t < T)
                     raw = quant_word(__ldg(reinterpret_cast<const uint2 *>(row + (size_t)t * SHERRY_TILE_K) + lane),
                                      inv);
-                D.xw[((size_t)b * D.Tp + t) * 32 + lane] = reorder_word(raw, lane);
+                D.xw[xw_word(P.xrows, D.Tp, b, t, lane)] = reorder_word(raw, lane);
             }
         } else if (local < D.xunits) {
             const int b = local / D.Tp, t = local - b * D.Tp;
@@ -303,7 +330,7 @@ __global__ void __launch_bounds__(256) xprep_kernel(const __grid_constant__ Xpre
             const uint32_t raw = t < T ? __ldg(reinterpret_cast<const uint32_t *>(
                                              D.x + (size_t)b * D.K + (size_t)t * SHERRY_TILE_K) + lane)
                                        : 0u;
-            D.xw[(size_t)local * 32 + lane] = reorder_word(raw, lane);
+            D.xw[xw_word(P.xrows, D.Tp, b, t, lane)] = reorder_word(raw, lane);
         } else {
             const int w = (local - D.xunits) * 32 + lane;
             if (w < D.zero_words) D.zero[w] = 0u;
@@ -408,7 +435,7 @@ __global__ void __launch_bounds__(kF32Threads) xprep_f32_kernel(const __grid_con
         if (D.q)
             reinterpret_cast<uint32_t *>(D.q + row + (size_t)t * SHERRY_TILE_K)[lane] = raw;
         else
-            D.xw[((size_t)b * D.Tp + t) * 32 + lane] = reorder_word(raw, lane);
+            D.xw[xw_word(P.xrows, D.Tp, b, t, lane)] = reorder_word(raw, lane);
     }
     // the GEMV's split-K words, cleared by its clusters together
     const int stride = P.B * kF32Cluster * kF32Threads;
@@ -605,9 +632,10 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const __grid_constan
             for (int nb = 0; nb < NB; nb++) {
                 const int b = nb * 8 + g;
                 const bool xvld = tv && b < P.B;
-                const uint4 *xp = D.xw + ((size_t)b * D.Tp + tile) * 8;
+                const int R = xgroup_rows(P.B);
 #pragma unroll
-                for (int k = 0; k < 8; k++) xv[nb][k] = xvld ? ld_x(xp + k) : make_uint4(0, 0, 0, 0);
+                for (int k = 0; k < 8; k++)
+                    xv[nb][k] = xvld ? ld_x(D.xw + xw_word(R, D.Tp, b, tile, 4 * k) / 4) : make_uint4(0, 0, 0, 0);
             }
             if (s + 1 < nslices) {  // prefetch the next slice's code words
                 const int nt = tile + 4;
@@ -860,6 +888,8 @@ __global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
     Consts C;
     load_consts(P, C);
     const int B = P.B;
+    const int xr = xgroup_rows(B);      // 4 or 8 rows per activation group
+    const size_t xstride = 4 * xr;     // uint4 between a tile's uint4 j and j + 1
 
     int start = b1;
     ItemCursor cur = {0, 0, 0};
@@ -920,12 +950,14 @@ __global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
         const int nreal = min(D.cpp, D.nchunk - first);
         const int c_begin = first + max(b0 - start, 0);
         const int c_end = first + min(b1 - start, nreal);
+        // lane (g, t) reads row g of each group (rows past the batch are padding
+        // whose columns are never stored; with 4-row groups lanes g >= 4 re-read
+        // rows g - 4), tile t of the chunk: chunk c at xstride * 8 uint4, uint4 j
+        // of the tile at xstride * j
         const uint4 *xrow[NB];
 #pragma unroll
-        for (int nb = 0; nb < NB; nb++) {
-            const int b = min(nb * 8 + g, B - 1);  // lanes past the batch: never stored
-            xrow[nb] = D.xw + (size_t)b * D.Tp * 8 + (size_t)t * 8;
-        }
+        for (int nb = 0; nb < NB; nb++)
+            xrow[nb] = D.xw + xw_word(xr, D.Tp, nb * xr + (g & (xr - 1)), t, 0) / 4;
 #pragma unroll
         for (int a = 0; a < 2; a++)
 #pragma unroll
@@ -936,7 +968,7 @@ __global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
             // tile t of the chunk, plane p, row g + 8 r: word t * 168 + 32 p + g + 8 r
             const uint32_t *st = ring + slot * kStageWords + t * kTileWordsPadded + g;
             // padded tiles hold zero activations, so no load is predicated
-            const size_t xoff = (size_t)c * kChunkTiles * 8;
+            const size_t xoff = (size_t)c * 8 * xstride;
             // the four rows of this lane (g, g + 8 of row block 0, g + 16, g + 24 of row
             // block 1) are decoded together, so each activation fragment is loaded once
             // for both row blocks, and the next position's fragments are loaded while
@@ -953,15 +985,15 @@ __global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
 #pragma unroll
             for (int nb = 0; nb < NB; nb++) {
                 xq[nb][0] = ld_x(xrow[nb] + xoff);
-                xq[nb][1] = ld_x(xrow[nb] + xoff + 1);
+                xq[nb][1] = ld_x(xrow[nb] + xoff + xstride);
             }
 #pragma unroll
             for (int i = 0; i < 4; i++) {
                 if (i < 3) {
 #pragma unroll
                     for (int nb = 0; nb < NB; nb++) {
-                        xn[nb][0] = ld_x(xrow[nb] + xoff + 2 * i + 2);
-                        xn[nb][1] = ld_x(xrow[nb] + xoff + 2 * i + 3);
+                        xn[nb][0] = ld_x(xrow[nb] + xoff + (2 * i + 2) * xstride);
+                        xn[nb][1] = ld_x(xrow[nb] + xoff + (2 * i + 3) * xstride);
                     }
                 }
                 const uint32_t tlo = C.tlo[i], thi = C.thi[i];
@@ -1756,6 +1788,7 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
     if (f32) std::memset(&fp, 0, sizeof(fp));
     xp.count = gp.count = fp.count = count;
     xp.B = gp.B = fp.B = B;
+    xp.xrows = fp.xrows = xgroup_rows(B);
     fp.total_clusters = count * B;
     gp.mul4 = 4u;
     gp.mul2 = 2u;
@@ -1781,7 +1814,7 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
         const GemvCall &c = calls[i];
         uint32_t *region = static_cast<uint32_t *>(workspace) + off;
         const int Tp = (int)padded_tiles(c.K);
-        const int xw_words = (int)round_words((int64_t)B * Tp * 32);
+        const int xw_words = (int)round_words(xw_rows(B) * Tp * 32);
         const int units32 = (int)((c.N + kUnitRows - 1) / kUnitRows);
         const int units = (units32 + nu - 1) / nu;
         const int nchunk = Tp / kChunkTiles;

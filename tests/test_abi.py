@@ -41,18 +41,23 @@ def test_packed_and_workspace_sizes():
     assert S.codes_shape(33, 2048) == (2, 16, 5, 32)
     assert S.packed_bytes(3, 100) == 0
     assert S.packed_bytes(0, 128) == 0
-    # re-ordered activations (B rows of K padded to 512) + partial sums and counters
+    # re-ordered activations (rows of K padded to 512; B >= 3 pads the batch
+    # rows to groups of 4, or of 8 above B = 4) + partial sums and counters
     # up to 4 chunks per row: re-ordered activations only, no split-K region
-    assert S.gemv_workspace_bytes(100, 384, 3) == 3 * 512
+    assert S.gemv_workspace_bytes(100, 384, 3) == 4 * 512
+    assert S.gemv_workspace_bytes(100, 384, 4) == 4 * 512
+    assert S.gemv_workspace_bytes(100, 384, 5) == 8 * 512
+    assert S.gemv_workspace_bytes(100, 384, 9) == 16 * 512
+    assert S.gemv_workspace_bytes(100, 384, 16) == 16 * 512
     assert S.gemv_workspace_bytes(40, 1024, 2) == 2 * 8 * 128
     assert S.gemv_workspace_bytes(2048, 2048, 1) == 2048
     # up to 16 chunks per row: one K-part, re-ordered activations only
     assert S.gemv_workspace_bytes(2048, 8192, 1) == 4 * 64 * 32
-    assert S.gemv_workspace_bytes(100, 8192, 3) == 3 * 4 * 64 * 32
+    assert S.gemv_workspace_bytes(100, 8192, 3) == 4 * 4 * 64 * 32
     # 34 chunks per row -> 3 K-parts: activations, then partial sums [B][N] and one
     # counter per 32-row unit, rounded to 256 bytes
     assert S.gemv_workspace_bytes(2048, 17408, 1) == 4 * 136 * 32 + 256 * ((4 * (2048 + 64) + 255) // 256)
-    assert S.gemv_workspace_bytes(100, 17408, 3) == 3 * 4 * 136 * 32 + 256 * ((4 * (300 + 4) + 255) // 256)
+    assert S.gemv_workspace_bytes(100, 17408, 3) == 4 * 4 * 136 * 32 + 256 * ((4 * (300 + 4) + 255) // 256)
     assert S.gemv_workspace_bytes(16, 128, 0) == 0
 
 
