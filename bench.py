@@ -850,46 +850,64 @@ def main():
     # ---------------- end to end through the public API with pinned host buffers
     # Every step copies its activations from pinned host memory to the device,
     # runs the grouped GEMV and copies all 112 outputs back to pinned host
-    # memory.  The outputs alternate between two device buffers and their
-    # copy-back runs on a second stream, so step i's copy-back overlaps step
-    # i+1's GEMV; a buffer is rewritten only after its previous copy-back ended.
+    # memory.  Activations and outputs alternate between two device buffers:
+    # step i + 1's activations are copied in (on a copy-in stream) while step
+    # i's GEMV runs, and step i's outputs are copied back (on a copy-out
+    # stream) while step i + 1's GEMV runs.  A buffer is rewritten only after
+    # the GEMV (activations) or the copy-back (outputs) that last read it ended.
     x_pinned = x_all.cpu().pin_memory()
+    x_alt = torch.empty_like(x_all)
+    xs_alt = {2048: x_alt[:, :2048], 8192: x_alt[:, 2048:]}
     y_alt = torch.empty_like(y_all)
     ys_alt, o = [], 0
     for _, _, n, _, _, _ in layers:
         ys_alt.append(y_alt[o:o + n].view(1, n))
         o += n
-    step_alt = S.GroupedGemv([(codes, scales, xs[k], y) for (_, _, n, k, codes, scales), y
+    step_alt = S.GroupedGemv([(codes, scales, xs_alt[k], y) for (_, _, n, k, codes, scales), y
                               in zip(layers, ys_alt)], B=1)
-    e2e_steps, y_bufs = (step, step_alt), (y_all, y_alt)
+    e2e_steps, x_bufs, y_bufs = (step, step_alt), (x_all, x_alt), (y_all, y_alt)
     y_pinned = [torch.empty_like(y_all, device="cpu").pin_memory() for _ in range(2)]
-    copy_stream = torch.cuda.Stream(dev)
-    done = [torch.cuda.Event(), torch.cuda.Event()]
-    freed = [torch.cuda.Event(), torch.cuda.Event()]
+    in_stream, out_stream = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    x_ready = [torch.cuda.Event(), torch.cuda.Event()]   # activations of buffer j landed
+    done = [torch.cuda.Event(), torch.cuda.Event()]      # GEMV on buffers j ended
+    freed = [torch.cuda.Event(), torch.cuda.Event()]     # copy-back of outputs j ended
     h2d = x_pinned.numel()
     d2h = 4 * y_all.numel()
     K_e2e = max(3, min(K, 2000))
 
-    def e2e_step(i):
+    def copy_in(i):
         j = i & 1
+        in_stream.wait_event(done[j])          # the GEMV that last read buffer j ended
+        with torch.cuda.stream(in_stream):
+            x_bufs[j].copy_(x_pinned, non_blocking=True)
+        x_ready[j].record(in_stream)
+
+    def e2e_step(i, last):
+        j = i & 1
+        if not last:
+            copy_in(i + 1)                     # next step's activations, during this GEMV
+        stream.wait_event(x_ready[j])
         stream.wait_event(freed[j])            # the buffer's previous copy-back ended
-        x_all.copy_(x_pinned, non_blocking=True)
         e2e_steps[j](sptr)
         done[j].record(stream)
-        copy_stream.wait_event(done[j])
-        with torch.cuda.stream(copy_stream):
+        out_stream.wait_event(done[j])
+        with torch.cuda.stream(out_stream):
             y_pinned[j].copy_(y_bufs[j], non_blocking=True)
-        freed[j].record(copy_stream)
-    for i in range(4):
-        e2e_step(i)
-    torch.cuda.synchronize(dev)
+        freed[j].record(out_stream)
+    for r in range(2):
+        copy_in(0)
+        for i in range(4):
+            e2e_step(i, i == 3)
+        torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
+    in_stream.wait_stream(stream)               # the first step's copy-in is inside the timed region
+    copy_in(0)
     for i in range(K_e2e):
-        e2e_step(i)
-    stream.wait_stream(copy_stream)             # the last copy-back is inside the timed region
+        e2e_step(i, i == K_e2e - 1)
+    stream.wait_stream(out_stream)              # the last copy-back is inside the timed region
     e1.record(stream)
     e1.synchronize()
     e2e_s = max_over_ranks(e0.elapsed_time(e1) / 1e3, dist if world > 1 else None, dev)
@@ -982,9 +1000,10 @@ def main():
                      "traffic": ncu_traffic, "traffic_unit": "bytes per launch"},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": K_e2e, "ms_per_step": e2e_s / K_e2e * 1e3,
-                "pipelining": "per step: H2D of x, sherry_gemv_grouped, D2H of all outputs; the "
-                              "D2H runs on a second stream from one of two output buffers, "
-                              "overlapping the next step's GEMV"},
+                "pipelining": "per step: H2D of x, sherry_gemv_grouped, D2H of all outputs; "
+                              "activations and outputs alternate between two device buffers, the "
+                              "H2D of step i+1 runs during step i's GEMV (copy-in stream) and the "
+                              "D2H of step i during step i+1's GEMV (copy-out stream)"},
     }
     if sharded_line is not None:
         line["sharded_step"] = sharded_line

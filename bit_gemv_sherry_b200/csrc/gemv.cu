@@ -107,7 +107,7 @@ struct XprepDesc {
     int K;
     int Tp;
     int unit_begin;       // first work unit of this GEMV
-    int xunits;           // int8: B * Tp (batch row, tile) units; bf16: (row, 4 tiles) units
+    int xunits;           // (batch row, 4 tiles) units: B * Tp / 4
     int zero_words;       // words at `zero` (0 if the rows are not split)
     int kind;             // 0: int8 activations, 1: bf16 activations quantized here
 };
@@ -289,7 +289,7 @@ __device__ __forceinline__ float row_absmax_bf16(const uint16_t *row, int K, int
     return m;
 }
 
-constexpr int kXqTiles = 4;  // tiles per bf16 quantize unit
+constexpr int kXqTiles = 4;  // tiles per re-order unit (one chunk of one batch row)
 
 __global__ void __launch_bounds__(256) xprep_kernel(const __grid_constant__ XprepParams P) {
     pdl_allow_dependents();
@@ -324,13 +324,19 @@ __global__ void __launch_bounds__(256) xprep_kernel(const __grid_constant__ Xpre
                 D.xw[xw_word(P.xrows, D.Tp, b, t, lane)] = reorder_word(raw, lane);
             }
         } else if (local < D.xunits) {
-            const int b = local / D.Tp, t = local - b * D.Tp;
+            // int8: unit = (row b, 4 tiles); the four tiles' loads are issued together
+            const int per_row = D.Tp / kXqTiles;
+            const int b = local / per_row, t0 = (local - b * per_row) * kXqTiles;
             const int T = D.K / SHERRY_TILE_K;
             // x rows are 4-byte aligned (x is, and K is a multiple of 128)
-            const uint32_t raw = t < T ? __ldg(reinterpret_cast<const uint32_t *>(
-                                             D.x + (size_t)b * D.K + (size_t)t * SHERRY_TILE_K) + lane)
-                                       : 0u;
-            D.xw[xw_word(P.xrows, D.Tp, b, t, lane)] = reorder_word(raw, lane);
+            const uint32_t *row = reinterpret_cast<const uint32_t *>(D.x + (size_t)b * D.K);
+            uint32_t raw[kXqTiles];
+#pragma unroll
+            for (int q = 0; q < kXqTiles; q++)
+                raw[q] = t0 + q < T ? __ldg(row + (size_t)(t0 + q) * (SHERRY_TILE_K / 4) + lane) : 0u;
+#pragma unroll
+            for (int q = 0; q < kXqTiles; q++)
+                D.xw[xw_word(P.xrows, D.Tp, b, t0 + q, lane)] = reorder_word(raw[q], lane);
         } else {
             const int w = (local - D.xunits) * 32 + lane;
             if (w < D.zero_words) D.zero[w] = 0u;
@@ -1832,7 +1838,7 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
         X.K = (int)c.K;
         X.Tp = Tp;
         X.unit_begin = wb;
-        X.xunits = bf ? B * ((Tp + kXqTiles - 1) / kXqTiles) : B * Tp;
+        X.xunits = B * (Tp / kXqTiles);
         X.zero_words = (int)split_words(c.N, c.K, B);
         X.kind = bf ? 1 : 0;
         if (f32) {
