@@ -867,7 +867,9 @@ __device__ __forceinline__ void pipe_finish(const GemvDesc &D, int unit, int B, 
     }
 }
 
-template <int NB, bool ACC_OUT>
+// XR: rows per activation group of the fragment-order layout, xgroup_rows(B)
+// (a template parameter so that every fragment load has a constant offset).
+template <int NB, bool ACC_OUT, int XR>
 __global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
     gemv_pipe_kernel(const __grid_constant__ GemvParams P) {
     pdl_allow_dependents();
@@ -894,8 +896,7 @@ __global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
     Consts C;
     load_consts(P, C);
     const int B = P.B;
-    const int xr = xgroup_rows(B);      // 4 or 8 rows per activation group
-    const size_t xstride = 4 * xr;     // uint4 between a tile's uint4 j and j + 1
+    constexpr int xstride = 4 * XR;     // uint4 between a tile's uint4 j and j + 1
 
     int start = b1;
     ItemCursor cur = {0, 0, 0};
@@ -963,7 +964,7 @@ __global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
         const uint4 *xrow[NB];
 #pragma unroll
         for (int nb = 0; nb < NB; nb++)
-            xrow[nb] = D.xw + xw_word(xr, D.Tp, nb * xr + (g & (xr - 1)), t, 0) / 4;
+            xrow[nb] = D.xw + xw_word(XR, D.Tp, nb * XR + (g & (XR - 1)), t, 0) / 4;
 #pragma unroll
         for (int a = 0; a < 2; a++)
 #pragma unroll
@@ -1688,14 +1689,14 @@ int grid_for(KernelT kernel, int threads, size_t smem, int want, int *cache) {
     return std::max(1, std::min(want, bps * sm_count()));
 }
 
-template <int NB, bool ACC>
+template <int NB, bool ACC, int XR>
 void launch_pipe(const GemvParams &gp, cudaStream_t stream) {
     static int cache[64] = {0};
     // one chunk per warp at most (items cut between warps are summed in shared memory)
     const size_t smem = PipeShape<NB>::kSmem;
     const int want = (gp.total_chunks + kPipeWarps - 1) / kPipeWarps;
-    const int grid = grid_for(gemv_pipe_kernel<NB, ACC>, kPipeThreads, smem, want, cache);
-    launch_pdl(gemv_pipe_kernel<NB, ACC>, grid, kPipeThreads, smem, stream, gp);
+    const int grid = grid_for(gemv_pipe_kernel<NB, ACC, XR>, kPipeThreads, smem, want, cache);
+    launch_pdl(gemv_pipe_kernel<NB, ACC, XR>, grid, kPipeThreads, smem, stream, gp);
 }
 
 template <int NBX, bool ACC, int XMODE, int NU>
@@ -1924,10 +1925,12 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
             if (acc_out) launch_dot<2, true, 0>(gp, nu, stream); else launch_dot<2, false, 0>(gp, nu, stream);
         }
     } else if (pipelined) {
-        if (B <= 8) {
-            if (acc_out) launch_pipe<1, true>(gp, stream); else launch_pipe<1, false>(gp, stream);
+        if (B <= 4) {
+            if (acc_out) launch_pipe<1, true, 4>(gp, stream); else launch_pipe<1, false, 4>(gp, stream);
+        } else if (B <= 8) {
+            if (acc_out) launch_pipe<1, true, 8>(gp, stream); else launch_pipe<1, false, 8>(gp, stream);
         } else {
-            if (acc_out) launch_pipe<2, true>(gp, stream); else launch_pipe<2, false>(gp, stream);
+            if (acc_out) launch_pipe<2, true, 8>(gp, stream); else launch_pipe<2, false, 8>(gp, stream);
         }
     } else {
         if (B <= 8) {

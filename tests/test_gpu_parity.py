@@ -84,6 +84,8 @@ GEMV_CASES = [(256, 1024, 1), (1, 128, 1), (17, 384, 3), (33, 640, 5), (40, 1152
               (19, 256, 9), (64, 512, 16), (2048, 2048, 1), (512, 2048, 4), (100, 3072, 2),
               (31, 8192, 1), (48, 8192, 16), (50, 1536, 2), (23, 512, 1), (70, 2560, 9),
               (129, 4096, 8), (37, 8192, 2), (130, 2048, 3),
+              # B = 5 ... 7 and 13 on the MMA kernel (activation groups of 8, padded rows)
+              (96, 1024, 5), (200, 512, 6), (45, 2048, 7), (33, 1536, 13),
               # rows split into K-parts (K > 8192), short last parts included:
               # 21 chunks = 11 + 10, 34 = 12 + 12 + 10, 40 = 3 x 14 - 2, 128 = 8 x 16
               (70, 10752, 1), (33, 17408, 2), (40, 20480, 9), (20, 65536, 1), (65, 17408, 16)]
