@@ -480,12 +480,36 @@ def time_3b_layer(S, torch, dev, reps=10):
     return out
 
 
+# Which activation each projection of a LLaMA layer reads: q, k and v the
+# attention input, o the attention output, gate and up the MLP input, down the
+# SwiGLU output.
+LAYER_INPUT = {"q": "attn_in", "k": "attn_in", "v": "attn_in", "o": "attn_out",
+               "gate": "mlp_in", "up": "mlp_in", "down": "mlp_act"}
+
+
+def layer_activations(torch, dev, entries, B, make, seed):
+    """One activation tensor per (layer, LLaMA input): the projections of a
+    layer that read the same input get the same tensor, as in the model
+    (q, k, v share one, gate and up another), so a grouped call prepares each
+    distinct input once.  entries: (layer, projection name, K) in stack order;
+    make(shape, gen) draws a tensor on the device.  Returns one tensor per entry."""
+    gen = torch.Generator(device=dev).manual_seed(seed)
+    made, out = {}, []
+    for layer, name, k in entries:
+        key = (layer, LAYER_INPUT[name])
+        if key not in made:
+            made[key] = make((B, k), gen)
+        out.append(made[key])
+    return out
+
+
 def time_3b_stack(S, torch, dev, peak_gbs, n_layers=16, reps=200, batches=(1, 4, 16)):
     """A 16-layer LLaMA-3.2-3B-shaped stack (7 projections per layer, 252 MB of
     codes > L2) at B = 1, 4, 16: one grouped call per step (re-order launch +
     GEMV launch), back to back.  The codes are random words on the device
     (every word is a valid code; the kernels' work does not depend on the
-    values), so no latents need to be made on the host."""
+    values), so no latents need to be made on the host.  Activations: int8
+    uniform in [-127, 127], one per (layer, LLaMA input), shared as in the model."""
     g = torch.Generator(device=dev).manual_seed(7)
     mats = []
     for layer in range(n_layers):
@@ -498,9 +522,12 @@ def time_3b_stack(S, torch, dev, peak_gbs, n_layers=16, reps=200, batches=(1, 4,
     out = {"layers": n_layers, "code_bytes": code_bytes, "codes": "random words on the device"}
     for B in batches:
         seed = {1: 1, 4: 2, 16: 3}.get(B, B)
-        xs = {k: torch.from_numpy(synth.int8_uniform((B, k), seed=seed)).to(dev) for k in (3072, 8192)}
+        entries = [(l, name, k) for l in range(n_layers) for name, _, k in synth.LLAMA_3B_LAYERS]
+        xs = layer_activations(torch, dev, entries, B,
+                               lambda shape, gen: torch.randint(-127, 128, shape, dtype=torch.int8,
+                                                                device=dev, generator=gen), seed)
         ys = [torch.empty((B, n), dtype=torch.float32, device=dev) for n, _, _, _ in mats]
-        step = S.GroupedGemv([(c, s, xs[k], y) for (n, k, c, s), y in zip(mats, ys)], B=B)
+        step = S.GroupedGemv([(c, s, x, y) for (n, k, c, s), x, y in zip(mats, xs, ys)], B=B)
         for _ in range(5):
             step()
         torch.cuda.synchronize()
@@ -531,12 +558,14 @@ def time_3b_stack(S, torch, dev, peak_gbs, n_layers=16, reps=200, batches=(1, 4,
 
 
 def time_bf16_stack(layers, S, torch, dev, reps=200):
-    """The same stack with bf16 activations: each step quantizes every GEMV's
-    activations per token (fused into the re-order launch) and runs the GEMVs."""
-    gen = torch.Generator(device="cpu").manual_seed(3)
-    xb = {k: torch.randn((1, k), generator=gen).to(torch.bfloat16).to(dev) for k in (2048, 8192)}
+    """The same stack with bf16 activations: each step quantizes every distinct
+    activation per token (fused into the re-order launch) and runs the GEMVs.
+    One bf16 input per (layer, LLaMA input), shared as in the model."""
+    xb = layer_activations(torch, dev, [(l, name, k) for l, name, _, k, _, _ in layers], 1,
+                           lambda shape, gen: torch.randn(shape, generator=gen, device=dev).to(
+                               torch.bfloat16), 3)
     ys = [torch.empty((1, n), dtype=torch.float32, device=dev) for _, _, n, _, _, _ in layers]
-    items = [(codes, scales, xb[k], y) for (_, _, n, k, codes, scales), y in zip(layers, ys)]
+    items = [(codes, scales, x, y) for (_, _, n, k, codes, scales), x, y in zip(layers, xb, ys)]
     step = S.GroupedGemvBf16(items, B=1)
     for _ in range(5):
         step()
@@ -550,7 +579,7 @@ def time_bf16_stack(layers, S, torch, dev, reps=200):
     t = e0.elapsed_time(e1) / 1e3 / reps
     code_bytes = sum(codes.numel() * 4 for _, _, _, _, codes, _ in layers)
     return {"us_per_step": t * 1e6, "weight_gbs": code_bytes / t / 1e9, "steps": reps,
-            "note": "bf16 activations quantized per token inside the step (x seed 3)"}
+            "note": "bf16 activations (one per layer input, seed 3) quantized per token inside the step"}
 
 
 def time_mlp_chain(layers, S, torch, dev, reps=200):

@@ -100,16 +100,15 @@ struct GemvParams {
 
 struct XprepDesc {
     const int8_t *x;
-    const uint16_t *xbf;  // bf16 activations to quantize (kind 1), else null
-    float *xscale;        // kind 1: per batch row activation scales written here
+    const uint16_t *xbf;  // bf16 activations to quantize (xprep_bf16_kernel), else null
+    float *xscale;        // bf16: per batch row activation scales written here
     uint32_t *xw;         // first word of this GEMV's workspace region
     uint32_t *zero;       // split-K partial sums and counters to clear
     int K;
     int Tp;
     int unit_begin;       // first work unit of this GEMV
-    int xunits;           // (batch row, 4 tiles) units: B * Tp / 4
+    int xunits;           // int8: (batch row, 4 tiles) warp units, B * Tp / 4; bf16: rows
     int zero_words;       // words at `zero` (0 if the rows are not split)
-    int kind;             // 0: int8 activations, 1: bf16 activations quantized here
 };
 
 struct XprepParams {
@@ -291,6 +290,74 @@ __device__ __forceinline__ float row_absmax_bf16(const uint16_t *row, int K, int
 
 constexpr int kXqTiles = 4;  // tiles per re-order unit (one chunk of one batch row)
 
+// bf16 front-end: one CTA per (GEMV, batch row), its warps taking the row's
+// tiles in turn.  Each warp loads its tiles once (rows up to kBfKeep tiles per
+// warp, K <= 8192, stay in registers between the passes), the CTA reduces the
+// token's absmax through shared memory, and each warp quantizes and re-orders
+// its tiles: one round trip to L2 per row instead of one per tile group.
+constexpr int kBfWarps = 8;
+constexpr int kBfKeep = 8;
+
+__device__ __forceinline__ float absmax4_bf16(uint2 v) {
+    return fmaxf(fmaxf(fabsf(bf16_lo(v.x)), fabsf(bf16_hi(v.x))),
+                 fmaxf(fabsf(bf16_lo(v.y)), fabsf(bf16_hi(v.y))));
+}
+
+__global__ void __launch_bounds__(kBfWarps * 32) xprep_bf16_kernel(const __grid_constant__ XprepParams P) {
+    pdl_allow_dependents();
+    pdl_wait();  // x may come from the kernel before; the last GEMV may still read xw
+    __shared__ float wmax[kBfWarps];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int u = blockIdx.x; u < P.total_units; u += gridDim.x) {
+        int lo = 0, hi = P.count - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (P.d[mid].unit_begin <= u) lo = mid; else hi = mid - 1;
+        }
+        const XprepDesc &D = P.d[lo];
+        const int local = u - D.unit_begin;
+        if (local < D.xunits) {
+            const int b = local;
+            const int T = D.K / SHERRY_TILE_K;
+            // four bf16 values per uint2: tile t, lane l at t * 32 + l
+            const uint2 *row = reinterpret_cast<const uint2 *>(D.xbf + (size_t)b * D.K);
+            uint2 keep[kBfKeep];
+            float m = 0.0f;
+#pragma unroll
+            for (int j = 0; j < kBfKeep; j++) {
+                const int t = warp + kBfWarps * j;
+                keep[j] = t < T ? __ldg(row + (size_t)t * 32 + lane) : make_uint2(0u, 0u);
+                m = fmaxf(m, absmax4_bf16(keep[j]));
+            }
+            for (int t = warp + kBfWarps * kBfKeep; t < T; t += kBfWarps)
+                m = fmaxf(m, absmax4_bf16(__ldg(row + (size_t)t * 32 + lane)));
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+            if (lane == 0) wmax[warp] = m;
+            __syncthreads();
+            float amax = wmax[0];
+#pragma unroll
+            for (int w = 1; w < kBfWarps; w++) amax = fmaxf(amax, wmax[w]);
+            const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+            if (threadIdx.x == 0) D.xscale[b] = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
+#pragma unroll
+            for (int j = 0; j < kBfKeep; j++) {
+                const int t = warp + kBfWarps * j;
+                if (t < D.Tp)
+                    D.xw[xw_word(P.xrows, D.Tp, b, t, lane)] =
+                        reorder_word(t < T ? quant_word(keep[j], inv) : 0u, lane);
+            }
+            for (int t = warp + kBfWarps * kBfKeep; t < D.Tp; t += kBfWarps)
+                D.xw[xw_word(P.xrows, D.Tp, b, t, lane)] =
+                    reorder_word(t < T ? quant_word(__ldg(row + (size_t)t * 32 + lane), inv) : 0u, lane);
+            __syncthreads();  // wmax is rewritten for the CTA's next row
+        } else {
+            const int w = (local - D.xunits) * (kBfWarps * 32) + (int)threadIdx.x;
+            if (w < D.zero_words) D.zero[w] = 0u;
+        }
+    }
+}
+
 __global__ void __launch_bounds__(256) xprep_kernel(const __grid_constant__ XprepParams P) {
     pdl_allow_dependents();
     pdl_wait();  // x may come from the kernel before; the last GEMV may still read xw
@@ -304,26 +371,7 @@ __global__ void __launch_bounds__(256) xprep_kernel(const __grid_constant__ Xpre
         }
         const XprepDesc &D = P.d[lo];
         const int local = u - D.unit_begin;
-        if (local < D.xunits && D.kind == 1) {
-            // bf16: unit = (row b, kXqTiles tiles); every unit of a row computes the
-            // row's absmax (the row is re-read from L2), then quantizes and re-orders
-            // its own tiles; the row's first unit stores the activation scale
-            const int per_row = (D.Tp + kXqTiles - 1) / kXqTiles;
-            const int b = local / per_row, g = local - b * per_row;
-            const int T = D.K / SHERRY_TILE_K;
-            const uint16_t *row = D.xbf + (size_t)b * D.K;
-            const float amax = row_absmax_bf16(row, D.K, lane);
-            const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
-            if (lane == 0 && g == 0) D.xscale[b] = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
-            const int t_end = min(D.Tp, (g + 1) * kXqTiles);
-            for (int t = g * kXqTiles; t < t_end; t++) {
-                uint32_t raw = 0u;
-                if (t < T)
-                    raw = quant_word(__ldg(reinterpret_cast<const uint2 *>(row + (size_t)t * SHERRY_TILE_K) + lane),
-                                     inv);
-                D.xw[xw_word(P.xrows, D.Tp, b, t, lane)] = reorder_word(raw, lane);
-            }
-        } else if (local < D.xunits) {
+        if (local < D.xunits) {
             // int8: unit = (row b, 4 tiles); the four tiles' loads are issued together
             const int per_row = D.Tp / kXqTiles;
             const int b = local / per_row, t0 = (local - b * per_row) * kXqTiles;
@@ -1736,6 +1784,30 @@ struct GemvCall {
     const float *xu = nullptr;  // with xf: SwiGLU up outputs, the activations being silu(xf) * xu
 };
 
+// First GEMV of a call that uses an activation pointer with a given K: a
+// small open-addressing table (SHERRY_MAX_GROUP entries at most).
+struct ActivationIndex {
+    static constexpr int kSlots = 4 * SHERRY_MAX_GROUP;
+    const void *ptr[kSlots] = {};
+    int64_t k[kSlots] = {};
+    int first[kSlots] = {};
+    // the GEMV that first used (p, K), registering gemv i if none did
+    int find_or_add(const void *p, int64_t K, int i) {
+        uint64_t h = (reinterpret_cast<uintptr_t>(p) >> 4) * 0x9E3779B97F4A7C15ull ^ (uint64_t)K;
+        for (int n = 0; n < kSlots; n++) {
+            const int s = (int)((h + (uint64_t)n) % kSlots);
+            if (!ptr[s]) {
+                ptr[s] = p;
+                k[s] = K;
+                first[s] = i;
+                return i;
+            }
+            if (ptr[s] == p && k[s] == K) return first[s];
+        }
+        return i;
+    }
+};
+
 // Words after a GEMV's region for the activation scales of the bf16 front-end.
 constexpr int64_t kActScaleWords = 64;  // >= SHERRY_MAX_GEMV_BATCH, 256-byte region
 
@@ -1812,6 +1884,7 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
             gp.thi[i] = hi[i];
         }
     }
+    ActivationIndex first_user;
     // items of the dot kernel (B <= 2) hold one or two 32-row units, the MMA kernel's one
     const bool dot = pipelined && B <= 2;
     const int nu = dot && chunks > (int64_t)kDotPairMinChunksPerSM * sm_count() ? 2 : 1;
@@ -1839,9 +1912,8 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
         X.K = (int)c.K;
         X.Tp = Tp;
         X.unit_begin = wb;
-        X.xunits = B * (Tp / kXqTiles);
+        X.xunits = bf ? B : B * (Tp / kXqTiles);
         X.zero_words = (int)split_words(c.N, c.K, B);
-        X.kind = bf ? 1 : 0;
         if (f32) {
             XprepF32Desc &F = fp.d[i];
             F.x = c.xf;
@@ -1875,8 +1947,21 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
         D.kparts = kparts;
         D.cpp = cpp;
         D.chunk_begin = cb;
+        // A GEMV whose activations an earlier GEMV of the call already prepares
+        // (same int8 or bf16 pointer, same K) reads that GEMV's region instead of
+        // re-ordering them again: q, k and v, or gate and up, share one copy.
+        // Only a call that prepares and runs (the run phase alone may not see x).
+        if (phase == kBoth && !f32) {
+            const int j = first_user.find_or_add(c.x ? (const void *)c.x : (const void *)c.xbf, c.K, i);
+            if (j != i) {
+                D.xw = gp.d[j].xw;
+                D.xscale = gp.d[j].xscale;
+                X.xunits = 0;
+            }
+        }
         off += ws_words(c.N, c.K, B) + (bf ? kActScaleWords : 0);
-        wb += X.xunits + (X.zero_words + 31) / 32;
+        // zero units: 32 words per warp (int8), 256 per CTA (bf16)
+        wb += X.xunits + (X.zero_words + (c.xbf ? kBfWarps * 32 : 32) - 1) / (c.xbf ? kBfWarps * 32 : 32);
         ub16 += (int)((c.N + 15) / 16);
         cb += units * nchunk;
         cb32 += units32 * nchunk;
@@ -1900,6 +1985,9 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
     if ((phase & kPrepare) && !raw_x && !raw_bf) {
         if (f32) {
             launch_xprep_f32(fp, stream);
+        } else if (calls[0].xbf) {  // a call's GEMVs are all bf16 or all int8
+            launch_pdl(xprep_bf16_kernel, std::max(1, std::min(wb, sm_count() * 8)), kBfWarps * 32, 0,
+                       stream, xp);
         } else {
             const int blocks = std::max(1, std::min((wb + 7) / 8, sm_count() * 8));
             launch_pdl(xprep_kernel, blocks, 256, 0, stream, xp);

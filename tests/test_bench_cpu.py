@@ -75,3 +75,24 @@ def test_clock_sampler_matches_the_gpu_by_uuid_or_pci_bus():
     one = bench.ClockSampler("0000", None)
     one.samples, one.seen = rows[:1], {rows[0][1]: rows[0][2]}
     assert one.summary(0.0, 2.0)["samples"] == 1
+
+
+def test_layer_activations_share_as_a_llama_layer():
+    import torch
+    spec = [("q", 8, 32), ("k", 4, 32), ("v", 4, 32), ("o", 8, 32), ("gate", 16, 32), ("up", 16, 32),
+            ("down", 8, 64)]
+    entries = [(l, name, k) for l in range(2) for name, _, k in spec]
+    calls = []
+
+    def make(shape, gen):
+        calls.append(shape)
+        return torch.randint(-127, 128, shape, dtype=torch.int8, generator=gen)
+
+    xs = bench.layer_activations(torch, torch.device("cpu"), entries, 3, make, 5)
+    assert len(xs) == 14 and len(calls) == 8          # 4 distinct inputs per layer
+    for base in (0, 7):
+        q, k, v, o, gate, up, down = xs[base:base + 7]
+        assert q is k and k is v and gate is up
+        assert len({id(q), id(o), id(gate), id(down)}) == 4
+        assert tuple(q.shape) == (3, 32) and tuple(down.shape) == (3, 64)
+    assert xs[0] is not xs[7]                          # layers do not share inputs

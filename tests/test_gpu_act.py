@@ -131,3 +131,29 @@ def test_gemv_bf16_large_group_through_the_reorder_launch(B):
         ref = (scales[rows][None, :] * s_ref[:, None]).astype(np.float32) * acc.astype(np.float32)
         assert np.array_equal(it[3].cpu().numpy()[:, rows], ref)
     assert S.device_error() == 0
+
+
+def test_gemv_bf16_grouped_shared_activations():
+    """bf16 GEMVs sharing one activation tensor, in a call that takes the
+    re-order launch (a split-K row rules out the in-kernel quantization): the
+    GEMVs after the first read its quantized copy and its token scales; y is
+    the oracle's bit for bit for every GEMV."""
+    cuda = torch.device("cuda")
+    B = 2
+    bits_a, bits_b = bf16_rows(B, 2048, seed=990), bf16_rows(B, 10752, seed=991)
+    xa, xb = to_bf16(bits_a), to_bf16(bits_b)
+    spec = [(96, 2048, xa, bits_a), (64, 10752, xb, bits_b), (200, 2048, xa, bits_a),
+            (33, 10752, xb, bits_b), (7, 2048, xa, bits_a)]
+    items, refs = [], []
+    for i, (n, k, xt, bits) in enumerate(spec):
+        codes, scales = oracle.pack(synth.latent_weights(n, k, seed=1000 + i))
+        q_ref, s_ref = oracle.quantize_act(bits)
+        acc = oracle.gemv_acc(codes, q_ref, n, k)
+        refs.append((scales[None, :] * s_ref[:, None]).astype(np.float32) * acc.astype(np.float32))
+        items.append((dev_codes(codes), dev(scales), xt,
+                      torch.full((B, n), float("nan"), dtype=torch.float32, device=cuda)))
+    S.gemv_bf16_grouped(items, B)
+    torch.cuda.synchronize()
+    for (_, _, _, y), ref in zip(items, refs):
+        assert np.array_equal(y.cpu().numpy(), ref)
+    assert S.device_error() == 0

@@ -401,3 +401,42 @@ def test_gemv_in_kernel_reorder_equals_reorder_launch(B):
         xo = buf[4:].view(B, K)                                             # 4-byte aligned only
         xo.copy_(tx)
         assert_y_matches(S.gemv(tc, ts, xo).cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("B", [3, 16])
+def test_gemv_grouped_shared_activations(B):
+    """GEMVs of one grouped call that share an activation tensor (q, k, v and
+    gate, up of a layer do) re-use one re-ordered copy of it; the same pointer
+    with another K (a prefix view) is a different activation and is prepared on
+    its own.  Shares in mixed order, one split-K row among them (whose partial
+    sums are still cleared), every output against the oracle; then the same
+    items through prepare + run, which prepares every GEMV's own copy."""
+    cuda = torch.device("cuda")
+    xa = synth.int8_uniform((B, 3072), seed=901)
+    xb = synth.int8_uniform((B, 10752), seed=902)
+    xa_d, xb_d = dev(xa), dev(xb)
+    xa_pre = xa_d[:, :1024]                       # same pointer as xa_d, K = 1024 (strided rows)
+    xa_pre_c = xa_pre.contiguous()
+    spec = [(96, 3072, xa_d, xa), (64, 10752, xb_d, xb), (33, 3072, xa_d, xa),
+            (70, 1024, xa_pre_c, np.ascontiguousarray(xa[:, :1024])), (128, 3072, xa_d, xa),
+            (40, 10752, xb_d, xb)]
+    items, refs = [], []
+    for i, (n, k, xt, xh) in enumerate(spec):
+        codes, scales = oracle.pack(synth.latent_weights(n, k, seed=910 + i))
+        items.append((dev_codes(codes), dev(scales), xt,
+                      torch.full((B, n), float("nan"), dtype=torch.float32, device=cuda)))
+        refs.append(oracle.gemv(codes, scales, xh, k))
+    S.gemv_grouped(items, B=B)
+    torch.cuda.synchronize()
+    for (_, _, _, y), ref in zip(items, refs):
+        assert_y_matches(y.cpu().numpy(), ref)
+    g = S.GroupedGemv(items, B=B)
+    for _ in range(2):
+        for it in items:
+            it[3].fill_(float("nan"))
+        g.prepare()
+        g.run()
+        torch.cuda.synchronize()
+        for (_, _, _, y), ref in zip(items, refs):
+            assert_y_matches(y.cpu().numpy(), ref)
+    assert S.device_error() == 0
