@@ -1785,18 +1785,29 @@ struct GemvCall {
 };
 
 // First GEMV of a call that uses an activation pointer with a given K: a
-// small open-addressing table (SHERRY_MAX_GROUP entries at most).
+// small open-addressing table (SHERRY_MAX_GROUP entries at most).  A slot is
+// live only if it carries the current call's stamp, so starting a call costs
+// one increment instead of clearing the table.
 struct ActivationIndex {
     static constexpr int kSlots = 4 * SHERRY_MAX_GROUP;
-    const void *ptr[kSlots] = {};
-    int64_t k[kSlots] = {};
-    int first[kSlots] = {};
-    // the GEMV that first used (p, K), registering gemv i if none did
+    const void *ptr[kSlots];
+    int64_t k[kSlots];
+    int first[kSlots];
+    uint32_t stamp[kSlots] = {};
+    uint32_t now = 0;
+    void start_call() {
+        if (++now == 0) {  // the stamps wrapped: clear them once
+            std::memset(stamp, 0, sizeof(stamp));
+            now = 1;
+        }
+    }
+    // the GEMV that first used (p, K) in this call, registering gemv i if none did
     int find_or_add(const void *p, int64_t K, int i) {
-        uint64_t h = (reinterpret_cast<uintptr_t>(p) >> 4) * 0x9E3779B97F4A7C15ull ^ (uint64_t)K;
+        const uint64_t h = (reinterpret_cast<uintptr_t>(p) >> 4) * 0x9E3779B97F4A7C15ull ^ (uint64_t)K;
         for (int n = 0; n < kSlots; n++) {
             const int s = (int)((h + (uint64_t)n) % kSlots);
-            if (!ptr[s]) {
+            if (stamp[s] != now) {
+                stamp[s] = now;
                 ptr[s] = p;
                 k[s] = K;
                 first[s] = i;
@@ -1884,7 +1895,8 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
             gp.thi[i] = hi[i];
         }
     }
-    ActivationIndex first_user;
+    static thread_local ActivationIndex first_user;
+    first_user.start_call();
     // items of the dot kernel (B <= 2) hold one or two 32-row units, the MMA kernel's one
     const bool dot = pipelined && B <= 2;
     const int nu = dot && chunks > (int64_t)kDotPairMinChunksPerSM * sm_count() ? 2 : 1;
