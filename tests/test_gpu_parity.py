@@ -103,7 +103,9 @@ def test_gemv_matches_oracle(N, K, B):
     assert_y_matches(y.cpu().numpy(), oracle.gemv(codes, scales, x, K))
 
 
-@pytest.mark.parametrize("N,K,B", [(37, 640, 1), (16, 1152, 7), (70, 384, 12)])
+@pytest.mark.parametrize("N,K,B", [(37, 640, 1), (16, 1152, 7), (70, 384, 12),
+                                   # the MMA kernel's accumulator form, each activation group size
+                                   (100, 512, 3), (64, 2048, 5), (33, 1024, 12), (40, 10752, 16)])
 def test_gemv_random_words_full_int8_range(N, K, B):
     # every 32-bit pattern is a valid code; activations cover [-128, 127]
     rng = np.random.default_rng(N + K + B)
