@@ -1870,12 +1870,22 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
     if (nf32 != 0 && nf32 != count) return SHERRY_ERR_UNSUPPORTED;
     const bool f32 = nf32 == count;
 
-    static thread_local XprepParams xp;
-    static thread_local XprepF32Params fp;
-    static thread_local GemvParams gp;
-    std::memset(&xp, 0, sizeof(xp));
-    std::memset(&gp, 0, sizeof(gp));
-    if (f32) std::memset(&fp, 0, sizeof(fp));
+    // Launch parameters live in thread-local storage (they are too large for the
+    // stack frame of every call).  Each is reached once through a reference, so
+    // the loops below do not pay a thread-local address lookup per access, and
+    // only the header and the descriptors in use are cleared (the kernels read
+    // no descriptor past `count`).
+    static thread_local XprepParams xp_tls;
+    static thread_local XprepF32Params fp_tls;
+    static thread_local GemvParams gp_tls;
+    static thread_local ActivationIndex index_tls;
+    XprepParams &xp = xp_tls;
+    XprepF32Params &fp = fp_tls;
+    GemvParams &gp = gp_tls;
+    ActivationIndex &first_user = index_tls;
+    std::memset(&xp, 0, offsetof(XprepParams, d) + (size_t)count * sizeof(XprepDesc));
+    std::memset(&gp, 0, offsetof(GemvParams, d) + (size_t)count * sizeof(GemvDesc));
+    if (f32) std::memset(&fp, 0, offsetof(XprepF32Params, d) + (size_t)count * sizeof(XprepF32Desc));
     xp.count = gp.count = fp.count = count;
     xp.B = gp.B = fp.B = B;
     xp.xrows = fp.xrows = xgroup_rows(B);
@@ -1895,7 +1905,6 @@ sherry_status gemv_launch(const GemvCall *calls, int count, int B, bool acc_out,
             gp.thi[i] = hi[i];
         }
     }
-    static thread_local ActivationIndex first_user;
     first_user.start_call();
     // items of the dot kernel (B <= 2) hold one or two 32-row units, the MMA kernel's one
     const bool dot = pipelined && B <= 2;

@@ -114,8 +114,21 @@ def _check(status, where):
         raise SherryError(status, where)
 
 
+# The raw handle of a device's current stream.  torch's private accessor skips
+# building a Stream object (about 2 us per call on the host); the public one is
+# the fallback.
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
+def _stream_handle(device):
+    if _raw_stream is not None:
+        idx = device.index if device.index is not None else torch.cuda.current_device()
+        return _raw_stream(idx)
+    return torch.cuda.current_stream(device).cuda_stream
+
+
 def _stream(t):
-    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+    return ctypes.c_void_p(_stream_handle(t.device))
 
 
 def _ptr(t):
@@ -137,7 +150,7 @@ _workspaces = {}
 def workspace(nbytes, device):
     """A cached device scratch buffer of at least `nbytes` for (device, current stream)."""
     device = torch.device(device)
-    key = (device.index, torch.cuda.current_stream(device).cuda_stream)
+    key = (device.index, _stream_handle(device))
     buf = _workspaces.get(key)
     if buf is None or buf.numel() < nbytes:
         buf = torch.empty(max(nbytes, 1 << 16), dtype=torch.uint8, device=device)
@@ -194,7 +207,7 @@ class GroupedPack:
 
     def __call__(self, stream=None):
         s = ctypes.c_void_p(stream if stream is not None
-                            else torch.cuda.current_stream(self.device).cuda_stream)
+                            else _stream_handle(self.device))
         _check(lib().sherry_pack_grouped(ctypes.cast(self.descs, ctypes.c_void_p), self.n, s),
                "sherry_pack_grouped")
 
@@ -432,7 +445,7 @@ class GroupedGemvF32:
 
     def __call__(self, stream=None):
         s = ctypes.c_void_p(stream if stream is not None
-                            else torch.cuda.current_stream(self.device).cuda_stream)
+                            else _stream_handle(self.device))
         _check(lib().sherry_gemv_f32_grouped(*self.args, s), "sherry_gemv_f32_grouped")
 
 
@@ -468,17 +481,17 @@ class GroupedGemv:
 
     def __call__(self, stream=None):
         s = ctypes.c_void_p(stream if stream is not None
-                            else torch.cuda.current_stream(self.device).cuda_stream)
+                            else _stream_handle(self.device))
         _check(lib().sherry_gemv_grouped(*self.args, s), "sherry_gemv_grouped")
 
     def prepare(self, stream=None):
         s = ctypes.c_void_p(stream if stream is not None
-                            else torch.cuda.current_stream(self.device).cuda_stream)
+                            else _stream_handle(self.device))
         _check(lib().sherry_gemv_prepare(*self.args, s), "sherry_gemv_prepare")
 
     def run(self, stream=None):
         s = ctypes.c_void_p(stream if stream is not None
-                            else torch.cuda.current_stream(self.device).cuda_stream)
+                            else _stream_handle(self.device))
         _check(lib().sherry_gemv_run(*self.args, s), "sherry_gemv_run")
 
 
@@ -507,7 +520,7 @@ class GroupedGemvBf16:
 
     def __call__(self, stream=None):
         s = ctypes.c_void_p(stream if stream is not None
-                            else torch.cuda.current_stream(self.device).cuda_stream)
+                            else _stream_handle(self.device))
         _check(lib().sherry_gemv_bf16_grouped(*self.args, s), "sherry_gemv_bf16_grouped")
 
 
@@ -610,7 +623,7 @@ class GroupedCmpGemv:
 
     def __call__(self, stream=None):
         s = ctypes.c_void_p(stream if stream is not None
-                            else torch.cuda.current_stream(self.device).cuda_stream)
+                            else _stream_handle(self.device))
         _check(lib().sherry_cmp_gemv_grouped(*self.args, s), "sherry_cmp_gemv_grouped")
 
 
