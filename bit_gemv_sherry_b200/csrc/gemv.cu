@@ -803,12 +803,17 @@ __device__ __forceinline__ ItemCursor cursor_at_chunk(const GemvParams &P, int c
     start = D.chunk_begin + r.unit * D.nchunk + r.kp * D.cpp;
     return r;
 }
-// First chunk of the item holding chunk c; total_chunks for c >= total_chunks.
-__device__ __forceinline__ int item_start_at_or_before(const GemvParams &P, int c) {
+// The item boundary nearest to chunk c (c <= total_chunks): the start of the
+// item holding c, or the start of the next one if that is nearer.  Monotone in
+// c, so consecutive CTAs get valid ranges; rounding to the nearer end keeps a
+// CTA's range within half an item of its share.
+__device__ __forceinline__ int item_boundary_near(const GemvParams &P, int c) {
     if (c >= P.total_chunks) return P.total_chunks;
     int start;
-    cursor_at_chunk(P, c, start);
-    return start;
+    const ItemCursor r = cursor_at_chunk(P, c, start);
+    const GemvDesc &D = P.d[r.id];
+    const int end = start + min(D.cpp, D.nchunk - r.kp * D.cpp);
+    return (c - start <= end - c) ? start : end;
 }
 __device__ __forceinline__ void cursor_next(const GemvParams &P, ItemCursor &c) {
     if (++c.kp == P.d[c.id].kparts) {
@@ -931,7 +936,7 @@ __global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
     // 1/gridDim of the chunks, its warps equal chunk shares of them
     if (threadIdx.x < 2) {
         const long long tc = P.total_chunks, nb = gridDim.x;
-        cta_bound[threadIdx.x] = item_start_at_or_before(P, (int)((blockIdx.x + threadIdx.x) * tc / nb));
+        cta_bound[threadIdx.x] = item_boundary_near(P, (int)((blockIdx.x + threadIdx.x) * tc / nb));
     }
     __syncthreads();
     const int cta_lo = cta_bound[0];
@@ -1176,21 +1181,32 @@ struct FmtTraits {
     static constexpr int kUnitChunkWords = kChunkTiles * kTileWords * kUnitRows;
 };
 
-// 8 warps per CTA.  B = 1 with two units per item: 2 CTAs (16 warps) per SM,
-// 90 KB of shared memory per CTA, up to 128 registers per thread.
+// Shared memory of a CTA of the small-batch kernel with `warps` warps: the
+// rings, the stages' mbarriers, the cut-item sums and starts.
+constexpr size_t dot_smem_bytes(int warps, int stage_words, int cut_words) {
+    return (size_t)warps * ((size_t)kDotRing * stage_words * 4 + kDotRing * 8 + (size_t)cut_words * 4 + 4);
+}
+
+// 8 or 16 warps per CTA (see kWarps).  B = 1 with two units per item: one CTA
+// of 16 warps per SM, 180 KB of shared memory, up to 128 registers per thread.
 // XMODE 2 adds to each stage the chunk's raw bf16 activations (1 KB per batch row).
 template <int NBX, int XMODE = 0, int FMT = kFmtSherry, int NU_ = kDotMaxUnits>
 struct DotShape {
     static constexpr int NU = NU_;
-    static constexpr int kWarps = 8;
-    static constexpr int kThreads = kWarps * 32;
     static constexpr int kChunkTilesF = FmtTraits<FMT>::kChunkTiles;
     static constexpr int kCodeWords = NU * FmtTraits<FMT>::kUnitChunkWords;
     static constexpr int kXWords = NBX * kChunkTilesF * 32;                     // int8, decode order
     static constexpr int kBfWords = XMODE == 2 ? NBX * kChunkTiles * 64 : 0;    // raw bf16
     static constexpr int kStageWords = kCodeWords + kXWords + kBfWords;
-    static constexpr int kRingWords = kWarps * kDotRing * kStageWords;
     static constexpr int kCutWords = NU * NBX * 32;
+    // Two-unit items (large calls) run one CTA of 16 warps per SM where its
+    // rings fit: a CTA's chunk range is rounded to whole items once per SM
+    // instead of once per half, which halves the spread of work between SMs
+    // (items of 16 chunks against ~200 chunks per SM on the 1B stack).
+    static constexpr int kWarps =
+        (NU == 2 && dot_smem_bytes(16, kStageWords, kCutWords) + 1024 <= 227u * 1024u) ? 16 : 8;
+    static constexpr int kThreads = kWarps * 32;
+    static constexpr int kRingWords = kWarps * kDotRing * kStageWords;
     // after the rings: the stages' mbarriers [warp][stage], then per warp the
     // row sums of a later piece of a cut item [NU][NBX][32] and that item's
     // first chunk
@@ -1389,7 +1405,7 @@ __global__ void __launch_bounds__(DotShape<NBX, XMODE, FMT, NU_>::kThreads,
     __shared__ int cta_bound[2];
     if (threadIdx.x < 2) {
         const long long tc = P.total_chunks, nb = gridDim.x;
-        cta_bound[threadIdx.x] = item_start_at_or_before(P, (int)((blockIdx.x + threadIdx.x) * tc / nb));
+        cta_bound[threadIdx.x] = item_boundary_near(P, (int)((blockIdx.x + threadIdx.x) * tc / nb));
     }
     if (lane == 0) {
 #pragma unroll
