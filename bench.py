@@ -220,19 +220,21 @@ def run_reference(args, rank):
     def step():
         for codes, scales, k in data:
             oracle.gemv(codes, scales, xs[k], k)
-    warmup = max(0, min(args.warmup, 1))
-    for _ in range(warmup):
-        step()
-    # one step = the whole stack; the number of timed steps is bounded so that
-    # the run stays within about a minute of oracle time
+    # one step = the whole stack.  The first warm-up step sizes the run: the
+    # warm-up and the timed steps asked for are each bounded to about a minute
+    # of oracle time, and the line reports the counts that ran.
     t0 = time.perf_counter()
     step()
     first = time.perf_counter() - t0
-    steps = max(1, min(args.steps, int(60.0 / max(first, 1e-3))))
-    t0 = time.perf_counter()
-    for _ in range(steps - 1):
+    per_minute = max(1, int(60.0 / max(first, 1e-3)))
+    warmup = max(1, min(args.warmup, per_minute))
+    for _ in range(warmup - 1):
         step()
-    dt = (time.perf_counter() - t0 + first) / steps
+    steps = max(1, min(args.steps, per_minute))
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        step()
+    dt = (time.perf_counter() - t0) / steps
     value = sample_bytes / dt / 1e9
     cores = oracle.num_threads()
     sample = "the whole stack per step (%d GEMVs, %d weights, %d code bytes), %d steps" % (
