@@ -743,16 +743,18 @@ __global__ void __launch_bounds__(kGemvThreads) gemv_kernel(const __grid_constan
 // ---------------------------------------------------------------------------
 // Pipelined kernel (K % 512 == 0, codes 16-byte aligned).
 //
-//   * work item = (32-row unit, K-part of at most 4 chunks = 2048 weights per
-//     row); thread (g, t) decodes rows g, g+8, g+16, g+24 of the unit for tile
-//     4c + t of chunk c, so the activation fragments it loads feed 32 MMAs;
+//   * work item = (32-row unit, K-part of at most kMaxPartChunks chunks = 8192
+//     weights per row); thread (g, t) decodes rows g, g+8, g+16, g+24 of the
+//     unit for tile 4c + t of chunk c, so the activation fragments it loads
+//     feed 32 MMAs;
 //   * a chunk of a unit (32 rows x 4 tiles) is one contiguous 2560-byte block
 //     of the code layout; each warp streams its items' chunks through a
 //     private ring of kRing shared-memory stages filled by cp.async with
-//     consecutive lanes on consecutive 16 bytes, so an SM keeps ~100 KB of
-//     fully coalesced HBM reads in flight;
+//     consecutive lanes on consecutive 16 bytes, so an SM (one CTA of 16
+//     warps) keeps ~80 KB of fully coalesced HBM reads in flight;
 //   * each CTA takes a run of whole items (in GEMV order) of about 1/gridDim
-//     of the chunks and its warps split the run into equal chunk ranges; an
+//     of the chunks, its ends rounded to the nearer item boundary, and its
+//     warps split the run into equal chunk ranges; an
 //     item cut by a warp boundary is summed in shared memory by the warp that
 //     holds its first chunk, after one CTA barrier;
 //   * a unit with several K-parts adds its partial int32 sums into part_acc
@@ -1137,7 +1139,8 @@ __global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
 //     NU rows per lane;
 //   * work is split by chunk count, a chunk being 4 tiles of every unit of a
 //     group.  Each CTA takes a run of whole items holding about 1/gridDim of
-//     the chunks and its warps split the run into equal chunk ranges, so no
+//     the chunks (its ends rounded to the nearer item boundary) and its warps
+//     split the run into equal chunk ranges, so no
 //     warp ends the launch with a whole extra item to do.  An item cut by a
 //     warp boundary is summed by the warps holding its pieces: later pieces
 //     leave their row sums in shared memory, and after one CTA barrier the
