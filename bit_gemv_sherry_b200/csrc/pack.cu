@@ -20,7 +20,7 @@
 namespace sherry {
 namespace {
 
-constexpr int kPackThreads = 256;
+constexpr int kPackThreads = 128;  // 4 warps: 0.83 ms for the 1B stack's latents against 0.85 with 8, 0.86 with 16
 constexpr int kPackWarps = kPackThreads / 32;
 constexpr int kPackBatch = 8;      // tiles loaded per batch
 // fewest tiles a warp of a multi-warp row takes: rows up to K = 8192 get one
@@ -82,7 +82,7 @@ __device__ __forceinline__ void store_words(uint32_t *tile_out, const TileBits &
 }
 
 // One launch packs a group of matrices; matrix i owns CTAs cta_begin[i] ..
-// cta_begin[i+1]-1.  CTA = 8 warps; `wpr` warps share one row, warp `sub` of
+// cta_begin[i+1]-1.  CTA = 4 warps; `wpr` warps share one row, warp `sub` of
 // a row takes the `tpw` consecutive tiles sub * tpw .. and loads them
 // kPackBatch at a time (all loads of a batch in flight before the first tile
 // is packed).  Each lane sums its kept |w| in double over all its tiles; the
@@ -185,7 +185,7 @@ sherry_status pack_launch(PackDesc *descs, int count, cudaStream_t stream) {
         PackDesc &d = descs[i];
         const int64_t T = d.K / SHERRY_TILE_K;
         d.Npad = (d.N + SHERRY_ROW_GROUP - 1) / SHERRY_ROW_GROUP * SHERRY_ROW_GROUP;
-        // warps per row: as many as keep at least kPackMinTiles tiles each (up to 8)
+        // warps per row: as many as keep at least kPackMinTiles tiles each (up to 4)
         int wpr = 1;
         while (wpr < kPackWarps && (int64_t)wpr * 2 * kPackMinTiles <= T) wpr *= 2;
         d.wpr = wpr;
