@@ -1165,7 +1165,10 @@ __global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
 // with 1; a 2048 x 8192 GEMV: 7.3 us with 1, 9.1 with 2.
 constexpr int kDotMaxUnits = 2;
 constexpr int kDotPairMinChunksPerSM = 64;
-constexpr int kDotRing = 2;                  // stages per warp
+// Stages per warp.  Deeper rings with fewer warps (the same shared memory)
+// measured slower on the 1B stack with two-unit items: 16 warps x 2 stages
+// 52.5 us, 12 x 3 54.5 us, 8 x 4 62.3 us.
+constexpr int kDotRing = 2;
 // bf16 calls up to this many 32-row chunks per SM quantize and re-order x in
 // the dot kernel (each warp takes the token's absmax from the row itself, so
 // large calls keep the front-end launch); int8 calls of any size re-order x
@@ -1189,8 +1192,8 @@ struct FmtTraits {
 
 // Shared memory of a CTA of the small-batch kernel with `warps` warps: the
 // rings, the stages' mbarriers, the cut-item sums and starts.
-constexpr size_t dot_smem_bytes(int warps, int stage_words, int cut_words) {
-    return (size_t)warps * ((size_t)kDotRing * stage_words * 4 + kDotRing * 8 + (size_t)cut_words * 4 + 4);
+constexpr size_t dot_smem_bytes(int warps, int ring, int stage_words, int cut_words) {
+    return (size_t)warps * ((size_t)ring * stage_words * 4 + ring * 8 + (size_t)cut_words * 4 + 4);
 }
 
 // 8 or 16 warps per CTA (see kWarps).  B = 1 with two units per item: one CTA
@@ -1209,15 +1212,17 @@ struct DotShape {
     // rings fit: a CTA's chunk range is rounded to whole items once per SM
     // instead of once per half, which halves the spread of work between SMs
     // (items of 16 chunks against ~200 chunks per SM on the 1B stack).
-    static constexpr int kWarps =
-        (NU == 2 && dot_smem_bytes(16, kStageWords, kCutWords) + 1024 <= 227u * 1024u) ? 16 : 8;
+    static constexpr bool kPair =
+        NU == 2 && dot_smem_bytes(16, kDotRing, kStageWords, kCutWords) + 1024 <= 227u * 1024u;
+    static constexpr int kWarps = kPair ? 16 : 8;
+    static constexpr int kRing = kDotRing;  // stages per warp
     static constexpr int kThreads = kWarps * 32;
-    static constexpr int kRingWords = kWarps * kDotRing * kStageWords;
+    static constexpr int kRingWords = kWarps * kRing * kStageWords;
     // after the rings: the stages' mbarriers [warp][stage], then per warp the
     // row sums of a later piece of a cut item [NU][NBX][32] and that item's
     // first chunk
     static constexpr size_t kBarOffset = (size_t)kRingWords * 4;
-    static constexpr size_t kCutOffset = kBarOffset + (size_t)kWarps * kDotRing * 8;
+    static constexpr size_t kCutOffset = kBarOffset + (size_t)kWarps * kRing * 8;
     static constexpr size_t kSmem = kCutOffset + ((size_t)kWarps * kCutWords + kWarps) * 4;
     // CTAs per SM that fit the 227 KB of shared memory (1 KB reserved per CTA)
     static constexpr int kFit = (int)((227u * 1024u) / (kSmem + 1024u));
@@ -1404,7 +1409,8 @@ __global__ void __launch_bounds__(DotShape<NBX, XMODE, FMT, NU_>::kThreads,
     extern __shared__ __align__(128) uint32_t dot_smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     uint8_t *smem_bytes = reinterpret_cast<uint8_t *>(dot_smem);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem_bytes + Shape::kBarOffset) + warp * kDotRing;
+    constexpr int RING = Shape::kRing;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem_bytes + Shape::kBarOffset) + warp * RING;
     int *cut_sum = reinterpret_cast<int *>(smem_bytes + Shape::kCutOffset);
     int *cut_start = cut_sum + kWarps * Shape::kCutWords;
     // chunk range [b0, b1) of this warp; threads 0 and 1 find the CTA's bounds
@@ -1415,7 +1421,7 @@ __global__ void __launch_bounds__(DotShape<NBX, XMODE, FMT, NU_>::kThreads,
     }
     if (lane == 0) {
 #pragma unroll
-        for (int s = 0; s < kDotRing; s++) mbar_init(&bars[s], 1);
+        for (int s = 0; s < RING; s++) mbar_init(&bars[s], 1);
         fence_mbar_init();
     }
     // T3: entry c of the table = the triple of code c as three ternary bytes
@@ -1434,7 +1440,7 @@ __global__ void __launch_bounds__(DotShape<NBX, XMODE, FMT, NU_>::kThreads,
     const int b1 = cta_lo + (int)((warp + 1) * len / kWarps);
     // -1: no cut item starts before b0; -2: empty range (skipped when summing)
     if (lane == 0) cut_start[warp] = b0 < b1 ? -1 : -2;
-    uint32_t *ring = dot_smem + (size_t)warp * kDotRing * SW;
+    uint32_t *ring = dot_smem + (size_t)warp * RING * SW;
     const uint32_t ring_addr = smem_u32(ring);
     Consts C;
     load_consts(P, C);
@@ -1537,6 +1543,9 @@ __global__ void __launch_bounds__(DotShape<NBX, XMODE, FMT, NU_>::kThreads,
         issue_x_and_advance(0);
         inflight = 1u;
     }
+    // stages 1 .. RING - 2: later chunks in flight before the first is waited for
+#pragma unroll
+    for (int s = 1; s + 1 < RING; s++) issue(s);
 
     // ---- consumer side ----
     int slot = 0;
@@ -1575,7 +1584,7 @@ __global__ void __launch_bounds__(DotShape<NBX, XMODE, FMT, NU_>::kThreads,
 #pragma unroll
             for (int b = 0; b < NBX; b++) acc[u][b][0] = acc[u][b][1] = 0;
         for (int c = c_begin; c < c_end; c++) {
-            issue(slot ^ 1);  // the next chunk into the stage the previous chunk used
+            issue(slot == 0 ? RING - 1 : slot - 1);  // the stage the previous chunk used
             if (!stage_wait(&bars[slot], (phase >> slot) & 1u)) {
                 failed = true;
                 break;
@@ -1654,7 +1663,7 @@ __global__ void __launch_bounds__(DotShape<NBX, XMODE, FMT, NU_>::kThreads,
             }
             }
             __syncwarp();  // every lane is done with this stage before it is refilled
-            slot ^= 1;
+            slot = slot + 1 == RING ? 0 : slot + 1;
         }
         if (failed) break;
 #pragma unroll
@@ -1681,7 +1690,7 @@ __global__ void __launch_bounds__(DotShape<NBX, XMODE, FMT, NU_>::kThreads,
         // land (bounded) and leave the CTA's item summing alone
         if (lane == 0) atomicCAS(&g_gemv_device_error, 0u, (unsigned int)SHERRY_ERR_TIMEOUT);
 #pragma unroll
-        for (int s = 0; s < kDotRing; s++)
+        for (int s = 0; s < RING; s++)
             if (inflight & (1u << s)) stage_wait(&bars[s], (phase >> s) & 1u);
         own_cut = false;
     }
