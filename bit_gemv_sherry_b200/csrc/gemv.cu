@@ -1165,9 +1165,10 @@ __global__ void __launch_bounds__(kPipeThreads, SHERRY_PIPE_MIN_BLOCKS)
 // with 1; a 2048 x 8192 GEMV: 7.3 us with 1, 9.1 with 2.
 constexpr int kDotMaxUnits = 2;
 constexpr int kDotPairMinChunksPerSM = 64;
-// Stages per warp.  Deeper rings with fewer warps (the same shared memory)
-// measured slower on the 1B stack with two-unit items: 16 warps x 2 stages
-// 52.5 us, 12 x 3 54.5 us, 8 x 4 62.3 us.
+// Stages per warp.  Measured on the 1B stack with two-unit items: 16 warps x
+// 2 stages of 4-tile chunks 52.5 us; deeper rings with fewer warps (the same
+// shared memory) 54.5 us (12 x 3) and 62.3 us (8 x 4); 16 warps x 4 stages
+// of 2-tile chunks 58.8 us.
 constexpr int kDotRing = 2;
 // bf16 calls up to this many 32-row chunks per SM quantize and re-order x in
 // the dot kernel (each warp takes the token's absmax from the row itself, so
@@ -1175,7 +1176,6 @@ constexpr int kDotRing = 2;
 // in the kernel (measured on the 16-layer 1B stack: 54.5 us per step against
 // 56.6 us with the re-order launch).
 constexpr int kRawBfMaxChunksPerSM = 64;
-constexpr int kDotCodeWords = kChunkTiles * kTileWords;  // 640 words: one unit's chunk
 // Weight formats the small-batch kernel streams: Sherry, and the two ternary
 // packings the pages compare it against (arXiv 2601.07892, abstract; Figure 2
 // caption): 2 bits per weight, aligned ("I2"), and three weights in five bits
@@ -1205,17 +1205,17 @@ struct DotShape {
     static constexpr int kChunkTilesF = FmtTraits<FMT>::kChunkTiles;
     static constexpr int kCodeWords = NU * FmtTraits<FMT>::kUnitChunkWords;
     static constexpr int kXWords = NBX * kChunkTilesF * 32;                     // int8, decode order
-    static constexpr int kBfWords = XMODE == 2 ? NBX * kChunkTiles * 64 : 0;    // raw bf16
+    static constexpr int kBfWords = XMODE == 2 ? NBX * kChunkTilesF * 64 : 0;   // raw bf16
     static constexpr int kStageWords = kCodeWords + kXWords + kBfWords;
     static constexpr int kCutWords = NU * NBX * 32;
     // Two-unit items (large calls) run one CTA of 16 warps per SM where its
     // rings fit: a CTA's chunk range is rounded to whole items once per SM
     // instead of once per half, which halves the spread of work between SMs
     // (items of 16 chunks against ~200 chunks per SM on the 1B stack).
-    static constexpr bool kPair =
-        NU == 2 && dot_smem_bytes(16, kDotRing, kStageWords, kCutWords) + 1024 <= 227u * 1024u;
-    static constexpr int kWarps = kPair ? 16 : 8;
     static constexpr int kRing = kDotRing;  // stages per warp
+    static constexpr bool kPair =
+        NU == 2 && dot_smem_bytes(16, kRing, kStageWords, kCutWords) + 1024 <= 227u * 1024u;
+    static constexpr int kWarps = kPair ? 16 : 8;
     static constexpr int kThreads = kWarps * 32;
     static constexpr int kRingWords = kWarps * kRing * kStageWords;
     // after the rings: the stages' mbarriers [warp][stage], then per warp the
@@ -1594,18 +1594,18 @@ __global__ void __launch_bounds__(DotShape<NBX, XMODE, FMT, NU_>::kThreads,
             uint32_t *st = ring + slot * SW;
             if (XRAW) {  // raw words of the chunk's tiles -> the decode order, in place
                 uint32_t *xr = st + Shape::kCodeWords;
-                uint32_t w[NBX][kChunkTiles];
+                uint32_t w[NBX][CT];
 #pragma unroll
                 for (int b = 0; b < NBX; b++)
 #pragma unroll
-                    for (int tt = 0; tt < kChunkTiles; tt++)
-                        w[b][tt] = b < B ? reorder_word(xr[(b * kChunkTiles + tt) * 32 + lane], lane) : 0u;
+                    for (int tt = 0; tt < CT; tt++)
+                        w[b][tt] = b < B ? reorder_word(xr[(b * CT + tt) * 32 + lane], lane) : 0u;
                 __syncwarp();
 #pragma unroll
                 for (int b = 0; b < NBX; b++)
 #pragma unroll
-                    for (int tt = 0; tt < kChunkTiles; tt++)
-                        if (b < B) xr[(b * kChunkTiles + tt) * 32 + lane] = w[b][tt];
+                    for (int tt = 0; tt < CT; tt++)
+                        if (b < B) xr[(b * CT + tt) * 32 + lane] = w[b][tt];
                 __syncwarp();
             }
             if (XBF) {  // bf16 of the chunk's tiles -> quantized words in the decode order
@@ -1614,10 +1614,10 @@ __global__ void __launch_bounds__(DotShape<NBX, XMODE, FMT, NU_>::kThreads,
 #pragma unroll
                 for (int b = 0; b < NBX; b++)
 #pragma unroll
-                    for (int tt = 0; tt < kChunkTiles; tt++)
+                    for (int tt = 0; tt < CT; tt++)
                         if (b < B)
-                            xq[(b * kChunkTiles + tt) * 32 + lane] =
-                                reorder_word(quant_word(xb[(b * kChunkTiles + tt) * 32 + lane], sx_inv[b]), lane);
+                            xq[(b * CT + tt) * 32 + lane] =
+                                reorder_word(quant_word(xb[(b * CT + tt) * 32 + lane], sx_inv[b]), lane);
                 __syncwarp();
             }
             if (FMT == kFmtI2) {
@@ -1626,11 +1626,11 @@ __global__ void __launch_bounds__(DotShape<NBX, XMODE, FMT, NU_>::kThreads,
                 dot_chunk_t3<NBX, NU>(st, Shape::kCodeWords, lane, t3_lut, acc);
             } else {
 #pragma unroll
-            for (int tt = 0; tt < kChunkTiles; tt++) {
+            for (int tt = 0; tt < CT; tt++) {
                 TileDecoder6 d[NU];
 #pragma unroll
                 for (int u = 0; u < NU; u++) {
-                    const uint32_t *cw = st + u * kDotCodeWords + tt * kTileWords + lane;
+                    const uint32_t *cw = st + u * UCW + tt * kTileWords + lane;
                     d[u].load(C, cw[0], cw[32], cw[64], cw[96], cw[128]);
                 }
                 // activation words of tile tt: batch row b at b * 128, word q at q
