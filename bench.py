@@ -40,8 +40,8 @@ L2_BYTES = 126 * 2 ** 20
 # dram__bytes_read.sum + dram__bytes_write.sum of one launch of the timed GEMV
 # kernel (gemv_dot_kernel<1,false,1>) on the 16-layer stack, B = 1, from an ncu
 # capture of this kernel version (profiles/gemv_dot_decode_stack_b1.md):
-# 153,637,120 read + 3,396,352 written (16-warp CTAs, nearest item boundaries).
-NCU_TRAFFIC_BYTES = 153637120 + 3396352
+# 153,628,928 read + 3,467,264 written (16-warp CTAs, nearest item boundaries).
+NCU_TRAFFIC_BYTES = 153628928 + 3467264
 
 
 def parse_args():
