@@ -30,7 +30,9 @@ def _x(B, K, seed):
 # array also holds the int32 partial sums and the per-unit counters, which each
 # call must find cleared by the call before it.
 @pytest.mark.parametrize("N,K,B", [(2048, 8192, 1), (1000, 2048, 5), (4096, 4096, 16),
-                                   (33, 384, 3), (2048, 16384, 4), (70, 17408, 1)])
+                                   (33, 384, 3), (2048, 16384, 4), (70, 17408, 1),
+                                   # the largest K: 16 K-parts, 2 MiB of activations
+                                   (40, 131072, 16)])
 def test_static_matches_workspace_gemv_two_calls_in_a_row(N, K, B):
     codes, scales = _layer(N, K, seed=900 + N % 97)
     x1, x2 = _x(B, K, seed=901), _x(B, K, seed=902)
