@@ -1,5 +1,7 @@
 // api.cu -- shared host utilities of libsherry: status strings, the last CUDA
 // error text, the device error word, and the packed-size query.
+#include <cuda.h>
+
 #include <cstdio>
 #include <cstring>
 
@@ -27,6 +29,31 @@ sherry_status launch_status(const char *what) {
         return SHERRY_ERR_CUDA;
     }
     return SHERRY_OK;
+}
+
+namespace {
+void *driver_entry(const char *name) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+        return nullptr;
+    return p;
+}
+}  // namespace
+
+unsigned long long context_id() {
+    using GetCurrentFn = CUresult (*)(CUcontext *);
+    using GetIdFn = CUresult (*)(CUcontext, unsigned long long *);
+    static const GetCurrentFn get_current =
+        reinterpret_cast<GetCurrentFn>(driver_entry("cuCtxGetCurrent"));
+    static const GetIdFn get_id = reinterpret_cast<GetIdFn>(driver_entry("cuCtxGetId"));
+    if (!get_current || !get_id) return 0;
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr || get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
 }
 
 int sm_count() {

@@ -6,6 +6,7 @@
 // the tcgen05 tensor-core instructions used by the GEMM.
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 #include <cuda_runtime.h>
 
@@ -26,6 +27,22 @@ inline bool valid_k(int64_t K) { return K >= SHERRY_TILE_K && K % SHERRY_TILE_K 
 
 // Number of SMs of the current device (cached per device).
 int sm_count();
+
+// Identifier of the CUDA context current on this thread, unique over the
+// process's lifetime (cuCtxGetId), or 0 if none is current or the driver
+// does not provide it.  Per-device set-up that lives in a context (kernel
+// attributes, the device address of a module variable) is cached with the
+// identifier of the context it was made in and made again when the current
+// context differs: a cudaDeviceReset ends the device's primary context, and
+// the next one starts with default attributes and a new module image.
+unsigned long long context_id();
+
+// Blocks per SM of a kernel launch shape, kept per device with the context
+// it was measured in (the shared-memory attribute is set in that context).
+struct OccupancyCache {
+    std::atomic<unsigned long long> ctx[64];
+    std::atomic<int> bps[64];
+};
 
 // Reads and clears the error word of the GEMV kernels (after a device sync).
 sherry_status gemv_device_error();

@@ -398,9 +398,9 @@ sherry_status gemm_launch(const uint32_t *codes, const float *scales, const int8
         set_last_error("cuTensorMapEncodeTiled", cudaErrorInvalidValue);
         return SHERRY_ERR_CUDA;
     }
-    // the shared-memory attribute is per device: set it once on each device
-    // this kernel runs on
-    static std::atomic<bool> attr_set[kMaxDevices];
+    // the shared-memory attribute lives in the device's context: set it once
+    // per device and context this kernel runs in
+    static std::atomic<unsigned long long> attr_ctx[kMaxDevices];
     int dev = 0;
     {
         const cudaError_t e = cudaGetDevice(&dev);
@@ -410,7 +410,8 @@ sherry_status gemm_launch(const uint32_t *codes, const float *scales, const int8
         }
     }
     if (dev < 0 || dev >= kMaxDevices) return SHERRY_ERR_UNSUPPORTED;
-    if (!attr_set[dev].load(std::memory_order_acquire)) {
+    const unsigned long long ctx = context_id();
+    if (ctx == 0 || attr_ctx[dev].load(std::memory_order_acquire) != ctx) {
         const cudaError_t e = cudaFuncSetAttribute(gemm_kernel<ACC>,
                                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                    (int)kSmemBytes);
@@ -418,7 +419,7 @@ sherry_status gemm_launch(const uint32_t *codes, const float *scales, const int8
             set_last_error("sherry_gemm (shared memory attribute)", e);
             return SHERRY_ERR_CUDA;
         }
-        attr_set[dev].store(true, std::memory_order_release);
+        attr_ctx[dev].store(context_id(), std::memory_order_release);
     }
     const int64_t tiles = ((N + kBM - 1) / kBM) * ((M + kBN - 1) / kBN);
     if (tiles > 0x7FFFFFFF) return SHERRY_ERR_UNSUPPORTED;
@@ -450,7 +451,7 @@ extern "C" sherry_status sherry_probe_mma_i8(int iters, int *ctas, sherry_stream
     using namespace sherry;
     if (!ctas) return SHERRY_ERR_NULL;
     if (iters < 1) return SHERRY_ERR_SHAPE;
-    static std::atomic<bool> attr_set[kMaxDevices];
+    static std::atomic<unsigned long long> attr_ctx[kMaxDevices];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) {
@@ -458,14 +459,15 @@ extern "C" sherry_status sherry_probe_mma_i8(int iters, int *ctas, sherry_stream
         return SHERRY_ERR_CUDA;
     }
     if (dev < 0 || dev >= kMaxDevices) return SHERRY_ERR_UNSUPPORTED;
-    if (!attr_set[dev].load(std::memory_order_acquire)) {
+    const unsigned long long ctx = context_id();
+    if (ctx == 0 || attr_ctx[dev].load(std::memory_order_acquire) != ctx) {
         e = cudaFuncSetAttribute(mma_probe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)kProbeSmem);
         if (e != cudaSuccess) {
             set_last_error("sherry_probe_mma_i8 (shared memory attribute)", e);
             return SHERRY_ERR_CUDA;
         }
-        attr_set[dev].store(true, std::memory_order_release);
+        attr_ctx[dev].store(context_id(), std::memory_order_release);
     }
     *ctas = sm_count();
     mma_probe_kernel<<<*ctas, kProbeThreads, kProbeSmem, reinterpret_cast<cudaStream_t>(stream)>>>(iters);

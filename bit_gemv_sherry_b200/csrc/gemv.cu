@@ -17,17 +17,20 @@
 //     bytes meet the multiply-accumulate.
 //
 // Kernels:
-//   gemv_dot_kernel   B <= 2 (the decode path): per-warp cp.async rings of
-//                     4-tile chunks, dp4a against broadcast activation words,
-//                     chunk-balanced warp ranges, items cut between warps
-//                     summed in shared memory.  Small int8 calls copy raw x
-//                     and re-order it in the kernel (no re-order launch).
-//   gemv_pipe_kernel  B >= 3: the same rings; the int8 MMA m16n8k32 takes the
-//                     decoded weights as its A fragment from registers and one
-//                     batch row per column, so batches up to 8 cost the same
-//                     MMA count as one.  Its activation fragments come from a
-//                     layout in fragment order (xw_word), so that each warp
-//                     load covers whole 128-byte lines.
+//   gemv_dot_kernel   B <= 2 (the decode path): per-warp rings of 4-tile
+//                     chunks filled by bulk copies (cp.async.bulk completing
+//                     on one mbarrier per stage), dp4a against broadcast
+//                     activation words, chunk-balanced warp ranges, items cut
+//                     between warps summed in shared memory.  Small int8 calls
+//                     copy raw x and re-order it in the kernel (no re-order
+//                     launch).
+//   gemv_pipe_kernel  B >= 3: per-warp 3-stage cp.async rings of code chunks;
+//                     the int8 MMA m16n8k32 takes the decoded weights as its A
+//                     fragment from registers and one batch row per column, so
+//                     batches up to 8 cost the same MMA count as one.  Its
+//                     activation fragments come from a layout in fragment
+//                     order (xw_word), so that each warp load covers whole
+//                     128-byte lines.
 //   gemv_kernel       the general fallback (K not a multiple of 512, or code
 //                     rows not 16-byte aligned), MMA from registers.
 //   xprep_kernel      re-orders int8 activations, or quantizes bf16 ones per
@@ -1752,25 +1755,28 @@ void launch_xprep_f32(const XprepF32Params &p, cudaStream_t stream) {
 }
 
 template <typename KernelT>
-int grid_for(KernelT kernel, int threads, size_t smem, int want, int *cache) {
+int grid_for(KernelT kernel, int threads, size_t smem, int want, OccupancyCache &cache) {
     int dev = 0;
     cudaGetDevice(&dev);
-    int &bps = cache[dev & 63];
-    if (bps == 0) {
+    const int d = dev & 63;
+    const unsigned long long now = context_id();
+    int bps = cache.bps[d].load(std::memory_order_acquire);
+    if (bps == 0 || now == 0 || cache.ctx[d].load(std::memory_order_acquire) != now) {
         if (smem > 48 * 1024)
             cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        int n = 0;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, smem) != cudaSuccess ||
-            n < 1)
-            n = 1;
-        bps = n;
+        bps = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bps, kernel, threads, smem) != cudaSuccess ||
+            bps < 1)
+            bps = 1;
+        cache.bps[d].store(bps, std::memory_order_release);
+        cache.ctx[d].store(context_id(), std::memory_order_release);  // current now, if it was not
     }
     return std::max(1, std::min(want, bps * sm_count()));
 }
 
 template <int NB, bool ACC, int XR>
 void launch_pipe(const GemvParams &gp, cudaStream_t stream) {
-    static int cache[64] = {0};
+    static OccupancyCache cache;
     // one chunk per warp at most (items cut between warps are summed in shared memory)
     const size_t smem = PipeShape<NB>::kSmem;
     const int want = (gp.total_chunks + kPipeWarps - 1) / kPipeWarps;
@@ -1780,7 +1786,7 @@ void launch_pipe(const GemvParams &gp, cudaStream_t stream) {
 
 template <int NBX, bool ACC, int XMODE, int NU>
 void launch_dot_nu(const GemvParams &gp, cudaStream_t stream) {
-    static int cache[64] = {0};
+    static OccupancyCache cache;
     using Shape = DotShape<NBX, XMODE, kFmtSherry, NU>;
     // one chunk (of a unit group) per warp at most: a small GEMV spreads over as
     // many SMs as it has chunks (items cut between warps are summed in shared memory)
@@ -1798,7 +1804,7 @@ void launch_dot(const GemvParams &gp, int nu, cudaStream_t stream) {
 
 template <int NB, bool ACC>
 void launch_regs(const GemvParams &gp, cudaStream_t stream) {
-    static int cache[64] = {0};
+    static OccupancyCache cache;
     const int want = (gp.total_units16 + kGemvWarps - 1) / kGemvWarps;
     const int grid = grid_for(gemv_kernel<NB, ACC>, kGemvThreads, 0, want, cache);
     launch_pdl(gemv_kernel<NB, ACC>, grid, kGemvThreads, 0, stream, gp);
@@ -2250,7 +2256,7 @@ int64_t cmp_ws_words(int fmt, int64_t K, int B) {
 
 template <int NBX, bool ACC, int FMT, int NU>
 void launch_dot_fmt_nu(const GemvParams &gp, cudaStream_t stream) {
-    static int cache[64] = {0};
+    static OccupancyCache cache;
     using Shape = DotShape<NBX, 0, FMT, NU>;
     const size_t smem = Shape::kSmem;
     const int want = (gp.total_chunks + Shape::kWarps - 1) / Shape::kWarps;
@@ -2583,9 +2589,10 @@ static __device__ __align__(256) uint32_t g_gemv_static_scratch[SHERRY_STATIC_SC
 constexpr int kStaticMaxDevices = 64;
 std::mutex g_static_mu;
 void *g_static_ptr[kStaticMaxDevices] = {};
+unsigned long long g_static_ctx[kStaticMaxDevices] = {};
 
 // Device address of the scratch array on the current device, looked up once
-// per device.
+// per device and context.
 sherry_status static_scratch(void **out) {
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
@@ -2594,16 +2601,19 @@ sherry_status static_scratch(void **out) {
         return SHERRY_ERR_CUDA;
     }
     if (dev < 0 || dev >= kStaticMaxDevices) return SHERRY_ERR_UNSUPPORTED;
+    const unsigned long long now = context_id();
     std::lock_guard<std::mutex> lock(g_static_mu);
-    if (g_static_ptr[dev] == nullptr) {
+    if (g_static_ptr[dev] == nullptr || now == 0 || g_static_ctx[dev] != now) {
         void *p = nullptr;
         err = cudaGetSymbolAddress(&p, g_gemv_static_scratch);
         if (err != cudaSuccess || p == nullptr) {
+            g_static_ptr[dev] = nullptr;
             set_last_error("sherry_gemv_static (cudaGetSymbolAddress)",
                            err != cudaSuccess ? err : cudaErrorInvalidSymbol);
             return SHERRY_ERR_CUDA;
         }
         g_static_ptr[dev] = p;
+        g_static_ctx[dev] = context_id();  // the lookup made the context current if it was not
     }
     *out = g_static_ptr[dev];
     return SHERRY_OK;

@@ -50,6 +50,10 @@
  *     errors at the caller's next synchronisation.
  *   - No C++ exception crosses this interface.  Calls are thread-safe; two
  *     calls that share an output or a workspace must not overlap on the GPU.
+ *   - Calls run on the current device.  What a call sets up there once (the
+ *     kernels' shared-memory attributes, the static scratch's device address)
+ *     is kept per device together with the CUDA context it was made in, and
+ *     made again when another context is current, e.g. after cudaDeviceReset.
  *   - Integer results are exact: the dot products are accumulated in int32,
  *     which cannot overflow for K <= SHERRY_MAX_K, and converted to fp32
  *     exactly (|acc| <= 3K/4 * 128 < 2^24), so y = fl32(s * acc) with one
@@ -299,8 +303,9 @@ sherry_status sherry_gemv_f32_grouped(const sherry_gemv_f32_desc *descs, int cou
  *   SHERRY_STATIC_SCRATCH_BYTES, otherwise the call returns
  *   SHERRY_ERR_WORKSPACE with the two sizes in sherry_last_error().
  *   Set-up: the first call on a device (with that device current) looks up
- *   the array's device address (cudaGetSymbolAddress) once and caches it;
- *   make that first call before any stream capture.
+ *   the array's device address (cudaGetSymbolAddress) and caches it for the
+ *   device's current context (looked up again in a new context, e.g. after
+ *   cudaDeviceReset); make that first call before any stream capture.
  *   Sharing: every call on a device uses the same array.  Each call re-writes
  *   the activations and zeroes the partial sums and counters it needs before
  *   its GEMV kernel reads them, so consecutive calls are independent; calls
